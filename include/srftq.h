@@ -1,0 +1,168 @@
+/*
+ * srftq.h -- C ABI of the B200 rotate-then-quantize KV-cache codec (libsrftq.so).
+ *
+ * The codec is the one of "When Quantization Is Free" (technical summary):
+ * every head-dim vector x of an fp16 KV cache is rotated by
+ * SRFT(x) = pack(F diag(s) x) (Methodology 1; F the unitary DFT, s a fixed
+ * random sign vector), rescaled per channel by lambda, quantised with group
+ * absmax to signed int4 (two codes per byte) or int8 (Methodology 2, steps
+ * 1-5; Methodology 3 for per-channel + per-group scaling), and
+ * dequantised by the exact inverse. The SRHT variant replaces F by the
+ * normalised Walsh-Hadamard matrix ("HyperQuant", Methodology 1: H D x).
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * Shapes: a call covers S slices (e.g. layer x {K,V}) of N rows, each row
+ * holding H heads of d-element vectors. Vector (s, r, h) of an array with
+ * slice stride T rows lives at element offset ((s*T + r)*H + h) * per_vector.
+ *
+ *   x       fp16 (IEEE binary16 bit patterns)  [S][T_x][H][d]
+ *   codes   uint8                               [S][T_o][H][d*bits/8]
+ *   scales  fp16 bit patterns                   [S][T_o][H][d/group]
+ *   signs   int8, one row per (slice, head)     [S][H][d]   (< 0 means -1,
+ *           anything else +1)
+ *   lambda  float32, one row per (slice, head)  [S][H][d]   (finite, > 0)
+ *
+ * Packed coordinate order of the rotated vector y (d reals):
+ *   y_0 = X_0, y_1 = X_{d/2}, y_{2k} = sqrt2 Re X_k, y_{2k+1} = sqrt2 Im X_k
+ *   (0 < k < d/2), X = F (s * x) with kernel exp(-2 pi i k n / d) / sqrt(d).
+ * SRHT: y = H_d (s * x) / sqrt(d), Sylvester natural order.
+ *
+ * Quantiser (per vector, per group g of `group` consecutive coordinates):
+ *   w_j = y_j / lambda_j;  a_g = max |w_j|;  qmax = 7 (int4) or 127 (int8)
+ *   sigma_g = fp16 round-to-nearest-even of (a_g / qmax), saturated at 65504
+ *   q_j = clamp(round-half-even(w_j / sigma_g), -qmax, qmax); 0 if sigma_g == 0
+ *   int4: element 2k in the low nibble of byte k, 2k+1 in the high nibble.
+ * Dequantiser: x_hat = s * R^T (lambda * sigma * q), rounded to fp16.
+ *
+ * Ownership and execution: every pointer is a device pointer owned by the
+ * caller; the library allocates no device memory and keeps no per-call
+ * state. Calls enqueue work on `stream` (a cudaStream_t; NULL = legacy
+ * default stream) and return without synchronising: SRFTQ_OK means
+ * "launched". A call with zero vectors launches nothing. Every other
+ * successful call launches exactly one kernel.
+ *
+ * Errors: argument errors are detected on the host before anything is
+ * launched and return a negative status. A launch failure returns
+ * SRFTQ_ERR_CUDA. Device-side guards (bounded waits) record into a
+ * library-wide word read by srftq_check_device(); they never trap.
+ *
+ * Alignment: every pointer must be 16-byte aligned; slice strides are in
+ * rows and must be >= N (slices may not overlap). Inputs and outputs must
+ * not overlap (no in-place use). Non-finite inputs give unspecified codes,
+ * never a fault.
+ *
+ * Supported: d in {16, 32, 64, 128, 256}; group a power of two with
+ * 8 <= group <= d; bits in {4, 8}; heads >= 1; rotation SRFT or SRHT.
+ */
+#ifndef SRFTQ_H
+#define SRFTQ_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Status codes returned by every entry point. */
+#define SRFTQ_OK                0
+#define SRFTQ_ERR_INVALID_ARG  (-1)  /* null pointer, bad size, overlap  */
+#define SRFTQ_ERR_UNSUPPORTED  (-2)  /* d / group / bits / rotation       */
+#define SRFTQ_ERR_MISALIGNED   (-3)  /* pointer not 16-byte aligned       */
+#define SRFTQ_ERR_CUDA         (-4)  /* CUDA runtime or driver error      */
+#define SRFTQ_ERR_DEVICE_CHECK (-5)  /* a device-side guard fired         */
+
+/* Rotation kinds. */
+#define SRFTQ_ROT_SRFT 0  /* sign-randomised real-packed FFT (Methodology 1) */
+#define SRFTQ_ROT_SRHT 1  /* sign-randomised Walsh-Hadamard ("HyperQuant")  */
+
+/* Codec configuration: head dimension, heads per row, group size, code
+ * width and rotation kind. Plain data; the caller owns it. */
+typedef struct srftq_desc {
+    int32_t d;
+    int32_t heads;
+    int32_t group;
+    int32_t bits;
+    int32_t rotation;
+} srftq_desc;
+
+/*
+ * srftq_quantize -- rotate, rescale and quantise S x N x H vectors.
+ * "When Quantization Is Free", Methodology 2, steps 1-5 (load and sign,
+ * FFT, Hermitian pack, lambda / group absmax / round, nibble packing).
+ *
+ *   x        [S][x_slice_stride_rows][H][d] fp16, read-only
+ *   signs    [S][H][d] int8;  lambda [S][H][d] float32
+ *   codes    [S][out_slice_stride_rows][H][d*bits/8] uint8, written
+ *   scales   [S][out_slice_stride_rows][H][d/group] fp16, written
+ * Only rows 0..n_rows-1 of every slice are read or written.
+ */
+int srftq_quantize(const srftq_desc* desc, int64_t n_slices, int64_t n_rows,
+                   const uint16_t* x, int64_t x_slice_stride_rows,
+                   const int8_t* signs, const float* lambda,
+                   uint8_t* codes, uint16_t* scales,
+                   int64_t out_slice_stride_rows, void* stream);
+
+/*
+ * srftq_dequantize -- the inverse of srftq_quantize: unpack, multiply by
+ * the group scale and lambda, apply R^T (inverse real FFT or WHT), multiply
+ * by the signs, round to fp16. Implied by the cache use in "When
+ * Quantization Is Free" (Methodology 2, the cache that holds the codes;
+ * Problem Statement, the cost of de-rotation).
+ *
+ *   codes, scales as written by srftq_quantize, slice stride in_slice_stride_rows
+ *   xhat     [S][out_slice_stride_rows][H][d] fp16, written
+ */
+int srftq_dequantize(const srftq_desc* desc, int64_t n_slices, int64_t n_rows,
+                     const uint8_t* codes, const uint16_t* scales,
+                     int64_t in_slice_stride_rows,
+                     const int8_t* signs, const float* lambda,
+                     uint16_t* xhat, int64_t out_slice_stride_rows, void* stream);
+
+/*
+ * srftq_calibrate_lambda -- per-channel lambda from calibration rows.
+ * lambda_out[s][h][j] = sqrt(mean over rows r < n_cal of y_{s,r,h,j}^2),
+ * 1 where that sum is zero; y is the rotation of x (no lambda). The
+ * statistic is the calibrated per-channel scale of "When Quantization Is
+ * Free", Methodology 2 step 4 and Methodology 3 (the pages leave the
+ * statistic open; the root mean square is the reading taken). The sum is
+ * accumulated in float64 in a fixed order, so the result is deterministic.
+ *
+ *   x          [S][x_slice_stride_rows][H][d] fp16 (rows 0..n_cal-1 read)
+ *   lambda_out [S][H][d] float32, written
+ */
+int srftq_calibrate_lambda(const srftq_desc* desc, int64_t n_slices, int64_t n_cal,
+                           const uint16_t* x, int64_t x_slice_stride_rows,
+                           const int8_t* signs, float* lambda_out, void* stream);
+
+/*
+ * srftq_rotate -- the rotation alone, float32 out (parity and debugging).
+ * y = R (s * x), divided by lambda when lambda_or_null is not NULL.
+ * "When Quantization Is Free", Methodology 1 (SRFT definition).
+ *
+ *   y_out [S][n_rows][H][d] float32, contiguous, written
+ */
+int srftq_rotate(const srftq_desc* desc, int64_t n_slices, int64_t n_rows,
+                 const uint16_t* x, int64_t x_slice_stride_rows,
+                 const int8_t* signs, const float* lambda_or_null,
+                 float* y_out, void* stream);
+
+/* Human-readable text for a status code (static storage, never NULL). */
+const char* srftq_status_string(int status);
+
+/*
+ * srftq_check_device -- synchronise `stream`, then read and clear the
+ * library-wide device guard word of the current device. Returns SRFTQ_OK
+ * if no guard fired since the last check, SRFTQ_ERR_DEVICE_CHECK if one
+ * did (a bounded wait gave up), SRFTQ_ERR_CUDA on a runtime error.
+ */
+int srftq_check_device(void* stream);
+
+/* Library version as 10000*major + 100*minor + patch. */
+int srftq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SRFTQ_H */

@@ -1,0 +1,28 @@
+"""B200-native rotate-then-quantize KV-cache codec (SRFT / SRHT, int4 / int8).
+
+The codec runs in libsrftq.so (hand-written CUDA for sm_100a, C ABI declared
+in include/srftq.h); this package holds its sources, the in-tree build and a
+thin ctypes binding. Importing the package does not load the library; the
+first call does, and fails loudly if it has not been built.
+"""
+
+from .binding import (  # noqa: F401
+    EXPORTED,
+    SRFT,
+    SRHT,
+    SrftqDesc,
+    SrftqError,
+    calibrate_lambda,
+    dequantize,
+    load_library,
+    make_desc,
+    quantize,
+    rotate,
+    srftq_calibrate_lambda,
+    srftq_check_device,
+    srftq_dequantize,
+    srftq_quantize,
+    srftq_rotate,
+    srftq_version,
+    status_string,
+)

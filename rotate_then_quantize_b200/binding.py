@@ -1,0 +1,224 @@
+"""ctypes binding of libsrftq.so (argument marshalling only).
+
+Every function named ``srftq_*`` here calls the C entry point of the same
+name declared in include/srftq.h; the arguments are torch tensors on a CUDA
+device (PyTorch provides device memory and streams, nothing else). All of the
+codec's work runs in the library's CUDA kernels: there is no fallback, and
+loading fails loudly when the library has not been built.
+
+Tensor views are accepted when each row's heads and elements are contiguous;
+a slice stride larger than the row count (for example ``cache[:, t0:t1]`` of
+a [S, T, H, d] buffer) is passed through as the slice stride in rows.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+PKG_DIR = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG_DIR, "libsrftq.so")
+
+SRFTQ_OK = 0
+SRFTQ_ERR_INVALID_ARG = -1
+SRFTQ_ERR_UNSUPPORTED = -2
+SRFTQ_ERR_MISALIGNED = -3
+SRFTQ_ERR_CUDA = -4
+SRFTQ_ERR_DEVICE_CHECK = -5
+
+SRFT = 0
+SRHT = 1
+
+# Every symbol include/srftq.h declares (checked by the CPU test suite).
+EXPORTED = ("srftq_quantize", "srftq_dequantize", "srftq_calibrate_lambda", "srftq_rotate",
+            "srftq_status_string", "srftq_check_device", "srftq_version")
+
+
+class SrftqDesc(ctypes.Structure):
+    _fields_ = [("d", ctypes.c_int32), ("heads", ctypes.c_int32), ("group", ctypes.c_int32),
+                ("bits", ctypes.c_int32), ("rotation", ctypes.c_int32)]
+
+
+class SrftqError(RuntimeError):
+    def __init__(self, fn, status, text):
+        super().__init__(f"{fn} failed: status {status} ({text})")
+        self.status = status
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Loads libsrftq.so once; raises if it is missing (no CPU fallback exists)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise FileNotFoundError(
+            f"{path} not found: build it with `python -m rotate_then_quantize_b200.build`")
+    lib = ctypes.CDLL(path)
+    P, I64, I32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+    D = ctypes.POINTER(SrftqDesc)
+    lib.srftq_quantize.argtypes = [D, I64, I64, P, I64, P, P, P, P, I64, P]
+    lib.srftq_dequantize.argtypes = [D, I64, I64, P, P, I64, P, P, P, I64, P]
+    lib.srftq_calibrate_lambda.argtypes = [D, I64, I64, P, I64, P, P, P]
+    lib.srftq_rotate.argtypes = [D, I64, I64, P, I64, P, P, P, P]
+    lib.srftq_status_string.argtypes = [I32]
+    lib.srftq_status_string.restype = ctypes.c_char_p
+    lib.srftq_check_device.argtypes = [P]
+    lib.srftq_version.argtypes = []
+    for name in ("srftq_quantize", "srftq_dequantize", "srftq_calibrate_lambda", "srftq_rotate",
+                 "srftq_check_device", "srftq_version"):
+        getattr(lib, name).restype = I32
+    _lib = lib
+    return lib
+
+
+def status_string(status: int) -> str:
+    return load_library().srftq_status_string(int(status)).decode()
+
+
+def _check(fn: str, status: int) -> None:
+    if status != SRFTQ_OK:
+        raise SrftqError(fn, status, status_string(status))
+
+
+def make_desc(d: int, heads: int, group: int, bits: int, rotation: int = SRFT) -> SrftqDesc:
+    return SrftqDesc(int(d), int(heads), int(group), int(bits), int(rotation))
+
+
+def _stream_handle(stream) -> int:
+    import torch
+
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream)
+
+
+def _rows_view(t, H: int, row_elems: int, name: str):
+    """(pointer, n_slices, n_rows, slice_stride_rows) of a [S, N, H, e] view."""
+    if t.dim() != 4 or t.shape[2] != H or t.shape[3] != row_elems:
+        raise ValueError(f"{name}: expected [S, N, {H}, {row_elems}], got {tuple(t.shape)}")
+    if t.stride(3) != 1 or t.stride(2) != row_elems or t.stride(1) != H * row_elems:
+        raise ValueError(f"{name}: heads and elements of a row must be contiguous")
+    if t.stride(0) % (H * row_elems) != 0:
+        raise ValueError(f"{name}: slice stride must be a whole number of rows")
+    stride_rows = t.stride(0) // (H * row_elems) if t.shape[0] > 1 else t.shape[1]
+    return t.data_ptr(), t.shape[0], t.shape[1], max(stride_rows, t.shape[1])
+
+
+def _table(t, S: int, H: int, d: int, name: str):
+    if tuple(t.shape) != (S, H, d) or not t.is_contiguous():
+        raise ValueError(f"{name}: expected contiguous [{S}, {H}, {d}], got {tuple(t.shape)}")
+    return t.data_ptr()
+
+
+def srftq_quantize(desc: SrftqDesc, x, signs, lam, codes, scales, stream=None) -> None:
+    """x [S,N,H,d] fp16 -> codes [S,N,H,d*bits/8] uint8, scales [S,N,H,d/G] fp16."""
+    lib = load_library()
+    px, S, N, xs = _rows_view(x, desc.heads, desc.d, "x")
+    pc, S2, N2, os_ = _rows_view(codes, desc.heads, desc.d * desc.bits // 8, "codes")
+    ps, S3, N3, os2 = _rows_view(scales, desc.heads, desc.d // desc.group, "scales")
+    if (S2, N2) != (S, N) or (S3, N3) != (S, N) or os2 != os_:
+        raise ValueError("codes/scales must match x's slices and rows and share a slice stride")
+    st = lib.srftq_quantize(ctypes.byref(desc), S, N, px, xs, _table(signs, S, desc.heads, desc.d, "signs"),
+                            _table(lam, S, desc.heads, desc.d, "lambda"), pc, ps, os_,
+                            _stream_handle(stream))
+    _check("srftq_quantize", st)
+
+
+def srftq_dequantize(desc: SrftqDesc, codes, scales, signs, lam, xhat, stream=None) -> None:
+    """codes, scales -> xhat [S,N,H,d] fp16 (the inverse of srftq_quantize)."""
+    lib = load_library()
+    pc, S, N, is_ = _rows_view(codes, desc.heads, desc.d * desc.bits // 8, "codes")
+    ps, S2, N2, is2 = _rows_view(scales, desc.heads, desc.d // desc.group, "scales")
+    px, S3, N3, os_ = _rows_view(xhat, desc.heads, desc.d, "xhat")
+    if (S2, N2) != (S, N) or (S3, N3) != (S, N) or is2 != is_:
+        raise ValueError("codes/scales/xhat shapes disagree")
+    st = lib.srftq_dequantize(ctypes.byref(desc), S, N, pc, ps, is_,
+                              _table(signs, S, desc.heads, desc.d, "signs"),
+                              _table(lam, S, desc.heads, desc.d, "lambda"), px, os_,
+                              _stream_handle(stream))
+    _check("srftq_dequantize", st)
+
+
+def srftq_calibrate_lambda(desc: SrftqDesc, x, signs, lam_out, n_cal: int, stream=None) -> None:
+    """lambda_out [S,H,d] float32 = RMS of the rotated first n_cal rows of x."""
+    lib = load_library()
+    px, S, N, xs = _rows_view(x, desc.heads, desc.d, "x")
+    if n_cal > N:
+        raise ValueError("n_cal exceeds the rows of x")
+    st = lib.srftq_calibrate_lambda(ctypes.byref(desc), S, int(n_cal), px, xs,
+                                    _table(signs, S, desc.heads, desc.d, "signs"),
+                                    _table(lam_out, S, desc.heads, desc.d, "lambda_out"),
+                                    _stream_handle(stream))
+    _check("srftq_calibrate_lambda", st)
+
+
+def srftq_rotate(desc: SrftqDesc, x, signs, y_out, lam=None, stream=None) -> None:
+    """y_out [S,N,H,d] float32 (contiguous) = R (s*x), divided by lambda if given."""
+    lib = load_library()
+    px, S, N, xs = _rows_view(x, desc.heads, desc.d, "x")
+    if tuple(y_out.shape) != (S, N, desc.heads, desc.d) or not y_out.is_contiguous():
+        raise ValueError("y_out must be a contiguous [S, N, H, d] float32 tensor")
+    pl = _table(lam, S, desc.heads, desc.d, "lambda") if lam is not None else None
+    st = lib.srftq_rotate(ctypes.byref(desc), S, N, px, xs,
+                          _table(signs, S, desc.heads, desc.d, "signs"), pl, y_out.data_ptr(),
+                          _stream_handle(stream))
+    _check("srftq_rotate", st)
+
+
+def srftq_check_device(stream=None) -> int:
+    """Synchronises the stream and returns (and clears) the device guard status."""
+    return int(load_library().srftq_check_device(_stream_handle(stream)))
+
+
+def srftq_version() -> int:
+    return int(load_library().srftq_version())
+
+
+# ---------------------------------------------------------------------------
+# Allocating conveniences (torch allocates; the library computes)
+# ---------------------------------------------------------------------------
+
+def quantize(x, signs, lam, group: int = 16, bits: int = 4, rotation: int = SRFT, stream=None):
+    """Returns (codes, scales) for x [S,N,H,d] fp16 on a CUDA device."""
+    import torch
+
+    S, N, H, d = x.shape
+    desc = make_desc(d, H, group, bits, rotation)
+    codes = torch.empty((S, N, H, d * bits // 8), dtype=torch.uint8, device=x.device)
+    scales = torch.empty((S, N, H, d // group), dtype=torch.float16, device=x.device)
+    srftq_quantize(desc, x, signs, lam, codes, scales, stream)
+    return codes, scales
+
+
+def dequantize(codes, scales, signs, lam, d: int, group: int = 16, bits: int = 4,
+               rotation: int = SRFT, stream=None):
+    import torch
+
+    S, N, H, _ = codes.shape
+    desc = make_desc(d, H, group, bits, rotation)
+    xhat = torch.empty((S, N, H, d), dtype=torch.float16, device=codes.device)
+    srftq_dequantize(desc, codes, scales, signs, lam, xhat, stream)
+    return xhat
+
+
+def calibrate_lambda(x, signs, n_cal: int = 512, rotation: int = SRFT, stream=None):
+    import torch
+
+    S, N, H, d = x.shape
+    desc = make_desc(d, H, 8, 4, rotation)
+    lam = torch.empty((S, H, d), dtype=torch.float32, device=x.device)
+    srftq_calibrate_lambda(desc, x, signs, lam, n_cal, stream)
+    return lam
+
+
+def rotate(x, signs, lam=None, rotation: int = SRFT, stream=None):
+    import torch
+
+    S, N, H, d = x.shape
+    desc = make_desc(d, H, 8, 4, rotation)
+    y = torch.empty((S, N, H, d), dtype=torch.float32, device=x.device)
+    srftq_rotate(desc, x, signs, y, lam, stream)
+    return y

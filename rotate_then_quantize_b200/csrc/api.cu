@@ -1,0 +1,252 @@
+// C ABI of libsrftq.so: argument validation, dispatch on the head dimension,
+// the device guard word and the tensor-map encoder. See include/srftq.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstdint>
+#include <mutex>
+
+#include "../../include/srftq.h"
+#include "common.cuh"
+#include "launch.cuh"
+
+// Library-wide device guard word (one per device that loads the module).
+__device__ unsigned g_srftq_guard;
+
+namespace srftq {
+namespace {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = []() -> EncodeTiledFn {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                         &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    return reinterpret_cast<EncodeTiledFn>(p);
+  }();
+  return fn;
+}
+
+constexpr int kMaxDevices = 64;
+std::atomic<int> g_num_sms[kMaxDevices];
+std::atomic<unsigned*> g_guard_ptr[kMaxDevices];
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool is_pow2(int64_t x) { return x > 0 && (x & (x - 1)) == 0; }
+
+int check_desc(const srftq_desc* d) {
+  if (!d) return SRFTQ_ERR_INVALID_ARG;
+  if (d->heads < 1) return SRFTQ_ERR_INVALID_ARG;
+  if (!(d->d == 16 || d->d == 32 || d->d == 64 || d->d == 128)) return SRFTQ_ERR_UNSUPPORTED;
+  if (d->bits != 4 && d->bits != 8) return SRFTQ_ERR_UNSUPPORTED;
+  if (!is_pow2(d->group) || d->group < 8 || d->group > d->d) return SRFTQ_ERR_UNSUPPORTED;
+  if (d->rotation != SRFTQ_ROT_SRFT && d->rotation != SRFTQ_ROT_SRHT) return SRFTQ_ERR_UNSUPPORTED;
+  return SRFTQ_OK;
+}
+
+// Byte range [lo, hi) touched by rows 0..n_rows-1 of S slices with a stride
+// of `stride` rows of `row_bytes` each.
+struct Range {
+  uintptr_t lo, hi;
+};
+
+Range extent(const void* p, int64_t S, int64_t stride, int64_t n_rows, int64_t row_bytes) {
+  const uintptr_t lo = reinterpret_cast<uintptr_t>(p);
+  const uint64_t rows = uint64_t(S - 1) * uint64_t(stride) + uint64_t(n_rows);
+  return {lo, lo + uintptr_t(rows * uint64_t(row_bytes))};
+}
+
+bool overlap(Range a, Range b) { return a.lo < b.hi && b.lo < a.hi; }
+
+template <typename Fn>
+int by_d(int d, Fn&& fn) {
+  switch (d) {
+    case 16: return fn(Int<16>{});
+    case 32: return fn(Int<32>{});
+    case 64: return fn(Int<64>{});
+    case 128: return fn(Int<128>{});
+    default: return SRFTQ_ERR_UNSUPPORTED;
+  }
+}
+
+}  // namespace
+
+int Runtime::encode_4d(CUtensorMap* map, CUtensorMapDataType dtype, void* base,
+                       const uint64_t dims[4], const uint64_t strides_bytes[3],
+                       const uint32_t box[4], CUtensorMapSwizzle swz) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return -1;
+  const cuuint64_t gd[4] = {dims[0], dims[1], dims[2], dims[3]};
+  const cuuint64_t gs[3] = {strides_bytes[0], strides_bytes[1], strides_bytes[2]};
+  const cuuint32_t bd[4] = {box[0], box[1], box[2], box[3]};
+  const cuuint32_t es[4] = {1, 1, 1, 1};
+  const CUresult r = fn(map, dtype, 4, base, gd, gs, bd, es, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? 0 : -1;
+}
+
+int Runtime::num_sms() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 1;
+  int n = g_num_sms[dev].load(std::memory_order_acquire);
+  if (n == 0) {
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1)
+      n = 1;
+    g_num_sms[dev].store(n, std::memory_order_release);
+  }
+  return n;
+}
+
+unsigned* Runtime::guard_word() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  unsigned* p = g_guard_ptr[dev].load(std::memory_order_acquire);
+  if (!p) {
+    void* q = nullptr;
+    if (cudaGetSymbolAddress(&q, g_srftq_guard) != cudaSuccess) return nullptr;
+    p = static_cast<unsigned*>(q);
+    g_guard_ptr[dev].store(p, std::memory_order_release);
+  }
+  return p;
+}
+
+}  // namespace srftq
+
+using namespace srftq;
+
+extern "C" {
+
+int srftq_quantize(const srftq_desc* desc, int64_t n_slices, int64_t n_rows, const uint16_t* x,
+                   int64_t x_slice_stride_rows, const int8_t* signs, const float* lambda,
+                   uint8_t* codes, uint16_t* scales, int64_t out_slice_stride_rows,
+                   void* stream) {
+  int rc = check_desc(desc);
+  if (rc != SRFTQ_OK) return rc;
+  if (n_slices < 0 || n_rows < 0) return SRFTQ_ERR_INVALID_ARG;
+  if (n_slices == 0 || n_rows == 0) return SRFTQ_OK;
+  if (x_slice_stride_rows < n_rows || out_slice_stride_rows < n_rows) return SRFTQ_ERR_INVALID_ARG;
+  if (!x || !signs || !lambda || !codes || !scales) return SRFTQ_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(signs) || !aligned16(lambda) || !aligned16(codes) ||
+      !aligned16(scales))
+    return SRFTQ_ERR_MISALIGNED;
+  const int64_t d = desc->d, H = desc->heads;
+  const Range rx = extent(x, n_slices, x_slice_stride_rows, n_rows, H * d * 2);
+  const Range rc_ = extent(codes, n_slices, out_slice_stride_rows, n_rows, H * d * desc->bits / 8);
+  const Range rs = extent(scales, n_slices, out_slice_stride_rows, n_rows, H * (d / desc->group) * 2);
+  const Range rsg = extent(signs, n_slices, H, H, d);
+  const Range rl = extent(lambda, n_slices, H, H, d * 4);
+  for (Range out : {rc_, rs})
+    for (Range in : {rx, rsg, rl})
+      if (overlap(out, in)) return SRFTQ_ERR_INVALID_ARG;
+  if (overlap(rc_, rs)) return SRFTQ_ERR_INVALID_ARG;
+  QuantCall c{desc->heads, desc->group, desc->bits, desc->rotation, n_slices, n_rows,
+              x, x_slice_stride_rows, signs, lambda, codes, scales, out_slice_stride_rows,
+              static_cast<cudaStream_t>(stream)};
+  return by_d(desc->d, [&](auto d_) { return launch_quantize<decltype(d_)::value>(c); });
+}
+
+int srftq_dequantize(const srftq_desc* desc, int64_t n_slices, int64_t n_rows,
+                     const uint8_t* codes, const uint16_t* scales, int64_t in_slice_stride_rows,
+                     const int8_t* signs, const float* lambda, uint16_t* xhat,
+                     int64_t out_slice_stride_rows, void* stream) {
+  int rc = check_desc(desc);
+  if (rc != SRFTQ_OK) return rc;
+  if (n_slices < 0 || n_rows < 0) return SRFTQ_ERR_INVALID_ARG;
+  if (n_slices == 0 || n_rows == 0) return SRFTQ_OK;
+  if (in_slice_stride_rows < n_rows || out_slice_stride_rows < n_rows) return SRFTQ_ERR_INVALID_ARG;
+  if (!codes || !scales || !signs || !lambda || !xhat) return SRFTQ_ERR_INVALID_ARG;
+  if (!aligned16(codes) || !aligned16(scales) || !aligned16(signs) || !aligned16(lambda) ||
+      !aligned16(xhat))
+    return SRFTQ_ERR_MISALIGNED;
+  const int64_t d = desc->d, H = desc->heads;
+  const Range rx = extent(xhat, n_slices, out_slice_stride_rows, n_rows, H * d * 2);
+  const Range rc_ = extent(codes, n_slices, in_slice_stride_rows, n_rows, H * d * desc->bits / 8);
+  const Range rs = extent(scales, n_slices, in_slice_stride_rows, n_rows, H * (d / desc->group) * 2);
+  const Range rsg = extent(signs, n_slices, H, H, d);
+  const Range rl = extent(lambda, n_slices, H, H, d * 4);
+  for (Range in : {rc_, rs, rsg, rl})
+    if (overlap(rx, in)) return SRFTQ_ERR_INVALID_ARG;
+  DequantCall c{desc->heads, desc->group, desc->bits, desc->rotation, n_slices, n_rows,
+                codes, scales, in_slice_stride_rows, signs, lambda, xhat, out_slice_stride_rows,
+                static_cast<cudaStream_t>(stream)};
+  return by_d(desc->d, [&](auto d_) { return launch_dequantize<decltype(d_)::value>(c); });
+}
+
+int srftq_calibrate_lambda(const srftq_desc* desc, int64_t n_slices, int64_t n_cal,
+                           const uint16_t* x, int64_t x_slice_stride_rows, const int8_t* signs,
+                           float* lambda_out, void* stream) {
+  int rc = check_desc(desc);
+  if (rc != SRFTQ_OK) return rc;
+  if (n_slices < 0 || n_cal < 1) return SRFTQ_ERR_INVALID_ARG;
+  if (n_slices == 0) return SRFTQ_OK;
+  if (x_slice_stride_rows < n_cal) return SRFTQ_ERR_INVALID_ARG;
+  if (!x || !signs || !lambda_out) return SRFTQ_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(signs) || !aligned16(lambda_out)) return SRFTQ_ERR_MISALIGNED;
+  const int64_t d = desc->d, H = desc->heads;
+  const Range rx = extent(x, n_slices, x_slice_stride_rows, n_cal, H * d * 2);
+  const Range rsg = extent(signs, n_slices, H, H, d);
+  const Range rl = extent(lambda_out, n_slices, H, H, d * 4);
+  if (overlap(rl, rx) || overlap(rl, rsg)) return SRFTQ_ERR_INVALID_ARG;
+  CalibCall c{desc->heads, desc->rotation, n_slices, n_cal, x, x_slice_stride_rows, signs,
+              lambda_out, static_cast<cudaStream_t>(stream)};
+  return by_d(desc->d, [&](auto d_) { return launch_calibrate<decltype(d_)::value>(c); });
+}
+
+int srftq_rotate(const srftq_desc* desc, int64_t n_slices, int64_t n_rows, const uint16_t* x,
+                 int64_t x_slice_stride_rows, const int8_t* signs, const float* lambda_or_null,
+                 float* y_out, void* stream) {
+  int rc = check_desc(desc);
+  if (rc != SRFTQ_OK) return rc;
+  if (n_slices < 0 || n_rows < 0) return SRFTQ_ERR_INVALID_ARG;
+  if (n_slices == 0 || n_rows == 0) return SRFTQ_OK;
+  if (x_slice_stride_rows < n_rows) return SRFTQ_ERR_INVALID_ARG;
+  if (!x || !signs || !y_out) return SRFTQ_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(signs) || !aligned16(y_out) ||
+      (lambda_or_null && !aligned16(lambda_or_null)))
+    return SRFTQ_ERR_MISALIGNED;
+  const int64_t d = desc->d, H = desc->heads;
+  const Range ry = extent(y_out, n_slices, n_rows, n_rows, H * d * 4);
+  const Range rx = extent(x, n_slices, x_slice_stride_rows, n_rows, H * d * 2);
+  const Range rsg = extent(signs, n_slices, H, H, d);
+  if (overlap(ry, rx) || overlap(ry, rsg)) return SRFTQ_ERR_INVALID_ARG;
+  if (lambda_or_null && overlap(ry, extent(lambda_or_null, n_slices, H, H, d * 4)))
+    return SRFTQ_ERR_INVALID_ARG;
+  RotateCall c{desc->heads, desc->rotation, n_slices, n_rows, x, x_slice_stride_rows, signs,
+               lambda_or_null, y_out, static_cast<cudaStream_t>(stream)};
+  return by_d(desc->d, [&](auto d_) { return launch_rotate<decltype(d_)::value>(c); });
+}
+
+const char* srftq_status_string(int status) {
+  switch (status) {
+    case SRFTQ_OK: return "ok";
+    case SRFTQ_ERR_INVALID_ARG: return "invalid argument";
+    case SRFTQ_ERR_UNSUPPORTED: return "unsupported configuration";
+    case SRFTQ_ERR_MISALIGNED: return "pointer not 16-byte aligned";
+    case SRFTQ_ERR_CUDA: return "CUDA error";
+    case SRFTQ_ERR_DEVICE_CHECK: return "device-side guard fired";
+    default: return "unknown status";
+  }
+}
+
+int srftq_check_device(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return SRFTQ_ERR_CUDA;
+  unsigned v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_srftq_guard, sizeof(v)) != cudaSuccess) return SRFTQ_ERR_CUDA;
+  if (v == 0) return SRFTQ_OK;
+  const unsigned zero = 0;
+  if (cudaMemcpyToSymbol(g_srftq_guard, &zero, sizeof(zero)) != cudaSuccess) return SRFTQ_ERR_CUDA;
+  return SRFTQ_ERR_DEVICE_CHECK;
+}
+
+int srftq_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,121 @@
+// Rotation-only and calibration kernels. They use the same per-thread
+// transforms as the codec kernels but plain global loads: neither is on the
+// bandwidth-critical path (the rotation kernel exists for parity checks, the
+// calibration reads n_cal rows per (slice, head) once).
+#pragma once
+
+#include <cuda_fp16.h>
+
+#include "codec.cuh"
+
+namespace srftq {
+
+// Loads vector `vec` (fp16, 16-byte aligned rows), applies the int8 sign
+// row and converts to float.
+template <int D>
+__device__ __forceinline__ void load_signed_vector(const uint16_t* x, const int8_t* sgn, float (&v)[D]) {
+  static_for<0, D / 8>([&](auto c_) {
+    constexpr int ci = decltype(c_)::value;
+    const uint4 raw = reinterpret_cast<const uint4*>(x)[ci];
+    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+    static_for<0, 4>([&](auto k_) {
+      constexpr int k = decltype(k_)::value;
+      const float2 f = __half22float2(u32_as_half2(w[k]));
+      const int j = 8 * ci + 2 * k;
+      v[j] = sgn[j] < 0 ? -f.x : f.x;
+      v[j + 1] = sgn[j + 1] < 0 ? -f.y : f.y;
+    });
+  });
+}
+
+struct RotateArgs {
+  int64_t n_slices, n_rows, x_slice_stride_rows;
+  int32_t heads;
+  const uint16_t* x;
+  const int8_t* signs;
+  const float* lambda;  // may be null
+  float* y;
+};
+
+// y = R (s * x) [/ lambda], one thread per vector, grid-stride.
+template <int D, int ROT>
+__global__ void __launch_bounds__(128) rotate_kernel(const RotateArgs a) {
+  const int64_t total = a.n_slices * a.n_rows * a.heads;
+  for (int64_t v_id = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; v_id < total;
+       v_id += int64_t(gridDim.x) * blockDim.x) {
+    const int h = int(v_id % a.heads);
+    const int64_t sr = v_id / a.heads;
+    const int64_t r = sr % a.n_rows;
+    const int64_t s = sr / a.n_rows;
+    const uint16_t* xv = a.x + ((s * a.x_slice_stride_rows + r) * a.heads + h) * D;
+    const int64_t tab = (s * a.heads + h) * D;
+    float v[D];
+    load_signed_vector<D>(xv, a.signs + tab, v);
+    rotate_forward_raw<ROT, D>(v);
+    float* yv = a.y + v_id * D;
+    static_for<0, D / 4>([&](auto c_) {
+      constexpr int ci = decltype(c_)::value;
+      float4 o;
+      float* op = &o.x;
+      static_for<0, 4>([&](auto k_) {
+        constexpr int j = 4 * ci + decltype(k_)::value;
+        const float g = gain_f<ROT, D>(j);
+        op[decltype(k_)::value] =
+            a.lambda ? v[j] * __fdiv_rn(g, a.lambda[tab + j]) : v[j] * g;
+      });
+      reinterpret_cast<float4*>(yv)[ci] = o;
+    });
+  }
+}
+
+struct CalibArgs {
+  int64_t n_cal, x_slice_stride_rows;
+  int32_t heads;
+  const uint16_t* x;
+  const int8_t* signs;
+  float* lambda_out;
+};
+
+constexpr int kCalibRows = 64;  // rows rotated per batch
+
+// One block per (slice, head). Threads 0..63 rotate one row each per batch
+// and write y^2 to shared memory; then thread j adds column j over the
+// batch's rows, in row order, into a float64 accumulator. The order of every
+// addition is fixed, so the result does not depend on scheduling.
+template <int D, int ROT>
+__global__ void __launch_bounds__(128) calibrate_kernel(const CalibArgs a) {
+  __shared__ float sq[kCalibRows][D + 1];
+  const int s = blockIdx.x / a.heads;
+  const int h = blockIdx.x % a.heads;
+  const int64_t tab = (int64_t(s) * a.heads + h) * D;
+  double acc = 0.0;
+  for (int64_t base = 0; base < a.n_cal; base += kCalibRows) {
+    if (threadIdx.x < kCalibRows) {
+      const int64_t r = base + threadIdx.x;
+      if (r < a.n_cal) {
+        const uint16_t* xv = a.x + ((int64_t(s) * a.x_slice_stride_rows + r) * a.heads + h) * D;
+        float v[D];
+        load_signed_vector<D>(xv, a.signs + tab, v);
+        rotate_forward_raw<ROT, D>(v);
+        static_for<0, D>([&](auto j_) {
+          constexpr int j = decltype(j_)::value;
+          const float y = v[j] * gain_f<ROT, D>(j);
+          sq[threadIdx.x][j] = y * y;
+        });
+      } else {
+        for (int j = 0; j < D; ++j) sq[threadIdx.x][j] = 0.0f;
+      }
+    }
+    __syncthreads();
+    if (threadIdx.x < D) {
+      for (int i = 0; i < kCalibRows; ++i) acc += double(sq[i][threadIdx.x]);
+    }
+    __syncthreads();
+  }
+  if (threadIdx.x < D) {
+    a.lambda_out[tab + threadIdx.x] =
+        acc > 0.0 ? float(sqrt(acc / double(a.n_cal))) : 1.0f;
+  }
+}
+
+}  // namespace srftq

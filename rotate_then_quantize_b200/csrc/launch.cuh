@@ -1,0 +1,77 @@
+// Host-side launch layer: tensor-map encoding, kernel configuration and
+// dispatch over the compile-time shapes. Each head dimension d is compiled
+// in its own translation unit (launch_d*.cu) from launch_impl.cuh.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "../../include/srftq.h"
+
+namespace srftq {
+
+struct QuantCall {
+  int32_t heads, group, bits, rotation;
+  int64_t n_slices, n_rows;
+  const uint16_t* x;
+  int64_t x_slice_stride_rows;
+  const int8_t* signs;
+  const float* lambda;
+  uint8_t* codes;
+  uint16_t* scales;
+  int64_t out_slice_stride_rows;
+  cudaStream_t stream;
+};
+
+struct DequantCall {
+  int32_t heads, group, bits, rotation;
+  int64_t n_slices, n_rows;
+  const uint8_t* codes;
+  const uint16_t* scales;
+  int64_t in_slice_stride_rows;
+  const int8_t* signs;
+  const float* lambda;
+  uint16_t* xhat;
+  int64_t out_slice_stride_rows;
+  cudaStream_t stream;
+};
+
+struct RotateCall {
+  int32_t heads, rotation;
+  int64_t n_slices, n_rows;
+  const uint16_t* x;
+  int64_t x_slice_stride_rows;
+  const int8_t* signs;
+  const float* lambda;
+  float* y;
+  cudaStream_t stream;
+};
+
+struct CalibCall {
+  int32_t heads, rotation;
+  int64_t n_slices, n_cal;
+  const uint16_t* x;
+  int64_t x_slice_stride_rows;
+  const int8_t* signs;
+  float* lambda_out;
+  cudaStream_t stream;
+};
+
+// Services the per-d units get from the API unit.
+struct Runtime {
+  // Encodes a rank-4 tiled tensor map; returns 0 on success.
+  static int encode_4d(CUtensorMap* map, CUtensorMapDataType dtype, void* base,
+                       const uint64_t dims[4], const uint64_t strides_bytes[3],
+                       const uint32_t box[4], CUtensorMapSwizzle swz);
+  static int num_sms();          // streaming multiprocessors of the current device
+  static unsigned* guard_word(); // device address of the guard word, current device
+};
+
+template <int D> int launch_quantize(const QuantCall& c);
+template <int D> int launch_dequantize(const DequantCall& c);
+template <int D> int launch_rotate(const RotateCall& c);
+template <int D> int launch_calibrate(const CalibCall& c);
+
+}  // namespace srftq

@@ -1,0 +1,234 @@
+// Per-d launch implementation, included by one translation unit per head
+// dimension (launch_d16.cu ... launch_d128.cu).
+#pragma once
+
+#include <atomic>
+#include <climits>
+#include <cstring>
+
+#include "aux.cuh"
+#include "codec.cuh"
+#include "launch.cuh"
+
+namespace srftq {
+
+// Warps per block, input stages and output staging buffers per warp.
+constexpr int kWPC = 4;
+constexpr int kNST = 2;
+constexpr int kNOUT = 2;
+
+inline CUtensorMapSwizzle swizzle_mode(int span) {
+  switch (span) {
+    case 32: return CU_TENSOR_MAP_SWIZZLE_32B;
+    case 64: return CU_TENSOR_MAP_SWIZZLE_64B;
+    case 128: return CU_TENSOR_MAP_SWIZZLE_128B;
+    default: return CU_TENSOR_MAP_SWIZZLE_NONE;
+  }
+}
+
+// Sets the dynamic shared-memory limit of kernel K once per device and
+// caches its occupancy (blocks per SM) for the block shape it is launched
+// with.
+template <auto K>
+int prepare_kernel(int smem_bytes, int threads, int* blocks_per_sm) {
+  static std::atomic<uint64_t> attr_done{0};
+  static std::atomic<int> bps{0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SRFTQ_ERR_CUDA;
+  const uint64_t bit = 1ull << (dev & 63);
+  if (!(attr_done.load(std::memory_order_acquire) & bit)) {
+    if (smem_bytes > 48 * 1024 &&
+        cudaFuncSetAttribute(K, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes) !=
+            cudaSuccess)
+      return SRFTQ_ERR_CUDA;
+    attr_done.fetch_or(bit, std::memory_order_acq_rel);
+  }
+  int b = bps.load(std::memory_order_acquire);
+  if (b == 0) {
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, K, threads, smem_bytes) != cudaSuccess)
+      return SRFTQ_ERR_CUDA;
+    if (b < 1) return SRFTQ_ERR_CUDA;
+    bps.store(b, std::memory_order_release);
+  }
+  *blocks_per_sm = b;
+  return SRFTQ_OK;
+}
+
+// Calls f(Int<BITS>, Int<G>, Int<ROT>) for the run-time configuration.
+template <int D, typename F>
+int dispatch_config(int bits, int group, int rot, F&& f) {
+  int rc = SRFTQ_ERR_UNSUPPORTED;
+  static_for<0, 2>([&](auto b_) {
+    constexpr int BITS = decltype(b_)::value == 0 ? 4 : 8;
+    static_for<3, ilog2(D) + 1>([&](auto lg_) {
+      constexpr int G = 1 << decltype(lg_)::value;
+      static_for<0, 2>([&](auto r_) {
+        constexpr int ROT = decltype(r_)::value;
+        if (bits == BITS && group == G && rot == ROT) rc = f(Int<BITS>{}, Int<G>{}, Int<ROT>{});
+      });
+    });
+  });
+  return rc;
+}
+
+inline int finish_launch() {
+  return cudaGetLastError() == cudaSuccess ? SRFTQ_OK : SRFTQ_ERR_CUDA;
+}
+
+template <int D, int BITS, int G, int ROT>
+int quantize_impl(const QuantCall& c) {
+  using S = Shape<D, BITS, G>;
+  using Lay = WarpLayout<D, BITS, G, kNST, kNOUT, true>;
+  const int64_t row_blocks = (c.n_rows + kTileRows - 1) / kTileRows;
+  const int64_t total = c.n_slices * row_blocks * c.heads;
+  if (total == 0) return SRFTQ_OK;
+  if (total > INT_MAX || c.n_rows > INT_MAX || c.n_slices > INT_MAX) return SRFTQ_ERR_UNSUPPORTED;
+
+  CUtensorMap tm_x, tm_c;
+  std::memset(&tm_c, 0, sizeof(tm_c));
+  {
+    const uint64_t dims[4] = {uint64_t(D), uint64_t(c.heads), uint64_t(c.n_rows),
+                              uint64_t(c.n_slices)};
+    const uint64_t str[3] = {uint64_t(S::XB), uint64_t(c.heads) * S::XB,
+                             uint64_t(c.x_slice_stride_rows) * c.heads * S::XB};
+    const uint32_t box[4] = {uint32_t(S::X_SPAN / 2), 1u, uint32_t(kTileRows), 1u};
+    if (Runtime::encode_4d(&tm_x, CU_TENSOR_MAP_DATA_TYPE_UINT16, const_cast<uint16_t*>(c.x), dims,
+                           str, box, swizzle_mode(S::X_SPAN)) != 0)
+      return SRFTQ_ERR_CUDA;
+  }
+  if constexpr (S::CODES_TMA) {
+    const uint64_t dims[4] = {uint64_t(S::CB), uint64_t(c.heads), uint64_t(c.n_rows),
+                              uint64_t(c.n_slices)};
+    const uint64_t str[3] = {uint64_t(S::CB), uint64_t(c.heads) * S::CB,
+                             uint64_t(c.out_slice_stride_rows) * c.heads * S::CB};
+    const uint32_t box[4] = {uint32_t(S::C_SPAN), 1u, uint32_t(kTileRows), 1u};
+    if (Runtime::encode_4d(&tm_c, CU_TENSOR_MAP_DATA_TYPE_UINT8, c.codes, dims, str, box,
+                           swizzle_mode(S::C_SPAN)) != 0)
+      return SRFTQ_ERR_CUDA;
+  }
+  unsigned* guard = Runtime::guard_word();
+  if (!guard) return SRFTQ_ERR_CUDA;
+  QuantArgs a;
+  a.g = TileGeom{c.heads, int32_t(row_blocks), int32_t(c.n_rows), int32_t(total)};
+  a.signs = c.signs;
+  a.lambda = c.lambda;
+  a.codes = c.codes;
+  a.scales = c.scales;
+  a.out_slice_stride_rows = c.out_slice_stride_rows;
+  a.guard = guard;
+
+  constexpr auto K = quantize_kernel<D, BITS, G, ROT, kWPC, kNST, kNOUT>;
+  const int smem = kWPC * Lay::kWarpBytes + kSmemSlack;
+  int bps = 0;
+  int rc = prepare_kernel<K>(smem, kWPC * 32, &bps);
+  if (rc != SRFTQ_OK) return rc;
+  const int64_t want = (total + kWPC - 1) / kWPC;
+  const int64_t cap = int64_t(Runtime::num_sms()) * bps;
+  const int grid = int(want < cap ? want : cap);
+  K<<<grid, kWPC * 32, smem, c.stream>>>(tm_x, tm_c, a);
+  return finish_launch();
+}
+
+template <int D, int BITS, int G, int ROT>
+int dequantize_impl(const DequantCall& c) {
+  using S = Shape<D, BITS, G>;
+  using Lay = WarpLayout<D, BITS, G, kNST, kNOUT, false>;
+  const int64_t row_blocks = (c.n_rows + kTileRows - 1) / kTileRows;
+  const int64_t total = c.n_slices * row_blocks * c.heads;
+  if (total == 0) return SRFTQ_OK;
+  if (total > INT_MAX || c.n_rows > INT_MAX || c.n_slices > INT_MAX) return SRFTQ_ERR_UNSUPPORTED;
+
+  CUtensorMap tm_c, tm_x;
+  std::memset(&tm_c, 0, sizeof(tm_c));
+  if constexpr (S::CODES_TMA) {
+    const uint64_t dims[4] = {uint64_t(S::CB), uint64_t(c.heads), uint64_t(c.n_rows),
+                              uint64_t(c.n_slices)};
+    const uint64_t str[3] = {uint64_t(S::CB), uint64_t(c.heads) * S::CB,
+                             uint64_t(c.in_slice_stride_rows) * c.heads * S::CB};
+    const uint32_t box[4] = {uint32_t(S::C_SPAN), 1u, uint32_t(kTileRows), 1u};
+    if (Runtime::encode_4d(&tm_c, CU_TENSOR_MAP_DATA_TYPE_UINT8, const_cast<uint8_t*>(c.codes),
+                           dims, str, box, swizzle_mode(S::C_SPAN)) != 0)
+      return SRFTQ_ERR_CUDA;
+  }
+  {
+    const uint64_t dims[4] = {uint64_t(D), uint64_t(c.heads), uint64_t(c.n_rows),
+                              uint64_t(c.n_slices)};
+    const uint64_t str[3] = {uint64_t(S::XB), uint64_t(c.heads) * S::XB,
+                             uint64_t(c.out_slice_stride_rows) * c.heads * S::XB};
+    const uint32_t box[4] = {uint32_t(S::X_SPAN / 2), 1u, uint32_t(kTileRows), 1u};
+    if (Runtime::encode_4d(&tm_x, CU_TENSOR_MAP_DATA_TYPE_UINT16, c.xhat, dims, str, box,
+                           swizzle_mode(S::X_SPAN)) != 0)
+      return SRFTQ_ERR_CUDA;
+  }
+  unsigned* guard = Runtime::guard_word();
+  if (!guard) return SRFTQ_ERR_CUDA;
+  DequantArgs a;
+  a.g = TileGeom{c.heads, int32_t(row_blocks), int32_t(c.n_rows), int32_t(total)};
+  a.signs = c.signs;
+  a.lambda = c.lambda;
+  a.codes = c.codes;
+  a.scales = c.scales;
+  a.in_slice_stride_rows = c.in_slice_stride_rows;
+  a.guard = guard;
+
+  constexpr auto K = dequantize_kernel<D, BITS, G, ROT, kWPC, kNST, kNOUT>;
+  const int smem = kWPC * Lay::kWarpBytes + kSmemSlack;
+  int bps = 0;
+  int rc = prepare_kernel<K>(smem, kWPC * 32, &bps);
+  if (rc != SRFTQ_OK) return rc;
+  const int64_t want = (total + kWPC - 1) / kWPC;
+  const int64_t cap = int64_t(Runtime::num_sms()) * bps;
+  const int grid = int(want < cap ? want : cap);
+  K<<<grid, kWPC * 32, smem, c.stream>>>(tm_c, tm_x, a);
+  return finish_launch();
+}
+
+template <int D>
+int launch_quantize(const QuantCall& c) {
+  return dispatch_config<D>(c.bits, c.group, c.rotation, [&](auto b_, auto g_, auto r_) {
+    return quantize_impl<D, decltype(b_)::value, decltype(g_)::value, decltype(r_)::value>(c);
+  });
+}
+
+template <int D>
+int launch_dequantize(const DequantCall& c) {
+  return dispatch_config<D>(c.bits, c.group, c.rotation, [&](auto b_, auto g_, auto r_) {
+    return dequantize_impl<D, decltype(b_)::value, decltype(g_)::value, decltype(r_)::value>(c);
+  });
+}
+
+template <int D>
+int launch_rotate(const RotateCall& c) {
+  const int64_t total = c.n_slices * c.n_rows * c.heads;
+  if (total == 0) return SRFTQ_OK;
+  RotateArgs a{c.n_slices, c.n_rows, c.x_slice_stride_rows, c.heads, c.x, c.signs, c.lambda, c.y};
+  const int64_t want = (total + 127) / 128;
+  const int64_t cap = int64_t(Runtime::num_sms()) * 16;
+  const int grid = int(want < cap ? want : cap);
+  if (c.rotation == kSRFT)
+    rotate_kernel<D, kSRFT><<<grid, 128, 0, c.stream>>>(a);
+  else
+    rotate_kernel<D, kSRHT><<<grid, 128, 0, c.stream>>>(a);
+  return finish_launch();
+}
+
+template <int D>
+int launch_calibrate(const CalibCall& c) {
+  const int64_t blocks = c.n_slices * c.heads;
+  if (blocks == 0) return SRFTQ_OK;
+  if (blocks > INT_MAX) return SRFTQ_ERR_UNSUPPORTED;
+  CalibArgs a{c.n_cal, c.x_slice_stride_rows, c.heads, c.x, c.signs, c.lambda_out};
+  if (c.rotation == kSRFT)
+    calibrate_kernel<D, kSRFT><<<int(blocks), 128, 0, c.stream>>>(a);
+  else
+    calibrate_kernel<D, kSRHT><<<int(blocks), 128, 0, c.stream>>>(a);
+  return finish_launch();
+}
+
+}  // namespace srftq
+
+#define SRFTQ_INSTANTIATE_D(D)                                        \
+  template int srftq::launch_quantize<D>(const srftq::QuantCall&);     \
+  template int srftq::launch_dequantize<D>(const srftq::DequantCall&); \
+  template int srftq::launch_rotate<D>(const srftq::RotateCall&);      \
+  template int srftq::launch_calibrate<D>(const srftq::CalibCall&);

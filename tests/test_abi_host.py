@@ -1,0 +1,127 @@
+"""Host-side checks of libsrftq.so that need no GPU.
+
+The library must load, export every entry point include/srftq.h declares, and
+reject bad arguments on the host with the documented status before anything
+would be launched (no call here reaches a kernel launch).
+"""
+
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import rotate_then_quantize_b200 as rq
+from rotate_then_quantize_b200 import binding as b
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "srftq.h")
+
+
+def _declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(srftq_[a-z_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(b.LIB_PATH):
+        pytest.fail("libsrftq.so is not built; run python -m rotate_then_quantize_b200.build")
+    return rq.load_library()
+
+
+def test_header_declares_the_boundary():
+    assert _declared() == sorted(b.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", b.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (srftq_\w+)", out))
+    for name in _declared():
+        assert name in exported, name
+        assert hasattr(lib, name)
+
+
+def test_version_and_status_strings(lib):
+    assert rq.srftq_version() >= 100
+    for st in (0, -1, -2, -3, -4, -5):
+        assert rq.status_string(st) != "unknown status"
+    assert rq.status_string(42) == "unknown status"
+
+
+def _q(lib, desc, S=1, N=8, x=16, xs=8, sg=16, lam=16, codes=16, sc=16, os_=8):
+    """srftq_quantize with fake (never dereferenced) addresses."""
+    return lib.srftq_quantize(ctypes.byref(desc) if desc is not None else None, S, N,
+                              x, xs, sg, lam, codes, sc, os_, None)
+
+
+FAKE = 1 << 40  # a 16-byte-aligned address far from anything; never touched
+
+
+def _addrs(n_bytes_apart=1 << 30):
+    return [FAKE + i * n_bytes_apart for i in range(6)]
+
+
+def test_quantize_rejects_bad_descriptors(lib):
+    x, sg, lam, codes, sc, _ = _addrs()
+    ok = dict(x=x, sg=sg, lam=lam, codes=codes, sc=sc)
+    assert _q(lib, None, **ok) == b.SRFTQ_ERR_INVALID_ARG
+    for d, heads, group, bits, rot, want in [
+        (96, 2, 16, 4, 0, b.SRFTQ_ERR_UNSUPPORTED),    # d not a supported power of two
+        (512, 2, 16, 4, 0, b.SRFTQ_ERR_UNSUPPORTED),
+        (128, 0, 16, 4, 0, b.SRFTQ_ERR_INVALID_ARG),   # no heads
+        (128, 2, 12, 4, 0, b.SRFTQ_ERR_UNSUPPORTED),   # group not a power of two
+        (128, 2, 4, 4, 0, b.SRFTQ_ERR_UNSUPPORTED),    # group below 8
+        (64, 2, 128, 4, 0, b.SRFTQ_ERR_UNSUPPORTED),   # group above d
+        (128, 2, 16, 3, 0, b.SRFTQ_ERR_UNSUPPORTED),   # bits
+        (128, 2, 16, 4, 2, b.SRFTQ_ERR_UNSUPPORTED),   # rotation
+    ]:
+        assert _q(lib, rq.make_desc(d, heads, group, bits, rot), **ok) == want, (d, heads, group, bits, rot)
+
+
+def test_quantize_rejects_bad_sizes_pointers_and_overlap(lib):
+    desc = rq.make_desc(128, 2, 16, 4)
+    x, sg, lam, codes, sc, _ = _addrs()
+    ok = dict(x=x, sg=sg, lam=lam, codes=codes, sc=sc)
+    assert _q(lib, desc, N=-1, **ok) == b.SRFTQ_ERR_INVALID_ARG
+    assert _q(lib, desc, S=-1, **ok) == b.SRFTQ_ERR_INVALID_ARG
+    assert _q(lib, desc, N=0, **ok) == b.SRFTQ_OK            # nothing to do, nothing launched
+    assert _q(lib, desc, S=0, **ok) == b.SRFTQ_OK
+    assert _q(lib, desc, S=2, N=8, xs=4, **ok) == b.SRFTQ_ERR_INVALID_ARG   # overlapping slices
+    assert _q(lib, desc, S=2, N=8, os_=4, **ok) == b.SRFTQ_ERR_INVALID_ARG
+    assert _q(lib, desc, **dict(ok, x=0)) == b.SRFTQ_ERR_INVALID_ARG
+    assert _q(lib, desc, **dict(ok, sc=0)) == b.SRFTQ_ERR_INVALID_ARG
+    assert _q(lib, desc, **dict(ok, x=x + 8)) == b.SRFTQ_ERR_MISALIGNED
+    assert _q(lib, desc, **dict(ok, codes=codes + 4)) == b.SRFTQ_ERR_MISALIGNED
+    # in-place: codes inside x
+    assert _q(lib, desc, **dict(ok, codes=x + 256)) == b.SRFTQ_ERR_INVALID_ARG
+    # scales overlapping codes
+    assert _q(lib, desc, **dict(ok, sc=codes + 16)) == b.SRFTQ_ERR_INVALID_ARG
+
+
+def test_dequantize_calibrate_rotate_validation(lib):
+    desc = rq.make_desc(64, 3, 16, 8, 1)
+    c, s, sg, lam, xh, y = _addrs()
+    D = ctypes.byref(desc)
+    assert lib.srftq_dequantize(D, 1, 8, c, s, 8, sg, lam, c, 8, None) == b.SRFTQ_ERR_INVALID_ARG
+    assert lib.srftq_dequantize(D, 1, 8, c + 2, s, 8, sg, lam, xh, 8, None) == b.SRFTQ_ERR_MISALIGNED
+    assert lib.srftq_dequantize(D, 1, 0, c, s, 8, sg, lam, xh, 8, None) == b.SRFTQ_OK
+    assert lib.srftq_calibrate_lambda(D, 1, 0, c, 8, sg, lam, None) == b.SRFTQ_ERR_INVALID_ARG
+    assert lib.srftq_calibrate_lambda(D, 1, 9, c, 8, sg, lam, None) == b.SRFTQ_ERR_INVALID_ARG
+    assert lib.srftq_calibrate_lambda(D, 0, 4, c, 8, sg, lam, None) == b.SRFTQ_OK
+    assert lib.srftq_calibrate_lambda(D, 1, 4, c, 8, sg, c, None) == b.SRFTQ_ERR_INVALID_ARG
+    assert lib.srftq_rotate(D, 1, 8, c, 8, sg, None, c, None) == b.SRFTQ_ERR_INVALID_ARG
+    assert lib.srftq_rotate(D, 1, 8, c, 8, sg, lam + 4, y, None) == b.SRFTQ_ERR_MISALIGNED
+    assert lib.srftq_rotate(D, 1, 0, c, 8, sg, None, y, None) == b.SRFTQ_OK
+
+
+def test_python_binding_rejects_bad_views():
+    torch = pytest.importorskip("torch")
+    x = torch.zeros((2, 8, 3, 64), dtype=torch.float16)
+    with pytest.raises(ValueError):
+        b._rows_view(x.transpose(1, 2), 3, 64, "x")
+    ptr, S, N, stride = b._rows_view(x[:, 2:6], 3, 64, "x")
+    assert (S, N, stride) == (2, 4, 8)

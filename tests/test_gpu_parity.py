@@ -1,0 +1,263 @@
+"""GPU parity: the CUDA library against the CPU oracle, through the C ABI.
+
+Small cases run every compiled configuration in full (several 32-row tiles,
+a ragged last tile, several slices and heads). The paper-shaped workloads run
+at full size in the same launch configuration the benchmark uses; the oracle
+checks a sample of rows from every slice, and properties that hold for any
+size are checked on every vector.
+"""
+
+import numpy as np
+import pytest
+
+import kv_synth
+import oracle
+import parity
+
+torch = pytest.importorskip("torch")
+import rotate_then_quantize_b200 as rq  # noqa: E402
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    if not torch.cuda.is_available():
+        pytest.fail("no CUDA device")
+    rq.load_library()
+    yield
+    assert rq.srftq_check_device() == 0, "a device-side guard fired"
+
+
+def _signs(rng, S, H, d):
+    return np.where(rng.random((S, H, d)) < 0.5, -1, 1).astype(np.int8)
+
+
+def _x(rng, S, N, H, d, outlier_p=0.01, scale=20.0):
+    x = rng.standard_normal((S, N, H, d))
+    x = np.where(rng.random(x.shape) < outlier_p, x * scale, x)
+    return x.astype(np.float16)
+
+
+def _t(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).to(DEV)
+
+
+def _np16(t):
+    return t.cpu().numpy().view(np.uint16)
+
+
+def run_and_check(x16, signs, lam, d, group, bits, rot, what):
+    """Rotation, quantisation and dequantisation of x16 on the GPU vs the oracle."""
+    xt, st, lt = _t(x16), _t(signs), _t(lam)
+    y = rq.rotate(xt, st, lt, rotation=rot).cpu().numpy()
+    y_ref = oracle.rotate(x16, signs, rot) / lam[:, None].astype(np.float64)
+    parity.assert_clean(parity.check_rotation(y, y_ref), f"{what} rotate")
+
+    codes, scales = rq.quantize(xt, st, lt, group, bits, rot)
+    ref = oracle.quantize(x16, signs, lam, group, bits, rot)
+    c_np, s_np = codes.cpu().numpy(), _np16(scales)
+    stats = parity.check_codes(ref, c_np, s_np, bits, group)
+    parity.assert_clean(stats, f"{what} codes")
+
+    xhat = rq.dequantize(codes, scales, st, lt, d, group, bits, rot)
+    deq = oracle.dequantize(c_np, s_np, signs, lam, d, group, bits, rot)
+    parity.assert_clean(parity.check_dequant(_np16(xhat), deq["bits"]), f"{what} dequant")
+    return stats
+
+
+def _configs():
+    out = []
+    for d in (16, 32, 64, 128):
+        for bits in (4, 8):
+            g = 8
+            while g <= d:
+                for rot in (rq.SRFT, rq.SRHT):
+                    out.append((d, bits, g, rot))
+                g *= 2
+    return out
+
+
+@pytest.mark.parametrize("d,bits,group,rot", _configs())
+def test_small_sweep(d, bits, group, rot):
+    rng = np.random.default_rng(1000 * d + 100 * bits + group + rot)
+    S, N, H = 2, 45, 3
+    x16 = _x(rng, S, N, H, d)
+    signs = _signs(rng, S, H, d)
+    lam = oracle.calibrate_lambda(x16, signs, 32, rot).astype(np.float32)
+    run_and_check(x16, signs, lam, d, group, bits, rot, f"d{d} b{bits} g{group} r{rot}")
+    lam_gpu = rq.calibrate_lambda(_t(x16), _t(signs), 32, rotation=rot).cpu().numpy()
+    parity.assert_clean(parity.check_lambda(lam_gpu, oracle.calibrate_lambda(x16, signs, 32, rot)),
+                        "lambda")
+
+
+@pytest.mark.parametrize("N", [1, 31, 32, 33, 97])
+@pytest.mark.parametrize("H", [1, 5])
+def test_ragged_rows_and_heads(N, H):
+    rng = np.random.default_rng(N * 7 + H)
+    d, group, bits = 64, 16, 4
+    x16 = _x(rng, 3, N, H, d)
+    signs = _signs(rng, 3, H, d)
+    lam = np.exp(rng.uniform(-1, 1, (3, H, d))).astype(np.float32)
+    run_and_check(x16, signs, lam, d, group, bits, rq.SRFT, f"N{N} H{H}")
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+def test_strided_views_and_guard_bands(bits):
+    """Slices with a row stride larger than the rows used (a cache written at a
+    row offset); rows outside the written window must keep their sentinel."""
+    rng = np.random.default_rng(bits)
+    S, T, H, d, group, N, off = 3, 100, 2, 128, 16, 37, 41
+    big = _x(rng, S, T, H, d)
+    signs = _signs(rng, S, H, d)
+    lam = np.exp(rng.uniform(-0.5, 0.5, (S, H, d))).astype(np.float32)
+    xt, st, lt = _t(big), _t(signs), _t(lam)
+    codes_big = torch.full((S, T, H, d * bits // 8), 0xAB, dtype=torch.uint8, device=DEV)
+    scales_big = torch.full((S, T, H, d // group), 7.0, dtype=torch.float16, device=DEV)
+    desc = rq.make_desc(d, H, group, bits)
+    rq.srftq_quantize(desc, xt[:, off:off + N], st, lt, codes_big[:, off:off + N],
+                      scales_big[:, off:off + N])
+    ref = oracle.quantize(big[:, off:off + N], signs, lam, group, bits)
+    c_np = codes_big.cpu().numpy()
+    s_np = _np16(scales_big)
+    parity.assert_clean(parity.check_codes(ref, c_np[:, off:off + N], s_np[:, off:off + N],
+                                           bits, group), "strided codes")
+    outside = np.ones(T, dtype=bool)
+    outside[off:off + N] = False
+    assert np.all(c_np[:, outside] == 0xAB)
+    assert np.all(s_np[:, outside] == np.float16(7.0).view(np.uint16))
+    # dequantise into a strided view, sentinel around it
+    xh_big = torch.full((S, T, H, d), -3.0, dtype=torch.float16, device=DEV)
+    rq.srftq_dequantize(desc, codes_big[:, off:off + N], scales_big[:, off:off + N], st, lt,
+                        xh_big[:, off:off + N])
+    deq = oracle.dequantize(c_np[:, off:off + N], s_np[:, off:off + N], signs, lam, d, group, bits)
+    xh = _np16(xh_big)
+    parity.assert_clean(parity.check_dequant(xh[:, off:off + N], deq["bits"]), "strided dequant")
+    assert np.all(xh[:, outside] == np.float16(-3.0).view(np.uint16))
+
+
+def test_degenerate_values():
+    """Zero vectors (sigma = 0), values driving sigma subnormal or saturated,
+    and exact ties; all decided as the oracle decides them."""
+    rng = np.random.default_rng(5)
+    S, N, H, d, group = 1, 64, 1, 64, 16
+    x = rng.standard_normal((S, N, H, d))
+    x[:, 0] = 0.0                              # all-zero vector
+    x[:, 1] = 1e-7 * rng.standard_normal(d)    # tiny: subnormal scales
+    x[:, 2] = 6e4 * np.sign(rng.standard_normal(d))  # near fp16 max
+    x[:, 3, :, 5] = 1.0                        # single spike
+    x16 = x.astype(np.float16)
+    signs = _signs(rng, S, H, d)
+    for lam_val in (1.0, 1e-3, 3e3):
+        lam = np.full((S, H, d), lam_val, dtype=np.float32)
+        for bits in (4, 8):
+            run_and_check(x16, signs, lam, d, group, bits, rq.SRFT, f"degenerate lam={lam_val}")
+
+
+def test_non_finite_inputs_do_not_fault():
+    rng = np.random.default_rng(9)
+    x16 = _x(rng, 1, 40, 2, 128)
+    x16[0, 3, 0, 7] = np.inf
+    x16[0, 5, 1, 0] = np.nan
+    signs = _signs(rng, 1, 2, 128)
+    lam = np.ones((1, 2, 128), np.float32)
+    codes, scales = rq.quantize(_t(x16), _t(signs), _t(lam), 16, 4)
+    rq.dequantize(codes, scales, _t(signs), _t(lam), 128, 16, 4)
+    torch.cuda.synchronize()
+    assert rq.srftq_check_device() == 0
+    # rows without non-finite values are still exact
+    clean = [r for r in range(40) if r not in (3, 5)]
+    ref = oracle.quantize(x16[:, clean], signs, lam, 16, 4)
+    parity.assert_clean(parity.check_codes(ref, codes.cpu().numpy()[:, clean],
+                                           _np16(scales)[:, clean], 4, 16), "finite rows")
+
+
+def test_empty_call_launches_nothing():
+    x = torch.empty((2, 0, 3, 64), dtype=torch.float16, device=DEV)
+    codes, scales = rq.quantize(x, torch.ones((2, 3, 64), dtype=torch.int8, device=DEV),
+                                torch.ones((2, 3, 64), device=DEV), 16, 4)
+    assert codes.numel() == 0 and scales.numel() == 0
+
+
+# ---------------------------------------------------------------------------
+# Paper-shaped workloads
+# ---------------------------------------------------------------------------
+
+def test_tiny_workload_full():
+    """4096 vectors, d=64, seeded exactly as specified; every output checked."""
+    w = kv_synth.WORKLOADS["tiny_d64"]
+    x16, signs = kv_synth.tiny_inputs()
+    lam64 = oracle.calibrate_lambda(x16, signs, w.n_cal)
+    lam_gpu = rq.calibrate_lambda(_t(x16), _t(signs), w.n_cal).cpu().numpy()
+    parity.assert_clean(parity.check_lambda(lam_gpu, lam64), "tiny lambda")
+    stats = run_and_check(x16, signs, lam64.astype(np.float32), w.d, w.group, w.bits, rq.SRFT,
+                          "tiny")
+    print("tiny codes:", stats)
+
+
+def _sample_rows(rng, N, k):
+    rows = np.unique(np.concatenate([rng.choice(N, size=k, replace=False), [0, N - 1]]))
+    return rows
+
+
+def _workload_check(name, rot, k_rows=48):
+    w = kv_synth.WORKLOADS[name]
+    rng = np.random.default_rng(17)
+    x = kv_synth.make_x_torch(w, DEV, seed=0)
+    signs = kv_synth.rademacher_signs(w.S, w.H, w.d, seed=1)
+    st = _t(signs)
+    # lambda: the oracle's, from the first n_cal rows of every slice
+    x_cal = x[:, :w.n_cal].cpu().numpy()
+    lam64 = oracle.calibrate_lambda(x_cal, signs, w.n_cal, rot)
+    lam = lam64.astype(np.float32)
+    lt = _t(lam)
+    lam_gpu = rq.calibrate_lambda(x, st, w.n_cal, rotation=rot).cpu().numpy()
+    parity.assert_clean(parity.check_lambda(lam_gpu, lam64), f"{name} lambda")
+
+    codes, scales = rq.quantize(x, st, lt, w.group, w.bits, rot)
+    xhat = rq.dequantize(codes, scales, st, lt, w.d, w.group, w.bits, rot)
+    torch.cuda.synchronize()
+
+    totals = {}
+    for s in range(w.S):
+        rows = _sample_rows(rng, w.N, k_rows)
+        xs = x[s:s + 1, rows].cpu().numpy()
+        ref = oracle.quantize(xs, signs[s:s + 1], lam[s:s + 1], w.group, w.bits, rot)
+        c_np = codes[s:s + 1, rows].cpu().numpy()
+        s_np = _np16(scales[s:s + 1, rows])
+        stats = parity.check_codes(ref, c_np, s_np, w.bits, w.group)
+        parity.assert_clean(stats, f"{name} slice {s} codes")
+        deq = oracle.dequantize(c_np, s_np, signs[s:s + 1], lam[s:s + 1], w.d, w.group, w.bits, rot)
+        parity.assert_clean(parity.check_dequant(_np16(xhat[s:s + 1, rows]), deq["bits"]),
+                            f"{name} slice {s} dequant")
+        for key, v in stats.items():
+            totals[key] = totals.get(key, 0) + v
+
+    # every vector: range of codes, and the orthogonal error bound
+    qmin_code = 0x8 if w.bits == 4 else 0x80
+    if w.bits == 4:
+        assert not bool(((codes & 0xF) == qmin_code).any() or ((codes >> 4) == qmin_code).any())
+    else:
+        assert not bool((codes == qmin_code).any())
+    sig = scales.float().repeat_interleave(w.group, dim=-1)
+    bound = torch.linalg.vector_norm(sig * lt[:, None] / 2, dim=-1)
+    err = torch.linalg.vector_norm(xhat.float() - x.float(), dim=-1)
+    slack = torch.linalg.vector_norm(xhat.float(), dim=-1) * 2.0 ** -11 + 1e-3 * bound + 1e-6
+    assert bool((err <= bound + slack).all()), float((err - bound - slack).max())
+    rel = (err / torch.linalg.vector_norm(x.float(), dim=-1).clamp_min(1e-12))
+    print(f"{name} rot{rot}: sampled code stats {totals}; rel-L2 error mean "
+          f"{float(rel.mean()):.4f} p99 {float(rel.quantile(0.99) if rel.numel() < 2**24 else rel[:2**24].quantile(0.99)):.4f}")
+    del x, codes, scales, xhat
+    torch.cuda.empty_cache()
+    return totals
+
+
+def test_qwen_like_workload_sampled():
+    _workload_check("qwen_like_d128", rq.SRFT)
+
+
+@pytest.mark.parametrize("rot", [0, 1])
+def test_longctx_int8_workload_sampled(rot):
+    _workload_check("longctx_int8_d128", rot)
