@@ -17,7 +17,9 @@ import ctypes
 import os
 
 PKG_DIR = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(PKG_DIR, "libsrftq.so")
+# SRFTQ_LIB may point at another build of the same library (e.g. a variant
+# under evaluation); by default the in-tree build is loaded.
+LIB_PATH = os.environ.get("SRFTQ_LIB") or os.path.join(PKG_DIR, "libsrftq.so")
 
 SRFTQ_OK = 0
 SRFTQ_ERR_INVALID_ARG = -1

@@ -52,8 +52,22 @@ def _compile(src: str, force: bool, verbose_ptxas: bool):
     return obj, r.stderr if verbose_ptxas else None
 
 
-def build(jobs: int | None = None, force: bool = False, verbose_ptxas: bool = False) -> str:
-    """Compiles every csrc/*.cu for sm_100a and links libsrftq.so; returns its path."""
+def build(jobs: int | None = None, force: bool = False, verbose_ptxas: bool = False,
+          defines: tuple = (), out_dir: str | None = None, src_dir: str | None = None) -> str:
+    """Compiles every csrc/*.cu for sm_100a and links libsrftq.so; returns its path.
+
+    `defines` (NAME=VALUE strings), `src_dir` and `out_dir` build a variant
+    of the library in a separate directory instead of the in-tree one."""
+    global BUILD, LIB, CSRC
+    if src_dir:
+        if not out_dir:
+            raise ValueError("a build from other sources needs its own out_dir")
+        CSRC = os.path.abspath(src_dir)
+    if defines or out_dir:
+        if not out_dir:
+            raise ValueError("a variant build needs its own out_dir")
+        BUILD, LIB = os.path.join(out_dir, "obj"), os.path.join(out_dir, "libsrftq.so")
+        FLAGS.extend(f"-D{d}" for d in defines)
     os.makedirs(BUILD, exist_ok=True)
     srcs = _sources()
     jobs = jobs or min(len(srcs), os.cpu_count() or 4)
@@ -84,8 +98,13 @@ def main(argv=None):
     ap.add_argument("--force", action="store_true")
     ap.add_argument("--ptxas-verbose", action="store_true",
                     help="write ptxas register/spill reports to _build/ptxas.log")
+    ap.add_argument("-D", dest="defines", action="append", default=[],
+                    help="extra preprocessor definition (variant builds)")
+    ap.add_argument("--out-dir", default=None, help="directory of a variant build")
+    ap.add_argument("--src", default=None, help="build these sources instead of csrc/")
     args = ap.parse_args(argv)
-    path = build(args.jobs, args.force, args.ptxas_verbose)
+    path = build(args.jobs, args.force, args.ptxas_verbose, tuple(args.defines), args.out_dir,
+                 args.src)
     print(path)
 
 

@@ -10,21 +10,22 @@
 
 namespace srftq {
 
-// Loads vector `vec` (fp16, 16-byte aligned rows), applies the int8 sign
-// row and converts to float.
+// Loads vector x (fp16, 16-byte aligned) as fp16 pairs and the fp16 +-1
+// sign pairs of its (slice, head) row.
 template <int D>
-__device__ __forceinline__ void load_signed_vector(const uint16_t* x, const int8_t* sgn, float (&v)[D]) {
+__device__ __forceinline__ void load_vector(const uint16_t* x, const int8_t* sgn,
+                                            uint32_t (&xw)[D / 2], uint32_t (&sgw)[D / 2]) {
   static_for<0, D / 8>([&](auto c_) {
     constexpr int ci = decltype(c_)::value;
     const uint4 raw = reinterpret_cast<const uint4*>(x)[ci];
-    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
-    static_for<0, 4>([&](auto k_) {
-      constexpr int k = decltype(k_)::value;
-      const float2 f = __half22float2(u32_as_half2(w[k]));
-      const int j = 8 * ci + 2 * k;
-      v[j] = sgn[j] < 0 ? -f.x : f.x;
-      v[j + 1] = sgn[j + 1] < 0 ? -f.y : f.y;
-    });
+    xw[4 * ci + 0] = raw.x;
+    xw[4 * ci + 1] = raw.y;
+    xw[4 * ci + 2] = raw.z;
+    xw[4 * ci + 3] = raw.w;
+  });
+  static_for<0, D / 2>([&](auto m_) {
+    constexpr int m = decltype(m_)::value;
+    sgw[m] = sign_halves(sgn[2 * m], sgn[2 * m + 1]);
   });
 }
 
@@ -49,21 +50,22 @@ __global__ void __launch_bounds__(128) rotate_kernel(const RotateArgs a) {
     const int64_t s = sr / a.n_rows;
     const uint16_t* xv = a.x + ((s * a.x_slice_stride_rows + r) * a.heads + h) * D;
     const int64_t tab = (s * a.heads + h) * D;
-    float v[D];
-    load_signed_vector<D>(xv, a.signs + tab, v);
-    rotate_forward_raw<ROT, D>(v);
+    uint32_t xw[D / 2], sgw[D / 2];
+    load_vector<D>(xv, a.signs + tab, xw, sgw);
+    float2 v[D / 2];
+    rotate_forward<ROT, D>(xw, sgw, v);
     float* yv = a.y + v_id * D;
     static_for<0, D / 4>([&](auto c_) {
       constexpr int ci = decltype(c_)::value;
-      float4 o;
-      float* op = &o.x;
+      float m[4];
       static_for<0, 4>([&](auto k_) {
         constexpr int j = 4 * ci + decltype(k_)::value;
         const float g = gain_f<ROT, D>(j);
-        op[decltype(k_)::value] =
-            a.lambda ? v[j] * __fdiv_rn(g, a.lambda[tab + j]) : v[j] * g;
+        m[decltype(k_)::value] = a.lambda ? __fdiv_rn(g, a.lambda[tab + j]) : g;
       });
-      reinterpret_cast<float4*>(yv)[ci] = o;
+      reinterpret_cast<float4*>(yv)[ci] = make_float4(v[2 * ci].x * m[0], v[2 * ci].y * m[1],
+                                                      v[2 * ci + 1].x * m[2],
+                                                      v[2 * ci + 1].y * m[3]);
     });
   }
 }
@@ -94,13 +96,16 @@ __global__ void __launch_bounds__(128) calibrate_kernel(const CalibArgs a) {
       const int64_t r = base + threadIdx.x;
       if (r < a.n_cal) {
         const uint16_t* xv = a.x + ((int64_t(s) * a.x_slice_stride_rows + r) * a.heads + h) * D;
-        float v[D];
-        load_signed_vector<D>(xv, a.signs + tab, v);
-        rotate_forward_raw<ROT, D>(v);
-        static_for<0, D>([&](auto j_) {
+        uint32_t xw[D / 2], sgw[D / 2];
+        load_vector<D>(xv, a.signs + tab, xw, sgw);
+        float2 v[D / 2];
+        rotate_forward<ROT, D>(xw, sgw, v);
+        static_for<0, D / 2>([&](auto j_) {
           constexpr int j = decltype(j_)::value;
-          const float y = v[j] * gain_f<ROT, D>(j);
-          sq[threadIdx.x][j] = y * y;
+          const float y0 = v[j].x * gain_f<ROT, D>(2 * j);
+          const float y1 = v[j].y * gain_f<ROT, D>(2 * j + 1);
+          sq[threadIdx.x][2 * j] = y0 * y0;
+          sq[threadIdx.x][2 * j + 1] = y1 * y1;
         });
       } else {
         for (int j = 0; j < D; ++j) sq[threadIdx.x][j] = 0.0f;

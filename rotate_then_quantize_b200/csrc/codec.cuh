@@ -6,19 +6,24 @@
 // memory. Every warp is an independent persistent pipeline: warp w of the
 // grid handles tiles w, w + W, w + 2W, ... (W = warps in the grid). A warp
 // owns NST input stages in shared memory; lane 0 issues, per stage, the TMA
-// box loads of the tile (32 rows x d fp16, 128-byte swizzled so that each
-// lane reading its own row hits distinct banks) plus 1-D bulk copies of that
+// box loads of the tile (32 rows, 128-byte swizzled so that each lane reading
+// its own row hits distinct banks) plus 1-D bulk copies of that
 // (slice, head)'s lambda row and sign row, all completing on one mbarrier.
-// The lanes then build the per-tile multiplier and sign-mask tables, pull
-// their vector into registers, hand the stage back to the TMA engine, and
-// compute. Codes leave through a swizzled shared staging buffer and a TMA
-// tensor store; scales are stored straight from registers.
+// The lanes build the per-(slice, head) multiplier and sign tables (only
+// when the pair changes), pull their vector into registers and compute; the
+// results (codes, or the dequantised fp16 vectors) are written to a swizzled
+// staging tile and fenced for the async proxy. Nothing on this path waits
+// for the TMA engine: at the start of the next tile, where the warp
+// converges anyway, lane 0 issues the TMA store of the staged tile and the
+// refill of the stage the previous tile consumed (NST - 1 tiles ahead).
+// The quantiser stores scales straight from registers; the dequantiser loads
+// them one tile ahead into registers.
 //
 // Quantiser stages follow "When Quantization Is Free", Methodology 2:
-// (1) load and sign multiply (an XOR of the fp16 sign bit in registers),
-// (2) the radix-2 FFT passes, (3) the Hermitian pack, (4) per-channel
-// lambda, group absmax and rounding to signed int4/int8, (5) nibble packing.
-// The dequantiser runs the same stages backwards.
+// (1) load and sign multiply (fused into the first butterfly pass, see
+// transform.cuh), (2) the radix-2 FFT passes, (3) the Hermitian pack,
+// (4) per-channel lambda, group absmax and rounding to signed int4/int8,
+// (5) nibble packing. The dequantiser runs the same stages backwards.
 #pragma once
 
 #include <cuda_fp16.h>
@@ -65,8 +70,11 @@ struct DequantArgs {
   const uint8_t* codes;   // direct path only (code bytes per vector < 16)
   const uint16_t* scales; // [S][T_in][H][d/G]
   int64_t in_slice_stride_rows;
+  uint16_t* xhat;         // [S][T_out][H][d]
+  int64_t out_slice_stride_rows;
   unsigned* guard;
 };
+
 
 // Static shape of one codec configuration.
 template <int D, int BITS, int G>
@@ -86,28 +94,41 @@ struct Shape {
   static constexpr int C_TILE = TR * CB;
   static constexpr int CW = (CB + 3) / 4;               // code words / vector
   static constexpr int NG = D / G;                      // groups / vector
+  static constexpr int SW = (NG + 1) / 2;               // scale words / vector
   static constexpr int QMAX = (1 << (BITS - 1)) - 1;
 };
 
 __host__ __device__ constexpr int align_up(int x, int a) { return (x + a - 1) / a * a; }
 
-// Per-warp shared-memory layout. Stage s: [x or codes tile][lambda row][sign row].
-template <int D, int BITS, int G, int NST, int NOUT, bool QUANT>
+// Per-warp shared-memory layout: NST input tiles (x for the quantiser, codes
+// for the dequantiser; 1024-byte aligned for the swizzled TMA boxes), one
+// output staging tile (codes, or the dequantised fp16 vectors), the NST
+// (lambda row, sign row) pairs that arrive with the input tiles, the
+// multiplier table (d floats), the sign table (d/2 words) and the barriers.
+template <int D, int BITS, int G, int NST, bool QUANT>
 struct WarpLayout {
   using S = Shape<D, BITS, G>;
   static constexpr int kInTile = QUANT ? S::X_TILE : (S::CODES_TMA ? S::C_TILE : 0);
-  static constexpr int kLamOff = align_up(kInTile, 16);
-  static constexpr int kSgnOff = kLamOff + 4 * D;
-  static constexpr int kStageTx = kInTile + 4 * D + D;
-  static constexpr int kStageBytes = align_up(kSgnOff + D, 1024);
+  static constexpr int kInBytes = align_up(kInTile, 1024);
   static constexpr int kOutTile = QUANT ? (S::CODES_TMA ? S::C_TILE : 0) : S::X_TILE;
   static constexpr int kOutBytes = align_up(kOutTile, 1024);
-  static constexpr int kOutOff = NST * kStageBytes;
-  static constexpr int kTableOff = kOutOff + NOUT * kOutBytes;
-  static constexpr int kMaskOff = kTableOff + 4 * D;
-  static constexpr int kBarOff = align_up(kMaskOff + 2 * D, 16);
+  static constexpr int kOutOff = NST * kInBytes;
+  static constexpr int kRowBytes = 4 * D + D;            // lambda row + sign row
+  static constexpr int kRowsOff = kOutOff + kOutBytes;
+  static constexpr int kStageTx = kInTile + kRowBytes;
+  static constexpr int kTableOff = kRowsOff + NST * kRowBytes;
+  static constexpr int kSignTabOff = kTableOff + 4 * D;
+  static constexpr int kBarOff = align_up(kSignTabOff + 2 * D, 16);
   static constexpr int kWarpBytes = align_up(kBarOff + 8 * NST, 1024);
 };
+
+// The launch reserves 1 KB of slack so the swizzled TMA boxes can start on a
+// 1024-byte boundary whatever the base of dynamic shared memory is.
+constexpr int kSmemSlack = 1024;
+
+__device__ __forceinline__ uint8_t* align_smem_1024(uint8_t* p) {
+  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
 
 // Gain of packed coordinate j as a float (see coordinate_gain).
 template <int ROT, int D>
@@ -123,49 +144,66 @@ __device__ __forceinline__ float gain_f(int j) {
   }
 }
 
-// Builds the sign-mask table (one 32-bit XOR mask per fp16 pair: bit 15 and
-// bit 31 set where the sign is negative) from a raw int8 sign row.
-template <int D>
-__device__ __forceinline__ void build_masks(const int8_t* sgn, uint32_t* mask, int lane) {
-  for (int w = lane; w < D / 2; w += 32) {
-    const uint32_t lo = sgn[2 * w] < 0 ? 0x00008000u : 0u;
-    const uint32_t hi = sgn[2 * w + 1] < 0 ? 0x80000000u : 0u;
-    mask[w] = lo | hi;
-  }
+// fp16 +-1.0 pair for int8 signs s0, s1 (negative means -1).
+__device__ __forceinline__ uint32_t sign_halves(int8_t s0, int8_t s1) {
+  return (s0 < 0 ? 0xBC00u : 0x3C00u) | ((s1 < 0 ? 0xBC00u : 0x3C00u) << 16);
 }
 
-__device__ __forceinline__ __half2 u32_as_half2(uint32_t u) {
-  __half2 h;
-  *reinterpret_cast<uint32_t*>(&h) = u;
-  return h;
+// XOR mask flipping the fp16 sign bits of a pair where the sign is negative.
+__device__ __forceinline__ uint32_t sign_mask(int8_t s0, int8_t s1) {
+  return (s0 < 0 ? 0x00008000u : 0u) | (s1 < 0 ? 0x80000000u : 0u);
 }
 
-__device__ __forceinline__ uint32_t half2_as_u32(__half2 h) {
-  return *reinterpret_cast<uint32_t*>(&h);
+// max(|a|, |b|, |c|) in one instruction.
+__device__ __forceinline__ float absmax3(float a, float b, float c) {
+  float r;
+  asm("max.abs.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
 }
+
+// Correctly rounded a / Q for the constant Q: q0 = a * RN(1/Q) is within an
+// ulp, the FMA remainder a - q0 Q is exact, and one correction step gives the
+// rounded quotient (Markstein's theorem on division by a reciprocal).
+template <int Q>
+__device__ __forceinline__ float div_by_const(float a) {
+  constexpr float inv = float(1.0 / double(Q));
+  const float q0 = a * inv;
+  const float r = fmaf(-q0, float(Q), a);
+  return fmaf(r, inv, q0);
+}
+
+__device__ __forceinline__ float rcp_approx(float x) {
+  float r;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// Whether the rounding step uses f32x2 FMAs (constant pairs in registers)
+// or scalar FMAs with an immediate.
+#ifndef SRFTQ_PACKED_ROUND
+#define SRFTQ_PACKED_ROUND 1
+#endif
 
 // 1.5 * 2^23: adding it to |v| < 2^22 rounds v to an integer (ties to even)
 // whose two's complement lands in the low bits of the float's encoding.
-constexpr float kMagic0 = 12582912.0f;
-
-// The launch reserves 1 KB of slack so the swizzled TMA boxes can start on a
-// 1024-byte boundary whatever the base of dynamic shared memory is.
-constexpr int kSmemSlack = 1024;
-
-__device__ __forceinline__ uint8_t* align_smem_1024(uint8_t* p) {
-  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
-}
+constexpr float kMagic = 12582912.0f;
 
 // ---------------------------------------------------------------------------
 // Quantiser
 // ---------------------------------------------------------------------------
 
-template <int D, int BITS, int G, int ROT, int WPC, int NST, int NOUT>
-__global__ void __launch_bounds__(WPC * 32)
+template <int D, int BITS, int G, int ROT, int WPC, int NST, int MINB>
+__global__ void __launch_bounds__(WPC * 32, MINB)
     quantize_kernel(const __grid_constant__ CUtensorMap tm_x,
                     const __grid_constant__ CUtensorMap tm_codes, const QuantArgs a) {
   using S = Shape<D, BITS, G>;
-  using Lay = WarpLayout<D, BITS, G, NST, NOUT, true>;
+  using Lay = WarpLayout<D, BITS, G, NST, true>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = align_smem_1024(smem_raw);
   const int warp = threadIdx.x >> 5;
@@ -173,7 +211,8 @@ __global__ void __launch_bounds__(WPC * 32)
   uint8_t* ws = smem + warp * Lay::kWarpBytes;
   uint64_t* bars = reinterpret_cast<uint64_t*>(ws + Lay::kBarOff);
   float* mult = reinterpret_cast<float*>(ws + Lay::kTableOff);
-  uint32_t* mask = reinterpret_cast<uint32_t*>(ws + Lay::kMaskOff);
+  uint32_t* stab = reinterpret_cast<uint32_t*>(ws + Lay::kSignTabOff);
+  uint8_t* ob = ws + Lay::kOutOff;   // codes staging tile
 
   const int total = a.g.total_tiles;
   const int nw = gridDim.x * WPC;
@@ -190,15 +229,22 @@ __global__ void __launch_bounds__(WPC * 32)
 
   auto issue = [&](int t, int st) {
     const TileCoord c = decode_tile(t, a.g);
-    uint8_t* sb = ws + st * Lay::kStageBytes;
+    uint8_t* sb = ws + st * Lay::kInBytes;
+    uint8_t* rb = ws + Lay::kRowsOff + st * Lay::kRowBytes;
     mbar_arrive_expect_tx(&bars[st], Lay::kStageTx);
 #pragma unroll
     for (int p = 0; p < S::X_PIECES; ++p)
       tma_load_4d(sb + p * (S::TR * S::X_SPAN), &tm_x, &bars[st], p * (S::X_SPAN / 2), c.h, c.r0,
                   c.s);
     const size_t row = static_cast<size_t>(c.s) * a.g.heads + c.h;
-    bulk_load(sb + Lay::kLamOff, a.lambda + row * D, 4 * D, &bars[st]);
-    bulk_load(sb + Lay::kSgnOff, a.signs + row * D, D, &bars[st]);
+    bulk_load(rb, a.lambda + row * D, 4 * D, &bars[st]);
+    bulk_load(rb + 4 * D, a.signs + row * D, D, &bars[st]);
+  };
+  auto store_codes = [&](const TileCoord& c) {
+#pragma unroll
+    for (int p = 0; p < S::C_PIECES; ++p)
+      tma_store_4d(&tm_codes, ob + p * (S::TR * S::C_SPAN), p * S::C_SPAN, c.h, c.r0, c.s);
+    bulk_commit();
   };
 
   if (lane == 0) {
@@ -209,11 +255,15 @@ __global__ void __launch_bounds__(WPC * 32)
   }
 
   int it = 0;
+  int table_sh = -1;          // (slice, head) the tables were built for
+  bool pending = false;       // a staged codes tile awaits its TMA store
+  TileCoord prev{0, 0, 0};
   for (int t = first; t < total; t += nw, ++it) {
     const int st = it % NST;
     const uint32_t parity = (it / NST) & 1;
     const TileCoord c = decode_tile(t, a.g);
-    uint8_t* sb = ws + st * Lay::kStageBytes;
+    const uint8_t* sb = ws + st * Lay::kInBytes;
+    const uint8_t* rb = ws + Lay::kRowsOff + st * Lay::kRowBytes;
 
     const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars[st], parity));
     if (!ok) {
@@ -229,89 +279,105 @@ __global__ void __launch_bounds__(WPC * 32)
       __syncwarp();
       return;
     }
-
-    // (a) per-(slice, head) tables: multiplier gain_j / lambda_j and sign masks
-    const float* lam_raw = reinterpret_cast<const float*>(sb + Lay::kLamOff);
-    const int8_t* sgn_raw = reinterpret_cast<const int8_t*>(sb + Lay::kSgnOff);
+    // Converged: the previous tile's codes are staged and fenced, and its
+    // input stage has been read. Store the one, refill the other.
     __syncwarp();
-    for (int j = lane; j < D; j += 32) mult[j] = __fdiv_rn(gain_f<ROT, D>(j), lam_raw[j]);
-    build_masks<D>(sgn_raw, mask, lane);
-    __syncwarp();
+    if (lane == 0) {
+      if (pending) store_codes(prev);
+      const int tn = t + (NST - 1) * nw;
+      if (it > 0 && tn < total) issue(tn, (it - 1) % NST);
+    }
+    pending = false;
 
-    // (b) this lane's vector: swizzled 16-byte chunks, sign XOR, fp16 -> fp32
-    float v[D];
+    // (a) per-(slice, head) tables: multiplier gain_j / lambda_j, fp16 signs
+    // (rebuilt only when the tile's (slice, head) differs from the last one)
+    const int sh = c.s * a.g.heads + c.h;
+    if (sh != table_sh) {
+      const float* lam_raw = reinterpret_cast<const float*>(rb);
+      const int8_t* sgn_raw = reinterpret_cast<const int8_t*>(rb + 4 * D);
+      for (int j = lane; j < D; j += 32) mult[j] = gain_f<ROT, D>(j) * rcp_approx(lam_raw[j]);
+      for (int w = lane; w < D / 2; w += 32) stab[w] = sign_halves(sgn_raw[2 * w], sgn_raw[2 * w + 1]);
+      __syncwarp();
+      table_sh = sh;
+    }
+
+    // (b) this lane's vector (swizzled 16-byte chunks) and the sign words
+    uint32_t xw[D / 2], sgw[D / 2];
     static_for<0, D / 8>([&](auto c_) {
       constexpr int ci = decltype(c_)::value;
       constexpr int piece = (ci * 16) / S::X_SPAN;
       constexpr int cc = ((ci * 16) % S::X_SPAN) / 16;
       const uint32_t off =
           piece * (S::TR * S::X_SPAN) + swizzle<S::X_SPAN>(lane * S::X_SPAN + cc * 16);
-      uint4 raw = *reinterpret_cast<const uint4*>(sb + off);
-      const uint4 m = *reinterpret_cast<const uint4*>(mask + 4 * ci);
-      raw.x ^= m.x;
-      raw.y ^= m.y;
-      raw.z ^= m.z;
-      raw.w ^= m.w;
-      const float2 f0 = __half22float2(u32_as_half2(raw.x));
-      const float2 f1 = __half22float2(u32_as_half2(raw.y));
-      const float2 f2 = __half22float2(u32_as_half2(raw.z));
-      const float2 f3 = __half22float2(u32_as_half2(raw.w));
-      v[8 * ci + 0] = f0.x;
-      v[8 * ci + 1] = f0.y;
-      v[8 * ci + 2] = f1.x;
-      v[8 * ci + 3] = f1.y;
-      v[8 * ci + 4] = f2.x;
-      v[8 * ci + 5] = f2.y;
-      v[8 * ci + 6] = f3.x;
-      v[8 * ci + 7] = f3.y;
+      const uint4 raw = *reinterpret_cast<const uint4*>(sb + off);
+      const uint4 sg = *reinterpret_cast<const uint4*>(stab + 4 * ci);
+      xw[4 * ci + 0] = raw.x;
+      xw[4 * ci + 1] = raw.y;
+      xw[4 * ci + 2] = raw.z;
+      xw[4 * ci + 3] = raw.w;
+      sgw[4 * ci + 0] = sg.x;
+      sgw[4 * ci + 1] = sg.y;
+      sgw[4 * ci + 2] = sg.z;
+      sgw[4 * ci + 3] = sg.w;
     });
-    __syncwarp();
-    if (lane == 0) {
-      const int tn = t + NST * nw;
-      if (tn < total) issue(tn, st);
-    }
 
     // (c) rotation, then w_j = y_j / lambda_j through the multiplier table
-    rotate_forward_raw<ROT, D>(v);
+    float2 v[D / 2];
+    rotate_forward<ROT, D>(xw, sgw, v);
     static_for<0, D / 4>([&](auto c_) {
       constexpr int ci = decltype(c_)::value;
       const float4 m4 = *reinterpret_cast<const float4*>(mult + 4 * ci);
-      v[4 * ci + 0] *= m4.x;
-      v[4 * ci + 1] *= m4.y;
-      v[4 * ci + 2] *= m4.z;
-      v[4 * ci + 3] *= m4.w;
+      v[2 * ci] = mul2(v[2 * ci], make_float2(m4.x, m4.y));
+      v[2 * ci + 1] = mul2(v[2 * ci + 1], make_float2(m4.z, m4.w));
     });
 
-    // (d) group absmax -> fp16 scale -> rounded codes (float-encoded integers)
-    uint32_t qb[D];
+    // (d) group absmax -> fp16 scale -> codes as float-encoded integers.
+    // With a normal, unsaturated scale |w/sigma| <= qmax * (1 + 2^-10) up to
+    // rounding, which rounds inside the range, so unless some group's scale
+    // is subnormal or saturated the whole vector is rounded without a clamp
+    // (sigma == 0 gives inv = 0 and code 0 either way). Both branches are
+    // straight-line code over all groups.
     uint16_t sig[S::NG];
+    float invs[S::NG];
+    bool clamp = false;
     static_for<0, S::NG>([&](auto g_) {
       constexpr int g = decltype(g_)::value;
+      constexpr int P0 = g * G / 2;   // first pair of the group
       float amax = 0.0f;
-      static_for<0, G>([&](auto j_) {
-        amax = fmaxf(amax, fabsf(v[g * G + decltype(j_)::value]));
+      static_for<0, G / 2>([&](auto p_) {
+        constexpr int p = P0 + decltype(p_)::value;
+        amax = absmax3(amax, v[p].x, v[p].y);
       });
-      const float sf = __fdiv_rn(amax, float(S::QMAX));
+      const float sf = div_by_const<S::QMAX>(amax);
       const __half hs = __float2half_rn(fminf(sf, 65504.0f));
       sig[g] = __half_as_ushort(hs);
       const float sg = __half2float(hs);
-      // With a normal, unsaturated scale |w/sigma| <= qmax * (1 + 2^-10), which
-      // rounds inside the range: no clamp needed.
-      if (sg >= 6.103515625e-05f && sf <= 65504.0f) {
-        const float inv = __frcp_rn(sg);
-        static_for<0, G>([&](auto j_) {
-          constexpr int j = g * G + decltype(j_)::value;
-          qb[j] = __float_as_uint(fmaf(v[j], inv, kMagic0));
-        });
-      } else {
-        const float inv = sg > 0.0f ? __frcp_rn(sg) : 0.0f;
-        static_for<0, G>([&](auto j_) {
-          constexpr int j = g * G + decltype(j_)::value;
-          const float q = fminf(fmaxf(v[j] * inv, -float(S::QMAX)), float(S::QMAX));
-          qb[j] = __float_as_uint(q + kMagic0);
-        });
-      }
+      invs[g] = sg > 0.0f ? rcp_approx(sg) : 0.0f;
+      clamp |= sg > 0.0f && !(sg >= 6.103515625e-05f && sf <= 65504.0f);
     });
+    uint32_t qb[D];
+    if (!clamp) {
+      static_for<0, D / 2>([&](auto p_) {
+        constexpr int p = decltype(p_)::value;
+#if SRFTQ_PACKED_ROUND
+        const float2 r = fma2(v[p], splat(invs[(2 * p) / G]), splat(kMagic));
+        qb[2 * p] = __float_as_uint(r.x);
+        qb[2 * p + 1] = __float_as_uint(r.y);
+#else
+        qb[2 * p] = __float_as_uint(fmaf(v[p].x, invs[(2 * p) / G], kMagic));
+        qb[2 * p + 1] = __float_as_uint(fmaf(v[p].y, invs[(2 * p) / G], kMagic));
+#endif
+      });
+    } else {
+      static_for<0, D / 2>([&](auto p_) {
+        constexpr int p = decltype(p_)::value;
+        const float inv = invs[(2 * p) / G];
+        const float q0 = fminf(fmaxf(v[p].x * inv, -float(S::QMAX)), float(S::QMAX));
+        const float q1 = fminf(fmaxf(v[p].y * inv, -float(S::QMAX)), float(S::QMAX));
+        qb[2 * p] = __float_as_uint(q0 + kMagic);
+        qb[2 * p + 1] = __float_as_uint(q1 + kMagic);
+      });
+    }
 
     // (e) pack. The low byte of every qb is its code in two's complement.
     // int4: byte k = code 2k in the low nibble | code 2k+1 in the high nibble;
@@ -338,10 +404,11 @@ __global__ void __launch_bounds__(WPC * 32)
     const bool valid = row < a.g.n_rows;
     const size_t vec = (static_cast<size_t>(c.s) * a.out_slice_stride_rows + row) * a.g.heads + c.h;
 
-    // (f) codes: swizzled staging + TMA store (rows past N are clipped by TMA)
+    // (f) codes: swizzled staging tile, stored by TMA at the next convergence
+    // (rows past N are clipped by TMA). The store issued at this tile's start
+    // read the staging tile long ago; the wait only confirms it.
     if constexpr (S::CODES_TMA) {
-      uint8_t* ob = ws + Lay::kOutOff + (it % NOUT) * Lay::kOutBytes;
-      if (lane == 0) bulk_wait_read<NOUT - 1>();
+      if (lane == 0) bulk_wait_read<0>();
       __syncwarp();
       static_for<0, S::CB / 16>([&](auto c_) {
         constexpr int ci = decltype(c_)::value;
@@ -353,22 +420,11 @@ __global__ void __launch_bounds__(WPC * 32)
             make_uint4(words[4 * ci], words[4 * ci + 1], words[4 * ci + 2], words[4 * ci + 3]);
       });
       fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) {
-#pragma unroll
-        for (int p = 0; p < S::C_PIECES; ++p)
-          tma_store_4d(&tm_codes, ob + p * (S::TR * S::C_SPAN), p * S::C_SPAN, c.h, c.r0, c.s);
-        bulk_commit();
-      }
+      pending = true;
+      prev = c;
     } else {
-      if (valid) {
-        uint8_t* dst = a.codes + vec * S::CB;
-        if constexpr (S::CB == 8) {
-          *reinterpret_cast<uint2*>(dst) = make_uint2(words[0], words[1]);
-        } else {
-          static_assert(S::CB == 8, "direct code path covers d=16 int4 only");
-        }
-      }
+      static_assert(S::CODES_TMA || S::CB == 8, "direct code path covers d=16 int4 only");
+      if (valid) *reinterpret_cast<uint2*>(a.codes + vec * S::CB) = make_uint2(words[0], words[1]);
     }
 
     // (g) scales straight from registers
@@ -396,8 +452,10 @@ __global__ void __launch_bounds__(WPC * 32)
       }
     }
   }
-  if constexpr (S::CODES_TMA) {
-    if (lane == 0) bulk_wait<0>();
+  __syncwarp();
+  if (lane == 0) {
+    if (pending) store_codes(prev);
+    bulk_wait<0>();
   }
 }
 
@@ -405,12 +463,37 @@ __global__ void __launch_bounds__(WPC * 32)
 // Dequantiser
 // ---------------------------------------------------------------------------
 
-template <int D, int BITS, int G, int ROT, int WPC, int NST, int NOUT>
-__global__ void __launch_bounds__(WPC * 32)
+// Codes of one 32-bit word to exact fp32 values q * sigma (int8: 4 codes;
+// int4: 8 codes, odd positions scaled by 16). The codes are spread into fp16
+// pairs 1024 + offset + code (one AND-XOR each), then `fma.rn.f32.f16`
+// multiplies by the fp16 scale and subtracts the offset's product exactly.
+template <int BITS, int HS>
+__device__ __forceinline__ void unpack_word(uint32_t w, uint32_t sgw, float c_even, float c_odd,
+                                            float2* out) {
+  const uint32_t w8 = w >> 8;
+  if constexpr (BITS == 4) {
+    const uint32_t h04 = (w & 0x000F000Fu) ^ 0x64086408u;   // 1024 + 8 + q
+    const uint32_t h15 = (w & 0x00F000F0u) ^ 0x64806480u;   // 1024 + 16 (8 + q)
+    const uint32_t h26 = (w8 & 0x000F000Fu) ^ 0x64086408u;
+    const uint32_t h37 = (w8 & 0x00F000F0u) ^ 0x64806480u;
+    out[0] = make_float2(fma_f16<0, HS>(h04, sgw, c_even), fma_f16<0, HS>(h15, sgw, c_odd));
+    out[1] = make_float2(fma_f16<0, HS>(h26, sgw, c_even), fma_f16<0, HS>(h37, sgw, c_odd));
+    out[2] = make_float2(fma_f16<1, HS>(h04, sgw, c_even), fma_f16<1, HS>(h15, sgw, c_odd));
+    out[3] = make_float2(fma_f16<1, HS>(h26, sgw, c_even), fma_f16<1, HS>(h37, sgw, c_odd));
+  } else {
+    const uint32_t h02 = (w & 0x00FF00FFu) ^ 0x64806480u;   // 1024 + 128 + q
+    const uint32_t h13 = (w8 & 0x00FF00FFu) ^ 0x64806480u;
+    out[0] = make_float2(fma_f16<0, HS>(h02, sgw, c_even), fma_f16<0, HS>(h13, sgw, c_even));
+    out[1] = make_float2(fma_f16<1, HS>(h02, sgw, c_even), fma_f16<1, HS>(h13, sgw, c_even));
+  }
+}
+
+template <int D, int BITS, int G, int ROT, int WPC, int NST, int MINB>
+__global__ void __launch_bounds__(WPC * 32, MINB)
     dequantize_kernel(const __grid_constant__ CUtensorMap tm_codes,
                       const __grid_constant__ CUtensorMap tm_xhat, const DequantArgs a) {
   using S = Shape<D, BITS, G>;
-  using Lay = WarpLayout<D, BITS, G, NST, NOUT, false>;
+  using Lay = WarpLayout<D, BITS, G, NST, false>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = align_smem_1024(smem_raw);
   const int warp = threadIdx.x >> 5;
@@ -418,7 +501,8 @@ __global__ void __launch_bounds__(WPC * 32)
   uint8_t* ws = smem + warp * Lay::kWarpBytes;
   uint64_t* bars = reinterpret_cast<uint64_t*>(ws + Lay::kBarOff);
   float* mult = reinterpret_cast<float*>(ws + Lay::kTableOff);
-  uint32_t* mask = reinterpret_cast<uint32_t*>(ws + Lay::kMaskOff);
+  uint32_t* mtab = reinterpret_cast<uint32_t*>(ws + Lay::kSignTabOff);
+  uint8_t* ob = ws + Lay::kOutOff;   // fp16 staging tile
 
   const int total = a.g.total_tiles;
   const int nw = gridDim.x * WPC;
@@ -435,7 +519,8 @@ __global__ void __launch_bounds__(WPC * 32)
 
   auto issue = [&](int t, int st) {
     const TileCoord c = decode_tile(t, a.g);
-    uint8_t* sb = ws + st * Lay::kStageBytes;
+    uint8_t* sb = ws + st * Lay::kInBytes;
+    uint8_t* rb = ws + Lay::kRowsOff + st * Lay::kRowBytes;
     mbar_arrive_expect_tx(&bars[st], Lay::kStageTx);
     if constexpr (S::CODES_TMA) {
 #pragma unroll
@@ -444,8 +529,14 @@ __global__ void __launch_bounds__(WPC * 32)
                     c.s);
     }
     const size_t row = static_cast<size_t>(c.s) * a.g.heads + c.h;
-    bulk_load(sb + Lay::kLamOff, a.lambda + row * D, 4 * D, &bars[st]);
-    bulk_load(sb + Lay::kSgnOff, a.signs + row * D, D, &bars[st]);
+    bulk_load(rb, a.lambda + row * D, 4 * D, &bars[st]);
+    bulk_load(rb + 4 * D, a.signs + row * D, D, &bars[st]);
+  };
+  auto store_xhat = [&](const TileCoord& c) {
+#pragma unroll
+    for (int p = 0; p < S::X_PIECES; ++p)
+      tma_store_4d(&tm_xhat, ob + p * (S::TR * S::X_SPAN), p * (S::X_SPAN / 2), c.h, c.r0, c.s);
+    bulk_commit();
   };
 
   if (lane == 0) {
@@ -455,19 +546,13 @@ __global__ void __launch_bounds__(WPC * 32)
     }
   }
 
-  int it = 0;
-  for (int t = first; t < total; t += nw, ++it) {
-    const int st = it % NST;
-    const uint32_t parity = (it / NST) & 1;
+  // the next tile's scales are loaded one tile ahead, into registers
+  auto load_scales = [&](int t, uint32_t (&sw)[S::SW]) {
     const TileCoord c = decode_tile(t, a.g);
-    uint8_t* sb = ws + st * Lay::kStageBytes;
     const int row = c.r0 + lane;
-    const bool valid = row < a.g.n_rows;
-    const size_t vec = (static_cast<size_t>(c.s) * a.in_slice_stride_rows + row) * a.g.heads + c.h;
-
-    // scales for this lane's vector (plain loads; rows past N read as zero)
-    uint32_t sw[(S::NG + 1) / 2];
-    if (valid) {
+    if (row < a.g.n_rows) {
+      const size_t vec =
+          (static_cast<size_t>(c.s) * a.in_slice_stride_rows + row) * a.g.heads + c.h;
       const uint16_t* src = a.scales + vec * S::NG;
       if constexpr (S::NG == 1) {
         sw[0] = src[0];
@@ -488,8 +573,30 @@ __global__ void __launch_bounds__(WPC * 32)
         });
       }
     } else {
-      static_for<0, (S::NG + 1) / 2>([&](auto k_) { sw[decltype(k_)::value] = 0u; });
+      static_for<0, S::SW>([&](auto k_) { sw[decltype(k_)::value] = 0u; });
     }
+  };
+  uint32_t sw_next[S::SW];
+  load_scales(first, sw_next);
+
+  int it = 0;
+  int table_sh = -1;          // (slice, head) the tables were built for
+  bool pending = false;       // a staged fp16 tile awaits its TMA store
+  TileCoord prev{0, 0, 0};
+  for (int t = first; t < total; t += nw, ++it) {
+    const int st = it % NST;
+    const uint32_t parity = (it / NST) & 1;
+    const TileCoord c = decode_tile(t, a.g);
+    const uint8_t* sb = ws + st * Lay::kInBytes;
+    const uint8_t* rb = ws + Lay::kRowsOff + st * Lay::kRowBytes;
+    const int row = c.r0 + lane;
+    const bool valid = row < a.g.n_rows;
+    const size_t vec = (static_cast<size_t>(c.s) * a.in_slice_stride_rows + row) * a.g.heads + c.h;
+
+    uint32_t sw[S::SW];
+    static_for<0, S::SW>([&](auto k_) { sw[decltype(k_)::value] = sw_next[decltype(k_)::value]; });
+    if (t + nw < total) load_scales(t + nw, sw_next);
+
     uint32_t words[S::CW];
     if constexpr (!S::CODES_TMA) {
       if (valid) {
@@ -514,14 +621,29 @@ __global__ void __launch_bounds__(WPC * 32)
       __syncwarp();
       return;
     }
+    // Converged: the previous tile's output is staged and fenced, and its
+    // input stage has been read. Store the one, refill the other.
+    __syncwarp();
+    if (lane == 0) {
+      if (pending) store_xhat(prev);
+      const int tn = t + (NST - 1) * nw;
+      if (it > 0 && tn < total) issue(tn, (it - 1) % NST);
+    }
+    pending = false;
 
-    // (a) tables: multiplier gain_j * lambda_j and sign masks
-    const float* lam_raw = reinterpret_cast<const float*>(sb + Lay::kLamOff);
-    const int8_t* sgn_raw = reinterpret_cast<const int8_t*>(sb + Lay::kSgnOff);
-    __syncwarp();
-    for (int j = lane; j < D; j += 32) mult[j] = gain_f<ROT, D>(j) * lam_raw[j];
-    build_masks<D>(sgn_raw, mask, lane);
-    __syncwarp();
+    // (a) tables: multiplier gain_j * lambda_j (int4: /16 at odd j, matching
+    // the x16 of the odd codes' unpacking) and output sign masks (rebuilt
+    // only when the tile's (slice, head) differs from the last one)
+    const int sh = c.s * a.g.heads + c.h;
+    if (sh != table_sh) {
+      const float* lam_raw = reinterpret_cast<const float*>(rb);
+      const int8_t* sgn_raw = reinterpret_cast<const int8_t*>(rb + 4 * D);
+      for (int j = lane; j < D; j += 32)
+        mult[j] = gain_f<ROT, D>(j) * lam_raw[j] * ((BITS == 4 && (j & 1)) ? 0.0625f : 1.0f);
+      for (int w = lane; w < D / 2; w += 32) mtab[w] = sign_mask(sgn_raw[2 * w], sgn_raw[2 * w + 1]);
+      __syncwarp();
+      table_sh = sh;
+    }
 
     // (b) codes of this lane's vector
     if constexpr (S::CODES_TMA) {
@@ -538,63 +660,57 @@ __global__ void __launch_bounds__(WPC * 32)
         words[4 * ci + 3] = u.w;
       });
     }
-    __syncwarp();
-    if (lane == 0) {
-      const int tn = t + NST * nw;
-      if (tn < total) issue(tn, st);
-    }
 
     // (c) yhat_j = q_j * sigma_g * lambda_j * gain_j
-    float v[D];
-    static_for<0, S::NG>([&](auto g_) {
-      constexpr int g = decltype(g_)::value;
-      const uint32_t sbits = (sw[g / 2] >> (16 * (g & 1))) & 0xFFFFu;
-      const float sg = __half2float(__ushort_as_half(static_cast<unsigned short>(sbits)));
-      static_for<0, G>([&](auto j_) {
-        constexpr int j = g * G + decltype(j_)::value;
-        float q;
-        if constexpr (BITS == 4) {
-          const uint32_t nib = (words[j / 8] >> (4 * (j % 8))) & 0xFu;
-          q = __uint_as_float(0x4B400000u | (nib ^ 0x8u)) - (kMagic0 + 8.0f);
-        } else {
-          const uint32_t byte = (words[j / 4] >> (8 * (j % 4))) & 0xFFu;
-          q = __uint_as_float(0x4B400000u | (byte ^ 0x80u)) - (kMagic0 + 128.0f);
-        }
-        v[j] = q * (sg * mult[j]);
-      });
+    float2 v[D / 2];
+    constexpr int CPW = 32 / BITS;   // codes per word
+    static_for<0, S::CW>([&](auto m_) {
+      constexpr int m = decltype(m_)::value;
+      constexpr int g = (m * CPW) / G;
+      const float sgf = __half2float(__ushort_as_half(
+          static_cast<unsigned short>((sw[g / 2] >> (16 * (g & 1))) & 0xFFFFu)));
+      const float c_even = BITS == 4 ? -1032.0f * sgf : -1152.0f * sgf;
+      const float c_odd = -1152.0f * sgf;
+      unpack_word<BITS, g & 1>(words[m], sw[g / 2], c_even, c_odd, &v[m * CPW / 2]);
+    });
+    static_for<0, D / 4>([&](auto c_) {
+      constexpr int ci = decltype(c_)::value;
+      const float4 m4 = *reinterpret_cast<const float4*>(mult + 4 * ci);
+      v[2 * ci] = mul2(v[2 * ci], make_float2(m4.x, m4.y));
+      v[2 * ci + 1] = mul2(v[2 * ci + 1], make_float2(m4.z, m4.w));
     });
 
     // (d) inverse rotation
-    rotate_inverse_raw<ROT, D>(v);
+    rotate_inverse<ROT, D>(v);
 
-    // (e) signs + fp16, swizzled staging, TMA store
-    uint8_t* ob = ws + Lay::kOutOff + (it % NOUT) * Lay::kOutBytes;
-    if (lane == 0) bulk_wait_read<NOUT - 1>();
+    // (e) signs + fp16 into the swizzled staging tile, stored by TMA at the
+    // next convergence. The store issued at this tile's start read the
+    // staging tile long ago; the wait only confirms it.
+    if (lane == 0) bulk_wait_read<0>();
     __syncwarp();
     static_for<0, D / 8>([&](auto c_) {
       constexpr int ci = decltype(c_)::value;
       constexpr int piece = (ci * 16) / S::X_SPAN;
       constexpr int cc = ((ci * 16) % S::X_SPAN) / 16;
-      const uint4 m = *reinterpret_cast<const uint4*>(mask + 4 * ci);
+      const uint4 mk = *reinterpret_cast<const uint4*>(mtab + 4 * ci);
       uint4 o;
-      o.x = half2_as_u32(__floats2half2_rn(v[8 * ci + 0], v[8 * ci + 1])) ^ m.x;
-      o.y = half2_as_u32(__floats2half2_rn(v[8 * ci + 2], v[8 * ci + 3])) ^ m.y;
-      o.z = half2_as_u32(__floats2half2_rn(v[8 * ci + 4], v[8 * ci + 5])) ^ m.z;
-      o.w = half2_as_u32(__floats2half2_rn(v[8 * ci + 6], v[8 * ci + 7])) ^ m.w;
+      o.x = pack_f16x2(v[4 * ci + 0].x, v[4 * ci + 0].y) ^ mk.x;
+      o.y = pack_f16x2(v[4 * ci + 1].x, v[4 * ci + 1].y) ^ mk.y;
+      o.z = pack_f16x2(v[4 * ci + 2].x, v[4 * ci + 2].y) ^ mk.z;
+      o.w = pack_f16x2(v[4 * ci + 3].x, v[4 * ci + 3].y) ^ mk.w;
       const uint32_t off =
           piece * (S::TR * S::X_SPAN) + swizzle<S::X_SPAN>(lane * S::X_SPAN + cc * 16);
       *reinterpret_cast<uint4*>(ob + off) = o;
     });
     fence_proxy_async_smem();
-    __syncwarp();
-    if (lane == 0) {
-#pragma unroll
-      for (int p = 0; p < S::X_PIECES; ++p)
-        tma_store_4d(&tm_xhat, ob + p * (S::TR * S::X_SPAN), p * (S::X_SPAN / 2), c.h, c.r0, c.s);
-      bulk_commit();
-    }
+    pending = true;
+    prev = c;
   }
-  if (lane == 0) bulk_wait<0>();
+  __syncwarp();
+  if (lane == 0) {
+    if (pending) store_xhat(prev);
+    bulk_wait<0>();
+  }
 }
 
 }  // namespace srftq

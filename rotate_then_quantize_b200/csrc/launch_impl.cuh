@@ -12,10 +12,30 @@
 
 namespace srftq {
 
-// Warps per block, input stages and output staging buffers per warp.
-constexpr int kWPC = 4;
-constexpr int kNST = 2;
-constexpr int kNOUT = 2;
+// Launch shapes: warps per block and the blocks per SM the register budget
+// is sized for (their product is the resident warps per SM), and input
+// stages per warp. Measured on B200 at d = 128: both kernels run fastest
+// with 8 warps per SM and the full register budget (the transform keeps
+// ~200 values live; at 12 warps per SM the 168-register cap costs more than
+// the extra warps recover).
+#ifndef SRFTQ_Q_WPC
+#define SRFTQ_Q_WPC 4
+#endif
+#ifndef SRFTQ_Q_MINB
+#define SRFTQ_Q_MINB 2
+#endif
+#ifndef SRFTQ_D_WPC
+#define SRFTQ_D_WPC 4
+#endif
+#ifndef SRFTQ_D_MINB
+#define SRFTQ_D_MINB 2
+#endif
+#ifndef SRFTQ_NST
+#define SRFTQ_NST 2
+#endif
+constexpr int kQWPC = SRFTQ_Q_WPC, kQMinBlocks = SRFTQ_Q_MINB;
+constexpr int kDWPC = SRFTQ_D_WPC, kDMinBlocks = SRFTQ_D_MINB;
+constexpr int kNST = SRFTQ_NST;
 
 inline CUtensorMapSwizzle swizzle_mode(int span) {
   switch (span) {
@@ -78,7 +98,7 @@ inline int finish_launch() {
 template <int D, int BITS, int G, int ROT>
 int quantize_impl(const QuantCall& c) {
   using S = Shape<D, BITS, G>;
-  using Lay = WarpLayout<D, BITS, G, kNST, kNOUT, true>;
+  using Lay = WarpLayout<D, BITS, G, kNST, true>;
   const int64_t row_blocks = (c.n_rows + kTileRows - 1) / kTileRows;
   const int64_t total = c.n_slices * row_blocks * c.heads;
   if (total == 0) return SRFTQ_OK;
@@ -117,22 +137,22 @@ int quantize_impl(const QuantCall& c) {
   a.out_slice_stride_rows = c.out_slice_stride_rows;
   a.guard = guard;
 
-  constexpr auto K = quantize_kernel<D, BITS, G, ROT, kWPC, kNST, kNOUT>;
-  const int smem = kWPC * Lay::kWarpBytes + kSmemSlack;
+  constexpr auto K = quantize_kernel<D, BITS, G, ROT, kQWPC, kNST, kQMinBlocks>;
+  const int smem = kQWPC * Lay::kWarpBytes + kSmemSlack;
   int bps = 0;
-  int rc = prepare_kernel<K>(smem, kWPC * 32, &bps);
+  int rc = prepare_kernel<K>(smem, kQWPC * 32, &bps);
   if (rc != SRFTQ_OK) return rc;
-  const int64_t want = (total + kWPC - 1) / kWPC;
+  const int64_t want = (total + kQWPC - 1) / kQWPC;
   const int64_t cap = int64_t(Runtime::num_sms()) * bps;
   const int grid = int(want < cap ? want : cap);
-  K<<<grid, kWPC * 32, smem, c.stream>>>(tm_x, tm_c, a);
+  K<<<grid, kQWPC * 32, smem, c.stream>>>(tm_x, tm_c, a);
   return finish_launch();
 }
 
 template <int D, int BITS, int G, int ROT>
 int dequantize_impl(const DequantCall& c) {
   using S = Shape<D, BITS, G>;
-  using Lay = WarpLayout<D, BITS, G, kNST, kNOUT, false>;
+  using Lay = WarpLayout<D, BITS, G, kNST, false>;
   const int64_t row_blocks = (c.n_rows + kTileRows - 1) / kTileRows;
   const int64_t total = c.n_slices * row_blocks * c.heads;
   if (total == 0) return SRFTQ_OK;
@@ -169,17 +189,19 @@ int dequantize_impl(const DequantCall& c) {
   a.codes = c.codes;
   a.scales = c.scales;
   a.in_slice_stride_rows = c.in_slice_stride_rows;
+  a.xhat = c.xhat;
+  a.out_slice_stride_rows = c.out_slice_stride_rows;
   a.guard = guard;
 
-  constexpr auto K = dequantize_kernel<D, BITS, G, ROT, kWPC, kNST, kNOUT>;
-  const int smem = kWPC * Lay::kWarpBytes + kSmemSlack;
+  constexpr auto K = dequantize_kernel<D, BITS, G, ROT, kDWPC, kNST, kDMinBlocks>;
+  const int smem = kDWPC * Lay::kWarpBytes + kSmemSlack;
   int bps = 0;
-  int rc = prepare_kernel<K>(smem, kWPC * 32, &bps);
+  int rc = prepare_kernel<K>(smem, kDWPC * 32, &bps);
   if (rc != SRFTQ_OK) return rc;
-  const int64_t want = (total + kWPC - 1) / kWPC;
+  const int64_t want = (total + kDWPC - 1) / kDWPC;
   const int64_t cap = int64_t(Runtime::num_sms()) * bps;
   const int grid = int(want < cap ? want : cap);
-  K<<<grid, kWPC * 32, smem, c.stream>>>(tm_c, tm_x, a);
+  K<<<grid, kDWPC * 32, smem, c.stream>>>(tm_c, tm_x, a);
   return finish_launch();
 }
 
