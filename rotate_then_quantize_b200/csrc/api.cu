@@ -46,9 +46,12 @@ bool is_pow2(int64_t x) { return x > 0 && (x & (x - 1)) == 0; }
 int check_desc(const srftq_desc* d) {
   if (!d) return SRFTQ_ERR_INVALID_ARG;
   if (d->heads < 1) return SRFTQ_ERR_INVALID_ARG;
-  if (!(d->d == 16 || d->d == 32 || d->d == 64 || d->d == 128)) return SRFTQ_ERR_UNSUPPORTED;
+  if (!(d->d == 16 || d->d == 32 || d->d == 64 || d->d == 128 || d->d == 256))
+    return SRFTQ_ERR_UNSUPPORTED;
   if (d->bits != 4 && d->bits != 8) return SRFTQ_ERR_UNSUPPORTED;
-  if (!is_pow2(d->group) || d->group < 8 || d->group > d->d) return SRFTQ_ERR_UNSUPPORTED;
+  // a group lies inside one thread's half of the vector at d = 256
+  const int gmax = d->d < 64 ? d->d : (d->d == 256 ? 64 : d->d);
+  if (!is_pow2(d->group) || d->group < 8 || d->group > gmax) return SRFTQ_ERR_UNSUPPORTED;
   if (d->rotation != SRFTQ_ROT_SRFT && d->rotation != SRFTQ_ROT_SRHT) return SRFTQ_ERR_UNSUPPORTED;
   return SRFTQ_OK;
 }
@@ -74,6 +77,7 @@ int by_d(int d, Fn&& fn) {
     case 32: return fn(Int<32>{});
     case 64: return fn(Int<64>{});
     case 128: return fn(Int<128>{});
+    case 256: return fn(Int<256>{});
     default: return SRFTQ_ERR_UNSUPPORTED;
   }
 }

@@ -74,4 +74,10 @@ template <int D> int launch_dequantize(const DequantCall& c);
 template <int D> int launch_rotate(const RotateCall& c);
 template <int D> int launch_calibrate(const CalibCall& c);
 
+// d = 256 has its own kernels (two threads per vector; launch_d256.cu).
+template <> int launch_quantize<256>(const QuantCall& c);
+template <> int launch_dequantize<256>(const DequantCall& c);
+template <> int launch_rotate<256>(const RotateCall& c);
+template <> int launch_calibrate<256>(const CalibCall& c);
+
 }  // namespace srftq

@@ -70,10 +70,10 @@ def run_and_check(x16, signs, lam, d, group, bits, rot, what):
 
 def _configs():
     out = []
-    for d in (16, 32, 64, 128):
+    for d in (16, 32, 64, 128, 256):
         for bits in (4, 8):
             g = 8
-            while g <= d:
+            while g <= min(d, 64 if d == 256 else d):
                 for rot in (rq.SRFT, rq.SRHT):
                     out.append((d, bits, g, rot))
                 g *= 2
@@ -104,12 +104,36 @@ def test_ragged_rows_and_heads(N, H):
     run_and_check(x16, signs, lam, d, group, bits, rq.SRFT, f"N{N} H{H}")
 
 
+@pytest.mark.parametrize("N", [1, 15, 16, 17, 47])
+@pytest.mark.parametrize("rot", [0, 1])
+def test_ragged_rows_d256(N, rot):
+    """d = 256 runs 16-row tiles with two threads per vector."""
+    rng = np.random.default_rng(N * 11 + rot)
+    d, group, bits, H = 256, 32, 4, 3
+    x16 = _x(rng, 2, N, H, d, outlier_p=0.005, scale=25.0)
+    signs = _signs(rng, 2, H, d)
+    lam = np.exp(rng.uniform(-1, 1, (2, H, d))).astype(np.float32)
+    run_and_check(x16, signs, lam, d, group, bits, rot, f"d256 N{N} r{rot}")
+
+
+def test_unsupported_groups_d256():
+    """Groups wider than one thread's half of a d = 256 vector are refused."""
+    x = torch.zeros((1, 4, 1, 256), dtype=torch.float16, device=DEV)
+    st = torch.ones((1, 1, 256), dtype=torch.int8, device=DEV)
+    lt = torch.ones((1, 1, 256), device=DEV)
+    for group in (128, 256):
+        with pytest.raises(rq.SrftqError) as e:
+            rq.quantize(x, st, lt, group, 4)
+        assert e.value.status == rq.binding.SRFTQ_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("d", [128, 256])
 @pytest.mark.parametrize("bits", [4, 8])
-def test_strided_views_and_guard_bands(bits):
+def test_strided_views_and_guard_bands(bits, d):
     """Slices with a row stride larger than the rows used (a cache written at a
     row offset); rows outside the written window must keep their sentinel."""
-    rng = np.random.default_rng(bits)
-    S, T, H, d, group, N, off = 3, 100, 2, 128, 16, 37, 41
+    rng = np.random.default_rng(bits + d)
+    S, T, H, group, N, off = 3, 100, 2, 16, 37, 41
     big = _x(rng, S, T, H, d)
     signs = _signs(rng, S, H, d)
     lam = np.exp(rng.uniform(-0.5, 0.5, (S, H, d))).astype(np.float32)
@@ -261,3 +285,7 @@ def test_qwen_like_workload_sampled():
 @pytest.mark.parametrize("rot", [0, 1])
 def test_longctx_int8_workload_sampled(rot):
     _workload_check("longctx_int8_d128", rot)
+
+
+def test_gemma_like_d256_workload_sampled():
+    _workload_check("gemma_like_d256", rq.SRFT)
