@@ -50,14 +50,16 @@ def parse_args(argv=None):
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="qwen_like_d128",
-                    choices=[k for k, w in kv_synth.WORKLOADS.items() if w.d <= 128 and w.S * w.N * w.H < 2**28])
+    ap.add_argument("--workload", default="qwen_like_d128", choices=list(kv_synth.WORKLOADS))
     ap.add_argument("--rotation", type=int, default=0, choices=[0, 1])
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample", type=int, default=8192,
-                    help="vectors per oracle step for the CPU baseline / reference arm")
+                    help="vectors per oracle step of the reference arm")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="CPU time the cpu_baseline leg spends (whole oracle steps on a "
+                         "65536-vector sample, repeated)")
     return ap.parse_args(argv)
 
 
@@ -176,18 +178,24 @@ def blas_threads():
         return 1
 
 
-def cpu_baseline(w, n_vectors, rot, steps=1):
+def cpu_baseline(w, rot, seconds, n_vectors=65536):
+    """The oracle, as it stands, on a 65536-vector sample of the workload,
+    repeated (whole steps) until `seconds` of wall time have passed."""
     x16, signs, nv = oracle_sample(w, n_vectors)
+    steps = 0
     t0 = time.perf_counter()
-    for _ in range(steps):
+    while True:
         oracle_step(w, x16, signs, rot)
-    dt = time.perf_counter() - t0
+        steps += 1
+        dt = time.perf_counter() - t0
+        if dt >= seconds:
+            break
     gbs = 2 * nv * w.bytes_per_vector() * steps / dt / 1e9
     return {"value": gbs, "unit": "GB/s", "cores": blas_threads(), "kind": "oracle",
             "vectors_per_s": nv * steps / dt, "seconds": dt,
-            "sample": f"{nv} vectors of slice 0 ({w.name}), calibrate+quantize+dequantize x{steps}; "
-                      f"float64 numpy, matrix products on {blas_threads()} BLAS threads, "
-                      f"elementwise steps single-threaded"}
+            "sample": f"{nv} vectors of slice 0 ({w.name}), calibrate+quantize+dequantize, "
+                      f"{steps} repetitions; float64 numpy, matrix products on "
+                      f"{blas_threads()} BLAS threads, elementwise steps single-threaded"}
 
 
 def run_reference(args):
@@ -234,10 +242,9 @@ def _config(w, args, extra=None):
 # GPU leg
 # ---------------------------------------------------------------------------
 
-def run_ours(args):
+def _setup_ranks():
+    """One process per GPU; NCCL only for the barrier and the max over ranks."""
     import torch
-
-    import rotate_then_quantize_b200 as rq
 
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -251,7 +258,24 @@ def run_ours(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=dev)
         pg = dist
+    return rank, world, local, dev, pg
 
+
+def _max_over_ranks(pg, dev, ms):
+    import torch
+
+    if pg is None:
+        return ms
+    t = torch.tensor([ms], device=dev, dtype=torch.float64)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+def run_ours(args):
+    import torch
+
+    import rotate_then_quantize_b200 as rq
+
+    rank, world, local, dev, pg = _setup_ranks()
     w = kv_synth.WORKLOADS[args.workload]
     rot = args.rotation
     rq.load_library()
@@ -297,13 +321,9 @@ def run_ours(args):
     end.record()
     barrier()
     clk = clocks.stop()
-    ms = start.elapsed_time(end)
+    ms = _max_over_ranks(pg, dev, start.elapsed_time(end))
     q_ms = [evs[k][0].elapsed_time(evs[k][1]) for k in range(K)]
     d_ms = [evs[k][1].elapsed_time(evs[k][2]) for k in range(K)]
-    if pg is not None:
-        t = torch.tensor([ms], device=dev, dtype=torch.float64)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        ms = float(t.item())
     if rq.srftq_check_device() != 0:
         raise RuntimeError("device guard fired during the timed steps")
 
@@ -315,7 +335,7 @@ def run_ours(args):
     dom = "quantize" if q_avg >= d_avg else "dequantize"
     dom_ms = max(q_avg, d_avg)
     achieved = bytes_launch / (dom_ms / 1e3) / 1e9
-    kname = "quantize_kernel" if dom == "quantize" else "dequantize_kernel"
+    kname = f"{dom}{'256' if w.d == 256 else ''}_kernel"
 
     e2e = None
     if not args.no_e2e:
@@ -336,11 +356,7 @@ def run_ours(args):
             e2e_step()
         e2.record()
         barrier()
-        ems = s2.elapsed_time(e2)
-        if pg is not None:
-            t = torch.tensor([ems], device=dev, dtype=torch.float64)
-            pg.all_reduce(t, op=pg.ReduceOp.MAX)
-            ems = float(t.item())
+        ems = _max_over_ranks(pg, dev, s2.elapsed_time(e2))
         e2e = {"value": step_bytes * args.e2e_steps * world / (ems / 1e3) / 1e9, "unit": "GB/s",
                "h2d_bytes_per_step": x.numel() * x.element_size(),
                "d2h_bytes_per_step": xhat.numel() * xhat.element_size(),
@@ -369,7 +385,198 @@ def run_ours(args):
     if e2e is not None:
         line["e2e"] = e2e
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(w, args.cpu_sample, rot)
+        line["cpu_baseline"] = cpu_baseline(w, rot, args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if pg is not None:
+        pg.barrier()
+        pg.destroy_process_group()
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# Decode-style streaming
+# ---------------------------------------------------------------------------
+
+def run_decode(args):
+    """Decode steps over an int4 cache of 32768 tokens x 32 sequences.
+
+    Cache layout per slice (layer x {K, V}): row = token * 32 + sequence, so
+    one decode step's new tokens are 32 consecutive rows. A step, per layer:
+    quantize the 32 new (K, V) tokens into the cache at the next row block,
+    then dequantize that layer's whole cache (both slices) into one fp16
+    scratch buffer of a layer's shape, as an attention kernel would consume
+    it. The comparator reads an fp16 cache of the same shape once per layer
+    (torch.sum over the scratch buffer)."""
+    import torch
+
+    import rotate_then_quantize_b200 as rq
+
+    rank, world, local, dev, pg = _setup_ranks()
+    w = kv_synth.WORKLOADS[args.workload]
+    B = 32
+    T0 = w.N // B
+    L = w.S // 2
+    rot = args.rotation
+    n_steps = args.warmup + args.steps + args.e2e_steps + 2
+    cap = (T0 + n_steps) * B
+    rq.load_library()
+    desc = rq.make_desc(w.d, w.H, w.group, w.bits, rot)
+    signs = torch.from_numpy(kv_synth.rademacher_signs(w.S, w.H, w.d, seed=1 + rank)).to(dev)
+    lam = torch.empty((w.S, w.H, w.d), dtype=torch.float32, device=dev)
+    codes = torch.empty((w.S, cap, w.H, w.d * w.bits // 8), dtype=torch.uint8, device=dev)
+    scales = torch.empty((w.S, cap, w.H, w.d // w.group), dtype=torch.float16, device=dev)
+    scratch = torch.empty((2, cap, w.H, w.d), dtype=torch.float16, device=dev)
+    # the existing cache: seeded fp16 N(0,1) per slice, calibrated and quantized
+    for s_ in range(w.S):
+        xs = kv_synth.make_x_torch(w, dev, seed=1000 * rank, n_rows=T0 * B,
+                                   slices=range(s_, s_ + 1), out=scratch[0:1, :T0 * B])
+        rq.srftq_calibrate_lambda(desc, xs, signs[s_:s_ + 1], lam[s_:s_ + 1], w.n_cal)
+        rq.srftq_quantize(desc, xs, signs[s_:s_ + 1], lam[s_:s_ + 1],
+                          codes[s_:s_ + 1, :T0 * B], scales[s_:s_ + 1, :T0 * B])
+    new_tok = kv_synth.make_x_torch(w, dev, seed=7 + 1000 * rank, n_rows=B)
+    torch.cuda.synchronize()
+    if rq.srftq_check_device() != 0:
+        raise RuntimeError("device guard fired while filling the cache")
+
+    state = {"t": 0}
+    vec_bytes = w.bytes_per_vector()
+
+    def step(ev=None):
+        r0 = (T0 + state["t"]) * B
+        n = r0 + B
+        for l in range(L):
+            sl = slice(2 * l, 2 * l + 2)
+            rq.srftq_quantize(desc, new_tok[sl], signs[sl], lam[sl], codes[sl, r0:n],
+                              scales[sl, r0:n])
+            if ev is not None:
+                ev[l][0].record()
+            rq.srftq_dequantize(desc, codes[sl, :n], scales[sl, :n], signs[sl], lam[sl],
+                                scratch[:, :n])
+            if ev is not None:
+                ev[l][1].record()
+        state["t"] += 1
+        return (w.S * B * w.H + w.S * n * w.H) * vec_bytes, w.S * n * w.H
+
+    def barrier():
+        torch.cuda.synchronize()
+        if pg is not None:
+            pg.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        step()
+    barrier()
+    K = args.steps
+    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(L)]
+           for _ in range(K)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    clocks.start()
+    barrier()
+    start.record()
+    tot_bytes = tot_vec = 0
+    for k in range(K):
+        b_, v_ = step(evs[k])
+        tot_bytes += b_
+        tot_vec += v_
+    end.record()
+    barrier()
+    clk = clocks.stop()
+    ms = _max_over_ranks(pg, dev, start.elapsed_time(end))
+    if rq.srftq_check_device() != 0:
+        raise RuntimeError("device guard fired during the timed steps")
+    d_ms = [evs[k][l][0].elapsed_time(evs[k][l][1]) for k in range(K) for l in range(L)]
+    n_last = (T0 + state["t"]) * B
+    deq_bytes = 2 * n_last * w.H * vec_bytes
+    d_avg = statistics.mean(d_ms)
+
+    # comparator: the same decode steps reading a contiguous fp16 cache of one
+    # layer's (K, V) shape instead, once per layer
+    fp16_layer = scratch[:, :n_last].contiguous()
+    fp16_bytes = 0
+    acc = torch.zeros((), dtype=torch.float32, device=dev)
+    for _ in range(2):
+        for l in range(L):
+            acc += torch.sum(fp16_layer, dtype=torch.float32)
+    barrier()
+    s3, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s3.record()
+    for k in range(K):
+        for l in range(L):
+            acc += torch.sum(fp16_layer, dtype=torch.float32)
+            fp16_bytes += fp16_layer.numel() * 2
+    e3.record()
+    barrier()
+    fp16_ms = _max_over_ranks(pg, dev, s3.elapsed_time(e3))
+    del fp16_layer
+
+    e2e = None
+    if not args.no_e2e:
+        tok_host = torch.empty(new_tok.shape, dtype=new_tok.dtype, pin_memory=True)
+        tok_host.copy_(new_tok)
+        out_host = torch.empty((2, B, w.H, w.d), dtype=torch.float16, pin_memory=True)
+
+        def e2e_step():
+            new_tok.copy_(tok_host, non_blocking=True)
+            r0 = (T0 + state["t"]) * B
+            step()
+            # the step's result: the last layer's appended tokens, dequantized
+            out_host.copy_(scratch[:, r0:r0 + B], non_blocking=True)
+
+        barrier()
+        s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s2.record()
+        e_bytes = 0
+        for _ in range(args.e2e_steps):
+            n = (T0 + state["t"] + 1) * B
+            e_bytes += (w.S * B * w.H + w.S * n * w.H) * vec_bytes
+            e2e_step()
+        e2.record()
+        barrier()
+        ems = _max_over_ranks(pg, dev, s2.elapsed_time(e2))
+        e2e = {"value": e_bytes * world / (ems / 1e3) / 1e9, "unit": "GB/s",
+               "h2d_bytes_per_step": new_tok.numel() * new_tok.element_size(),
+               "d2h_bytes_per_step": 2 * B * w.H * w.d * 2,
+               "ms_per_step": ems / args.e2e_steps, "steps": args.e2e_steps,
+               "path": "new tokens pinned host -> device, the step's quantize+dequantize "
+                       "launches, the appended tokens' dequantized rows device -> host"}
+
+    peak, peak_src = read_peak()
+    achieved = deq_bytes / (d_avg / 1e3) / 1e9
+    line = {
+        "metric": METRIC, "value": tot_bytes * world / (ms / 1e3) / 1e9, "unit": "GB/s",
+        "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": ms / K,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic",
+        "config": _config(w, args, extra={
+            "sequences": B, "cached_tokens": T0, "layers": L,
+            "step": "per layer: quantize 32 new K and V tokens into the cache, then "
+                    "dequantize the layer's whole K and V cache into an fp16 scratch"}),
+        "vectors_per_s": tot_vec * world / (ms / 1e3),
+        "fp16_read": {"GBps": fp16_bytes / (fp16_ms / 1e3) / 1e9,
+                      "ms_per_step": fp16_ms / K,
+                      "bytes_per_step": fp16_bytes // K,
+                      "how": "torch.sum over an fp16 buffer of one layer's K and V cache "
+                             "shape, once per layer"},
+        "int4_step_over_fp16_read_time": (ms / K) / (fp16_ms / K),
+        "int4_step_over_fp16_read_at_peak": (ms / K) / (fp16_bytes / K / (read_peak()[0] * 1e6)),
+        "kernels": {"dequantize_ms_per_layer": d_avg,
+                    "dequantize_GBps": achieved,
+                    "launches_per_step": 2 * L},
+        "roofline": {"bound": "hbm", "kernel": "dequantize_kernel", "achieved": achieved,
+                     "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)"
+                     if peak_src == "measured" else "fallback 6.65 TB/s",
+                     "algorithmic_bytes_per_launch": deq_bytes,
+                     "traffic": read_traffic("dequantize_kernel", w.name)},
+        "gpu_launches": 2 * L * K,
+        "clocks": clk,
+    }
+    if e2e is not None:
+        line["e2e"] = e2e
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, rot, args.cpu_seconds)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if pg is not None:
@@ -382,6 +589,8 @@ def main(argv=None):
     args = parse_args(argv)
     if args.impl == "reference":
         return run_reference(args)
+    if args.workload == "decode_stream_d128":
+        return run_decode(args)
     return run_ours(args)
 
 

@@ -14,7 +14,8 @@ Tolerances (fixed before any kernel ran):
   edge qmax + 1/2); such codes must differ by exactly one step and are
   counted.
 * dequantised output: |xhat_gpu - xhat_ref| <= 1e-3 * max(1, |xhat_ref|),
-  with xhat_ref computed by the oracle from the GPU's own codes and scales;
+  both sides dequantising the oracle's codes and scales (or, for a GPU
+  round trip, the vectors whose GPU codes and scales equal the oracle's);
   values beyond the binary16 range round to the same infinity on both sides
   and count as equal.
 * lambda (calibration): relative 1e-5.

@@ -62,10 +62,24 @@ def run_and_check(x16, signs, lam, d, group, bits, rot, what):
     stats = parity.check_codes(ref, c_np, s_np, bits, group)
     parity.assert_clean(stats, f"{what} codes")
 
-    xhat = rq.dequantize(codes, scales, st, lt, d, group, bits, rot)
-    deq = oracle.dequantize(c_np, s_np, signs, lam, d, group, bits, rot)
+    # the dequantiser runs on the oracle's codes, so both sides see the same input
+    deq = oracle.dequantize(ref["codes"], ref["scales"], signs, lam, d, group, bits, rot)
+    xhat = rq.dequantize(_t(ref["codes"]), _t(ref["scales"].view(np.float16)), st, lt, d, group,
+                         bits, rot)
     parity.assert_clean(parity.check_dequant(_np16(xhat), deq["bits"]), f"{what} dequant")
+    # and the GPU round trip, where its codes equal the oracle's
+    xhat_rt = rq.dequantize(codes, scales, st, lt, d, group, bits, rot)
+    check_dequant_where_codes_match(_np16(xhat_rt), c_np, s_np, ref, deq, f"{what} round trip")
     return stats
+
+
+def check_dequant_where_codes_match(xh_bits, c_np, s_np, ref, deq, what):
+    """Dequantised vectors of the GPU's own codes against the oracle's
+    dequantisation of the oracle's codes, on the vectors whose codes and
+    scales are identical (all but the flagged rounding-boundary cases)."""
+    same = np.all(c_np == ref["codes"], axis=-1) & np.all(s_np == ref["scales"], axis=-1)
+    parity.assert_clean(parity.check_dequant(xh_bits[same], deq["bits"][same]), what)
+    return int((~same).sum())
 
 
 def _configs():
@@ -152,11 +166,14 @@ def test_strided_views_and_guard_bands(bits, d):
     outside[off:off + N] = False
     assert np.all(c_np[:, outside] == 0xAB)
     assert np.all(s_np[:, outside] == np.float16(7.0).view(np.uint16))
-    # dequantise into a strided view, sentinel around it
+    # dequantise the oracle's codes, placed in the strided window, into a
+    # strided view with a sentinel around it
+    codes_big[:, off:off + N] = _t(ref["codes"])
+    scales_big[:, off:off + N] = _t(ref["scales"].view(np.float16))
     xh_big = torch.full((S, T, H, d), -3.0, dtype=torch.float16, device=DEV)
     rq.srftq_dequantize(desc, codes_big[:, off:off + N], scales_big[:, off:off + N], st, lt,
                         xh_big[:, off:off + N])
-    deq = oracle.dequantize(c_np[:, off:off + N], s_np[:, off:off + N], signs, lam, d, group, bits)
+    deq = oracle.dequantize(ref["codes"], ref["scales"], signs, lam, d, group, bits)
     xh = _np16(xh_big)
     parity.assert_clean(parity.check_dequant(xh[:, off:off + N], deq["bits"]), "strided dequant")
     assert np.all(xh[:, outside] == np.float16(-3.0).view(np.uint16))
@@ -253,9 +270,16 @@ def _workload_check(name, rot, k_rows=48):
         s_np = _np16(scales[s:s + 1, rows])
         stats = parity.check_codes(ref, c_np, s_np, w.bits, w.group)
         parity.assert_clean(stats, f"{name} slice {s} codes")
-        deq = oracle.dequantize(c_np, s_np, signs[s:s + 1], lam[s:s + 1], w.d, w.group, w.bits, rot)
-        parity.assert_clean(parity.check_dequant(_np16(xhat[s:s + 1, rows]), deq["bits"]),
-                            f"{name} slice {s} dequant")
+        deq = oracle.dequantize(ref["codes"], ref["scales"], signs[s:s + 1], lam[s:s + 1], w.d,
+                                w.group, w.bits, rot)
+        # the full-size launch's output where its codes equal the oracle's ...
+        check_dequant_where_codes_match(_np16(xhat[s:s + 1, rows]), c_np, s_np, ref, deq,
+                                        f"{name} slice {s} dequant")
+        # ... and the dequantiser on the oracle's own codes for the sampled rows
+        xh_ref_in = rq.dequantize(_t(ref["codes"]), _t(ref["scales"].view(np.float16)),
+                                  st[s:s + 1], lt[s:s + 1], w.d, w.group, w.bits, rot)
+        parity.assert_clean(parity.check_dequant(_np16(xh_ref_in), deq["bits"]),
+                            f"{name} slice {s} dequant of the oracle's codes")
         for key, v in stats.items():
             totals[key] = totals.get(key, 0) + v
 
@@ -289,3 +313,43 @@ def test_longctx_int8_workload_sampled(rot):
 
 def test_gemma_like_d256_workload_sampled():
     _workload_check("gemma_like_d256", rq.SRFT)
+
+
+@pytest.mark.parametrize("rot", [0, 1])
+def test_decode_streaming_appends(rot):
+    """Decode-style use: a cache with spare capacity is filled, then each step
+    appends one token for every sequence (rows token * B + sequence) and the
+    whole cache is dequantized. Appended codes must equal a one-shot
+    quantization of all tokens; untouched capacity keeps its sentinel."""
+    rng = np.random.default_rng(31 + rot)
+    S, B, T0, steps, H, d, group, bits = 4, 4, 20, 3, 2, 128, 16, 4
+    cap = (T0 + steps + 2) * B
+    x_all = _x(rng, S, (T0 + steps) * B, H, d, outlier_p=0.0)
+    signs = _signs(rng, S, H, d)
+    st = _t(signs)
+    lam_np = oracle.calibrate_lambda(x_all[:, :T0 * B], signs, 16, rot).astype(np.float32)
+    lam = _t(lam_np)
+    codes = torch.full((S, cap, H, d * bits // 8), 0x5A, dtype=torch.uint8, device=DEV)
+    scales = torch.full((S, cap, H, d // group), 9.0, dtype=torch.float16, device=DEV)
+    xhat = torch.full((S, cap, H, d), 5.0, dtype=torch.float16, device=DEV)
+    desc = rq.make_desc(d, H, group, bits, rot)
+    rq.srftq_quantize(desc, _t(x_all[:, :T0 * B]), st, lam, codes[:, :T0 * B], scales[:, :T0 * B])
+    for t in range(steps):
+        r0 = (T0 + t) * B
+        for layer in range(S // 2):
+            sl = slice(2 * layer, 2 * layer + 2)
+            rq.srftq_quantize(desc, _t(x_all[sl, r0:r0 + B]), st[sl], lam[sl], codes[sl, r0:r0 + B],
+                              scales[sl, r0:r0 + B])
+            rq.srftq_dequantize(desc, codes[sl, :r0 + B], scales[sl, :r0 + B], st[sl], lam[sl],
+                                xhat[sl, :r0 + B])
+    n = (T0 + steps) * B
+    ref = oracle.quantize(x_all, signs, lam_np, group, bits, rot)
+    c_np, s_np = codes.cpu().numpy(), _np16(scales)
+    parity.assert_clean(parity.check_codes(ref, c_np[:, :n], s_np[:, :n], bits, group), "append codes")
+    deq = oracle.dequantize(ref["codes"], ref["scales"], signs, lam_np, d, group, bits, rot)
+    xh = _np16(xhat)
+    check_dequant_where_codes_match(xh[:, :n], c_np[:, :n], s_np[:, :n], ref, deq,
+                                    "streamed dequant")
+    assert np.all(c_np[:, n:] == 0x5A)
+    assert np.all(s_np[:, n:] == np.float16(9.0).view(np.uint16))
+    assert np.all(xh[:, n:] == np.float16(5.0).view(np.uint16))
