@@ -37,9 +37,10 @@ constexpr int kTileRows = 32;
 
 struct TileGeom {
   int32_t heads;       // H
-  int32_t row_blocks;  // ceil(N / 32)
+  int32_t row_blocks;  // ceil(N / rows per tile)
   int32_t n_rows;      // N
   int32_t total_tiles; // S * row_blocks * H
+  int32_t n_slices;    // S
 };
 
 struct TileCoord {
@@ -51,6 +52,38 @@ __device__ __forceinline__ TileCoord decode_tile(int t, const TileGeom& g) {
   const int q = t / g.heads;
   const int rb = q % g.row_blocks;
   return {q / g.row_blocks, rb * kTileRows, h};
+}
+
+// Position of a warp's tile t = (s * row_blocks + rb) * H + h as digits. A
+// warp walks t, t + W, t + 2W, ... by adding the digits of the stride W with
+// carries, so no division is left in the loop.
+struct TileWalk {
+  int s, rb, h;
+
+  __device__ __forceinline__ void set(int t, const TileGeom& g) {
+    h = t % g.heads;
+    const int q = t / g.heads;
+    rb = q % g.row_blocks;
+    s = q / g.row_blocks;
+  }
+  __device__ __forceinline__ void advance(const TileWalk& step, const TileGeom& g) {
+    int hh = h + step.h;
+    int c = hh >= g.heads;
+    h = c ? hh - g.heads : hh;
+    int r = rb + step.rb + c;
+    c = r >= g.row_blocks;
+    rb = c ? r - g.row_blocks : r;
+    s += step.s + c;
+  }
+  __device__ __forceinline__ bool valid(const TileGeom& g) const { return s < g.n_slices; }
+};
+
+// The 1024-byte aligned start of dynamic shared memory, kept as a pointer
+// into the shared window so that every access derived from it compiles to
+// 32-bit shared loads and stores.
+__device__ __forceinline__ uint8_t* smem_base_1024(uint8_t* raw) {
+  const uint32_t a = static_cast<uint32_t>(__cvta_generic_to_shared(raw));
+  return raw + ((0u - a) & 1023u);
 }
 
 struct QuantArgs {
@@ -198,6 +231,87 @@ constexpr float kMagic = 12582912.0f;
 // Quantiser
 // ---------------------------------------------------------------------------
 
+// Three-input max / min (one instruction each on sm_100).
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+__device__ __forceinline__ float min3f(float a, float b, float c) {
+  float r;
+  asm("min.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// Largest and smallest of the n group absmaxes.
+template <int N>
+__device__ __forceinline__ void range_of(const float (&a)[N], float& hi, float& lo) {
+  if constexpr (N == 1) {
+    hi = lo = a[0];
+  } else {
+    hi = fmaxf(a[0], a[1]);
+    lo = fminf(a[0], a[1]);
+    static_for<2, N>([&](auto i_) {
+      constexpr int i = decltype(i_)::value;
+      if constexpr (i % 2 == 0 && i + 1 < N) {
+        hi = max3f(hi, a[i], a[i + 1]);
+        lo = min3f(lo, a[i], a[i + 1]);
+      } else if constexpr (i % 2 == 0) {
+        hi = fmaxf(hi, a[i]);
+        lo = fminf(lo, a[i]);
+      }
+    });
+  }
+}
+
+// Packed form of div_by_const: two correctly rounded quotients a / Q.
+template <int Q>
+__device__ __forceinline__ float2 div_by_const2(float2 a) {
+  constexpr float inv = float(1.0 / double(Q));
+  const float2 q0 = mul2(a, splat(inv));
+  const float2 r = fma2(q0, splat(-float(Q)), a);
+  return fma2(r, splat(inv), q0);
+}
+
+__device__ __forceinline__ float2 unpack_f16x2(uint32_t h) {
+  return __half22float2(*reinterpret_cast<const __half2*>(&h));
+}
+
+// Scales and reciprocals of all groups of one vector from the group absmax
+// a_g: sigma_g = fp16_rn(a_g / QMAX), written as packed fp16 words (low half
+// = even group), inv_g = 1 / sigma_g. FAST: every sigma_g is a normal fp16
+// and a_g / QMAX does not exceed 65504 (checked by the caller); otherwise
+// saturation at 65504, sigma = 0 (inv = 0, all codes 0) and subnormal scales
+// are handled, and CLAMP reports that the codes need clamping.
+template <int NG, int QMAX, bool FAST>
+__device__ __forceinline__ void group_scales(const float (&am)[NG], uint32_t (&sw)[(NG + 1) / 2],
+                                             float (&inv)[NG]) {
+  if constexpr (NG == 1) {
+    float sf = div_by_const<QMAX>(am[0]);
+    if constexpr (!FAST) sf = fminf(sf, 65504.0f);
+    const __half hs = __float2half_rn(sf);
+    sw[0] = __half_as_ushort(hs);
+    const float sg = __half2float(hs);
+    inv[0] = FAST ? rcp_approx(sg) : (sg > 0.0f ? rcp_approx(sg) : 0.0f);
+  } else {
+    static_for<0, NG / 2>([&](auto k_) {
+      constexpr int k = decltype(k_)::value;
+      float2 sf = div_by_const2<QMAX>(make_float2(am[2 * k], am[2 * k + 1]));
+      if constexpr (!FAST) sf = make_float2(fminf(sf.x, 65504.0f), fminf(sf.y, 65504.0f));
+      const uint32_t h2 = pack_f16x2(sf.x, sf.y);
+      sw[k] = h2;
+      const float2 sg = unpack_f16x2(h2);
+      if constexpr (FAST) {
+        inv[2 * k] = rcp_approx(sg.x);
+        inv[2 * k + 1] = rcp_approx(sg.y);
+      } else {
+        inv[2 * k] = sg.x > 0.0f ? rcp_approx(sg.x) : 0.0f;
+        inv[2 * k + 1] = sg.y > 0.0f ? rcp_approx(sg.y) : 0.0f;
+      }
+    });
+  }
+}
+
 template <int D, int BITS, int G, int ROT, int WPC, int NST, int MINB>
 __global__ void __launch_bounds__(WPC * 32, MINB)
     quantize_kernel(const __grid_constant__ CUtensorMap tm_x,
@@ -205,7 +319,7 @@ __global__ void __launch_bounds__(WPC * 32, MINB)
   using S = Shape<D, BITS, G>;
   using Lay = WarpLayout<D, BITS, G, NST, true>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t* smem = align_smem_1024(smem_raw);
+  uint8_t* smem = smem_base_1024(smem_raw);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   uint8_t* ws = smem + warp * Lay::kWarpBytes;
@@ -214,10 +328,12 @@ __global__ void __launch_bounds__(WPC * 32, MINB)
   uint32_t* stab = reinterpret_cast<uint32_t*>(ws + Lay::kSignTabOff);
   uint8_t* ob = ws + Lay::kOutOff;   // codes staging tile
 
-  const int total = a.g.total_tiles;
   const int nw = gridDim.x * WPC;
   const int first = blockIdx.x * WPC + warp;
-  if (first >= total) return;
+  if (first >= a.g.total_tiles) return;
+  TileWalk cur, step;
+  cur.set(first, a.g);
+  step.set(nw, a.g);
 
   if (lane == 0) {
     prefetch_tensormap(&tm_x);
@@ -227,41 +343,47 @@ __global__ void __launch_bounds__(WPC * 32, MINB)
   }
   __syncwarp();
 
-  auto issue = [&](int t, int st) {
-    const TileCoord c = decode_tile(t, a.g);
+  auto issue = [&](const TileWalk& c, int st) {
     uint8_t* sb = ws + st * Lay::kInBytes;
     uint8_t* rb = ws + Lay::kRowsOff + st * Lay::kRowBytes;
     mbar_arrive_expect_tx(&bars[st], Lay::kStageTx);
 #pragma unroll
     for (int p = 0; p < S::X_PIECES; ++p)
-      tma_load_4d(sb + p * (S::TR * S::X_SPAN), &tm_x, &bars[st], p * (S::X_SPAN / 2), c.h, c.r0,
-                  c.s);
+      tma_load_4d(sb + p * (S::TR * S::X_SPAN), &tm_x, &bars[st], p * (S::X_SPAN / 2), c.h,
+                  c.rb * kTileRows, c.s);
     const size_t row = static_cast<size_t>(c.s) * a.g.heads + c.h;
     bulk_load(rb, a.lambda + row * D, 4 * D, &bars[st]);
     bulk_load(rb + 4 * D, a.signs + row * D, D, &bars[st]);
   };
-  auto store_codes = [&](const TileCoord& c) {
+  auto store_codes = [&](const TileWalk& c) {
 #pragma unroll
     for (int p = 0; p < S::C_PIECES; ++p)
-      tma_store_4d(&tm_codes, ob + p * (S::TR * S::C_SPAN), p * S::C_SPAN, c.h, c.r0, c.s);
+      tma_store_4d(&tm_codes, ob + p * (S::TR * S::C_SPAN), p * S::C_SPAN, c.h,
+                   c.rb * kTileRows, c.s);
     bulk_commit();
   };
 
+  // Lane 0 issues the first NST tiles; `ahead` is then the next tile to
+  // issue and `issued` counts the tiles issued so far.
+  TileWalk ahead = cur;
+  int issued = 0;
   if (lane == 0) {
     for (int k = 0; k < NST; ++k) {
-      const int t = first + k * nw;
-      if (t < total) issue(t, k);
+      if (ahead.valid(a.g)) {
+        issue(ahead, k);
+        ++issued;
+      }
+      ahead.advance(step, a.g);
     }
   }
 
   int it = 0;
   int table_sh = -1;          // (slice, head) the tables were built for
   bool pending = false;       // a staged codes tile awaits its TMA store
-  TileCoord prev{0, 0, 0};
-  for (int t = first; t < total; t += nw, ++it) {
+  TileWalk prev = cur;
+  for (; cur.valid(a.g); ++it) {
     const int st = it % NST;
     const uint32_t parity = (it / NST) & 1;
-    const TileCoord c = decode_tile(t, a.g);
     const uint8_t* sb = ws + st * Lay::kInBytes;
     const uint8_t* rb = ws + Lay::kRowsOff + st * Lay::kRowBytes;
 
@@ -269,11 +391,9 @@ __global__ void __launch_bounds__(WPC * 32, MINB)
     if (!ok) {
       if (lane == 0) {
         atomicOr(a.guard, kGuardWaitTimeout);
-        // give the other stages' copies (again boundedly) a chance to land
-        for (int k = 1; k < NST; ++k) {
-          const int tk = t + k * nw;
-          if (tk < total) (void)mbar_wait_bounded(&bars[(it + k) % NST], ((it + k) / NST) & 1);
-        }
+        // give the other issued stages' copies (again boundedly) a chance to land
+        for (int k = it + 1; k < issued; ++k)
+          (void)mbar_wait_bounded(&bars[k % NST], (k / NST) & 1);
         bulk_wait<0>();
       }
       __syncwarp();
@@ -284,14 +404,19 @@ __global__ void __launch_bounds__(WPC * 32, MINB)
     __syncwarp();
     if (lane == 0) {
       if (pending) store_codes(prev);
-      const int tn = t + (NST - 1) * nw;
-      if (it > 0 && tn < total) issue(tn, (it - 1) % NST);
+      if (it > 0) {
+        if (ahead.valid(a.g)) {
+          issue(ahead, (it - 1) % NST);
+          ++issued;
+        }
+        ahead.advance(step, a.g);
+      }
     }
     pending = false;
 
     // (a) per-(slice, head) tables: multiplier gain_j / lambda_j, fp16 signs
     // (rebuilt only when the tile's (slice, head) differs from the last one)
-    const int sh = c.s * a.g.heads + c.h;
+    const int sh = cur.s * a.g.heads + cur.h;
     if (sh != table_sh) {
       const float* lam_raw = reinterpret_cast<const float*>(rb);
       const int8_t* sgn_raw = reinterpret_cast<const int8_t*>(rb + 4 * D);
@@ -303,12 +428,12 @@ __global__ void __launch_bounds__(WPC * 32, MINB)
 
     // (b) this lane's vector (swizzled 16-byte chunks) and the sign words
     uint32_t xw[D / 2], sgw[D / 2];
+    const uint32_t row_off = lane * S::X_SPAN;
     static_for<0, D / 8>([&](auto c_) {
       constexpr int ci = decltype(c_)::value;
       constexpr int piece = (ci * 16) / S::X_SPAN;
       constexpr int cc = ((ci * 16) % S::X_SPAN) / 16;
-      const uint32_t off =
-          piece * (S::TR * S::X_SPAN) + swizzle<S::X_SPAN>(lane * S::X_SPAN + cc * 16);
+      const uint32_t off = piece * (S::TR * S::X_SPAN) + swizzle<S::X_SPAN>(row_off + cc * 16);
       const uint4 raw = *reinterpret_cast<const uint4*>(sb + off);
       const uint4 sg = *reinterpret_cast<const uint4*>(stab + 4 * ci);
       xw[4 * ci + 0] = raw.x;
@@ -332,43 +457,40 @@ __global__ void __launch_bounds__(WPC * 32, MINB)
     });
 
     // (d) group absmax -> fp16 scale -> codes as float-encoded integers.
-    // With a normal, unsaturated scale |w/sigma| <= qmax * (1 + 2^-10) up to
-    // rounding, which rounds inside the range, so unless some group's scale
-    // is subnormal or saturated the whole vector is rounded without a clamp
-    // (sigma == 0 gives inv = 0 and code 0 either way). Both branches are
-    // straight-line code over all groups.
-    uint16_t sig[S::NG];
-    float invs[S::NG];
-    bool clamp = false;
+    // When every group's scale is a normal fp16 and no a_g / qmax exceeds
+    // 65504, |w / sigma| <= qmax * (1 + 2^-10) up to rounding, which rounds
+    // inside the range: that common case (decided once per vector from the
+    // largest and smallest absmax) runs without clamps; a vector with a zero,
+    // subnormal-scale or saturating group takes the clamped block.
+    float am[S::NG];
     static_for<0, S::NG>([&](auto g_) {
       constexpr int g = decltype(g_)::value;
       constexpr int P0 = g * G / 2;   // first pair of the group
-      float amax = 0.0f;
-      static_for<0, G / 2>([&](auto p_) {
+      float m = absmax3(0.0f, v[P0].x, v[P0].y);
+      static_for<1, G / 2>([&](auto p_) {
         constexpr int p = P0 + decltype(p_)::value;
-        amax = absmax3(amax, v[p].x, v[p].y);
+        m = absmax3(m, v[p].x, v[p].y);
       });
-      const float sf = div_by_const<S::QMAX>(amax);
-      const __half hs = __float2half_rn(fminf(sf, 65504.0f));
-      sig[g] = __half_as_ushort(hs);
-      const float sg = __half2float(hs);
-      invs[g] = sg > 0.0f ? rcp_approx(sg) : 0.0f;
-      clamp |= sg > 0.0f && !(sg >= 6.103515625e-05f && sf <= 65504.0f);
+      am[g] = m;
     });
+    float a_hi, a_lo;
+    range_of(am, a_hi, a_lo);
+    constexpr float kHi = 65504.0f * float(S::QMAX);            // no saturation
+    constexpr float kLo = 6.103515625e-05f * float(S::QMAX);    // sigma >= 2^-14
+    uint32_t sw[(S::NG + 1) / 2];
     uint32_t qb[D];
-    if (!clamp) {
+    if (a_hi <= kHi && a_lo >= kLo) {
+      float invs[S::NG];
+      group_scales<S::NG, S::QMAX, true>(am, sw, invs);
       static_for<0, D / 2>([&](auto p_) {
         constexpr int p = decltype(p_)::value;
-#if SRFTQ_PACKED_ROUND
         const float2 r = fma2(v[p], splat(invs[(2 * p) / G]), splat(kMagic));
         qb[2 * p] = __float_as_uint(r.x);
         qb[2 * p + 1] = __float_as_uint(r.y);
-#else
-        qb[2 * p] = __float_as_uint(fmaf(v[p].x, invs[(2 * p) / G], kMagic));
-        qb[2 * p + 1] = __float_as_uint(fmaf(v[p].y, invs[(2 * p) / G], kMagic));
-#endif
       });
     } else {
+      float invs[S::NG];
+      group_scales<S::NG, S::QMAX, false>(am, sw, invs);
       static_for<0, D / 2>([&](auto p_) {
         constexpr int p = decltype(p_)::value;
         const float inv = invs[(2 * p) / G];
@@ -400,9 +522,10 @@ __global__ void __launch_bounds__(WPC * 32, MINB)
       });
     }
 
-    const int row = c.r0 + lane;
+    const int row = cur.rb * kTileRows + lane;
     const bool valid = row < a.g.n_rows;
-    const size_t vec = (static_cast<size_t>(c.s) * a.out_slice_stride_rows + row) * a.g.heads + c.h;
+    const size_t vec =
+        (static_cast<size_t>(cur.s) * a.out_slice_stride_rows + row) * a.g.heads + cur.h;
 
     // (f) codes: swizzled staging tile, stored by TMA at the next convergence
     // (rows past N are clipped by TMA). The store issued at this tile's start
@@ -410,47 +533,41 @@ __global__ void __launch_bounds__(WPC * 32, MINB)
     if constexpr (S::CODES_TMA) {
       if (lane == 0) bulk_wait_read<0>();
       __syncwarp();
+      const uint32_t crow = lane * S::C_SPAN;
       static_for<0, S::CB / 16>([&](auto c_) {
         constexpr int ci = decltype(c_)::value;
         constexpr int piece = (ci * 16) / S::C_SPAN;
         constexpr int cc = ((ci * 16) % S::C_SPAN) / 16;
-        const uint32_t off =
-            piece * (S::TR * S::C_SPAN) + swizzle<S::C_SPAN>(lane * S::C_SPAN + cc * 16);
+        const uint32_t off = piece * (S::TR * S::C_SPAN) + swizzle<S::C_SPAN>(crow + cc * 16);
         *reinterpret_cast<uint4*>(ob + off) =
             make_uint4(words[4 * ci], words[4 * ci + 1], words[4 * ci + 2], words[4 * ci + 3]);
       });
       fence_proxy_async_smem();
       pending = true;
-      prev = c;
+      prev = cur;
     } else {
       static_assert(S::CODES_TMA || S::CB == 8, "direct code path covers d=16 int4 only");
       if (valid) *reinterpret_cast<uint2*>(a.codes + vec * S::CB) = make_uint2(words[0], words[1]);
     }
 
-    // (g) scales straight from registers
+    // (g) scales straight from registers (packed fp16 words)
     if (valid) {
       uint16_t* dst = a.scales + vec * S::NG;
       if constexpr (S::NG == 1) {
-        dst[0] = sig[0];
+        dst[0] = static_cast<uint16_t>(sw[0]);
+      } else if constexpr (S::NG == 2) {
+        *reinterpret_cast<uint32_t*>(dst) = sw[0];
+      } else if constexpr (S::NG == 4) {
+        *reinterpret_cast<uint2*>(dst) = make_uint2(sw[0], sw[1]);
       } else {
-        uint32_t sw[S::NG / 2];
-        static_for<0, S::NG / 2>([&](auto k_) {
+        static_for<0, S::NG / 8>([&](auto k_) {
           constexpr int k = decltype(k_)::value;
-          sw[k] = uint32_t(sig[2 * k]) | (uint32_t(sig[2 * k + 1]) << 16);
+          reinterpret_cast<uint4*>(dst)[k] =
+              make_uint4(sw[4 * k], sw[4 * k + 1], sw[4 * k + 2], sw[4 * k + 3]);
         });
-        if constexpr (S::NG == 2) {
-          *reinterpret_cast<uint32_t*>(dst) = sw[0];
-        } else if constexpr (S::NG == 4) {
-          *reinterpret_cast<uint2*>(dst) = make_uint2(sw[0], sw[1]);
-        } else {
-          static_for<0, S::NG / 8>([&](auto k_) {
-            constexpr int k = decltype(k_)::value;
-            reinterpret_cast<uint4*>(dst)[k] =
-                make_uint4(sw[4 * k], sw[4 * k + 1], sw[4 * k + 2], sw[4 * k + 3]);
-          });
-        }
       }
     }
+    cur.advance(step, a.g);
   }
   __syncwarp();
   if (lane == 0) {
@@ -495,7 +612,7 @@ __global__ void __launch_bounds__(WPC * 32, MINB)
   using S = Shape<D, BITS, G>;
   using Lay = WarpLayout<D, BITS, G, NST, false>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t* smem = align_smem_1024(smem_raw);
+  uint8_t* smem = smem_base_1024(smem_raw);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   uint8_t* ws = smem + warp * Lay::kWarpBytes;
@@ -504,10 +621,12 @@ __global__ void __launch_bounds__(WPC * 32, MINB)
   uint32_t* mtab = reinterpret_cast<uint32_t*>(ws + Lay::kSignTabOff);
   uint8_t* ob = ws + Lay::kOutOff;   // fp16 staging tile
 
-  const int total = a.g.total_tiles;
   const int nw = gridDim.x * WPC;
   const int first = blockIdx.x * WPC + warp;
-  if (first >= total) return;
+  if (first >= a.g.total_tiles) return;
+  TileWalk cur, step;
+  cur.set(first, a.g);
+  step.set(nw, a.g);
 
   if (lane == 0) {
     if constexpr (S::CODES_TMA) prefetch_tensormap(&tm_codes);
@@ -517,39 +636,43 @@ __global__ void __launch_bounds__(WPC * 32, MINB)
   }
   __syncwarp();
 
-  auto issue = [&](int t, int st) {
-    const TileCoord c = decode_tile(t, a.g);
+  auto issue = [&](const TileWalk& c, int st) {
     uint8_t* sb = ws + st * Lay::kInBytes;
     uint8_t* rb = ws + Lay::kRowsOff + st * Lay::kRowBytes;
     mbar_arrive_expect_tx(&bars[st], Lay::kStageTx);
     if constexpr (S::CODES_TMA) {
 #pragma unroll
       for (int p = 0; p < S::C_PIECES; ++p)
-        tma_load_4d(sb + p * (S::TR * S::C_SPAN), &tm_codes, &bars[st], p * S::C_SPAN, c.h, c.r0,
-                    c.s);
+        tma_load_4d(sb + p * (S::TR * S::C_SPAN), &tm_codes, &bars[st], p * S::C_SPAN, c.h,
+                    c.rb * kTileRows, c.s);
     }
     const size_t row = static_cast<size_t>(c.s) * a.g.heads + c.h;
     bulk_load(rb, a.lambda + row * D, 4 * D, &bars[st]);
     bulk_load(rb + 4 * D, a.signs + row * D, D, &bars[st]);
   };
-  auto store_xhat = [&](const TileCoord& c) {
+  auto store_xhat = [&](const TileWalk& c) {
 #pragma unroll
     for (int p = 0; p < S::X_PIECES; ++p)
-      tma_store_4d(&tm_xhat, ob + p * (S::TR * S::X_SPAN), p * (S::X_SPAN / 2), c.h, c.r0, c.s);
+      tma_store_4d(&tm_xhat, ob + p * (S::TR * S::X_SPAN), p * (S::X_SPAN / 2), c.h,
+                   c.rb * kTileRows, c.s);
     bulk_commit();
   };
 
+  TileWalk ahead = cur;
+  int issued = 0;
   if (lane == 0) {
     for (int k = 0; k < NST; ++k) {
-      const int t = first + k * nw;
-      if (t < total) issue(t, k);
+      if (ahead.valid(a.g)) {
+        issue(ahead, k);
+        ++issued;
+      }
+      ahead.advance(step, a.g);
     }
   }
 
   // the next tile's scales are loaded one tile ahead, into registers
-  auto load_scales = [&](int t, uint32_t (&sw)[S::SW]) {
-    const TileCoord c = decode_tile(t, a.g);
-    const int row = c.r0 + lane;
+  auto load_scales = [&](const TileWalk& c, uint32_t (&sw)[S::SW]) {
+    const int row = c.rb * kTileRows + lane;
     if (row < a.g.n_rows) {
       const size_t vec =
           (static_cast<size_t>(c.s) * a.in_slice_stride_rows + row) * a.g.heads + c.h;
@@ -577,29 +700,31 @@ __global__ void __launch_bounds__(WPC * 32, MINB)
     }
   };
   uint32_t sw_next[S::SW];
-  load_scales(first, sw_next);
+  load_scales(cur, sw_next);
 
   int it = 0;
   int table_sh = -1;          // (slice, head) the tables were built for
   bool pending = false;       // a staged fp16 tile awaits its TMA store
-  TileCoord prev{0, 0, 0};
-  for (int t = first; t < total; t += nw, ++it) {
+  TileWalk prev = cur;
+  for (; cur.valid(a.g); ++it) {
     const int st = it % NST;
     const uint32_t parity = (it / NST) & 1;
-    const TileCoord c = decode_tile(t, a.g);
     const uint8_t* sb = ws + st * Lay::kInBytes;
     const uint8_t* rb = ws + Lay::kRowsOff + st * Lay::kRowBytes;
-    const int row = c.r0 + lane;
+    const int row = cur.rb * kTileRows + lane;
     const bool valid = row < a.g.n_rows;
-    const size_t vec = (static_cast<size_t>(c.s) * a.in_slice_stride_rows + row) * a.g.heads + c.h;
 
     uint32_t sw[S::SW];
     static_for<0, S::SW>([&](auto k_) { sw[decltype(k_)::value] = sw_next[decltype(k_)::value]; });
-    if (t + nw < total) load_scales(t + nw, sw_next);
+    TileWalk nxt = cur;
+    nxt.advance(step, a.g);
+    if (nxt.valid(a.g)) load_scales(nxt, sw_next);
 
     uint32_t words[S::CW];
     if constexpr (!S::CODES_TMA) {
       if (valid) {
+        const size_t vec =
+            (static_cast<size_t>(cur.s) * a.in_slice_stride_rows + row) * a.g.heads + cur.h;
         const uint2 u = *reinterpret_cast<const uint2*>(a.codes + vec * S::CB);
         words[0] = u.x;
         words[1] = u.y;
@@ -612,10 +737,8 @@ __global__ void __launch_bounds__(WPC * 32, MINB)
     if (!ok) {
       if (lane == 0) {
         atomicOr(a.guard, kGuardWaitTimeout);
-        for (int k = 1; k < NST; ++k) {
-          const int tk = t + k * nw;
-          if (tk < total) (void)mbar_wait_bounded(&bars[(it + k) % NST], ((it + k) / NST) & 1);
-        }
+        for (int k = it + 1; k < issued; ++k)
+          (void)mbar_wait_bounded(&bars[k % NST], (k / NST) & 1);
         bulk_wait<0>();
       }
       __syncwarp();
@@ -626,15 +749,20 @@ __global__ void __launch_bounds__(WPC * 32, MINB)
     __syncwarp();
     if (lane == 0) {
       if (pending) store_xhat(prev);
-      const int tn = t + (NST - 1) * nw;
-      if (it > 0 && tn < total) issue(tn, (it - 1) % NST);
+      if (it > 0) {
+        if (ahead.valid(a.g)) {
+          issue(ahead, (it - 1) % NST);
+          ++issued;
+        }
+        ahead.advance(step, a.g);
+      }
     }
     pending = false;
 
     // (a) tables: multiplier gain_j * lambda_j (int4: /16 at odd j, matching
     // the x16 of the odd codes' unpacking) and output sign masks (rebuilt
     // only when the tile's (slice, head) differs from the last one)
-    const int sh = c.s * a.g.heads + c.h;
+    const int sh = cur.s * a.g.heads + cur.h;
     if (sh != table_sh) {
       const float* lam_raw = reinterpret_cast<const float*>(rb);
       const int8_t* sgn_raw = reinterpret_cast<const int8_t*>(rb + 4 * D);
@@ -647,12 +775,12 @@ __global__ void __launch_bounds__(WPC * 32, MINB)
 
     // (b) codes of this lane's vector
     if constexpr (S::CODES_TMA) {
+      const uint32_t crow = lane * S::C_SPAN;
       static_for<0, S::CB / 16>([&](auto c_) {
         constexpr int ci = decltype(c_)::value;
         constexpr int piece = (ci * 16) / S::C_SPAN;
         constexpr int cc = ((ci * 16) % S::C_SPAN) / 16;
-        const uint32_t off =
-            piece * (S::TR * S::C_SPAN) + swizzle<S::C_SPAN>(lane * S::C_SPAN + cc * 16);
+        const uint32_t off = piece * (S::TR * S::C_SPAN) + swizzle<S::C_SPAN>(crow + cc * 16);
         const uint4 u = *reinterpret_cast<const uint4*>(sb + off);
         words[4 * ci] = u.x;
         words[4 * ci + 1] = u.y;
@@ -688,6 +816,7 @@ __global__ void __launch_bounds__(WPC * 32, MINB)
     // staging tile long ago; the wait only confirms it.
     if (lane == 0) bulk_wait_read<0>();
     __syncwarp();
+    const uint32_t xrow = lane * S::X_SPAN;
     static_for<0, D / 8>([&](auto c_) {
       constexpr int ci = decltype(c_)::value;
       constexpr int piece = (ci * 16) / S::X_SPAN;
@@ -698,13 +827,13 @@ __global__ void __launch_bounds__(WPC * 32, MINB)
       o.y = pack_f16x2(v[4 * ci + 1].x, v[4 * ci + 1].y) ^ mk.y;
       o.z = pack_f16x2(v[4 * ci + 2].x, v[4 * ci + 2].y) ^ mk.z;
       o.w = pack_f16x2(v[4 * ci + 3].x, v[4 * ci + 3].y) ^ mk.w;
-      const uint32_t off =
-          piece * (S::TR * S::X_SPAN) + swizzle<S::X_SPAN>(lane * S::X_SPAN + cc * 16);
+      const uint32_t off = piece * (S::TR * S::X_SPAN) + swizzle<S::X_SPAN>(xrow + cc * 16);
       *reinterpret_cast<uint4*>(ob + off) = o;
     });
     fence_proxy_async_smem();
     pending = true;
-    prev = c;
+    prev = cur;
+    cur = nxt;
   }
   __syncwarp();
   if (lane == 0) {

@@ -129,7 +129,8 @@ int quantize_impl(const QuantCall& c) {
   unsigned* guard = Runtime::guard_word();
   if (!guard) return SRFTQ_ERR_CUDA;
   QuantArgs a;
-  a.g = TileGeom{c.heads, int32_t(row_blocks), int32_t(c.n_rows), int32_t(total)};
+  a.g = TileGeom{c.heads, int32_t(row_blocks), int32_t(c.n_rows), int32_t(total),
+                 int32_t(c.n_slices)};
   a.signs = c.signs;
   a.lambda = c.lambda;
   a.codes = c.codes;
@@ -183,7 +184,8 @@ int dequantize_impl(const DequantCall& c) {
   unsigned* guard = Runtime::guard_word();
   if (!guard) return SRFTQ_ERR_CUDA;
   DequantArgs a;
-  a.g = TileGeom{c.heads, int32_t(row_blocks), int32_t(c.n_rows), int32_t(total)};
+  a.g = TileGeom{c.heads, int32_t(row_blocks), int32_t(c.n_rows), int32_t(total),
+                 int32_t(c.n_slices)};
   a.signs = c.signs;
   a.lambda = c.lambda;
   a.codes = c.codes;

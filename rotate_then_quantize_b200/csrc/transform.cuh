@@ -233,6 +233,33 @@ __host__ __device__ constexpr double srft_coordinate_gain(int j, int d) {
   return 0.70710678118654752440;
 }
 
+// Hermitian step of one bin K (0 < K < L, L = D/2) from E = Z_K + conj Z_{L-K}
+// and O = Z_K - conj Z_{L-K}: with W = exp(-2 pi i / D),
+//   xk = 2 X_K = E - i W^K O,   xm = conj(2 X_{L-K}) = E + i W^K O,
+// stored as xk = (Re, Im) of 2 X_K and xm = (Re, Im) of 2 X_{L-K}. The
+// twiddle enters as c (a + t b) with |t| <= 1, six FMAs for both bins.
+template <int D, int K>
+__device__ __forceinline__ void hermitian_out(float Er, float Ei, float Or, float Oi, float2& xk,
+                                              float2& xm) {
+  constexpr double cw = ct::cos2pi(K, D);
+  constexpr double sw = ct::sin2pi(K, D);
+  if constexpr (ct::dabs(cw) >= ct::dabs(sw)) {
+    constexpr float t = float(sw / cw);
+    constexpr float c = float(cw);
+    const float P = fmaf(-t, Or, Oi);   // (cw Oi - sw Or) / cw
+    const float Qv = fmaf(t, Oi, Or);   // (sw Oi + cw Or) / cw
+    xk = make_float2(fmaf(c, P, Er), fmaf(-c, Qv, Ei));
+    xm = make_float2(fmaf(-c, P, Er), fmaf(-c, Qv, -Ei));
+  } else {
+    constexpr float t = float(cw / sw);
+    constexpr float c = float(sw);
+    const float P = fmaf(-t, Oi, Or);   // -(cw Oi - sw Or) / sw
+    const float Qv = fmaf(t, Or, Oi);   // (sw Oi + cw Or) / sw
+    xk = make_float2(fmaf(-c, P, Er), fmaf(-c, Qv, Ei));
+    xm = make_float2(fmaf(c, P, Er), fmaf(-c, Qv, -Ei));
+  }
+}
+
 // Forward SRFT from fp16: xw[m] holds (x_{2m}, x_{2m+1}), sw[m] the fp16
 // signs (s_{2m}, s_{2m+1}) as +-1.0. Output v[j] = (raw_{2j}, raw_{2j+1}),
 // the unnormalised packed spectrum: raw_0 = X_0, raw_1 = X_L, raw_L / raw_{L+1}
@@ -256,37 +283,33 @@ __device__ __forceinline__ void srft_forward(const uint32_t (&xw)[D / 2],
     lane<Q, i + 1>(PI) = fma_f16<1, 1>(xa, sa, -ti);
   });
   packed_passes<Q, -1, 2>(PR, PI);
-  last_pass<Q, -1>(PR, PI);
-  // now PR[k] = (Re Z_k, Re Z_{k+Q}), PI[k] = (Im Z_k, Im Z_{k+Q})
 
-  // Hermitian step for the bin pair (k, L-k):
-  //   E = Z_k + conj Z_{L-k}, O = Z_k - conj Z_{L-k},
-  //   2 X_k = E - i W^k O, 2 X_{L-k} = conj(E + i W^k O), W = exp(-2 pi i / d).
+  // Last pass (span Q) fused with the Hermitian step. Butterfly k gives
+  // (Z_k, Z_{k+Q}) in the lanes of PR[k] / PI[k]; butterfly Q-k gives
+  // (Z_{Q-k}, Z_{L-k}), written here lane-swapped as (Z_{L-k}, Z_{Q-k}), so
+  // that each lane of the pair holds a bin and its Hermitian partner: the
+  // sums and differences E = Z_k + conj Z_{L-k}, O = Z_k - conj Z_{L-k} of
+  // the bins k and k+Q then take four packed instructions.
+  butterfly<-1, 0, Q>(PR[0].x, PI[0].x, PR[0].y, PI[0].y);   // Z_0, Z_Q
   v[0] = make_float2(PR[0].x + PI[0].x, PR[0].x - PI[0].x);
-  static_for<1, Q>([&](auto k_) {
-    constexpr int k = decltype(k_)::value;
-    const float ar = PR[k].x, ai = PI[k].x;            // Z_k
-    const float br = PR[Q - k].y, bi = PI[Q - k].y;    // Z_{L-k}
-    const float Er = ar + br, Ei = ai - bi, Or = ar - br, Oi = ai + bi;
-    constexpr double cw = ct::cos2pi(k, D);
-    constexpr double sw_ = ct::sin2pi(k, D);
-    if constexpr (cw >= sw_) {
-      constexpr float t = float(sw_ / cw);
-      constexpr float c = float(cw);
-      const float P = fmaf(-t, Or, Oi);   // (cw Oi - sw Or) / cw
-      const float Qv = fmaf(t, Oi, Or);   // (sw Oi + cw Or) / cw
-      v[k] = make_float2(fmaf(c, P, Er), fmaf(-c, Qv, Ei));
-      v[L - k] = make_float2(fmaf(-c, P, Er), fmaf(-c, Qv, -Ei));
-    } else {
-      constexpr float t = float(cw / sw_);
-      constexpr float c = float(sw_);
-      const float P = fmaf(-t, Oi, Or);   // -(cw Oi - sw Or) / sw
-      const float Qv = fmaf(t, Or, Oi);   // (sw Oi + cw Or) / sw
-      v[k] = make_float2(fmaf(-c, P, Er), fmaf(-c, Qv, Ei));
-      v[L - k] = make_float2(fmaf(c, P, Er), fmaf(-c, Qv, -Ei));
-    }
-  });
   v[Q] = make_float2(PR[0].y, PI[0].y);
+  {
+    constexpr int k = Q / 2;   // Z_{Q/2} and Z_{3Q/2} are each other's partner
+    butterfly<-1, k, Q>(PR[k].x, PI[k].x, PR[k].y, PI[k].y);
+    const float ar = PR[k].x, ai = PI[k].x, br = PR[k].y, bi = PI[k].y;
+    hermitian_out<D, k>(ar + br, ai - bi, ar - br, ai + bi, v[k], v[L - k]);
+  }
+  static_for<1, Q / 2>([&](auto k_) {
+    constexpr int k = decltype(k_)::value;
+    butterfly<-1, k, Q>(PR[k].x, PI[k].x, PR[k].y, PI[k].y);
+    float a_r = PR[Q - k].x, a_i = PI[Q - k].x, b_r = PR[Q - k].y, b_i = PI[Q - k].y;
+    butterfly<-1, Q - k, Q>(a_r, a_i, b_r, b_i);   // a = Z_{Q-k}, b = Z_{L-k}
+    const float2 Vr = make_float2(b_r, a_r), Vi = make_float2(b_i, a_i);
+    const float2 Er = add2(PR[k], Vr), Ei = sub2(PI[k], Vi);
+    const float2 Or = sub2(PR[k], Vr), Oi = add2(PI[k], Vi);
+    hermitian_out<D, k>(Er.x, Ei.x, Or.x, Oi.x, v[k], v[L - k]);
+    hermitian_out<D, k + Q>(Er.y, Ei.y, Or.y, Oi.y, v[k + Q], v[Q - k]);
+  });
 }
 
 // Inverse SRFT: input v[j] = (c_{2j}, c_{2j+1}) with c_j = coordinate gain
@@ -301,11 +324,13 @@ __device__ __forceinline__ void srft_inverse(float2 (&v)[D / 2]) {
   // Z_k is written to the bit-reversed slot a_{bitrev(k)} for the DIT passes.
   lane<Q, 0>(PR) = v[0].x + v[0].y;
   lane<Q, 0>(PI) = v[0].x - v[0].y;
+  const float2 pm = make_float2(1.0f, -1.0f), mp = make_float2(-1.0f, 1.0f);
   static_for<1, Q>([&](auto k_) {
     constexpr int k = decltype(k_)::value;
     constexpr int ik = bitrev(k, LOG), ilk = bitrev(L - k, LOG);
-    const float ar = v[k].x, ai = v[k].y, br = v[L - k].x, bi = v[L - k].y;
-    const float Er = ar + br, Ei = ai - bi, Or = ar - br, Oi = ai + bi;
+    const float2 E = fma2(v[L - k], pm, v[k]);   // (ar + br, ai - bi)
+    const float2 O = fma2(v[L - k], mp, v[k]);   // (ar - br, ai + bi)
+    const float Er = E.x, Ei = E.y, Or = O.x, Oi = O.y;
     constexpr double cw = ct::cos2pi(k, D);
     constexpr double sw_ = ct::sin2pi(k, D);
     if constexpr (cw >= sw_) {
