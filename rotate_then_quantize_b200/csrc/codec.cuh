@@ -1,21 +1,22 @@
 // Fused quantise / dequantise kernels (one thread per head-dim vector).
 //
-// Work decomposition. A *tile* is 32 consecutive rows of one (slice, head):
-// vectors (s, r0..r0+31, h). Tiles are numbered with the head fastest, then
-// the row block, then the slice, so consecutive tile numbers cover adjacent
-// memory. Every warp is an independent persistent pipeline: warp w of the
-// grid handles tiles w, w + W, w + 2W, ... (W = warps in the grid). A warp
-// owns NST input stages in shared memory; lane 0 issues, per stage, the TMA
-// box loads of the tile (32 rows, 128-byte swizzled so that each lane reading
-// its own row hits distinct banks) plus 1-D bulk copies of that
-// (slice, head)'s lambda row and sign row, all completing on one mbarrier.
-// The lanes build the per-(slice, head) multiplier and sign tables (only
-// when the pair changes), pull their vector into registers and compute; the
-// results (codes, or the dequantised fp16 vectors) are written to a swizzled
-// staging tile and fenced for the async proxy. Nothing on this path waits
-// for the TMA engine: at the start of the next tile, where the warp
-// converges anyway, lane 0 issues the TMA store of the staged tile and the
-// refill of the stage the previous tile consumed (NST - 1 tiles ahead).
+// Work decomposition. A *tile* is the 32 vectors of HPT consecutive heads
+// (HPT = the largest power of two <= 8 dividing H) of 32 / HPT consecutive
+// rows of one slice: a contiguous block of memory when HPT = H. Lane l holds
+// head l % HPT of row l / HPT. Tiles are numbered (s, head block, row block)
+// with the row block fastest, and warp w of the grid takes one contiguous
+// range of tile numbers, so each warp streams consecutive memory and its
+// (slice, head block) -- and with it the per-head multiplier and sign tables
+// -- changes only at the ends of a range. A warp owns NST input stages in
+// shared memory; lane 0 issues the TMA box loads of a tile (128-byte
+// swizzled rows, so each lane reading its own row hits distinct banks), all
+// completing on one mbarrier. The lanes pull their vector into registers and
+// compute; the results (codes, or the dequantised fp16 vectors) are written
+// to a swizzled staging tile and fenced for the async proxy. Nothing on this
+// path waits for the TMA engine: as soon as the lanes have read a stage into
+// registers (where the warp converges anyway), lane 0 issues the refill of
+// that stage with the tile NST ahead and the TMA store of the previously
+// staged tile, so every copy overlaps a whole tile of compute.
 // The quantiser stores scales straight from registers; the dequantiser loads
 // them one tile ahead into registers.
 //
@@ -39,9 +40,19 @@ struct TileGeom {
   int32_t heads;       // H
   int32_t row_blocks;  // ceil(N / rows per tile)
   int32_t n_rows;      // N
-  int32_t total_tiles; // S * row_blocks * H
+  int32_t total_tiles; // S * head_blocks * row_blocks
   int32_t n_slices;    // S
+  int32_t hpt_log2;    // log2(heads per tile); heads x rows per tile = 32
+  int32_t head_blocks; // H / heads per tile
 };
+
+// Heads per tile for H heads: the largest power of two <= kMaxHPT dividing H.
+constexpr int kMaxHPT = 8;
+__host__ __device__ constexpr int heads_per_tile_log2(int H) {
+  int l = 0;
+  while ((2 << l) <= kMaxHPT && H % (2 << l) == 0) ++l;
+  return l;
+}
 
 struct TileCoord {
   int s, r0, h;
@@ -54,28 +65,40 @@ __device__ __forceinline__ TileCoord decode_tile(int t, const TileGeom& g) {
   return {q / g.row_blocks, rb * kTileRows, h};
 }
 
-// Position of a warp's tile t = (s * row_blocks + rb) * H + h as digits. A
-// warp walks t, t + W, t + 2W, ... by adding the digits of the stride W with
-// carries, so no division is left in the loop.
+// A warp's current tile as digits (s, hb, rb) of t = (s * head_blocks + hb)
+// * row_blocks + rb, and the number of tiles left in its range. Stepping
+// carries rb into hb into s: no division inside the loop.
 struct TileWalk {
-  int s, rb, h;
+  int s, hb, rb, left;
 
-  __device__ __forceinline__ void set(int t, const TileGeom& g) {
-    h = t % g.heads;
-    const int q = t / g.heads;
-    rb = q % g.row_blocks;
-    s = q / g.row_blocks;
+  // First tile of warp w of nw (balanced contiguous ranges); false if the
+  // warp has none.
+  __device__ __forceinline__ bool start(int w, int nw, const TileGeom& g) {
+    const int T = g.total_tiles;
+    const int base = T / nw, rem = T % nw;
+    const int t0 = w * base + (w < rem ? w : rem);
+    left = base + (w < rem ? 1 : 0);
+    rb = t0 % g.row_blocks;
+    const int q = t0 / g.row_blocks;
+    hb = q % g.head_blocks;
+    s = q / g.head_blocks;
+    return left > 0;
   }
-  __device__ __forceinline__ void advance(const TileWalk& step, const TileGeom& g) {
-    int hh = h + step.h;
-    int c = hh >= g.heads;
-    h = c ? hh - g.heads : hh;
-    int r = rb + step.rb + c;
-    c = r >= g.row_blocks;
-    rb = c ? r - g.row_blocks : r;
-    s += step.s + c;
+  __device__ __forceinline__ void advance(const TileGeom& g) {
+    const int r = rb + 1;
+    int c = r >= g.row_blocks;
+    rb = c ? 0 : r;
+    const int h = hb + c;
+    c = h >= g.head_blocks;
+    hb = c ? 0 : h;
+    s += c;
+    --left;
   }
-  __device__ __forceinline__ bool valid(const TileGeom& g) const { return s < g.n_slices; }
+  __device__ __forceinline__ bool valid() const { return left > 0; }
+  // identity of the (slice, head block) the tables belong to
+  __device__ __forceinline__ int table_key(const TileGeom& g) const {
+    return s * g.head_blocks + hb;
+  }
 };
 
 // The 1024-byte aligned start of dynamic shared memory, kept as a pointer
@@ -135,9 +158,11 @@ __host__ __device__ constexpr int align_up(int x, int a) { return (x + a - 1) / 
 
 // Per-warp shared-memory layout: NST input tiles (x for the quantiser, codes
 // for the dequantiser; 1024-byte aligned for the swizzled TMA boxes), one
-// output staging tile (codes, or the dequantised fp16 vectors), the NST
-// (lambda row, sign row) pairs that arrive with the input tiles, the
-// multiplier table (d floats), the sign table (d/2 words) and the barriers.
+// output staging tile (codes, or the dequantised fp16 vectors), the per-head
+// multiplier tables (d floats each) and sign tables (d/2 words each) of up to
+// kMaxHPT heads, and the barriers. Each head's table is padded by 16 bytes so
+// that the lanes of different heads reading the same column hit distinct
+// banks.
 template <int D, int BITS, int G, int NST, bool QUANT>
 struct WarpLayout {
   using S = Shape<D, BITS, G>;
@@ -146,12 +171,12 @@ struct WarpLayout {
   static constexpr int kOutTile = QUANT ? (S::CODES_TMA ? S::C_TILE : 0) : S::X_TILE;
   static constexpr int kOutBytes = align_up(kOutTile, 1024);
   static constexpr int kOutOff = NST * kInBytes;
-  static constexpr int kRowBytes = 4 * D + D;            // lambda row + sign row
-  static constexpr int kRowsOff = kOutOff + kOutBytes;
-  static constexpr int kStageTx = kInTile + kRowBytes;
-  static constexpr int kTableOff = kRowsOff + NST * kRowBytes;
-  static constexpr int kSignTabOff = kTableOff + 4 * D;
-  static constexpr int kBarOff = align_up(kSignTabOff + 2 * D, 16);
+  static constexpr int kStageTx = kInTile;
+  static constexpr int kMultStride = D + 4;          // floats per head
+  static constexpr int kSignStride = D / 2 + 4;      // words per head
+  static constexpr int kTableOff = kOutOff + kOutBytes;
+  static constexpr int kSignTabOff = kTableOff + 4 * kMaxHPT * kMultStride;
+  static constexpr int kBarOff = align_up(kSignTabOff + 4 * kMaxHPT * kSignStride, 16);
   static constexpr int kWarpBytes = align_up(kBarOff + 8 * NST, 1024);
 };
 
@@ -312,6 +337,72 @@ __device__ __forceinline__ void group_scales(const float (&am)[NG], uint32_t (&s
   }
 }
 
+// Builds the tables of the HPT heads of (slice s, head block hb) from global
+// memory (all lanes; rare: a warp's head block changes only at the ends of
+// its tile range). QUANT: multiplier gain_j / lambda_j and fp16 +-1 sign
+// pairs; otherwise multiplier gain_j * lambda_j (int4: / 16 at odd j,
+// matching the x16 of the odd codes' unpacking) and fp16 sign-bit masks.
+template <int D, int BITS, int ROT, bool QUANT, int MS, int SS>
+__device__ __forceinline__ void build_tables(float* mult, uint32_t* stab, const float* lambda,
+                                             const int8_t* signs, int s, int hb, int H,
+                                             int hpt_log2, int lane) {
+  // The HPT heads' lambda rows (HPT * D floats) and sign rows (HPT * D
+  // bytes) are contiguous; every lane issues all of its 16-byte loads before
+  // using any, so a rebuild costs one memory round trip.
+  constexpr int kL4 = (kMaxHPT * D / 4 + 31) / 32;    // float4 loads per lane, at most
+  constexpr int kS16 = (kMaxHPT * D / 16 + 31) / 32;  // 16-sign loads per lane, at most
+  const int hpt = 1 << hpt_log2;
+  const size_t h0 = static_cast<size_t>(s) * H + static_cast<size_t>(hb) * hpt;
+  const float4* lam4 = reinterpret_cast<const float4*>(lambda + h0 * D);
+  const uint4* sg16 = reinterpret_cast<const uint4*>(signs + h0 * D);
+  const int n4 = (hpt * D) / 4, n16 = (hpt * D) / 16;
+  float4 l[kL4];
+  uint4 g[kS16];
+#pragma unroll
+  for (int k = 0; k < kL4; ++k) {
+    const int i = lane + 32 * k;
+    if (i < n4) l[k] = __ldg(lam4 + i);
+  }
+#pragma unroll
+  for (int k = 0; k < kS16; ++k) {
+    const int i = lane + 32 * k;
+    if (i < n16) g[k] = __ldg(sg16 + i);
+  }
+  __syncwarp();   // every lane is done reading the old tables
+#pragma unroll
+  for (int k = 0; k < kL4; ++k) {
+    const int i = lane + 32 * k;
+    if (i < n4) {
+      const int h = (4 * i) / D, j = (4 * i) % D;
+      const float lv[4] = {l[k].x, l[k].y, l[k].z, l[k].w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        float m;
+        if constexpr (QUANT)
+          m = gain_f<ROT, D>(j + e) * rcp_approx(lv[e]);
+        else
+          m = gain_f<ROT, D>(j + e) * lv[e] * ((BITS == 4 && ((j + e) & 1)) ? 0.0625f : 1.0f);
+        mult[h * MS + j + e] = m;
+      }
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < kS16; ++k) {
+    const int i = lane + 32 * k;
+    if (i < n16) {
+      const int h = (16 * i) / D, w0 = ((16 * i) % D) / 2;
+      const uint32_t wd[4] = {g[k].x, g[k].y, g[k].z, g[k].w};
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const int8_t s0 = static_cast<int8_t>(wd[e / 2] >> (16 * (e & 1)));
+        const int8_t s1 = static_cast<int8_t>(wd[e / 2] >> (16 * (e & 1) + 8));
+        stab[h * SS + w0 + e] = QUANT ? sign_halves(s0, s1) : sign_mask(s0, s1);
+      }
+    }
+  }
+  __syncwarp();
+}
+
 template <int D, int BITS, int G, int ROT, int WPC, int NST, int MINB>
 __global__ void __launch_bounds__(WPC * 32, MINB)
     quantize_kernel(const __grid_constant__ CUtensorMap tm_x,
@@ -320,7 +411,7 @@ __global__ void __launch_bounds__(WPC * 32, MINB)
   using Lay = WarpLayout<D, BITS, G, NST, true>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = smem_base_1024(smem_raw);
-  const int warp = threadIdx.x >> 5;
+  const int warp = WPC == 1 ? 0 : int(threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   uint8_t* ws = smem + warp * Lay::kWarpBytes;
   uint64_t* bars = reinterpret_cast<uint64_t*>(ws + Lay::kBarOff);
@@ -328,12 +419,15 @@ __global__ void __launch_bounds__(WPC * 32, MINB)
   uint32_t* stab = reinterpret_cast<uint32_t*>(ws + Lay::kSignTabOff);
   uint8_t* ob = ws + Lay::kOutOff;   // codes staging tile
 
-  const int nw = gridDim.x * WPC;
-  const int first = blockIdx.x * WPC + warp;
-  if (first >= a.g.total_tiles) return;
-  TileWalk cur, step;
-  cur.set(first, a.g);
-  step.set(nw, a.g);
+  TileWalk cur;
+  if (!cur.start(blockIdx.x * WPC + warp, gridDim.x * WPC, a.g)) return;
+  const int hpt_log2 = a.g.hpt_log2;
+  const int hpt = 1 << hpt_log2;
+  const int rpt = kTileRows >> hpt_log2;
+  const int hl = lane & (hpt - 1);         // this lane's head inside the tile
+  const int rl = lane >> hpt_log2;         // and its row
+  const float* mrow = mult + hl * Lay::kMultStride;
+  const uint32_t* srow = stab + hl * Lay::kSignStride;
 
   if (lane == 0) {
     prefetch_tensormap(&tm_x);
@@ -345,21 +439,17 @@ __global__ void __launch_bounds__(WPC * 32, MINB)
 
   auto issue = [&](const TileWalk& c, int st) {
     uint8_t* sb = ws + st * Lay::kInBytes;
-    uint8_t* rb = ws + Lay::kRowsOff + st * Lay::kRowBytes;
     mbar_arrive_expect_tx(&bars[st], Lay::kStageTx);
 #pragma unroll
     for (int p = 0; p < S::X_PIECES; ++p)
-      tma_load_4d(sb + p * (S::TR * S::X_SPAN), &tm_x, &bars[st], p * (S::X_SPAN / 2), c.h,
-                  c.rb * kTileRows, c.s);
-    const size_t row = static_cast<size_t>(c.s) * a.g.heads + c.h;
-    bulk_load(rb, a.lambda + row * D, 4 * D, &bars[st]);
-    bulk_load(rb + 4 * D, a.signs + row * D, D, &bars[st]);
+      tma_load_4d(sb + p * (S::TR * S::X_SPAN), &tm_x, &bars[st], p * (S::X_SPAN / 2),
+                  c.hb * hpt, c.rb * rpt, c.s);
   };
   auto store_codes = [&](const TileWalk& c) {
 #pragma unroll
     for (int p = 0; p < S::C_PIECES; ++p)
-      tma_store_4d(&tm_codes, ob + p * (S::TR * S::C_SPAN), p * S::C_SPAN, c.h,
-                   c.rb * kTileRows, c.s);
+      tma_store_4d(&tm_codes, ob + p * (S::TR * S::C_SPAN), p * S::C_SPAN, c.hb * hpt,
+                   c.rb * rpt, c.s);
     bulk_commit();
   };
 
@@ -368,24 +458,29 @@ __global__ void __launch_bounds__(WPC * 32, MINB)
   TileWalk ahead = cur;
   int issued = 0;
   if (lane == 0) {
-    for (int k = 0; k < NST; ++k) {
-      if (ahead.valid(a.g)) {
-        issue(ahead, k);
-        ++issued;
-      }
-      ahead.advance(step, a.g);
+    for (int k = 0; k < NST && ahead.valid(); ++k) {
+      issue(ahead, k);
+      ++issued;
+      ahead.advance(a.g);
     }
   }
 
   int it = 0;
-  int table_sh = -1;          // (slice, head) the tables were built for
+  int table_key = -1;         // (slice, head block) the tables were built for
   bool pending = false;       // a staged codes tile awaits its TMA store
   TileWalk prev = cur;
-  for (; cur.valid(a.g); ++it) {
+  for (; cur.valid(); ++it) {
     const int st = it % NST;
     const uint32_t parity = (it / NST) & 1;
     const uint8_t* sb = ws + st * Lay::kInBytes;
-    const uint8_t* rb = ws + Lay::kRowsOff + st * Lay::kRowBytes;
+
+    // (a) per-head tables, rebuilt only when the (slice, head block) changes
+    const int key = cur.table_key(a.g);
+    if (key != table_key) {
+      build_tables<D, BITS, ROT, true, Lay::kMultStride, Lay::kSignStride>(
+          mult, stab, a.lambda, a.signs, cur.s, cur.hb, a.g.heads, hpt_log2, lane);
+      table_key = key;
+    }
 
     const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars[st], parity));
     if (!ok) {
@@ -399,43 +494,15 @@ __global__ void __launch_bounds__(WPC * 32, MINB)
       __syncwarp();
       return;
     }
-    // Converged: the previous tile's codes are staged and fenced, and its
-    // input stage has been read. Store the one, refill the other.
-    __syncwarp();
-    if (lane == 0) {
-      if (pending) store_codes(prev);
-      if (it > 0) {
-        if (ahead.valid(a.g)) {
-          issue(ahead, (it - 1) % NST);
-          ++issued;
-        }
-        ahead.advance(step, a.g);
-      }
-    }
-    pending = false;
-
-    // (a) per-(slice, head) tables: multiplier gain_j / lambda_j, fp16 signs
-    // (rebuilt only when the tile's (slice, head) differs from the last one)
-    const int sh = cur.s * a.g.heads + cur.h;
-    if (sh != table_sh) {
-      const float* lam_raw = reinterpret_cast<const float*>(rb);
-      const int8_t* sgn_raw = reinterpret_cast<const int8_t*>(rb + 4 * D);
-      for (int j = lane; j < D; j += 32) mult[j] = gain_f<ROT, D>(j) * rcp_approx(lam_raw[j]);
-      for (int w = lane; w < D / 2; w += 32) stab[w] = sign_halves(sgn_raw[2 * w], sgn_raw[2 * w + 1]);
-      __syncwarp();
-      table_sh = sh;
-    }
-
     // (b) this lane's vector (swizzled 16-byte chunks) and the sign words
     uint32_t xw[D / 2], sgw[D / 2];
-    const uint32_t row_off = lane * S::X_SPAN;
+    const uint32_t xrow = swz_row<S::X_SPAN>(smem_addr(sb), lane);
     static_for<0, D / 8>([&](auto c_) {
       constexpr int ci = decltype(c_)::value;
       constexpr int piece = (ci * 16) / S::X_SPAN;
       constexpr int cc = ((ci * 16) % S::X_SPAN) / 16;
-      const uint32_t off = piece * (S::TR * S::X_SPAN) + swizzle<S::X_SPAN>(row_off + cc * 16);
-      const uint4 raw = *reinterpret_cast<const uint4*>(sb + off);
-      const uint4 sg = *reinterpret_cast<const uint4*>(stab + 4 * ci);
+      const uint4 raw = lds128(swz_chunk<S::X_SPAN>(xrow, cc) + piece * (S::TR * S::X_SPAN));
+      const uint4 sg = *reinterpret_cast<const uint4*>(srow + 4 * ci);
       xw[4 * ci + 0] = raw.x;
       xw[4 * ci + 1] = raw.y;
       xw[4 * ci + 2] = raw.z;
@@ -445,13 +512,26 @@ __global__ void __launch_bounds__(WPC * 32, MINB)
       sgw[4 * ci + 2] = sg.z;
       sgw[4 * ci + 3] = sg.w;
     });
+    // Converged: every lane has read this stage and has staged and fenced
+    // the previous tile's codes. Store those, and refill this stage with the
+    // tile NST ahead right away, so the copy overlaps all of this tile's work.
+    __syncwarp();
+    if (lane == 0) {
+      if (pending) store_codes(prev);
+      if (ahead.valid()) {
+        issue(ahead, st);
+        ++issued;
+        ahead.advance(a.g);
+      }
+    }
+    pending = false;
 
     // (c) rotation, then w_j = y_j / lambda_j through the multiplier table
     float2 v[D / 2];
     rotate_forward<ROT, D>(xw, sgw, v);
     static_for<0, D / 4>([&](auto c_) {
       constexpr int ci = decltype(c_)::value;
-      const float4 m4 = *reinterpret_cast<const float4*>(mult + 4 * ci);
+      const float4 m4 = *reinterpret_cast<const float4*>(mrow + 4 * ci);
       v[2 * ci] = mul2(v[2 * ci], make_float2(m4.x, m4.y));
       v[2 * ci + 1] = mul2(v[2 * ci + 1], make_float2(m4.z, m4.w));
     });
@@ -522,10 +602,10 @@ __global__ void __launch_bounds__(WPC * 32, MINB)
       });
     }
 
-    const int row = cur.rb * kTileRows + lane;
+    const int row = cur.rb * rpt + rl;
     const bool valid = row < a.g.n_rows;
-    const size_t vec =
-        (static_cast<size_t>(cur.s) * a.out_slice_stride_rows + row) * a.g.heads + cur.h;
+    const size_t vec = (static_cast<size_t>(cur.s) * a.out_slice_stride_rows + row) * a.g.heads +
+                       cur.hb * hpt + hl;
 
     // (f) codes: swizzled staging tile, stored by TMA at the next convergence
     // (rows past N are clipped by TMA). The store issued at this tile's start
@@ -533,14 +613,13 @@ __global__ void __launch_bounds__(WPC * 32, MINB)
     if constexpr (S::CODES_TMA) {
       if (lane == 0) bulk_wait_read<0>();
       __syncwarp();
-      const uint32_t crow = lane * S::C_SPAN;
+      const uint32_t crow = swz_row<S::C_SPAN>(smem_addr(ob), lane);
       static_for<0, S::CB / 16>([&](auto c_) {
         constexpr int ci = decltype(c_)::value;
         constexpr int piece = (ci * 16) / S::C_SPAN;
         constexpr int cc = ((ci * 16) % S::C_SPAN) / 16;
-        const uint32_t off = piece * (S::TR * S::C_SPAN) + swizzle<S::C_SPAN>(crow + cc * 16);
-        *reinterpret_cast<uint4*>(ob + off) =
-            make_uint4(words[4 * ci], words[4 * ci + 1], words[4 * ci + 2], words[4 * ci + 3]);
+        sts128(swz_chunk<S::C_SPAN>(crow, cc) + piece * (S::TR * S::C_SPAN),
+               make_uint4(words[4 * ci], words[4 * ci + 1], words[4 * ci + 2], words[4 * ci + 3]));
       });
       fence_proxy_async_smem();
       pending = true;
@@ -567,7 +646,7 @@ __global__ void __launch_bounds__(WPC * 32, MINB)
         });
       }
     }
-    cur.advance(step, a.g);
+    cur.advance(a.g);
   }
   __syncwarp();
   if (lane == 0) {
@@ -613,7 +692,7 @@ __global__ void __launch_bounds__(WPC * 32, MINB)
   using Lay = WarpLayout<D, BITS, G, NST, false>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = smem_base_1024(smem_raw);
-  const int warp = threadIdx.x >> 5;
+  const int warp = WPC == 1 ? 0 : int(threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   uint8_t* ws = smem + warp * Lay::kWarpBytes;
   uint64_t* bars = reinterpret_cast<uint64_t*>(ws + Lay::kBarOff);
@@ -621,12 +700,15 @@ __global__ void __launch_bounds__(WPC * 32, MINB)
   uint32_t* mtab = reinterpret_cast<uint32_t*>(ws + Lay::kSignTabOff);
   uint8_t* ob = ws + Lay::kOutOff;   // fp16 staging tile
 
-  const int nw = gridDim.x * WPC;
-  const int first = blockIdx.x * WPC + warp;
-  if (first >= a.g.total_tiles) return;
-  TileWalk cur, step;
-  cur.set(first, a.g);
-  step.set(nw, a.g);
+  TileWalk cur;
+  if (!cur.start(blockIdx.x * WPC + warp, gridDim.x * WPC, a.g)) return;
+  const int hpt_log2 = a.g.hpt_log2;
+  const int hpt = 1 << hpt_log2;
+  const int rpt = kTileRows >> hpt_log2;
+  const int hl = lane & (hpt - 1);
+  const int rl = lane >> hpt_log2;
+  const float* mrow = mult + hl * Lay::kMultStride;
+  const uint32_t* mkrow = mtab + hl * Lay::kSignStride;
 
   if (lane == 0) {
     if constexpr (S::CODES_TMA) prefetch_tensormap(&tm_codes);
@@ -638,44 +720,40 @@ __global__ void __launch_bounds__(WPC * 32, MINB)
 
   auto issue = [&](const TileWalk& c, int st) {
     uint8_t* sb = ws + st * Lay::kInBytes;
-    uint8_t* rb = ws + Lay::kRowsOff + st * Lay::kRowBytes;
-    mbar_arrive_expect_tx(&bars[st], Lay::kStageTx);
     if constexpr (S::CODES_TMA) {
+      mbar_arrive_expect_tx(&bars[st], Lay::kStageTx);
 #pragma unroll
       for (int p = 0; p < S::C_PIECES; ++p)
-        tma_load_4d(sb + p * (S::TR * S::C_SPAN), &tm_codes, &bars[st], p * S::C_SPAN, c.h,
-                    c.rb * kTileRows, c.s);
+        tma_load_4d(sb + p * (S::TR * S::C_SPAN), &tm_codes, &bars[st], p * S::C_SPAN,
+                    c.hb * hpt, c.rb * rpt, c.s);
+    } else {
+      mbar_arrive(&bars[st]);   // no asynchronous input: the phase completes at once
     }
-    const size_t row = static_cast<size_t>(c.s) * a.g.heads + c.h;
-    bulk_load(rb, a.lambda + row * D, 4 * D, &bars[st]);
-    bulk_load(rb + 4 * D, a.signs + row * D, D, &bars[st]);
   };
   auto store_xhat = [&](const TileWalk& c) {
 #pragma unroll
     for (int p = 0; p < S::X_PIECES; ++p)
-      tma_store_4d(&tm_xhat, ob + p * (S::TR * S::X_SPAN), p * (S::X_SPAN / 2), c.h,
-                   c.rb * kTileRows, c.s);
+      tma_store_4d(&tm_xhat, ob + p * (S::TR * S::X_SPAN), p * (S::X_SPAN / 2), c.hb * hpt,
+                   c.rb * rpt, c.s);
     bulk_commit();
   };
 
   TileWalk ahead = cur;
   int issued = 0;
   if (lane == 0) {
-    for (int k = 0; k < NST; ++k) {
-      if (ahead.valid(a.g)) {
-        issue(ahead, k);
-        ++issued;
-      }
-      ahead.advance(step, a.g);
+    for (int k = 0; k < NST && ahead.valid(); ++k) {
+      issue(ahead, k);
+      ++issued;
+      ahead.advance(a.g);
     }
   }
 
   // the next tile's scales are loaded one tile ahead, into registers
   auto load_scales = [&](const TileWalk& c, uint32_t (&sw)[S::SW]) {
-    const int row = c.rb * kTileRows + lane;
+    const int row = c.rb * rpt + rl;
     if (row < a.g.n_rows) {
-      const size_t vec =
-          (static_cast<size_t>(c.s) * a.in_slice_stride_rows + row) * a.g.heads + c.h;
+      const size_t vec = (static_cast<size_t>(c.s) * a.in_slice_stride_rows + row) * a.g.heads +
+                         c.hb * hpt + hl;
       const uint16_t* src = a.scales + vec * S::NG;
       if constexpr (S::NG == 1) {
         sw[0] = src[0];
@@ -703,34 +781,41 @@ __global__ void __launch_bounds__(WPC * 32, MINB)
   load_scales(cur, sw_next);
 
   int it = 0;
-  int table_sh = -1;          // (slice, head) the tables were built for
+  int table_key = -1;         // (slice, head block) the tables were built for
   bool pending = false;       // a staged fp16 tile awaits its TMA store
   TileWalk prev = cur;
-  for (; cur.valid(a.g); ++it) {
+  for (; cur.valid(); ++it) {
     const int st = it % NST;
     const uint32_t parity = (it / NST) & 1;
     const uint8_t* sb = ws + st * Lay::kInBytes;
-    const uint8_t* rb = ws + Lay::kRowsOff + st * Lay::kRowBytes;
-    const int row = cur.rb * kTileRows + lane;
+    const int row = cur.rb * rpt + rl;
     const bool valid = row < a.g.n_rows;
 
     uint32_t sw[S::SW];
     static_for<0, S::SW>([&](auto k_) { sw[decltype(k_)::value] = sw_next[decltype(k_)::value]; });
     TileWalk nxt = cur;
-    nxt.advance(step, a.g);
-    if (nxt.valid(a.g)) load_scales(nxt, sw_next);
+    nxt.advance(a.g);
+    if (nxt.valid()) load_scales(nxt, sw_next);
 
     uint32_t words[S::CW];
     if constexpr (!S::CODES_TMA) {
       if (valid) {
-        const size_t vec =
-            (static_cast<size_t>(cur.s) * a.in_slice_stride_rows + row) * a.g.heads + cur.h;
+        const size_t vec = (static_cast<size_t>(cur.s) * a.in_slice_stride_rows + row) *
+                               a.g.heads + cur.hb * hpt + hl;
         const uint2 u = *reinterpret_cast<const uint2*>(a.codes + vec * S::CB);
         words[0] = u.x;
         words[1] = u.y;
       } else {
         words[0] = words[1] = 0u;
       }
+    }
+
+    // (a) per-head tables, rebuilt only when the (slice, head block) changes
+    const int key = cur.table_key(a.g);
+    if (key != table_key) {
+      build_tables<D, BITS, ROT, false, Lay::kMultStride, Lay::kSignStride>(
+          mult, mtab, a.lambda, a.signs, cur.s, cur.hb, a.g.heads, hpt_log2, lane);
+      table_key = key;
     }
 
     const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars[st], parity));
@@ -744,50 +829,33 @@ __global__ void __launch_bounds__(WPC * 32, MINB)
       __syncwarp();
       return;
     }
-    // Converged: the previous tile's output is staged and fenced, and its
-    // input stage has been read. Store the one, refill the other.
-    __syncwarp();
-    if (lane == 0) {
-      if (pending) store_xhat(prev);
-      if (it > 0) {
-        if (ahead.valid(a.g)) {
-          issue(ahead, (it - 1) % NST);
-          ++issued;
-        }
-        ahead.advance(step, a.g);
-      }
-    }
-    pending = false;
-
-    // (a) tables: multiplier gain_j * lambda_j (int4: /16 at odd j, matching
-    // the x16 of the odd codes' unpacking) and output sign masks (rebuilt
-    // only when the tile's (slice, head) differs from the last one)
-    const int sh = cur.s * a.g.heads + cur.h;
-    if (sh != table_sh) {
-      const float* lam_raw = reinterpret_cast<const float*>(rb);
-      const int8_t* sgn_raw = reinterpret_cast<const int8_t*>(rb + 4 * D);
-      for (int j = lane; j < D; j += 32)
-        mult[j] = gain_f<ROT, D>(j) * lam_raw[j] * ((BITS == 4 && (j & 1)) ? 0.0625f : 1.0f);
-      for (int w = lane; w < D / 2; w += 32) mtab[w] = sign_mask(sgn_raw[2 * w], sgn_raw[2 * w + 1]);
-      __syncwarp();
-      table_sh = sh;
-    }
-
     // (b) codes of this lane's vector
     if constexpr (S::CODES_TMA) {
-      const uint32_t crow = lane * S::C_SPAN;
+      const uint32_t crow = swz_row<S::C_SPAN>(smem_addr(sb), lane);
       static_for<0, S::CB / 16>([&](auto c_) {
         constexpr int ci = decltype(c_)::value;
         constexpr int piece = (ci * 16) / S::C_SPAN;
         constexpr int cc = ((ci * 16) % S::C_SPAN) / 16;
-        const uint32_t off = piece * (S::TR * S::C_SPAN) + swizzle<S::C_SPAN>(crow + cc * 16);
-        const uint4 u = *reinterpret_cast<const uint4*>(sb + off);
+        const uint4 u = lds128(swz_chunk<S::C_SPAN>(crow, cc) + piece * (S::TR * S::C_SPAN));
         words[4 * ci] = u.x;
         words[4 * ci + 1] = u.y;
         words[4 * ci + 2] = u.z;
         words[4 * ci + 3] = u.w;
       });
     }
+    // Converged: every lane has read this stage and has staged and fenced
+    // the previous tile's output. Store that, and refill this stage with the
+    // tile NST ahead right away.
+    __syncwarp();
+    if (lane == 0) {
+      if (pending) store_xhat(prev);
+      if (ahead.valid()) {
+        issue(ahead, st);
+        ++issued;
+        ahead.advance(a.g);
+      }
+    }
+    pending = false;
 
     // (c) yhat_j = q_j * sigma_g * lambda_j * gain_j
     float2 v[D / 2];
@@ -803,7 +871,7 @@ __global__ void __launch_bounds__(WPC * 32, MINB)
     });
     static_for<0, D / 4>([&](auto c_) {
       constexpr int ci = decltype(c_)::value;
-      const float4 m4 = *reinterpret_cast<const float4*>(mult + 4 * ci);
+      const float4 m4 = *reinterpret_cast<const float4*>(mrow + 4 * ci);
       v[2 * ci] = mul2(v[2 * ci], make_float2(m4.x, m4.y));
       v[2 * ci + 1] = mul2(v[2 * ci + 1], make_float2(m4.z, m4.w));
     });
@@ -816,19 +884,18 @@ __global__ void __launch_bounds__(WPC * 32, MINB)
     // staging tile long ago; the wait only confirms it.
     if (lane == 0) bulk_wait_read<0>();
     __syncwarp();
-    const uint32_t xrow = lane * S::X_SPAN;
+    const uint32_t xrow = swz_row<S::X_SPAN>(smem_addr(ob), lane);
     static_for<0, D / 8>([&](auto c_) {
       constexpr int ci = decltype(c_)::value;
       constexpr int piece = (ci * 16) / S::X_SPAN;
       constexpr int cc = ((ci * 16) % S::X_SPAN) / 16;
-      const uint4 mk = *reinterpret_cast<const uint4*>(mtab + 4 * ci);
+      const uint4 mk = *reinterpret_cast<const uint4*>(mkrow + 4 * ci);
       uint4 o;
       o.x = pack_f16x2(v[4 * ci + 0].x, v[4 * ci + 0].y) ^ mk.x;
       o.y = pack_f16x2(v[4 * ci + 1].x, v[4 * ci + 1].y) ^ mk.y;
       o.z = pack_f16x2(v[4 * ci + 2].x, v[4 * ci + 2].y) ^ mk.z;
       o.w = pack_f16x2(v[4 * ci + 3].x, v[4 * ci + 3].y) ^ mk.w;
-      const uint32_t off = piece * (S::TR * S::X_SPAN) + swizzle<S::X_SPAN>(xrow + cc * 16);
-      *reinterpret_cast<uint4*>(ob + off) = o;
+      sts128(swz_chunk<S::X_SPAN>(xrow, cc) + piece * (S::TR * S::X_SPAN), o);
     });
     fence_proxy_async_smem();
     pending = true;

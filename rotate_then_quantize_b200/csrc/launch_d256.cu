@@ -6,6 +6,10 @@
 namespace srftq {
 namespace {
 
+// d = 256 launch shape: one warp per block, 8 blocks per SM, and two input
+// stages (these kernels refill a stage at the start of the next tile).
+constexpr int kWPC256 = 1, kMinBlocks256 = 8, kNST256 = 2;
+
 // Calls f(Int<BITS>, Int<G>, Int<ROT>) for the run-time configuration.
 template <typename F>
 int dispatch_config256(int bits, int group, int rot, F&& f) {
@@ -45,7 +49,7 @@ int encode_codes256(CUtensorMap* tm, const uint8_t* base, int cb, int64_t H, int
 template <int BITS, int G, int ROT>
 int quantize256_impl(const QuantCall& c) {
   using S = Shape256<BITS, G>;
-  using Lay = WarpLayout256<BITS, G, kNST, true>;
+  using Lay = WarpLayout256<BITS, G, kNST256, true>;
   const int64_t row_blocks = (c.n_rows + kTileRows256 - 1) / kTileRows256;
   const int64_t total = c.n_slices * row_blocks * c.heads;
   if (total == 0) return SRFTQ_OK;
@@ -67,22 +71,22 @@ int quantize256_impl(const QuantCall& c) {
   a.out_slice_stride_rows = c.out_slice_stride_rows;
   a.guard = guard;
 
-  constexpr auto K = quantize256_kernel<BITS, G, ROT, kQWPC, kNST, kQMinBlocks>;
-  const int smem = kQWPC * Lay::kWarpBytes + kSmemSlack;
+  constexpr auto K = quantize256_kernel<BITS, G, ROT, kWPC256, kNST256, kMinBlocks256>;
+  const int smem = kWPC256 * Lay::kWarpBytes + kSmemSlack;
   int bps = 0;
-  const int rc = prepare_kernel<K>(smem, kQWPC * 32, &bps);
+  const int rc = prepare_kernel<K>(smem, kWPC256 * 32, &bps);
   if (rc != SRFTQ_OK) return rc;
-  const int64_t want = (total + kQWPC - 1) / kQWPC;
+  const int64_t want = (total + kWPC256 - 1) / kWPC256;
   const int64_t cap = int64_t(Runtime::num_sms()) * bps;
   const int grid = int(want < cap ? want : cap);
-  K<<<grid, kQWPC * 32, smem, c.stream>>>(tm_x, tm_c, a);
+  K<<<grid, kWPC256 * 32, smem, c.stream>>>(tm_x, tm_c, a);
   return finish_launch();
 }
 
 template <int BITS, int G, int ROT>
 int dequantize256_impl(const DequantCall& c) {
   using S = Shape256<BITS, G>;
-  using Lay = WarpLayout256<BITS, G, kNST, false>;
+  using Lay = WarpLayout256<BITS, G, kNST256, false>;
   const int64_t row_blocks = (c.n_rows + kTileRows256 - 1) / kTileRows256;
   const int64_t total = c.n_slices * row_blocks * c.heads;
   if (total == 0) return SRFTQ_OK;
@@ -106,15 +110,15 @@ int dequantize256_impl(const DequantCall& c) {
   a.out_slice_stride_rows = c.out_slice_stride_rows;
   a.guard = guard;
 
-  constexpr auto K = dequantize256_kernel<BITS, G, ROT, kDWPC, kNST, kDMinBlocks>;
-  const int smem = kDWPC * Lay::kWarpBytes + kSmemSlack;
+  constexpr auto K = dequantize256_kernel<BITS, G, ROT, kWPC256, kNST256, kMinBlocks256>;
+  const int smem = kWPC256 * Lay::kWarpBytes + kSmemSlack;
   int bps = 0;
-  const int rc = prepare_kernel<K>(smem, kDWPC * 32, &bps);
+  const int rc = prepare_kernel<K>(smem, kWPC256 * 32, &bps);
   if (rc != SRFTQ_OK) return rc;
-  const int64_t want = (total + kDWPC - 1) / kDWPC;
+  const int64_t want = (total + kWPC256 - 1) / kWPC256;
   const int64_t cap = int64_t(Runtime::num_sms()) * bps;
   const int grid = int(want < cap ? want : cap);
-  K<<<grid, kDWPC * 32, smem, c.stream>>>(tm_c, tm_x, a);
+  K<<<grid, kWPC256 * 32, smem, c.stream>>>(tm_c, tm_x, a);
   return finish_launch();
 }
 

@@ -14,27 +14,36 @@ namespace srftq {
 
 // Launch shapes: warps per block and the blocks per SM the register budget
 // is sized for (their product is the resident warps per SM), and input
-// stages per warp. Measured on B200 at d = 128: both kernels run fastest
-// with 8 warps per SM and the full register budget (the transform keeps
-// ~200 values live; at 12 warps per SM the 168-register cap costs more than
-// the extra warps recover).
+// stages per warp. Measured on B200: one warp per block (a block's only
+// warp has index 0, so the tile walk and the TMA operands are warp-uniform
+// and live in uniform registers); one input stage, refilled as soon as it is
+// read, hides the load as well as two and leaves shared memory for the
+// per-head tables; d = 128 runs 8 warps per SM with the full register
+// budget (at 12 the transform spills), d <= 64 runs 12.
 #ifndef SRFTQ_Q_WPC
-#define SRFTQ_Q_WPC 4
+#define SRFTQ_Q_WPC 1
 #endif
 #ifndef SRFTQ_Q_MINB
-#define SRFTQ_Q_MINB 2
+#define SRFTQ_Q_MINB 0   // 0: by head dimension (q_min_blocks)
 #endif
 #ifndef SRFTQ_D_WPC
-#define SRFTQ_D_WPC 4
+#define SRFTQ_D_WPC 1
 #endif
 #ifndef SRFTQ_D_MINB
-#define SRFTQ_D_MINB 2
+#define SRFTQ_D_MINB 0   // 0: by head dimension (q_min_blocks)
 #endif
 #ifndef SRFTQ_NST
-#define SRFTQ_NST 2
+#define SRFTQ_NST 1
 #endif
-constexpr int kQWPC = SRFTQ_Q_WPC, kQMinBlocks = SRFTQ_Q_MINB;
-constexpr int kDWPC = SRFTQ_D_WPC, kDMinBlocks = SRFTQ_D_MINB;
+constexpr int kQWPC = SRFTQ_Q_WPC;
+constexpr int kDWPC = SRFTQ_D_WPC;
+// Blocks per SM the register budget is sized for: d <= 64 keeps its vector
+// in <= 168 registers without spills, so 12 one-warp blocks fit; d = 128
+// needs the full 255 registers (8 blocks).
+template <int D, int MINB>
+constexpr int min_blocks() {
+  return MINB > 0 ? MINB : (D <= 64 ? 12 : 8);
+}
 constexpr int kNST = SRFTQ_NST;
 
 inline CUtensorMapSwizzle swizzle_mode(int span) {
@@ -95,14 +104,27 @@ inline int finish_launch() {
   return cudaGetLastError() == cudaSuccess ? SRFTQ_OK : SRFTQ_ERR_CUDA;
 }
 
+// Tile geometry for H heads: HPT = 2^hpt_log2 heads x (32 / HPT) rows.
+inline TileGeom make_geom(int64_t n_slices, int64_t n_rows, int heads, int64_t* total) {
+  const int lg = heads_per_tile_log2(heads);
+  const int64_t rpt = kTileRows >> lg;
+  const int64_t row_blocks = (n_rows + rpt - 1) / rpt;
+  const int64_t head_blocks = heads >> lg;
+  *total = n_slices * head_blocks * row_blocks;
+  return TileGeom{heads, int32_t(row_blocks), int32_t(n_rows), int32_t(*total),
+                  int32_t(n_slices), lg, int32_t(head_blocks)};
+}
+
 template <int D, int BITS, int G, int ROT>
 int quantize_impl(const QuantCall& c) {
   using S = Shape<D, BITS, G>;
   using Lay = WarpLayout<D, BITS, G, kNST, true>;
-  const int64_t row_blocks = (c.n_rows + kTileRows - 1) / kTileRows;
-  const int64_t total = c.n_slices * row_blocks * c.heads;
-  if (total == 0) return SRFTQ_OK;
-  if (total > INT_MAX || c.n_rows > INT_MAX || c.n_slices > INT_MAX) return SRFTQ_ERR_UNSUPPORTED;
+  if (c.n_slices == 0 || c.n_rows == 0) return SRFTQ_OK;
+  if (c.n_rows > INT_MAX || c.n_slices > INT_MAX) return SRFTQ_ERR_UNSUPPORTED;
+  int64_t total = 0;
+  const TileGeom g = make_geom(c.n_slices, c.n_rows, c.heads, &total);
+  if (total > INT_MAX) return SRFTQ_ERR_UNSUPPORTED;
+  const uint32_t hpt = 1u << g.hpt_log2, rpt = uint32_t(kTileRows) >> g.hpt_log2;
 
   CUtensorMap tm_x, tm_c;
   std::memset(&tm_c, 0, sizeof(tm_c));
@@ -111,7 +133,7 @@ int quantize_impl(const QuantCall& c) {
                               uint64_t(c.n_slices)};
     const uint64_t str[3] = {uint64_t(S::XB), uint64_t(c.heads) * S::XB,
                              uint64_t(c.x_slice_stride_rows) * c.heads * S::XB};
-    const uint32_t box[4] = {uint32_t(S::X_SPAN / 2), 1u, uint32_t(kTileRows), 1u};
+    const uint32_t box[4] = {uint32_t(S::X_SPAN / 2), hpt, rpt, 1u};
     if (Runtime::encode_4d(&tm_x, CU_TENSOR_MAP_DATA_TYPE_UINT16, const_cast<uint16_t*>(c.x), dims,
                            str, box, swizzle_mode(S::X_SPAN)) != 0)
       return SRFTQ_ERR_CUDA;
@@ -121,7 +143,7 @@ int quantize_impl(const QuantCall& c) {
                               uint64_t(c.n_slices)};
     const uint64_t str[3] = {uint64_t(S::CB), uint64_t(c.heads) * S::CB,
                              uint64_t(c.out_slice_stride_rows) * c.heads * S::CB};
-    const uint32_t box[4] = {uint32_t(S::C_SPAN), 1u, uint32_t(kTileRows), 1u};
+    const uint32_t box[4] = {uint32_t(S::C_SPAN), hpt, rpt, 1u};
     if (Runtime::encode_4d(&tm_c, CU_TENSOR_MAP_DATA_TYPE_UINT8, c.codes, dims, str, box,
                            swizzle_mode(S::C_SPAN)) != 0)
       return SRFTQ_ERR_CUDA;
@@ -129,8 +151,7 @@ int quantize_impl(const QuantCall& c) {
   unsigned* guard = Runtime::guard_word();
   if (!guard) return SRFTQ_ERR_CUDA;
   QuantArgs a;
-  a.g = TileGeom{c.heads, int32_t(row_blocks), int32_t(c.n_rows), int32_t(total),
-                 int32_t(c.n_slices)};
+  a.g = g;
   a.signs = c.signs;
   a.lambda = c.lambda;
   a.codes = c.codes;
@@ -138,7 +159,7 @@ int quantize_impl(const QuantCall& c) {
   a.out_slice_stride_rows = c.out_slice_stride_rows;
   a.guard = guard;
 
-  constexpr auto K = quantize_kernel<D, BITS, G, ROT, kQWPC, kNST, kQMinBlocks>;
+  constexpr auto K = quantize_kernel<D, BITS, G, ROT, kQWPC, kNST, min_blocks<D, SRFTQ_Q_MINB>()>;
   const int smem = kQWPC * Lay::kWarpBytes + kSmemSlack;
   int bps = 0;
   int rc = prepare_kernel<K>(smem, kQWPC * 32, &bps);
@@ -154,10 +175,12 @@ template <int D, int BITS, int G, int ROT>
 int dequantize_impl(const DequantCall& c) {
   using S = Shape<D, BITS, G>;
   using Lay = WarpLayout<D, BITS, G, kNST, false>;
-  const int64_t row_blocks = (c.n_rows + kTileRows - 1) / kTileRows;
-  const int64_t total = c.n_slices * row_blocks * c.heads;
-  if (total == 0) return SRFTQ_OK;
-  if (total > INT_MAX || c.n_rows > INT_MAX || c.n_slices > INT_MAX) return SRFTQ_ERR_UNSUPPORTED;
+  if (c.n_slices == 0 || c.n_rows == 0) return SRFTQ_OK;
+  if (c.n_rows > INT_MAX || c.n_slices > INT_MAX) return SRFTQ_ERR_UNSUPPORTED;
+  int64_t total = 0;
+  const TileGeom g = make_geom(c.n_slices, c.n_rows, c.heads, &total);
+  if (total > INT_MAX) return SRFTQ_ERR_UNSUPPORTED;
+  const uint32_t hpt = 1u << g.hpt_log2, rpt = uint32_t(kTileRows) >> g.hpt_log2;
 
   CUtensorMap tm_c, tm_x;
   std::memset(&tm_c, 0, sizeof(tm_c));
@@ -166,7 +189,7 @@ int dequantize_impl(const DequantCall& c) {
                               uint64_t(c.n_slices)};
     const uint64_t str[3] = {uint64_t(S::CB), uint64_t(c.heads) * S::CB,
                              uint64_t(c.in_slice_stride_rows) * c.heads * S::CB};
-    const uint32_t box[4] = {uint32_t(S::C_SPAN), 1u, uint32_t(kTileRows), 1u};
+    const uint32_t box[4] = {uint32_t(S::C_SPAN), hpt, rpt, 1u};
     if (Runtime::encode_4d(&tm_c, CU_TENSOR_MAP_DATA_TYPE_UINT8, const_cast<uint8_t*>(c.codes),
                            dims, str, box, swizzle_mode(S::C_SPAN)) != 0)
       return SRFTQ_ERR_CUDA;
@@ -176,7 +199,7 @@ int dequantize_impl(const DequantCall& c) {
                               uint64_t(c.n_slices)};
     const uint64_t str[3] = {uint64_t(S::XB), uint64_t(c.heads) * S::XB,
                              uint64_t(c.out_slice_stride_rows) * c.heads * S::XB};
-    const uint32_t box[4] = {uint32_t(S::X_SPAN / 2), 1u, uint32_t(kTileRows), 1u};
+    const uint32_t box[4] = {uint32_t(S::X_SPAN / 2), hpt, rpt, 1u};
     if (Runtime::encode_4d(&tm_x, CU_TENSOR_MAP_DATA_TYPE_UINT16, c.xhat, dims, str, box,
                            swizzle_mode(S::X_SPAN)) != 0)
       return SRFTQ_ERR_CUDA;
@@ -184,8 +207,7 @@ int dequantize_impl(const DequantCall& c) {
   unsigned* guard = Runtime::guard_word();
   if (!guard) return SRFTQ_ERR_CUDA;
   DequantArgs a;
-  a.g = TileGeom{c.heads, int32_t(row_blocks), int32_t(c.n_rows), int32_t(total),
-                 int32_t(c.n_slices)};
+  a.g = g;
   a.signs = c.signs;
   a.lambda = c.lambda;
   a.codes = c.codes;
@@ -195,7 +217,7 @@ int dequantize_impl(const DequantCall& c) {
   a.out_slice_stride_rows = c.out_slice_stride_rows;
   a.guard = guard;
 
-  constexpr auto K = dequantize_kernel<D, BITS, G, ROT, kDWPC, kNST, kDMinBlocks>;
+  constexpr auto K = dequantize_kernel<D, BITS, G, ROT, kDWPC, kNST, min_blocks<D, SRFTQ_D_MINB>()>;
   const int smem = kDWPC * Lay::kWarpBytes + kSmemSlack;
   int bps = 0;
   int rc = prepare_kernel<K>(smem, kDWPC * 32, &bps);

@@ -35,6 +35,11 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                : "memory");
 }
 
+// Plain arrival (count 1) without transaction bytes.
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
@@ -124,6 +129,43 @@ __device__ __forceinline__ uint32_t swizzle(uint32_t off) {
     constexpr uint32_t mask = SPAN / 16 - 1;
     return off ^ (((off >> 7) & mask) << 4);
   }
+}
+
+// 16-byte shared-memory load / store at a 32-bit shared address.
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr));
+  return v;
+}
+
+__device__ __forceinline__ void sts128(uint32_t addr, uint4 v) {
+  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y),
+               "r"(v.z), "r"(v.w)
+               : "memory");
+}
+
+// Row r of a swizzled TMA box of rows of SPAN bytes: the 16-byte chunk c of
+// the row sits at  base + r * SPAN + ((c ^ (r' & mask)) << 4), r' = the
+// 128-byte line index of the row. For a row whose offset has no bits inside
+// the chunk field, that is (base + r * SPAN + (x << 4)) ^ (c << 4) with
+// x = r' & mask: swz_row() returns that per-row term, swz_chunk() applies
+// the chunk XOR (base 1024-aligned, piece offsets multiples of 1024).
+template <int SPAN>
+__device__ __forceinline__ uint32_t swz_row(uint32_t base, uint32_t r) {
+  const uint32_t off = r * SPAN;
+  if constexpr (SPAN <= 16) {
+    return base + off;
+  } else {
+    constexpr uint32_t mask = SPAN / 16 - 1;
+    return base + (off | (((off >> 7) & mask) << 4));
+  }
+}
+
+template <int SPAN>
+__device__ __forceinline__ uint32_t swz_chunk(uint32_t row_addr, uint32_t c) {
+  return SPAN <= 16 ? row_addr + 16 * c : row_addr ^ (16 * c);
 }
 
 }  // namespace srftq

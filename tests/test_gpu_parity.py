@@ -118,6 +118,19 @@ def test_ragged_rows_and_heads(N, H):
     run_and_check(x16, signs, lam, d, group, bits, rq.SRFT, f"N{N} H{H}")
 
 
+@pytest.mark.parametrize("H", [2, 4, 6, 8, 12, 16])
+@pytest.mark.parametrize("d,bits,group", [(64, 4, 16), (128, 8, 32)])
+def test_head_block_tiles(H, d, bits, group):
+    """Tiles span up to 8 heads of 32 / heads-per-tile rows; cover every
+    heads-per-tile value, several head blocks per slice and ragged rows."""
+    rng = np.random.default_rng(100 * H + d)
+    S, N = 2, 29
+    x16 = _x(rng, S, N, H, d)
+    signs = _signs(rng, S, H, d)
+    lam = np.exp(rng.uniform(-1, 1, (S, H, d))).astype(np.float32)
+    run_and_check(x16, signs, lam, d, group, bits, rq.SRFT, f"H{H} d{d}")
+
+
 @pytest.mark.parametrize("N", [1, 15, 16, 17, 47])
 @pytest.mark.parametrize("rot", [0, 1])
 def test_ragged_rows_d256(N, rot):
