@@ -24,7 +24,6 @@ from __future__ import annotations
 
 import argparse
 import hashlib
-import glob
 import json
 import os
 import statistics
@@ -47,11 +46,13 @@ FALLBACK_HBM_GBS = 6650.0
 def parse_args(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
-    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="qwen_like_d128", choices=list(kv_synth.WORKLOADS))
     ap.add_argument("--rotation", type=int, default=0, choices=[0, 1])
+    ap.add_argument("--slices", type=int, default=None,
+                    help="run the workload on its first SLICES slices only (smaller captures)")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -73,18 +74,34 @@ def read_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def csrc_hash():
+# Sources each timed kernel is compiled from: a committed DRAM-traffic figure
+# is used only while these files are unchanged.
+KERNEL_SOURCES = {
+    "quantize_kernel": ("codec.cuh", "transform.cuh", "common.cuh", "ptx.cuh", "launch.cuh",
+                        "launch_impl.cuh"),
+    "dequantize_kernel": ("codec.cuh", "transform.cuh", "common.cuh", "ptx.cuh", "launch.cuh",
+                          "launch_impl.cuh"),
+    "quantize256_kernel": ("codec256.cuh", "transform256.cuh", "codec.cuh", "transform.cuh",
+                           "common.cuh", "ptx.cuh", "launch.cuh", "launch_impl.cuh",
+                           "launch_d256.cu"),
+    "dequantize256_kernel": ("codec256.cuh", "transform256.cuh", "codec.cuh", "transform.cuh",
+                             "common.cuh", "ptx.cuh", "launch.cuh", "launch_impl.cuh",
+                             "launch_d256.cu"),
+}
+
+
+def csrc_hash(kernel: str) -> str:
     h = hashlib.sha256()
-    for p in sorted(glob.glob(os.path.join(ROOT, "rotate_then_quantize_b200", "csrc", "*"))):
-        with open(p, "rb") as f:
-            h.update(os.path.basename(p).encode())
+    for name in sorted(KERNEL_SOURCES.get(kernel, ())):
+        with open(os.path.join(ROOT, "rotate_then_quantize_b200", "csrc", name), "rb") as f:
+            h.update(name.encode())
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
 def read_traffic(kernel: str, workload: str):
     """Per-launch DRAM bytes from the committed ncu summary, if it was taken
-    on the current kernel sources; null otherwise."""
+    on the current sources of that kernel; null otherwise."""
     p = os.path.join(ROOT, "profiles", "dram_traffic.json")
     try:
         with open(p) as f:
@@ -92,7 +109,7 @@ def read_traffic(kernel: str, workload: str):
     except Exception:
         return None
     ent = data.get(f"{kernel}:{workload}")
-    if not ent or ent.get("csrc_sha") != csrc_hash():
+    if not ent or ent.get("sources_sha") != csrc_hash(kernel):
         return None
     return ent.get("dram_bytes_per_launch")
 
@@ -202,7 +219,7 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    w = kv_synth.WORKLOADS[args.workload]
+    w = workload(args)
     x16, signs, nv = oracle_sample(w, args.cpu_sample)
     for _ in range(args.warmup):
         oracle_step(w, x16, signs, args.rotation)
@@ -270,13 +287,25 @@ def _max_over_ranks(pg, dev, ms):
     pg.all_reduce(t, op=pg.ReduceOp.MAX)
     return float(t.item())
 
+def workload(args):
+    """The named workload, cut to its first --slices slices if given."""
+    import dataclasses
+
+    w = kv_synth.WORKLOADS[args.workload]
+    if args.slices is not None:
+        if not 1 <= args.slices <= w.S:
+            raise SystemExit(f"--slices must be in 1..{w.S}")
+        w = dataclasses.replace(w, S=args.slices)
+    return w
+
+
 def run_ours(args):
     import torch
 
     import rotate_then_quantize_b200 as rq
 
     rank, world, local, dev, pg = _setup_ranks()
-    w = kv_synth.WORKLOADS[args.workload]
+    w = workload(args)
     rot = args.rotation
     rq.load_library()
     x = kv_synth.make_x_torch(w, dev, seed=1000 * rank)
@@ -413,7 +442,7 @@ def run_decode(args):
     import rotate_then_quantize_b200 as rq
 
     rank, world, local, dev, pg = _setup_ranks()
-    w = kv_synth.WORKLOADS[args.workload]
+    w = workload(args)
     B = 32
     T0 = w.N // B
     L = w.S // 2
