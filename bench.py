@@ -278,6 +278,16 @@ def _setup_ranks():
     return rank, world, local, dev, pg
 
 
+def job_gbps(bytes_per_rank_step: float, steps: int, world: int, ms_max: float) -> float:
+    """Whole-job throughput: every rank's bytes over the slowest rank's time."""
+    return bytes_per_rank_step * steps * world / (ms_max / 1e3) / 1e9
+
+
+def rank_seeds(rank: int) -> tuple:
+    """(data seed, sign seed) of a replica: every rank codes its own cache."""
+    return 1000 * rank, 1 + rank
+
+
 def _max_over_ranks(pg, dev, ms):
     import torch
 
@@ -308,8 +318,9 @@ def run_ours(args):
     w = workload(args)
     rot = args.rotation
     rq.load_library()
-    x = kv_synth.make_x_torch(w, dev, seed=1000 * rank)
-    signs = torch.from_numpy(kv_synth.rademacher_signs(w.S, w.H, w.d, seed=1 + rank)).to(dev)
+    data_seed, sign_seed = rank_seeds(rank)
+    x = kv_synth.make_x_torch(w, dev, seed=data_seed)
+    signs = torch.from_numpy(kv_synth.rademacher_signs(w.S, w.H, w.d, seed=sign_seed)).to(dev)
     lam = torch.empty((w.S, w.H, w.d), dtype=torch.float32, device=dev)
     codes = torch.empty((w.S, w.N, w.H, w.d * w.bits // 8), dtype=torch.uint8, device=dev)
     scales = torch.empty((w.S, w.N, w.H, w.d // w.group), dtype=torch.float16, device=dev)
@@ -358,7 +369,7 @@ def run_ours(args):
 
     bytes_launch = w.vectors * w.bytes_per_vector()
     step_bytes = 2 * bytes_launch
-    value = step_bytes * K * world / (ms / 1e3) / 1e9
+    value = job_gbps(step_bytes, K, world, ms)
     peak, peak_src = read_peak()
     q_avg, d_avg = statistics.mean(q_ms), statistics.mean(d_ms)
     dom = "quantize" if q_avg >= d_avg else "dequantize"
