@@ -260,28 +260,13 @@ __device__ __forceinline__ void hermitian_out(float Er, float Ei, float Or, floa
   }
 }
 
-// Forward SRFT from fp16: xw[m] holds (x_{2m}, x_{2m+1}), sw[m] the fp16
-// signs (s_{2m}, s_{2m+1}) as +-1.0. Output v[j] = (raw_{2j}, raw_{2j+1}),
-// the unnormalised packed spectrum: raw_0 = X_0, raw_1 = X_L, raw_L / raw_{L+1}
-// = Re / Im Z_{L/2}, and 2 Re X_k / 2 Im X_k elsewhere.
+// Passes 2 .. log2(L) of the forward FFT, the last pass and the Hermitian
+// step, from pass-1 output in the packed bit-reversed arrangement PR / PI
+// (see the file comment) to the unnormalised packed spectrum v.
 template <int D>
-__device__ __forceinline__ void srft_forward(const uint32_t (&xw)[D / 2],
-                                             const uint32_t (&sw)[D / 2], float2 (&v)[D / 2]) {
-  constexpr int L = D / 2, Q = L / 2, LOG = ilog2(L);
-  float2 PR[Q], PI[Q];
-  // pass 1 (span 1) straight from fp16: a_i = z_m, a_{i+1} = z_{m+Q} with
-  // m = bitrev(i), i even; (a_i, a_{i+1}) <- (a_i + a_{i+1}, a_i - a_{i+1}).
-  static_for<0, Q>([&](auto p_) {
-    constexpr int i = 2 * decltype(p_)::value;
-    constexpr int m = bitrev(i, LOG);
-    const uint32_t xa = xw[m], sa = sw[m], xb = xw[m + Q], sb = sw[m + Q];
-    const float tr = fma_f16<0, 0>(xb, sb, 0.0f);
-    const float ti = fma_f16<1, 1>(xb, sb, 0.0f);
-    lane<Q, i>(PR) = fma_f16<0, 0>(xa, sa, tr);
-    lane<Q, i + 1>(PR) = fma_f16<0, 0>(xa, sa, -tr);
-    lane<Q, i>(PI) = fma_f16<1, 1>(xa, sa, ti);
-    lane<Q, i + 1>(PI) = fma_f16<1, 1>(xa, sa, -ti);
-  });
+__device__ __forceinline__ void srft_forward_rest(float2 (&PR)[D / 4], float2 (&PI)[D / 4],
+                                                  float2 (&v)[D / 2]) {
+  constexpr int L = D / 2, Q = L / 2;
   packed_passes<Q, -1, 2>(PR, PI);
 
   // Last pass (span Q) fused with the Hermitian step. Butterfly k gives
@@ -310,6 +295,31 @@ __device__ __forceinline__ void srft_forward(const uint32_t (&xw)[D / 2],
     hermitian_out<D, k>(Er.x, Ei.x, Or.x, Oi.x, v[k], v[L - k]);
     hermitian_out<D, k + Q>(Er.y, Ei.y, Or.y, Oi.y, v[k + Q], v[Q - k]);
   });
+}
+
+// Forward SRFT from fp16: xw[m] holds (x_{2m}, x_{2m+1}), sw[m] the fp16
+// signs (s_{2m}, s_{2m+1}) as +-1.0. Output v[j] = (raw_{2j}, raw_{2j+1}),
+// the unnormalised packed spectrum: raw_0 = X_0, raw_1 = X_L, raw_L / raw_{L+1}
+// = Re / Im Z_{L/2}, and 2 Re X_k / 2 Im X_k elsewhere.
+template <int D>
+__device__ __forceinline__ void srft_forward(const uint32_t (&xw)[D / 2],
+                                             const uint32_t (&sw)[D / 2], float2 (&v)[D / 2]) {
+  constexpr int L = D / 2, Q = L / 2, LOG = ilog2(L);
+  float2 PR[Q], PI[Q];
+  // pass 1 (span 1) straight from fp16: a_i = z_m, a_{i+1} = z_{m+Q} with
+  // m = bitrev(i), i even; (a_i, a_{i+1}) <- (a_i + a_{i+1}, a_i - a_{i+1}).
+  static_for<0, Q>([&](auto p_) {
+    constexpr int i = 2 * decltype(p_)::value;
+    constexpr int m = bitrev(i, LOG);
+    const uint32_t xa = xw[m], sa = sw[m], xb = xw[m + Q], sb = sw[m + Q];
+    const float tr = fma_f16<0, 0>(xb, sb, 0.0f);
+    const float ti = fma_f16<1, 1>(xb, sb, 0.0f);
+    lane<Q, i>(PR) = fma_f16<0, 0>(xa, sa, tr);
+    lane<Q, i + 1>(PR) = fma_f16<0, 0>(xa, sa, -tr);
+    lane<Q, i>(PI) = fma_f16<1, 1>(xa, sa, ti);
+    lane<Q, i + 1>(PI) = fma_f16<1, 1>(xa, sa, -ti);
+  });
+  srft_forward_rest<D>(PR, PI, v);
 }
 
 // Inverse SRFT: input v[j] = (c_{2j}, c_{2j+1}) with c_j = coordinate gain

@@ -119,7 +119,7 @@ def test_ragged_rows_and_heads(N, H):
 
 
 @pytest.mark.parametrize("H", [2, 4, 6, 8, 12, 16])
-@pytest.mark.parametrize("d,bits,group", [(64, 4, 16), (128, 8, 32)])
+@pytest.mark.parametrize("d,bits,group", [(64, 4, 16), (128, 8, 32), (256, 4, 32), (256, 8, 64)])
 def test_head_block_tiles(H, d, bits, group):
     """Tiles span up to 8 heads of 32 / heads-per-tile rows; cover every
     heads-per-tile value, several head blocks per slice and ragged rows."""
