@@ -4,6 +4,7 @@
 // calibration reads n_cal rows per (slice, head) once).
 #pragma once
 
+#include <cooperative_groups.h>
 #include <cuda_fp16.h>
 
 #include "codec.cuh"
@@ -78,20 +79,32 @@ struct CalibArgs {
   float* lambda_out;
 };
 
-constexpr int kCalibRows = 64;  // rows rotated per batch
+constexpr int kCalibRows = 64;     // rows rotated per batch
+constexpr int kCalibCluster = 8;   // blocks (a thread-block cluster) per (slice, head)
 
-// One block per (slice, head). Threads 0..63 rotate one row each per batch
-// and write y^2 to shared memory; then thread j adds column j over the
-// batch's rows, in row order, into a float64 accumulator. The order of every
-// addition is fixed, so the result does not depend on scheduling.
+// One cluster of kCalibCluster blocks per (slice, head); block r of the
+// cluster takes the batches of 64 rows starting at 64 (r + kCalibCluster b),
+// so n_cal = 512 is one batch per block. Threads 0..63 rotate one row each
+// and write y^2 to shared memory; thread j then adds column j over the
+// batch's rows, in row order, into a float64 accumulator. Rank 0 adds the
+// blocks' partial sums in rank order, reading them from the other blocks'
+// shared memory (distributed shared memory of the cluster). Every addition
+// happens in a fixed order, so the result does not depend on scheduling.
 template <int D, int ROT>
-__global__ void __launch_bounds__(128) calibrate_kernel(const CalibArgs a) {
+__global__ void __cluster_dims__(kCalibCluster, 1, 1) __launch_bounds__(128)
+    calibrate_kernel(const CalibArgs a) {
   __shared__ float sq[kCalibRows][D + 1];
-  const int s = blockIdx.x / a.heads;
-  const int h = blockIdx.x % a.heads;
+  __shared__ double part[D];
+  namespace cg = cooperative_groups;
+  cg::cluster_group cluster = cg::this_cluster();
+  const int rank = static_cast<int>(cluster.block_rank());
+  const int sh = blockIdx.x / kCalibCluster;
+  const int s = sh / a.heads;
+  const int h = sh % a.heads;
   const int64_t tab = (int64_t(s) * a.heads + h) * D;
   double acc = 0.0;
-  for (int64_t base = 0; base < a.n_cal; base += kCalibRows) {
+  for (int64_t base = int64_t(kCalibRows) * rank; base < a.n_cal;
+       base += int64_t(kCalibRows) * kCalibCluster) {
     if (threadIdx.x < kCalibRows) {
       const int64_t r = base + threadIdx.x;
       if (r < a.n_cal) {
@@ -117,10 +130,15 @@ __global__ void __launch_bounds__(128) calibrate_kernel(const CalibArgs a) {
     }
     __syncthreads();
   }
-  if (threadIdx.x < D) {
+  if (threadIdx.x < D) part[threadIdx.x] = acc;
+  cluster.sync();
+  if (rank == 0 && threadIdx.x < D) {
+    double total = 0.0;
+    for (int r = 0; r < kCalibCluster; ++r) total += cluster.map_shared_rank(part, r)[threadIdx.x];
     a.lambda_out[tab + threadIdx.x] =
-        acc > 0.0 ? float(sqrt(acc / double(a.n_cal))) : 1.0f;
+        total > 0.0 ? float(sqrt(total / double(a.n_cal))) : 1.0f;
   }
+  cluster.sync();   // the other blocks keep their shared memory until rank 0 is done
 }
 
 }  // namespace srftq

@@ -99,17 +99,27 @@ __global__ void __launch_bounds__(128) rotate256_kernel(const RotateArgs a) {
   }
 }
 
-// One block per (slice, head): 64 rows per batch, two threads per row.
+// One cluster of kCalibCluster blocks per (slice, head), block r taking the
+// batches of 64 rows starting at 64 (r + kCalibCluster b); two threads per
+// row; rank 0 adds the blocks' float64 partial sums in rank order through
+// distributed shared memory (as calibrate_kernel).
 template <int ROT>
-__global__ void __launch_bounds__(128) calibrate256_kernel(const CalibArgs a) {
+__global__ void __cluster_dims__(kCalibCluster, 1, 1) __launch_bounds__(128)
+    calibrate256_kernel(const CalibArgs a) {
   __shared__ float sq[kCalibRows / 2][257];
-  const int s = blockIdx.x / a.heads;
-  const int h = blockIdx.x % a.heads;
+  __shared__ double part[256];
+  namespace cg = cooperative_groups;
+  cg::cluster_group cluster = cg::this_cluster();
+  const int rank = static_cast<int>(cluster.block_rank());
+  const int shd = blockIdx.x / kCalibCluster;
+  const int s = shd / a.heads;
+  const int h = shd % a.heads;
   const int64_t tab = (int64_t(s) * a.heads + h) * 256;
   const bool p = threadIdx.x & 1;
   const int rl = threadIdx.x >> 1;   // row within a batch of 64 (two threads per row)
   double acc0 = 0.0, acc1 = 0.0;
-  for (int64_t b = 0; b < a.n_cal; b += 64) {
+  for (int64_t b = int64_t(kCalibRows) * rank; b < a.n_cal;
+       b += int64_t(kCalibRows) * kCalibCluster) {
     const int64_t rr = b + rl;
     const bool valid = rr < a.n_cal;
     const int64_t rc = valid ? rr : 0;
@@ -136,10 +146,20 @@ __global__ void __launch_bounds__(128) calibrate256_kernel(const CalibArgs a) {
       __syncthreads();
     }
   }
-  a.lambda_out[tab + threadIdx.x] =
-      acc0 > 0.0 ? float(sqrt(acc0 / double(a.n_cal))) : 1.0f;
-  a.lambda_out[tab + threadIdx.x + 128] =
-      acc1 > 0.0 ? float(sqrt(acc1 / double(a.n_cal))) : 1.0f;
+  part[threadIdx.x] = acc0;
+  part[threadIdx.x + 128] = acc1;
+  cluster.sync();
+  if (rank == 0) {
+    double t0 = 0.0, t1 = 0.0;
+    for (int r = 0; r < kCalibCluster; ++r) {
+      const double* q = cluster.map_shared_rank(part, r);
+      t0 += q[threadIdx.x];
+      t1 += q[threadIdx.x + 128];
+    }
+    a.lambda_out[tab + threadIdx.x] = t0 > 0.0 ? float(sqrt(t0 / double(a.n_cal))) : 1.0f;
+    a.lambda_out[tab + threadIdx.x + 128] = t1 > 0.0 ? float(sqrt(t1 / double(a.n_cal))) : 1.0f;
+  }
+  cluster.sync();   // the other blocks keep their shared memory until rank 0 is done
 }
 
 }  // namespace srftq

@@ -260,7 +260,7 @@ int launch_rotate(const RotateCall& c) {
 
 template <int D>
 int launch_calibrate(const CalibCall& c) {
-  const int64_t blocks = c.n_slices * c.heads;
+  const int64_t blocks = c.n_slices * c.heads * kCalibCluster;   // one cluster per (slice, head)
   if (blocks == 0) return SRFTQ_OK;
   if (blocks > INT_MAX) return SRFTQ_ERR_UNSUPPORTED;
   CalibArgs a{c.n_cal, c.x_slice_stride_rows, c.heads, c.x, c.signs, c.lambda_out};

@@ -131,6 +131,23 @@ def test_head_block_tiles(H, d, bits, group):
     run_and_check(x16, signs, lam, d, group, bits, rq.SRFT, f"H{H} d{d}")
 
 
+@pytest.mark.parametrize("n_cal", [1, 64, 100, 512, 700, 1100])
+@pytest.mark.parametrize("d", [64, 256])
+def test_calibration_row_counts(n_cal, d):
+    """Calibration runs one 8-block cluster per (slice, head), block r taking
+    the 64-row batches 64 (r + 8 b): cover fewer rows than one batch, ragged
+    batches, exactly one batch per block and several batches per block."""
+    rng = np.random.default_rng(n_cal + d)
+    S, H = 2, 3
+    x16 = _x(rng, S, max(n_cal, 8), H, d)
+    signs = _signs(rng, S, H, d)
+    for rot in (rq.SRFT, rq.SRHT):
+        lam_gpu = rq.calibrate_lambda(_t(x16), _t(signs), n_cal, rotation=rot).cpu().numpy()
+        parity.assert_clean(
+            parity.check_lambda(lam_gpu, oracle.calibrate_lambda(x16, signs, n_cal, rot)),
+            f"lambda n_cal={n_cal} d={d} rot={rot}")
+
+
 @pytest.mark.parametrize("N", [1, 15, 16, 17, 47])
 @pytest.mark.parametrize("rot", [0, 1])
 def test_ragged_rows_d256(N, rot):
