@@ -81,13 +81,19 @@ KERNEL_SOURCES = {
                         "launch_impl.cuh"),
     "dequantize_kernel": ("codec.cuh", "transform.cuh", "common.cuh", "ptx.cuh", "launch.cuh",
                           "launch_impl.cuh"),
-    "quantize256_kernel": ("codec256.cuh", "transform256.cuh", "codec.cuh", "transform.cuh",
-                           "common.cuh", "ptx.cuh", "launch.cuh", "launch_impl.cuh",
-                           "launch_d256.cu"),
-    "dequantize256_kernel": ("codec256.cuh", "transform256.cuh", "codec.cuh", "transform.cuh",
-                             "common.cuh", "ptx.cuh", "launch.cuh", "launch_impl.cuh",
-                             "launch_d256.cu"),
+    "quantize_split_kernel": ("codec_split.cuh", "codec.cuh", "transform.cuh", "common.cuh",
+                              "ptx.cuh", "launch.cuh", "launch_impl.cuh", "launch_split.cuh",
+                              "launch_d256.cu"),
+    "dequantize_split_kernel": ("codec_split.cuh", "codec.cuh", "transform.cuh", "common.cuh",
+                                "ptx.cuh", "launch.cuh", "launch_impl.cuh", "launch_split.cuh",
+                                "launch_d256.cu"),
 }
+
+
+def codec_kernel(kind: str, d: int) -> str:
+    """Name of the kernel that runs `kind` ("quantize" / "dequantize") for a
+    head dimension: d = 256 runs on the two-warp kernels."""
+    return f"{kind}{'_split' if d == 256 else ''}_kernel"
 
 
 def csrc_hash(kernel: str) -> str:
@@ -375,7 +381,7 @@ def run_ours(args):
     dom = "quantize" if q_avg >= d_avg else "dequantize"
     dom_ms = max(q_avg, d_avg)
     achieved = bytes_launch / (dom_ms / 1e3) / 1e9
-    kname = f"{dom}{'256' if w.d == 256 else ''}_kernel"
+    kname = codec_kernel(dom, w.d)
 
     e2e = None
     if not args.no_e2e:
@@ -604,12 +610,13 @@ def run_decode(args):
         "kernels": {"dequantize_ms_per_layer": d_avg,
                     "dequantize_GBps": achieved,
                     "launches_per_step": 2 * L},
-        "roofline": {"bound": "hbm", "kernel": "dequantize_kernel", "achieved": achieved,
+        "roofline": {"bound": "hbm", "kernel": codec_kernel("dequantize", w.d),
+                     "achieved": achieved,
                      "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)"
                      if peak_src == "measured" else "fallback 6.65 TB/s",
                      "algorithmic_bytes_per_launch": deq_bytes,
-                     "traffic": read_traffic("dequantize_kernel", w.name)},
+                     "traffic": read_traffic(codec_kernel("dequantize", w.d), w.name)},
         "gpu_launches": 2 * L * K,
         "clocks": clk,
     }

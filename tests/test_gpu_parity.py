@@ -119,7 +119,8 @@ def test_ragged_rows_and_heads(N, H):
 
 
 @pytest.mark.parametrize("H", [2, 4, 6, 8, 12, 16])
-@pytest.mark.parametrize("d,bits,group", [(64, 4, 16), (128, 8, 32), (256, 4, 32), (256, 8, 64)])
+@pytest.mark.parametrize("d,bits,group", [(64, 4, 16), (128, 4, 16), (128, 8, 32), (128, 4, 64),
+                                           (256, 4, 32), (256, 8, 64)])
 def test_head_block_tiles(H, d, bits, group):
     """Tiles span up to 8 heads of 32 / heads-per-tile rows; cover every
     heads-per-tile value, several head blocks per slice and ragged rows."""
@@ -150,14 +151,17 @@ def test_calibration_row_counts(n_cal, d):
 
 @pytest.mark.parametrize("N", [1, 15, 16, 17, 47])
 @pytest.mark.parametrize("rot", [0, 1])
-def test_ragged_rows_d256(N, rot):
-    """d = 256 runs 16-row tiles with two threads per vector."""
-    rng = np.random.default_rng(N * 11 + rot)
-    d, group, bits, H = 256, 32, 4, 3
+@pytest.mark.parametrize("d,group", [(128, 16), (256, 32)])
+def test_ragged_rows_d128_d256(N, rot, d, group):
+    """Ragged row counts leave part of the last tile empty: at d = 128 (one
+    thread per vector) and at d = 256 (two warps sharing a tile, both of
+    which must skip the missing rows)."""
+    rng = np.random.default_rng(N * 11 + rot + d)
+    bits, H = 4, 3
     x16 = _x(rng, 2, N, H, d, outlier_p=0.005, scale=25.0)
     signs = _signs(rng, 2, H, d)
     lam = np.exp(rng.uniform(-1, 1, (2, H, d))).astype(np.float32)
-    run_and_check(x16, signs, lam, d, group, bits, rot, f"d256 N{N} r{rot}")
+    run_and_check(x16, signs, lam, d, group, bits, rot, f"d{d} N{N} r{rot}")
 
 
 def test_unsupported_groups_d256():
