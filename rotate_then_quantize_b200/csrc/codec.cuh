@@ -342,22 +342,23 @@ __device__ __forceinline__ void group_scales(const float (&am)[NG], uint32_t (&s
 // its tile range). QUANT: multiplier gain_j / lambda_j and fp16 +-1 sign
 // pairs; otherwise multiplier gain_j * lambda_j (int4: / 16 at odd j,
 // matching the x16 of the odd codes' unpacking) and fp16 sign-bit masks.
-template <int D, int BITS, int ROT, bool QUANT, int MS, int SS>
+template <int D, int BITS, int ROT, bool QUANT, int MS, int SS, bool MULT = true,
+          bool SIGNS = true>
 __device__ __forceinline__ void build_tables(float* mult, uint32_t* stab, const float* lambda,
                                              const int8_t* signs, int s, int hb, int H,
                                              int hpt_log2, int lane) {
   // The HPT heads' lambda rows (HPT * D floats) and sign rows (HPT * D
   // bytes) are contiguous; every lane issues all of its 16-byte loads before
   // using any, so a rebuild costs one memory round trip.
-  constexpr int kL4 = (kMaxHPT * D / 4 + 31) / 32;    // float4 loads per lane, at most
-  constexpr int kS16 = (kMaxHPT * D / 16 + 31) / 32;  // 16-sign loads per lane, at most
+  constexpr int kL4 = MULT ? (kMaxHPT * D / 4 + 31) / 32 : 0;    // float4 loads per lane, at most
+  constexpr int kS16 = SIGNS ? (kMaxHPT * D / 16 + 31) / 32 : 0;  // 16-sign loads per lane, at most
   const int hpt = 1 << hpt_log2;
   const size_t h0 = static_cast<size_t>(s) * H + static_cast<size_t>(hb) * hpt;
   const float4* lam4 = reinterpret_cast<const float4*>(lambda + h0 * D);
   const uint4* sg16 = reinterpret_cast<const uint4*>(signs + h0 * D);
   const int n4 = (hpt * D) / 4, n16 = (hpt * D) / 16;
-  float4 l[kL4];
-  uint4 g[kS16];
+  float4 l[kL4 > 0 ? kL4 : 1];
+  uint4 g[kS16 > 0 ? kS16 : 1];
 #pragma unroll
   for (int k = 0; k < kL4; ++k) {
     const int i = lane + 32 * k;
@@ -401,6 +402,80 @@ __device__ __forceinline__ void build_tables(float* mult, uint32_t* stab, const 
     }
   }
   __syncwarp();
+}
+
+// Group absmax -> fp16 scales -> codes of one vector w (pairs v[p] =
+// (w_{2p}, w_{2p+1}), already divided by lambda): sw = the packed fp16 scale
+// pairs, words = the packed codes (int4: byte k = code 2k in the low nibble,
+// code 2k+1 in the high nibble; int8: one byte per code).
+template <int D, int BITS, int G>
+__device__ __forceinline__ void quantize_codes(const float2 (&v)[D / 2],
+                                               uint32_t (&sw)[Shape<D, BITS, G>::SW],
+                                               uint32_t (&words)[Shape<D, BITS, G>::CW]) {
+  using S = Shape<D, BITS, G>;
+  // Group absmax -> fp16 scale -> codes as float-encoded integers.
+  // When every group's scale is a normal fp16 and no a_g / qmax exceeds
+  // 65504, |w / sigma| <= qmax * (1 + 2^-10) up to rounding, which rounds
+  // inside the range: that common case (decided once per vector from the
+  // largest and smallest absmax) runs without clamps; a vector with a zero,
+  // subnormal-scale or saturating group takes the clamped block.
+  float am[S::NG];
+  static_for<0, S::NG>([&](auto g_) {
+    constexpr int g = decltype(g_)::value;
+    constexpr int P0 = g * G / 2;   // first pair of the group
+    float m = absmax3(0.0f, v[P0].x, v[P0].y);
+    static_for<1, G / 2>([&](auto p_) {
+      constexpr int p = P0 + decltype(p_)::value;
+      m = absmax3(m, v[p].x, v[p].y);
+    });
+    am[g] = m;
+  });
+  float a_hi, a_lo;
+  range_of(am, a_hi, a_lo);
+  constexpr float kHi = 65504.0f * float(S::QMAX);            // no saturation
+  constexpr float kLo = 6.103515625e-05f * float(S::QMAX);    // sigma >= 2^-14
+  uint32_t qb[D];
+  if (a_hi <= kHi && a_lo >= kLo) {
+    float invs[S::NG];
+    group_scales<S::NG, S::QMAX, true>(am, sw, invs);
+    static_for<0, D / 2>([&](auto p_) {
+      constexpr int p = decltype(p_)::value;
+      const float2 r = fma2(v[p], splat(invs[(2 * p) / G]), splat(kMagic));
+      qb[2 * p] = __float_as_uint(r.x);
+      qb[2 * p + 1] = __float_as_uint(r.y);
+    });
+  } else {
+    float invs[S::NG];
+    group_scales<S::NG, S::QMAX, false>(am, sw, invs);
+    static_for<0, D / 2>([&](auto p_) {
+      constexpr int p = decltype(p_)::value;
+      const float inv = invs[(2 * p) / G];
+      const float q0 = fminf(fmaxf(v[p].x * inv, -float(S::QMAX)), float(S::QMAX));
+      const float q1 = fminf(fmaxf(v[p].y * inv, -float(S::QMAX)), float(S::QMAX));
+      qb[2 * p] = __float_as_uint(q0 + kMagic);
+      qb[2 * p + 1] = __float_as_uint(q1 + kMagic);
+    });
+  }
+
+  // Pack. The low byte of every qb is its code in two's complement.
+  // int4: byte k = code 2k in the low nibble | code 2k+1 in the high nibble;
+  // gather the even and the odd codes' bytes, then merge the nibbles.
+  if constexpr (BITS == 4) {
+    static_for<0, D / 8>([&](auto m_) {
+      constexpr int m = decltype(m_)::value;
+      const uint32_t ev = __byte_perm(__byte_perm(qb[8 * m + 0], qb[8 * m + 2], 0x0040),
+                                      __byte_perm(qb[8 * m + 4], qb[8 * m + 6], 0x0040), 0x5410);
+      const uint32_t od = __byte_perm(__byte_perm(qb[8 * m + 1], qb[8 * m + 3], 0x0040),
+                                      __byte_perm(qb[8 * m + 5], qb[8 * m + 7], 0x0040), 0x5410);
+      words[m] = (ev & 0x0F0F0F0Fu) | ((od << 4) & 0xF0F0F0F0u);
+    });
+  } else {
+    static_for<0, D / 4>([&](auto m_) {
+      constexpr int m = decltype(m_)::value;
+      words[m] = __byte_perm(__byte_perm(qb[4 * m], qb[4 * m + 1], 0x0040),
+                             __byte_perm(qb[4 * m + 2], qb[4 * m + 3], 0x0040), 0x5410);
+    });
+  }
 }
 
 template <int D, int BITS, int G, int ROT, int WPC, int NST, int MINB>
@@ -536,71 +611,10 @@ __global__ void __launch_bounds__(WPC * 32, MINB)
       v[2 * ci + 1] = mul2(v[2 * ci + 1], make_float2(m4.z, m4.w));
     });
 
-    // (d) group absmax -> fp16 scale -> codes as float-encoded integers.
-    // When every group's scale is a normal fp16 and no a_g / qmax exceeds
-    // 65504, |w / sigma| <= qmax * (1 + 2^-10) up to rounding, which rounds
-    // inside the range: that common case (decided once per vector from the
-    // largest and smallest absmax) runs without clamps; a vector with a zero,
-    // subnormal-scale or saturating group takes the clamped block.
-    float am[S::NG];
-    static_for<0, S::NG>([&](auto g_) {
-      constexpr int g = decltype(g_)::value;
-      constexpr int P0 = g * G / 2;   // first pair of the group
-      float m = absmax3(0.0f, v[P0].x, v[P0].y);
-      static_for<1, G / 2>([&](auto p_) {
-        constexpr int p = P0 + decltype(p_)::value;
-        m = absmax3(m, v[p].x, v[p].y);
-      });
-      am[g] = m;
-    });
-    float a_hi, a_lo;
-    range_of(am, a_hi, a_lo);
-    constexpr float kHi = 65504.0f * float(S::QMAX);            // no saturation
-    constexpr float kLo = 6.103515625e-05f * float(S::QMAX);    // sigma >= 2^-14
-    uint32_t sw[(S::NG + 1) / 2];
-    uint32_t qb[D];
-    if (a_hi <= kHi && a_lo >= kLo) {
-      float invs[S::NG];
-      group_scales<S::NG, S::QMAX, true>(am, sw, invs);
-      static_for<0, D / 2>([&](auto p_) {
-        constexpr int p = decltype(p_)::value;
-        const float2 r = fma2(v[p], splat(invs[(2 * p) / G]), splat(kMagic));
-        qb[2 * p] = __float_as_uint(r.x);
-        qb[2 * p + 1] = __float_as_uint(r.y);
-      });
-    } else {
-      float invs[S::NG];
-      group_scales<S::NG, S::QMAX, false>(am, sw, invs);
-      static_for<0, D / 2>([&](auto p_) {
-        constexpr int p = decltype(p_)::value;
-        const float inv = invs[(2 * p) / G];
-        const float q0 = fminf(fmaxf(v[p].x * inv, -float(S::QMAX)), float(S::QMAX));
-        const float q1 = fminf(fmaxf(v[p].y * inv, -float(S::QMAX)), float(S::QMAX));
-        qb[2 * p] = __float_as_uint(q0 + kMagic);
-        qb[2 * p + 1] = __float_as_uint(q1 + kMagic);
-      });
-    }
-
-    // (e) pack. The low byte of every qb is its code in two's complement.
-    // int4: byte k = code 2k in the low nibble | code 2k+1 in the high nibble;
-    // gather the even and the odd codes' bytes, then merge the nibbles.
+    // (d), (e) scales and packed codes
+    uint32_t sw[S::SW];
     uint32_t words[S::CW];
-    if constexpr (BITS == 4) {
-      static_for<0, D / 8>([&](auto m_) {
-        constexpr int m = decltype(m_)::value;
-        const uint32_t ev = __byte_perm(__byte_perm(qb[8 * m + 0], qb[8 * m + 2], 0x0040),
-                                        __byte_perm(qb[8 * m + 4], qb[8 * m + 6], 0x0040), 0x5410);
-        const uint32_t od = __byte_perm(__byte_perm(qb[8 * m + 1], qb[8 * m + 3], 0x0040),
-                                        __byte_perm(qb[8 * m + 5], qb[8 * m + 7], 0x0040), 0x5410);
-        words[m] = (ev & 0x0F0F0F0Fu) | ((od << 4) & 0xF0F0F0F0u);
-      });
-    } else {
-      static_for<0, D / 4>([&](auto m_) {
-        constexpr int m = decltype(m_)::value;
-        words[m] = __byte_perm(__byte_perm(qb[4 * m], qb[4 * m + 1], 0x0040),
-                               __byte_perm(qb[4 * m + 2], qb[4 * m + 3], 0x0040), 0x5410);
-      });
-    }
+    quantize_codes<D, BITS, G>(v, sw, words);
 
     const int row = cur.rb * rpt + rl;
     const bool valid = row < a.g.n_rows;
