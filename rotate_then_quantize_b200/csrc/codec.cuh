@@ -342,23 +342,22 @@ __device__ __forceinline__ void group_scales(const float (&am)[NG], uint32_t (&s
 // its tile range). QUANT: multiplier gain_j / lambda_j and fp16 +-1 sign
 // pairs; otherwise multiplier gain_j * lambda_j (int4: / 16 at odd j,
 // matching the x16 of the odd codes' unpacking) and fp16 sign-bit masks.
-template <int D, int BITS, int ROT, bool QUANT, int MS, int SS, bool MULT = true,
-          bool SIGNS = true>
+template <int D, int BITS, int ROT, bool QUANT, int MS, int SS>
 __device__ __forceinline__ void build_tables(float* mult, uint32_t* stab, const float* lambda,
                                              const int8_t* signs, int s, int hb, int H,
                                              int hpt_log2, int lane) {
   // The HPT heads' lambda rows (HPT * D floats) and sign rows (HPT * D
   // bytes) are contiguous; every lane issues all of its 16-byte loads before
   // using any, so a rebuild costs one memory round trip.
-  constexpr int kL4 = MULT ? (kMaxHPT * D / 4 + 31) / 32 : 0;    // float4 loads per lane, at most
-  constexpr int kS16 = SIGNS ? (kMaxHPT * D / 16 + 31) / 32 : 0;  // 16-sign loads per lane, at most
+  constexpr int kL4 = (kMaxHPT * D / 4 + 31) / 32;    // float4 loads per lane, at most
+  constexpr int kS16 = (kMaxHPT * D / 16 + 31) / 32;  // 16-sign loads per lane, at most
   const int hpt = 1 << hpt_log2;
   const size_t h0 = static_cast<size_t>(s) * H + static_cast<size_t>(hb) * hpt;
   const float4* lam4 = reinterpret_cast<const float4*>(lambda + h0 * D);
   const uint4* sg16 = reinterpret_cast<const uint4*>(signs + h0 * D);
   const int n4 = (hpt * D) / 4, n16 = (hpt * D) / 16;
-  float4 l[kL4 > 0 ? kL4 : 1];
-  uint4 g[kS16 > 0 ? kS16 : 1];
+  float4 l[kL4];
+  uint4 g[kS16];
 #pragma unroll
   for (int k = 0; k < kL4; ++k) {
     const int i = lane + 32 * k;

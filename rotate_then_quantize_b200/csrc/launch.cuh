@@ -74,9 +74,6 @@ template <int D> int launch_dequantize(const DequantCall& c);
 template <int D> int launch_rotate(const RotateCall& c);
 template <int D> int launch_calibrate(const CalibCall& c);
 
-// d = 128 quantises SRFT on the tensor cores (launch_d128.cu).
-template <> int launch_quantize<128>(const QuantCall& c);
-
 // d = 256 has its own kernels (two threads per vector; launch_d256.cu).
 template <> int launch_quantize<256>(const QuantCall& c);
 template <> int launch_dequantize<256>(const DequantCall& c);
