@@ -373,6 +373,8 @@ def run_ours(args):
     if rq.srftq_check_device() != 0:
         raise RuntimeError("device guard fired during the timed steps")
 
+    quality = round_trip_error(x, xhat)
+
     bytes_launch = w.vectors * w.bytes_per_vector()
     step_bytes = 2 * bytes_launch
     value = job_gbps(step_bytes, K, world, ms)
@@ -427,6 +429,7 @@ def run_ours(args):
                      "traffic": read_traffic(kname, w.name)},
         "gpu_launches": 3 * K,
         "clocks": clk,
+        "quality": quality,
     }
     if e2e is not None:
         line["e2e"] = e2e
@@ -438,6 +441,32 @@ def run_ours(args):
         pg.barrier()
         pg.destroy_process_group()
     return 0
+
+
+def round_trip_error(x, xhat, chunk_rows: int = 4096) -> dict:
+    """Per-vector relative L2 error ||xhat - x|| / ||x|| of the last step's
+    round trip (quantize then dequantize), outside the timed region:
+    mean, median, 99th percentile and maximum over every vector with a
+    non-zero norm. Computed in float32 slice by slice."""
+    import torch
+
+    errs = []
+    d = x.shape[-1]
+    xf, hf = x.reshape(-1, d), xhat.reshape(-1, d)
+    for i in range(0, xf.shape[0], chunk_rows * 64):
+        a = xf[i:i + chunk_rows * 64].float()
+        b = hf[i:i + chunk_rows * 64].float()
+        n = a.norm(dim=1)
+        keep = n > 0
+        errs.append(((b - a).norm(dim=1)[keep] / n[keep]).cpu())
+    e = torch.cat(errs)
+    if e.numel() == 0:
+        return {"rel_l2_mean": None}
+    q = torch.quantile(e[torch.randperm(e.numel())[:1 << 24]] if e.numel() > (1 << 24) else e,
+                       torch.tensor([0.5, 0.99]))
+    return {"rel_l2_mean": float(e.mean()), "rel_l2_p50": float(q[0]),
+            "rel_l2_p99": float(q[1]), "rel_l2_max": float(e.max()), "vectors": int(e.numel()),
+            "what": "per-vector ||xhat - x|| / ||x|| of the last timed step"}
 
 
 # ---------------------------------------------------------------------------

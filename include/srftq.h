@@ -160,6 +160,19 @@ const char* srftq_status_string(int status);
  */
 int srftq_check_device(void* stream);
 
+/*
+ * srftq_probe_wait_timeout -- exercises the device-side failure path. Launches
+ * one thread that waits on a shared-memory barrier nothing ever arrives on,
+ * polling it `polls` times (1 <= polls <= 4194304, the codec kernels' own
+ * limit) before it gives up and records the timeout in the guard word, as
+ * every codec kernel does when one of its waits runs out. Nothing faults and
+ * the context stays usable: the next srftq_check_device on the same stream
+ * returns SRFTQ_ERR_DEVICE_CHECK (and clears the word). Returns
+ * SRFTQ_ERR_INVALID_ARG for `polls` out of range, SRFTQ_ERR_CUDA if the
+ * launch fails, else SRFTQ_OK (launched, asynchronous).
+ */
+int srftq_probe_wait_timeout(uint32_t polls, void* stream);
+
 /* Library version as 10000*major + 100*minor + patch. */
 int srftq_version(void);
 

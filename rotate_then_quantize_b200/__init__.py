@@ -21,6 +21,7 @@ from .binding import (  # noqa: F401
     srftq_calibrate_lambda,
     srftq_check_device,
     srftq_dequantize,
+    srftq_probe_wait_timeout,
     srftq_quantize,
     srftq_rotate,
     srftq_version,

@@ -33,7 +33,8 @@ SRHT = 1
 
 # Every symbol include/srftq.h declares (checked by the CPU test suite).
 EXPORTED = ("srftq_quantize", "srftq_dequantize", "srftq_calibrate_lambda", "srftq_rotate",
-            "srftq_status_string", "srftq_check_device", "srftq_version")
+            "srftq_status_string", "srftq_check_device", "srftq_probe_wait_timeout",
+            "srftq_version")
 
 
 class SrftqDesc(ctypes.Structure):
@@ -68,9 +69,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.srftq_status_string.argtypes = [I32]
     lib.srftq_status_string.restype = ctypes.c_char_p
     lib.srftq_check_device.argtypes = [P]
+    lib.srftq_probe_wait_timeout.argtypes = [ctypes.c_uint32, P]
     lib.srftq_version.argtypes = []
     for name in ("srftq_quantize", "srftq_dequantize", "srftq_calibrate_lambda", "srftq_rotate",
-                 "srftq_check_device", "srftq_version"):
+                 "srftq_check_device", "srftq_probe_wait_timeout", "srftq_version"):
         getattr(lib, name).restype = I32
     _lib = lib
     return lib
@@ -168,6 +170,11 @@ def srftq_rotate(desc: SrftqDesc, x, signs, y_out, lam=None, stream=None) -> Non
                           _table(signs, S, desc.heads, desc.d, "signs"), pl, y_out.data_ptr(),
                           _stream_handle(stream))
     _check("srftq_rotate", st)
+
+
+def srftq_probe_wait_timeout(polls: int, stream=None) -> int:
+    """Launches the device-side timeout probe (see include/srftq.h); returns the status."""
+    return int(load_library().srftq_probe_wait_timeout(int(polls), _stream_handle(stream)))
 
 
 def srftq_check_device(stream=None) -> int:

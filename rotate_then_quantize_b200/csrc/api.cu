@@ -10,9 +10,23 @@
 #include "../../include/srftq.h"
 #include "common.cuh"
 #include "launch.cuh"
+#include "ptx.cuh"
 
 // Library-wide device guard word (one per device that loads the module).
 __device__ unsigned g_srftq_guard;
+
+namespace srftq {
+// One thread waits on a barrier that nothing arrives on, `polls` times at
+// most, then records the timeout like the codec kernels' bounded waits.
+__global__ void probe_wait_timeout_kernel(unsigned* guard, uint32_t polls) {
+  __shared__ uint64_t bar;
+  mbar_init(&bar, 1);
+  fence_barrier_init();
+  for (uint32_t i = 0; i < polls; ++i)
+    if (mbar_try_wait(&bar, 0)) return;
+  atomicOr(guard, kGuardWaitTimeout);
+}
+}  // namespace srftq
 
 namespace srftq {
 namespace {
@@ -249,6 +263,14 @@ int srftq_check_device(void* stream) {
   const unsigned zero = 0;
   if (cudaMemcpyToSymbol(g_srftq_guard, &zero, sizeof(zero)) != cudaSuccess) return SRFTQ_ERR_CUDA;
   return SRFTQ_ERR_DEVICE_CHECK;
+}
+
+int srftq_probe_wait_timeout(uint32_t polls, void* stream) {
+  if (polls == 0 || polls > srftq::kWaitLimit) return SRFTQ_ERR_INVALID_ARG;
+  unsigned* guard = srftq::Runtime::guard_word();
+  if (!guard) return SRFTQ_ERR_CUDA;
+  srftq::probe_wait_timeout_kernel<<<1, 1, 0, static_cast<cudaStream_t>(stream)>>>(guard, polls);
+  return cudaGetLastError() == cudaSuccess ? SRFTQ_OK : SRFTQ_ERR_CUDA;
 }
 
 int srftq_version(void) { return 100; }

@@ -45,6 +45,12 @@ def test_library_exports_every_declared_symbol(lib):
         assert hasattr(lib, name)
 
 
+def test_timeout_probe_rejects_out_of_range_polls(lib):
+    # validated before any launch: no GPU is touched
+    assert lib.srftq_probe_wait_timeout(0, None) == b.SRFTQ_ERR_INVALID_ARG
+    assert lib.srftq_probe_wait_timeout((1 << 22) + 1, None) == b.SRFTQ_ERR_INVALID_ARG
+
+
 def test_version_and_status_strings(lib):
     assert rq.srftq_version() >= 100
     for st in (0, -1, -2, -3, -4, -5):

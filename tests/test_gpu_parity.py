@@ -249,6 +249,23 @@ def test_non_finite_inputs_do_not_fault():
                                            _np16(scales)[:, clean], 4, 16), "finite rows")
 
 
+def test_bounded_wait_that_runs_out_is_reported_and_the_context_stays_usable():
+    """Failure detection without a fault: a wait on a barrier nothing arrives
+    on gives up after its poll limit, records the timeout in the guard word
+    (as every codec kernel's bounded wait does), and the next check reports
+    it; the same context then runs a codec call cleanly."""
+    assert rq.srftq_check_device() == 0
+    assert rq.srftq_probe_wait_timeout(1 << 12) == 0
+    assert rq.srftq_check_device() == rq.binding.SRFTQ_ERR_DEVICE_CHECK
+    assert rq.srftq_check_device() == 0          # the check cleared the word
+    rng = np.random.default_rng(5)
+    x16 = _x(rng, 1, 40, 2, 128)
+    signs = _signs(rng, 1, 2, 128)
+    lam = np.exp(rng.uniform(-1, 1, (1, 2, 128))).astype(np.float32)
+    run_and_check(x16, signs, lam, 128, 16, 4, rq.SRFT, "after timeout probe")
+    assert rq.srftq_check_device() == 0
+
+
 def test_empty_call_launches_nothing():
     x = torch.empty((2, 0, 3, 64), dtype=torch.float16, device=DEV)
     codes, scales = rq.quantize(x, torch.ones((2, 3, 64), dtype=torch.int8, device=DEV),
