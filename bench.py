@@ -387,30 +387,8 @@ def run_ours(args):
 
     e2e = None
     if not args.no_e2e:
-        x_host = torch.empty(x.shape, dtype=x.dtype, pin_memory=True)
-        x_host.copy_(x)
-        xhat_host = torch.empty(x.shape, dtype=x.dtype, pin_memory=True)
-
-        def e2e_step():
-            x.copy_(x_host, non_blocking=True)
-            step()
-            xhat_host.copy_(xhat, non_blocking=True)
-
-        e2e_step()
-        barrier()
-        s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        s2.record()
-        for _ in range(args.e2e_steps):
-            e2e_step()
-        e2.record()
-        barrier()
-        ems = _max_over_ranks(pg, dev, s2.elapsed_time(e2))
-        e2e = {"value": step_bytes * args.e2e_steps * world / (ems / 1e3) / 1e9, "unit": "GB/s",
-               "h2d_bytes_per_step": x.numel() * x.element_size(),
-               "d2h_bytes_per_step": xhat.numel() * xhat.element_size(),
-               "ms_per_step": ems / args.e2e_steps, "steps": args.e2e_steps,
-               "path": "pinned host -> device copy, srftq_calibrate_lambda + srftq_quantize + "
-                       "srftq_dequantize, device -> pinned host copy of the dequantized cache"}
+        e2e = run_e2e(args, rq, desc, w, x, signs, lam, codes, scales, xhat, barrier, pg, dev,
+                      step_bytes, world)
 
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": K,
@@ -441,6 +419,80 @@ def run_ours(args):
         pg.barrier()
         pg.destroy_process_group()
     return 0
+
+
+def e2e_chunks(n_slices: int, target: int = 8) -> list:
+    """Slice ranges [a, b) of the pipelined end-to-end step: about `target`
+    chunks of whole slices (calibration is per slice, so chunks never split
+    one)."""
+    n = max(1, min(target, n_slices))
+    bounds = [round(i * n_slices / n) for i in range(n + 1)]
+    return [(bounds[i], bounds[i + 1]) for i in range(n) if bounds[i + 1] > bounds[i]]
+
+
+def run_e2e(args, rq, desc, w, x, signs, lam, codes, scales, xhat, barrier, pg, dev,
+            step_bytes, world) -> dict:
+    """The step end to end through the C ABI: the fp16 cache comes from pinned
+    host memory and the dequantised cache goes back to it, every step. The
+    step is pipelined over chunks of whole slices on three streams (copy in,
+    compute, copy out, ordered by events), so that host->device copies,
+    kernels and device->host copies of different chunks overlap; PCIe
+    carries both directions at once."""
+    import torch
+
+    x_host = torch.empty(x.shape, dtype=x.dtype, pin_memory=True)
+    x_host.copy_(x)
+    xhat_host = torch.empty(x.shape, dtype=x.dtype, pin_memory=True)
+    chunks = e2e_chunks(w.S)
+    s_in, s_cmp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    main = torch.cuda.current_stream()
+
+    def e2e_step():
+        start_ev = torch.cuda.Event()
+        start_ev.record(main)
+        done = []
+        for a, b in chunks:
+            e_in, e_cmp = torch.cuda.Event(), torch.cuda.Event()
+            with torch.cuda.stream(s_in):
+                s_in.wait_event(start_ev)
+                x[a:b].copy_(x_host[a:b], non_blocking=True)
+                e_in.record(s_in)
+            with torch.cuda.stream(s_cmp):
+                s_cmp.wait_event(e_in)
+                rq.srftq_calibrate_lambda(desc, x[a:b], signs[a:b], lam[a:b], w.n_cal, s_cmp)
+                rq.srftq_quantize(desc, x[a:b], signs[a:b], lam[a:b], codes[a:b], scales[a:b],
+                                  s_cmp)
+                rq.srftq_dequantize(desc, codes[a:b], scales[a:b], signs[a:b], lam[a:b],
+                                    xhat[a:b], s_cmp)
+                e_cmp.record(s_cmp)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(e_cmp)
+                xhat_host[a:b].copy_(xhat[a:b], non_blocking=True)
+                e_out = torch.cuda.Event()
+                e_out.record(s_out)
+            done.append(e_out)
+        for e in done:
+            main.wait_event(e)
+
+    e2e_step()
+    barrier()
+    s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s2.record(main)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    e2.record(main)
+    barrier()
+    ems = _max_over_ranks(pg, dev, s2.elapsed_time(e2))
+    if rq.srftq_check_device() != 0:
+        raise RuntimeError("device guard fired during the end-to-end steps")
+    return {"value": step_bytes * args.e2e_steps * world / (ems / 1e3) / 1e9, "unit": "GB/s",
+            "h2d_bytes_per_step": x.numel() * x.element_size(),
+            "d2h_bytes_per_step": xhat.numel() * xhat.element_size(),
+            "ms_per_step": ems / args.e2e_steps, "steps": args.e2e_steps,
+            "chunks": len(chunks),
+            "path": "pinned host -> device copy, srftq_calibrate_lambda + srftq_quantize + "
+                    "srftq_dequantize, device -> pinned host copy of the dequantized cache; "
+                    f"pipelined over {len(chunks)} chunks of slices on three streams"}
 
 
 def round_trip_error(x, xhat, chunk_rows: int = 4096) -> dict:
