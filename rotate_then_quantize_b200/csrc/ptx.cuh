@@ -1,6 +1,6 @@
 // Thin inline-PTX wrappers for sm_100a: mbarriers, TMA tiled loads and
-// stores, 1-D bulk copies and async-proxy fences. Only the forms without
-// cluster multicast are used anywhere in this library.
+// stores, 1-D bulk copies and async-proxy fences. Every copy here reads
+// and writes this CTA's own shared memory only.
 #pragma once
 
 #include <cuda.h>

@@ -78,3 +78,12 @@ def test_reference_arm_runs_on_rank_zero_only(monkeypatch, capsys):
     args = bench.parse_args(["--impl", "reference", "--gpus", "2", "--steps", "1", "--warmup", "0"])
     assert bench.run_reference(args) == 0
     assert capsys.readouterr().out == ""
+
+
+def test_end_to_end_chunks_cover_every_slice_once():
+    for n in (1, 2, 3, 4, 7, 8, 9, 56, 64, 100):
+        chunks = bench.e2e_chunks(n)
+        assert 1 <= len(chunks) <= 8
+        covered = [s for a, b in chunks for s in range(a, b)]
+        assert covered == list(range(n))
+        assert all(b > a for a, b in chunks)
