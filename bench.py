@@ -545,7 +545,7 @@ def run_decode(args):
     T0 = w.N // B
     L = w.S // 2
     rot = args.rotation
-    n_steps = args.warmup + args.steps + args.e2e_steps + 2
+    n_steps = args.warmup + 2 * args.steps + args.e2e_steps + 5
     cap = (T0 + n_steps) * B
     rq.load_library()
     desc = rq.make_desc(w.d, w.H, w.group, w.bits, rot)
@@ -638,6 +638,59 @@ def run_decode(args):
     fp16_ms = _max_over_ranks(pg, dev, s3.elapsed_time(e3))
     del fp16_layer
 
+    # The same decode steps in the rotated domain (R orthogonal: (R q) . (R x)
+    # = q . x): the layer's K and V dequantised without the inverse transform,
+    # the step's 32 x H queries rotated with K's signs and the 32 x H attention
+    # outputs unrotated with V's signs.
+    q_tok = new_tok[0:1]
+    q_rot = torch.empty((1, B, w.H, w.d), dtype=torch.float32, device=dev)
+    o_rot = torch.randn((1, B, w.H, w.d), dtype=torch.float32, device=dev)
+    o_out = torch.empty_like(o_rot)
+
+    def step_rot(ev=None):
+        r0 = (T0 + state["t"]) * B
+        n = r0 + B
+        for l in range(L):
+            sl = slice(2 * l, 2 * l + 2)
+            rq.srftq_quantize(desc, new_tok[sl], signs[sl], lam[sl], codes[sl, r0:n],
+                              scales[sl, r0:n])
+            rq.srftq_rotate(desc, q_tok, signs[2 * l:2 * l + 1], q_rot)
+            if ev is not None:
+                ev[l][0].record()
+            rq.srftq_dequantize_rotated(desc, codes[sl, :n], scales[sl, :n], lam[sl],
+                                        scratch[:, :n])
+            if ev is not None:
+                ev[l][1].record()
+            rq.srftq_unrotate(desc, o_rot, signs[2 * l + 1:2 * l + 2], o_out)
+        state["t"] += 1
+
+    for _ in range(2):
+        step_rot()
+    barrier()
+    evr = [[[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(L)]
+           for _ in range(K)]
+    s4, e4 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s4.record()
+    for k in range(K):
+        step_rot(evr[k])
+    e4.record()
+    barrier()
+    rot_ms = _max_over_ranks(pg, dev, s4.elapsed_time(e4))
+    if rq.srftq_check_device() != 0:
+        raise RuntimeError("device guard fired during the rotated-domain steps")
+    r_avg = statistics.mean(evr[k][l][0].elapsed_time(evr[k][l][1])
+                            for k in range(K) for l in range(L))
+    n_rot = (T0 + state["t"]) * B
+    rot_bytes = 2 * n_rot * w.H * vec_bytes
+    rotated = {"ms_per_step": rot_ms / K,
+               "dequantize_rotated_ms_per_layer": r_avg,
+               "dequantize_rotated_GBps": rot_bytes / (r_avg / 1e3) / 1e9,
+               "dequantize_rotated_frac_of_peak": rot_bytes / (r_avg / 1e3) / 1e9 / read_peak()[0],
+               "step_over_fp16_read_time": (rot_ms / K) / (fp16_ms / K),
+               "step": "per layer: quantize 32 new K and V tokens, rotate 32 x H queries, "
+                       "dequantize the layer's K and V cache in the rotated domain into an "
+                       "fp16 scratch, unrotate 32 x H outputs"}
+
     e2e = None
     if not args.no_e2e:
         tok_host = torch.empty(new_tok.shape, dtype=new_tok.dtype, pin_memory=True)
@@ -687,6 +740,7 @@ def run_decode(args):
                       "how": "torch.sum over an fp16 buffer of one layer's K and V cache "
                              "shape, once per layer"},
         "int4_step_over_fp16_read_time": (ms / K) / (fp16_ms / K),
+        "rotated_domain": rotated,
         "int4_step_over_fp16_read_at_peak": (ms / K) / (fp16_bytes / K / (read_peak()[0] * 1e6)),
         "kernels": {"dequantize_ms_per_layer": d_avg,
                     "dequantize_GBps": achieved,

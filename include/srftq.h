@@ -149,6 +149,39 @@ int srftq_rotate(const srftq_desc* desc, int64_t n_slices, int64_t n_rows,
                  const int8_t* signs, const float* lambda_or_null,
                  float* y_out, void* stream);
 
+/*
+ * srftq_dequantize_rotated -- dequantises into the rotated domain: for every
+ * vector, yhat'_j = lambda_j * sigma_g(j) * q_j (fp16, round to nearest
+ * even), the reconstruction R xhat of the cached vector with neither the
+ * inverse transform nor the signs applied. R is orthogonal ("When
+ * Quantization Is Free", Methodology 1), so attention can score the rotated
+ * query R q against these vectors, (R q) . yhat' = q . xhat, accumulate the
+ * value vectors in the rotated domain and undo the rotation once per output
+ * with srftq_unrotate. desc->rotation is not used (no transform runs).
+ *
+ *   codes  [S][in_stride][H][d*bits/8], scales [S][in_stride][H][d/group]
+ *   lambda [S][H][d] float32 (the quantiser's)
+ *   out    [S][out_stride][H][d] fp16, written
+ *
+ * Same argument rules as srftq_dequantize (signs are not read).
+ */
+int srftq_dequantize_rotated(const srftq_desc* desc, int64_t n_slices, int64_t n_rows,
+                             const uint8_t* codes, const uint16_t* scales,
+                             int64_t in_slice_stride_rows, const float* lambda, uint16_t* out,
+                             int64_t out_slice_stride_rows, void* stream);
+
+/*
+ * srftq_unrotate -- the inverse rotation x = s * R^T y, float32 in and out
+ * (y in the packed rotated coordinates of srftq_rotate without lambda).
+ * "When Quantization Is Free", Methodology 1 (R orthogonal, R^T = R^-1).
+ *
+ *   y [S][y_stride][H][d] float32, signs [S][H][d] int8,
+ *   x [S][x_stride][H][d] float32, written (must not overlap y or signs)
+ */
+int srftq_unrotate(const srftq_desc* desc, int64_t n_slices, int64_t n_rows, const float* y,
+                   int64_t y_slice_stride_rows, const int8_t* signs, float* x,
+                   int64_t x_slice_stride_rows, void* stream);
+
 /* Human-readable text for a status code (static storage, never NULL). */
 const char* srftq_status_string(int status);
 

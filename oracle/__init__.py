@@ -32,6 +32,7 @@ from .srft_oracle import (  # noqa: F401
     binary16_bits_to_float,
     calibrate_lambda,
     dequantize,
+    dequantize_rotated,
     float_to_binary16_bits,
     pack_codes,
     qmax_for,

@@ -336,6 +336,25 @@ def dequantize(codes: np.ndarray, scales: np.ndarray, signs: np.ndarray,
     return {"bits": float_to_binary16_bits(xhat64), "xhat64": xhat64, "yhat": yhat}
 
 
+def dequantize_rotated(codes: np.ndarray, scales: np.ndarray, lam: np.ndarray, d: int,
+                       group: int, bits: int) -> dict:
+    """The dequantised cache left in the rotated domain: yhat_j = q_j * sigma_g
+    * lambda_j (the first half of ``dequantize``, before R^T), float64, and
+    its binary16 rounding (ties to even) as ``bits``. Since R is orthogonal
+    ("When Quantization Is Free", Methodology 1), (R q) . yhat = q . (R^T yhat)
+    for any query q: attention can run on these vectors with a rotated query.
+    """
+    q = unpack_codes(codes, bits)
+    if q.shape[-1] != d:
+        raise ValueError("codes do not match d")
+    sig = binary16_bits_to_float(scales)
+    S, N, H, _ = q.shape
+    qg = q.reshape(S, N, H, d // group, group).astype(np.float64)
+    yhat = (qg * sig[..., None]).reshape(S, N, H, d)
+    yhat = yhat * np.asarray(lam, dtype=np.float32).astype(np.float64)[:, None, :, :]
+    return {"bits": float_to_binary16_bits(yhat), "yhat": yhat}
+
+
 def calibrate_lambda(x: np.ndarray, signs: np.ndarray, n_cal: int,
                      kind: int = SRFT) -> np.ndarray:
     """Per-channel lambda [S, H, d] (float64) from the first n_cal rows.

@@ -14,6 +14,7 @@ from .binding import (  # noqa: F401
     SrftqError,
     calibrate_lambda,
     dequantize,
+    dequantize_rotated,
     load_library,
     make_desc,
     quantize,
@@ -21,9 +22,12 @@ from .binding import (  # noqa: F401
     srftq_calibrate_lambda,
     srftq_check_device,
     srftq_dequantize,
+    srftq_dequantize_rotated,
     srftq_probe_wait_timeout,
     srftq_quantize,
     srftq_rotate,
+    srftq_unrotate,
     srftq_version,
     status_string,
+    unrotate,
 )

@@ -33,8 +33,8 @@ SRHT = 1
 
 # Every symbol include/srftq.h declares (checked by the CPU test suite).
 EXPORTED = ("srftq_quantize", "srftq_dequantize", "srftq_calibrate_lambda", "srftq_rotate",
-            "srftq_status_string", "srftq_check_device", "srftq_probe_wait_timeout",
-            "srftq_version")
+            "srftq_dequantize_rotated", "srftq_unrotate", "srftq_status_string",
+            "srftq_check_device", "srftq_probe_wait_timeout", "srftq_version")
 
 
 class SrftqDesc(ctypes.Structure):
@@ -66,13 +66,16 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.srftq_dequantize.argtypes = [D, I64, I64, P, P, I64, P, P, P, I64, P]
     lib.srftq_calibrate_lambda.argtypes = [D, I64, I64, P, I64, P, P, P]
     lib.srftq_rotate.argtypes = [D, I64, I64, P, I64, P, P, P, P]
+    lib.srftq_dequantize_rotated.argtypes = [D, I64, I64, P, P, I64, P, P, I64, P]
+    lib.srftq_unrotate.argtypes = [D, I64, I64, P, I64, P, P, I64, P]
     lib.srftq_status_string.argtypes = [I32]
     lib.srftq_status_string.restype = ctypes.c_char_p
     lib.srftq_check_device.argtypes = [P]
     lib.srftq_probe_wait_timeout.argtypes = [ctypes.c_uint32, P]
     lib.srftq_version.argtypes = []
     for name in ("srftq_quantize", "srftq_dequantize", "srftq_calibrate_lambda", "srftq_rotate",
-                 "srftq_check_device", "srftq_probe_wait_timeout", "srftq_version"):
+                 "srftq_dequantize_rotated", "srftq_unrotate", "srftq_check_device",
+                 "srftq_probe_wait_timeout", "srftq_version"):
         getattr(lib, name).restype = I32
     _lib = lib
     return lib
@@ -172,6 +175,33 @@ def srftq_rotate(desc: SrftqDesc, x, signs, y_out, lam=None, stream=None) -> Non
     _check("srftq_rotate", st)
 
 
+def srftq_dequantize_rotated(desc: SrftqDesc, codes, scales, lam, out, stream=None) -> None:
+    """codes, scales -> out [S,N,H,d] fp16 = lambda * sigma * q (the rotated domain)."""
+    lib = load_library()
+    pc, S, N, is_ = _rows_view(codes, desc.heads, desc.d * desc.bits // 8, "codes")
+    ps, S2, N2, is2 = _rows_view(scales, desc.heads, desc.d // desc.group, "scales")
+    po, S3, N3, os_ = _rows_view(out, desc.heads, desc.d, "out")
+    if (S2, N2) != (S, N) or (S3, N3) != (S, N) or is2 != is_:
+        raise ValueError("codes/scales/out shapes disagree")
+    st = lib.srftq_dequantize_rotated(ctypes.byref(desc), S, N, pc, ps, is_,
+                                      _table(lam, S, desc.heads, desc.d, "lambda"), po, os_,
+                                      _stream_handle(stream))
+    _check("srftq_dequantize_rotated", st)
+
+
+def srftq_unrotate(desc: SrftqDesc, y, signs, x_out, stream=None) -> None:
+    """x_out [S,N,H,d] float32 = s * R^T y for y [S,N,H,d] float32."""
+    lib = load_library()
+    py, S, N, ys = _rows_view(y, desc.heads, desc.d, "y")
+    px, S2, N2, xs = _rows_view(x_out, desc.heads, desc.d, "x_out")
+    if (S2, N2) != (S, N):
+        raise ValueError("y/x_out shapes disagree")
+    st = lib.srftq_unrotate(ctypes.byref(desc), S, N, py, ys,
+                            _table(signs, S, desc.heads, desc.d, "signs"), px, xs,
+                            _stream_handle(stream))
+    _check("srftq_unrotate", st)
+
+
 def srftq_probe_wait_timeout(polls: int, stream=None) -> int:
     """Launches the device-side timeout probe (see include/srftq.h); returns the status."""
     return int(load_library().srftq_probe_wait_timeout(int(polls), _stream_handle(stream)))
@@ -231,3 +261,25 @@ def rotate(x, signs, lam=None, rotation: int = SRFT, stream=None):
     y = torch.empty((S, N, H, d), dtype=torch.float32, device=x.device)
     srftq_rotate(desc, x, signs, y, lam, stream)
     return y
+
+
+def dequantize_rotated(codes, scales, lam, d: int, group: int = 16, bits: int = 4, stream=None):
+    """Returns lambda * sigma * q [S,N,H,d] fp16: the cache in the rotated domain."""
+    import torch
+
+    S, N, H, _ = codes.shape
+    desc = make_desc(d, H, group, bits, SRFT)
+    out = torch.empty((S, N, H, d), dtype=torch.float16, device=codes.device)
+    srftq_dequantize_rotated(desc, codes, scales, lam, out, stream)
+    return out
+
+
+def unrotate(y, signs, rotation: int = SRFT, stream=None):
+    """Returns s * R^T y [S,N,H,d] float32 for y [S,N,H,d] float32."""
+    import torch
+
+    S, N, H, d = y.shape
+    desc = make_desc(d, H, 8, 4, rotation)
+    x = torch.empty((S, N, H, d), dtype=torch.float32, device=y.device)
+    srftq_unrotate(desc, y, signs, x, stream)
+    return x

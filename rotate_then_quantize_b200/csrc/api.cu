@@ -265,6 +265,51 @@ int srftq_check_device(void* stream) {
   return SRFTQ_ERR_DEVICE_CHECK;
 }
 
+int srftq_dequantize_rotated(const srftq_desc* desc, int64_t n_slices, int64_t n_rows,
+                             const uint8_t* codes, const uint16_t* scales,
+                             int64_t in_slice_stride_rows, const float* lambda, uint16_t* out,
+                             int64_t out_slice_stride_rows, void* stream) {
+  int rc = check_desc(desc);
+  if (rc != SRFTQ_OK) return rc;
+  if (n_slices < 0 || n_rows < 0) return SRFTQ_ERR_INVALID_ARG;
+  if (n_slices == 0 || n_rows == 0) return SRFTQ_OK;
+  if (in_slice_stride_rows < n_rows || out_slice_stride_rows < n_rows) return SRFTQ_ERR_INVALID_ARG;
+  if (!codes || !scales || !lambda || !out) return SRFTQ_ERR_INVALID_ARG;
+  if (!aligned16(codes) || !aligned16(scales) || !aligned16(lambda) || !aligned16(out))
+    return SRFTQ_ERR_MISALIGNED;
+  const int64_t d = desc->d, H = desc->heads;
+  const Range ro = extent(out, n_slices, out_slice_stride_rows, n_rows, H * d * 2);
+  const Range rc_ = extent(codes, n_slices, in_slice_stride_rows, n_rows, H * d * desc->bits / 8);
+  const Range rs = extent(scales, n_slices, in_slice_stride_rows, n_rows, H * (d / desc->group) * 2);
+  const Range rl = extent(lambda, n_slices, H, H, d * 4);
+  for (Range in : {rc_, rs, rl})
+    if (overlap(ro, in)) return SRFTQ_ERR_INVALID_ARG;
+  RotDequantCall c{desc->heads, desc->group, desc->bits, n_slices, n_rows, codes, scales,
+                   in_slice_stride_rows, lambda, out, out_slice_stride_rows,
+                   static_cast<cudaStream_t>(stream)};
+  return by_d(desc->d, [&](auto d_) { return launch_dequantize_rotated<decltype(d_)::value>(c); });
+}
+
+int srftq_unrotate(const srftq_desc* desc, int64_t n_slices, int64_t n_rows, const float* y,
+                   int64_t y_slice_stride_rows, const int8_t* signs, float* x,
+                   int64_t x_slice_stride_rows, void* stream) {
+  int rc = check_desc(desc);
+  if (rc != SRFTQ_OK) return rc;
+  if (n_slices < 0 || n_rows < 0) return SRFTQ_ERR_INVALID_ARG;
+  if (n_slices == 0 || n_rows == 0) return SRFTQ_OK;
+  if (y_slice_stride_rows < n_rows || x_slice_stride_rows < n_rows) return SRFTQ_ERR_INVALID_ARG;
+  if (!y || !signs || !x) return SRFTQ_ERR_INVALID_ARG;
+  if (!aligned16(y) || !aligned16(signs) || !aligned16(x)) return SRFTQ_ERR_MISALIGNED;
+  const int64_t d = desc->d, H = desc->heads;
+  const Range rx = extent(x, n_slices, x_slice_stride_rows, n_rows, H * d * 4);
+  const Range ry = extent(y, n_slices, y_slice_stride_rows, n_rows, H * d * 4);
+  const Range rsg = extent(signs, n_slices, H, H, d);
+  if (overlap(rx, ry) || overlap(rx, rsg)) return SRFTQ_ERR_INVALID_ARG;
+  UnrotateCall c{desc->heads, desc->rotation, n_slices, n_rows, y, y_slice_stride_rows, signs,
+                 x, x_slice_stride_rows, static_cast<cudaStream_t>(stream)};
+  return by_d(desc->d, [&](auto d_) { return launch_unrotate<decltype(d_)::value>(c); });
+}
+
 int srftq_probe_wait_timeout(uint32_t polls, void* stream) {
   if (polls == 0 || polls > srftq::kWaitLimit) return SRFTQ_ERR_INVALID_ARG;
   unsigned* guard = srftq::Runtime::guard_word();

@@ -49,6 +49,29 @@ struct RotateCall {
   cudaStream_t stream;
 };
 
+struct RotDequantCall {
+  int32_t heads, group, bits;
+  int64_t n_slices, n_rows;
+  const uint8_t* codes;
+  const uint16_t* scales;
+  int64_t in_slice_stride_rows;
+  const float* lambda;
+  uint16_t* out;
+  int64_t out_slice_stride_rows;
+  cudaStream_t stream;
+};
+
+struct UnrotateCall {
+  int32_t heads, rotation;
+  int64_t n_slices, n_rows;
+  const float* y;
+  int64_t y_slice_stride_rows;
+  const int8_t* signs;
+  float* x;
+  int64_t x_slice_stride_rows;
+  cudaStream_t stream;
+};
+
 struct CalibCall {
   int32_t heads, rotation;
   int64_t n_slices, n_cal;
@@ -73,11 +96,14 @@ template <int D> int launch_quantize(const QuantCall& c);
 template <int D> int launch_dequantize(const DequantCall& c);
 template <int D> int launch_rotate(const RotateCall& c);
 template <int D> int launch_calibrate(const CalibCall& c);
+template <int D> int launch_dequantize_rotated(const RotDequantCall& c);
+template <int D> int launch_unrotate(const UnrotateCall& c);
 
 // d = 256 has its own kernels (two threads per vector; launch_d256.cu).
 template <> int launch_quantize<256>(const QuantCall& c);
 template <> int launch_dequantize<256>(const DequantCall& c);
 template <> int launch_rotate<256>(const RotateCall& c);
 template <> int launch_calibrate<256>(const CalibCall& c);
+template <> int launch_unrotate<256>(const UnrotateCall& c);
 
 }  // namespace srftq

@@ -49,4 +49,22 @@ int launch_calibrate<256>(const CalibCall& c) {
   return finish_launch();
 }
 
+template <>
+int launch_unrotate<256>(const UnrotateCall& c) {
+  const int64_t total = c.n_slices * c.n_rows * c.heads;
+  if (total == 0) return SRFTQ_OK;
+  UnrotateArgs a{c.n_slices, c.n_rows, c.y_slice_stride_rows, c.x_slice_stride_rows, c.heads,
+                 c.y, c.signs, c.x};
+  const int64_t want = (2 * total + 127) / 128;
+  const int64_t cap = int64_t(Runtime::num_sms()) * 16;
+  const int grid = int(want < cap ? want : cap);
+  if (c.rotation == kSRFT)
+    unrotate256_kernel<kSRFT><<<grid, 128, 0, c.stream>>>(a);
+  else
+    unrotate256_kernel<kSRHT><<<grid, 128, 0, c.stream>>>(a);
+  return finish_launch();
+}
+
 }  // namespace srftq
+
+template int srftq::launch_dequantize_rotated<256>(const srftq::RotDequantCall&);

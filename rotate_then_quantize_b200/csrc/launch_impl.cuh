@@ -9,6 +9,7 @@
 #include "aux.cuh"
 #include "codec.cuh"
 #include "launch.cuh"
+#include "rotated.cuh"
 
 namespace srftq {
 
@@ -271,10 +272,54 @@ int launch_calibrate(const CalibCall& c) {
   return finish_launch();
 }
 
+template <int D>
+int launch_dequantize_rotated(const RotDequantCall& c) {
+  const int64_t per_slice = c.n_rows * c.heads * (D / 8);
+  if (per_slice == 0 || c.n_slices == 0) return SRFTQ_OK;
+  if (per_slice >= (int64_t(1) << 32)) return SRFTQ_ERR_UNSUPPORTED;   // 32-bit in-slice index
+  RotDequantArgs a{c.n_slices, c.n_rows, c.in_slice_stride_rows, c.out_slice_stride_rows,
+                   c.heads, c.codes, c.scales, c.lambda, c.out};
+  // y walks the slices; x covers a slice, about 8 blocks of 256 per SM in all
+  const int64_t gy = c.n_slices < 65535 ? c.n_slices : 65535;
+  const int64_t cap_x = (int64_t(Runtime::num_sms()) * 8 + gy - 1) / gy;
+  const int64_t want_x = (per_slice + 1023) / 1024;   // 4 chunks per thread and step
+  const dim3 grid(unsigned(want_x < cap_x ? want_x : cap_x), unsigned(gy));
+  int rc = SRFTQ_ERR_UNSUPPORTED;
+  static_for<0, 2>([&](auto b_) {
+    constexpr int BITS = decltype(b_)::value == 0 ? 4 : 8;
+    static_for<3, ilog2(D) + 1>([&](auto lg_) {
+      constexpr int G = 1 << decltype(lg_)::value;
+      if (c.bits == BITS && c.group == G) {
+        dequantize_rotated_kernel<D, BITS, G><<<grid, 256, 0, c.stream>>>(a);
+        rc = finish_launch();
+      }
+    });
+  });
+  return rc;
+}
+
+template <int D>
+int launch_unrotate(const UnrotateCall& c) {
+  const int64_t total = c.n_slices * c.n_rows * c.heads;
+  if (total == 0) return SRFTQ_OK;
+  UnrotateArgs a{c.n_slices, c.n_rows, c.y_slice_stride_rows, c.x_slice_stride_rows, c.heads,
+                 c.y, c.signs, c.x};
+  const int64_t want = (total + 127) / 128;
+  const int64_t cap = int64_t(Runtime::num_sms()) * 16;
+  const int grid = int(want < cap ? want : cap);
+  if (c.rotation == kSRFT)
+    unrotate_kernel<D, kSRFT><<<grid, 128, 0, c.stream>>>(a);
+  else
+    unrotate_kernel<D, kSRHT><<<grid, 128, 0, c.stream>>>(a);
+  return finish_launch();
+}
+
 }  // namespace srftq
 
 #define SRFTQ_INSTANTIATE_D(D)                                        \
   template int srftq::launch_quantize<D>(const srftq::QuantCall&);     \
   template int srftq::launch_dequantize<D>(const srftq::DequantCall&); \
   template int srftq::launch_rotate<D>(const srftq::RotateCall&);      \
-  template int srftq::launch_calibrate<D>(const srftq::CalibCall&);
+  template int srftq::launch_calibrate<D>(const srftq::CalibCall&);       \
+  template int srftq::launch_dequantize_rotated<D>(const srftq::RotDequantCall&); \
+  template int srftq::launch_unrotate<D>(const srftq::UnrotateCall&);

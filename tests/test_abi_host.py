@@ -126,6 +126,25 @@ def test_dequantize_calibrate_rotate_validation(lib):
     assert lib.srftq_rotate(D, 1, 0, c, 8, sg, None, y, None) == b.SRFTQ_OK
 
 
+def test_rotated_domain_calls_validate_before_launching(lib):
+    desc = rq.make_desc(64, 3, 16, 8, 0)
+    c, s, sg, lam, xh, y = _addrs()
+    D = ctypes.byref(desc)
+    R = lib.srftq_dequantize_rotated
+    assert R(D, 1, 8, c, s, 8, lam, c, 8, None) == b.SRFTQ_ERR_INVALID_ARG      # out overlaps codes
+    assert R(D, 1, 8, c, s, 8, None, xh, 8, None) == b.SRFTQ_ERR_INVALID_ARG   # no lambda
+    assert R(D, 1, 8, c, s + 2, 8, lam, xh, 8, None) == b.SRFTQ_ERR_MISALIGNED
+    assert R(D, 1, 8, c, s, 4, lam, xh, 8, None) == b.SRFTQ_ERR_INVALID_ARG    # stride < rows
+    assert R(D, 0, 8, c, s, 8, lam, xh, 8, None) == b.SRFTQ_OK                 # nothing to do
+    assert R(None, 1, 8, c, s, 8, lam, xh, 8, None) == b.SRFTQ_ERR_INVALID_ARG
+    U = lib.srftq_unrotate
+    assert U(D, 1, 8, y, 8, sg, y, 8, None) == b.SRFTQ_ERR_INVALID_ARG         # in place
+    assert U(D, 1, 8, y, 8, sg, y + 16, 8, None) == b.SRFTQ_ERR_INVALID_ARG    # overlap
+    assert U(D, 1, 8, y + 8, 8, sg, xh, 8, None) == b.SRFTQ_ERR_MISALIGNED
+    assert U(D, 1, 8, y, 8, None, xh, 8, None) == b.SRFTQ_ERR_INVALID_ARG
+    assert U(D, 1, 0, y, 8, sg, xh, 8, None) == b.SRFTQ_OK
+
+
 def test_python_binding_rejects_bad_views():
     torch = pytest.importorskip("torch")
     x = torch.zeros((2, 8, 3, 64), dtype=torch.float16)

@@ -7,6 +7,8 @@ checks a sample of rows from every slice, and properties that hold for any
 size are checked on every vector.
 """
 
+import math
+
 import numpy as np
 import pytest
 
@@ -404,3 +406,104 @@ def test_decode_streaming_appends(rot):
     assert np.all(c_np[:, n:] == 0x5A)
     assert np.all(s_np[:, n:] == np.float16(9.0).view(np.uint16))
     assert np.all(xh[:, n:] == np.float16(5.0).view(np.uint16))
+
+
+# ---------------------------------------------------------------------------
+# Decode in the rotated domain: R orthogonal, so (R q) . (R x) = q . x
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("d,bits,group", [(16, 4, 8), (64, 4, 16), (128, 4, 16), (128, 8, 32),
+                                          (128, 4, 128), (256, 4, 32), (256, 8, 64)])
+def test_dequantize_rotated_matches_oracle(d, bits, group):
+    rng = np.random.default_rng(7 * d + bits + group)
+    S, N, H = 2, 37, 3
+    x16 = _x(rng, S, N, H, d)
+    signs = _signs(rng, S, H, d)
+    lam = np.exp(rng.uniform(-1, 1, (S, H, d))).astype(np.float32)
+    ref = oracle.quantize(x16, signs, lam, group, bits)
+    out = rq.dequantize_rotated(_t(ref["codes"]), _t(ref["scales"].view(np.float16)), _t(lam),
+                                d, group, bits)
+    want = oracle.dequantize_rotated(ref["codes"], ref["scales"], lam, d, group, bits)
+    parity.assert_clean(parity.check_dequant(_np16(out), want["bits"]),
+                        f"rotated dequant d{d} b{bits} g{group}")
+    # a strided window of a larger cache leaves the rows around it untouched
+    big = torch.full((S, N + 9, H, d), 7.0, dtype=torch.float16, device=DEV)
+    desc = rq.make_desc(d, H, group, bits)
+    rq.srftq_dequantize_rotated(desc, _t(ref["codes"]), _t(ref["scales"].view(np.float16)),
+                                _t(lam), big[:, 4:4 + N])
+    assert torch.equal(big[:, 4:4 + N], out)
+    assert torch.all(big[:, :4] == 7.0) and torch.all(big[:, 4 + N:] == 7.0)
+
+
+@pytest.mark.parametrize("d", [16, 32, 64, 128, 256])
+@pytest.mark.parametrize("rot", [0, 1])
+def test_unrotate_matches_oracle_and_inverts_rotate(d, rot):
+    rng = np.random.default_rng(13 * d + rot)
+    S, N, H = 2, 21, 3
+    y = rng.standard_normal((S, N, H, d)).astype(np.float32)
+    signs = _signs(rng, S, H, d)
+    x = rq.unrotate(_t(y), _t(signs), rotation=rot).cpu().numpy()
+    parity.assert_clean(parity.check_rotation(x, oracle.unrotate(y, signs, rot)), f"unrotate d{d}")
+    x16 = _x(rng, S, N, H, d)
+    back = rq.unrotate(rq.rotate(_t(x16), _t(signs), rotation=rot), _t(signs),
+                       rotation=rot).cpu().numpy()
+    parity.assert_clean(parity.check_rotation(back, x16.astype(np.float64)), f"round trip d{d}")
+
+
+@pytest.mark.parametrize("rot", [0, 1])
+def test_decode_attention_in_the_rotated_domain(rot):
+    """One decode query per head against an int4 K/V cache, run entirely in
+    the rotated domain on the GPU (rotate q with K's signs, score against the
+    rotated-domain K cache, softmax, accumulate the rotated-domain V cache,
+    unrotate the output with V's signs) and compared with float64 attention
+    over the oracle's dequantised K and V."""
+    rng = np.random.default_rng(21 + rot)
+    T, H, d, group, bits = 300, 4, 128, 16, 4
+    # the decode-stream cache's distribution: N(0, 1), no outliers
+    k16 = _x(rng, 1, T, H, d, outlier_p=0.0)
+    v16 = _x(rng, 1, T, H, d, outlier_p=0.0)
+    sk, sv = _signs(rng, 1, H, d), _signs(rng, 1, H, d)
+    lk = oracle.calibrate_lambda(k16, sk, 128, rot).astype(np.float32)
+    lv = oracle.calibrate_lambda(v16, sv, 128, rot).astype(np.float32)
+    qk = oracle.quantize(k16, sk, lk, group, bits, rot)
+    qv = oracle.quantize(v16, sv, lv, group, bits, rot)
+    q16 = _x(rng, 1, 1, H, d, outlier_p=0.0)
+
+    q_rot = rq.rotate(_t(q16), _t(sk), rotation=rot)[0, 0]                      # [H, d]
+    k_rot = rq.dequantize_rotated(_t(qk["codes"]), _t(qk["scales"].view(np.float16)), _t(lk),
+                                  d, group, bits)[0].float()                     # [T, H, d]
+    v_rot = rq.dequantize_rotated(_t(qv["codes"]), _t(qv["scales"].view(np.float16)), _t(lv),
+                                  d, group, bits)[0].float()
+    scores = torch.einsum("hd,thd->ht", q_rot, k_rot) / math.sqrt(d)
+    p = torch.softmax(scores, dim=1)
+    o_rot = torch.einsum("ht,thd->hd", p, v_rot)
+    o = rq.unrotate(o_rot[None, None].contiguous(), _t(sv), rotation=rot)[0, 0].cpu().numpy()
+
+    # (1) the same arithmetic in float64: attention over the oracle's own
+    # fp16-rounded rotated-domain K and V (bit-equal to the GPU's, checked by
+    # test_dequantize_rotated_matches_oracle), the rotated query, R^T of the
+    # output; only float32 accumulation on the GPU differs (~1e-6 relative)
+    ky16 = oracle.binary16_bits_to_float(
+        oracle.dequantize_rotated(qk["codes"], qk["scales"], lk, d, group, bits)["bits"])[0]
+    vy16 = oracle.binary16_bits_to_float(
+        oracle.dequantize_rotated(qv["codes"], qv["scales"], lv, d, group, bits)["bits"])[0]
+    qy = oracle.rotate(q16, sk, rot)[0, 0]
+    # (2) exact attention over the dequantised cache (no fp16 storage)
+    kx = oracle.dequantize(qk["codes"], qk["scales"], sk, lk, d, group, bits, rot)["xhat64"][0]
+    vx = oracle.dequantize(qv["codes"], qv["scales"], sv, lv, d, group, bits, rot)["xhat64"][0]
+    for h in range(H):
+        s16 = ky16[:, h, :] @ qy[h] / math.sqrt(d)
+        p16 = np.exp(s16 - s16.max())
+        p16 /= p16.sum()
+        o16 = oracle.unrotate((p16 @ vy16[:, h, :])[None, None, None, :], sv[:, h:h + 1, :],
+                              rot)[0, 0, 0]
+        err16 = np.abs(o[h] - o16) / np.maximum(1.0, np.abs(o16))
+        assert err16.max() < 1e-4, ("same arithmetic", h, float(err16.max()))
+        s_ref = kx[:, h, :] @ q16[0, 0, h, :].astype(np.float64) / math.sqrt(d)
+        p_ref = np.exp(s_ref - s_ref.max())
+        p_ref /= p_ref.sum()
+        o_ref = p_ref @ vx[:, h, :]
+        # fp16 storage of K and V moves the output by ~1e-4 on this unit-scale
+        # data; 2e-3 only guards against gross disagreement
+        err = np.abs(o[h] - o_ref) / np.maximum(1.0, np.abs(o_ref))
+        assert err.max() < 2e-3, ("exact attention", h, float(err.max()))

@@ -352,3 +352,49 @@ def test_calibration_energy_invariant(kind):
     x2 = x.copy()
     x2[:, 24:] *= 100.0
     assert np.array_equal(oracle.calibrate_lambda(x2, signs, 24, kind), lam)
+
+
+@pytest.mark.parametrize("kind", [oracle.SRFT, oracle.SRHT])
+def test_rotated_domain_attention_equals_plain_attention(kind):
+    """Orthogonality ("When Quantization Is Free", Methodology 1) carried
+    through decode attention: with K and V quantised, scoring the rotated
+    query against the rotated-domain cache gives the scores of the plain query
+    against the dequantised cache, and undoing the rotation of the
+    rotated-domain output gives the plain output, to float64 rounding."""
+    rng = np.random.default_rng(11)
+    S, T, H, d, group, bits = 1, 37, 2, 64, 16, 4
+    k16 = rng.standard_normal((S, T, H, d)).astype(np.float16)
+    v16 = rng.standard_normal((S, T, H, d)).astype(np.float16)
+    sk = np.where(rng.random((S, H, d)) < 0.5, -1, 1).astype(np.int8)
+    sv = np.where(rng.random((S, H, d)) < 0.5, -1, 1).astype(np.int8)
+    lk = np.exp(rng.uniform(-0.5, 0.5, (S, H, d))).astype(np.float32)
+    lv = np.exp(rng.uniform(-0.5, 0.5, (S, H, d))).astype(np.float32)
+    qk, qv = (oracle.quantize(k16, sk, lk, group, bits, kind),
+              oracle.quantize(v16, sv, lv, group, bits, kind))
+    kx = oracle.dequantize(qk["codes"], qk["scales"], sk, lk, d, group, bits, kind)["xhat64"]
+    vx = oracle.dequantize(qv["codes"], qv["scales"], sv, lv, d, group, bits, kind)["xhat64"]
+    ky = oracle.dequantize_rotated(qk["codes"], qk["scales"], lk, d, group, bits)["yhat"]
+    vy = oracle.dequantize_rotated(qv["codes"], qv["scales"], lv, d, group, bits)["yhat"]
+    q = rng.standard_normal((S, 1, H, d)).astype(np.float16)
+    q_rot = oracle.rotate(q, sk, kind)                       # R_K q, float64
+    for h in range(H):
+        plain = kx[0, :, h, :] @ q[0, 0, h, :].astype(np.float64)
+        rotated = ky[0, :, h, :] @ q_rot[0, 0, h, :]
+        np.testing.assert_allclose(rotated, plain, rtol=1e-12, atol=1e-12)
+        p = np.exp(plain - plain.max())
+        p /= p.sum()
+        out_plain = p @ vx[0, :, h, :]
+        out_rot = (p @ vy[0, :, h, :])[None, None, None, :]
+        sv_h = sv[:, h:h + 1, :]
+        out = oracle.unrotate(out_rot, sv_h, kind)[0, 0, 0]
+        np.testing.assert_allclose(out, out_plain, rtol=1e-12, atol=1e-12)
+
+
+def test_rotated_dequantisation_is_the_scaled_codes():
+    """Hand-worked: codes (-7, 3) in one byte, sigma = 0.5, lambda = (2, 4)
+    give (-7 * 0.5 * 2, 3 * 0.5 * 4) = (-7, 6)."""
+    codes = np.array([[[[0x39]]]], dtype=np.uint8)          # low nibble -7, high 3
+    scales = oracle.float_to_binary16_bits(np.array([[[[0.5]]]]))
+    lam = np.array([[[2.0, 4.0]]], dtype=np.float32)
+    out = oracle.dequantize_rotated(codes, scales, lam, 2, 2, 4)
+    np.testing.assert_array_equal(out["yhat"][0, 0, 0], [-7.0, 6.0])
