@@ -25,6 +25,7 @@ from __future__ import annotations
 import argparse
 import hashlib
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -545,7 +546,7 @@ def run_decode(args):
     T0 = w.N // B
     L = w.S // 2
     rot = args.rotation
-    n_steps = args.warmup + 2 * args.steps + args.e2e_steps + 5
+    n_steps = args.warmup + 3 * args.steps + args.e2e_steps + 8
     cap = (T0 + n_steps) * B
     rq.load_library()
     desc = rq.make_desc(w.d, w.H, w.group, w.bits, rot)
@@ -682,6 +683,58 @@ def run_decode(args):
                             for k in range(K) for l in range(L))
     n_rot = (T0 + state["t"]) * B
     rot_bytes = 2 * n_rot * w.H * vec_bytes
+    # The same decode steps with attention fused into the dequantisation: one
+    # query per (sequence, KV head) attends over the layer's K and V codes;
+    # no fp16 cache is written and no inverse transform runs per token.
+    q_dec = torch.randn((B, w.H, w.d), device=dev).to(torch.float16)
+    att_out = torch.empty((B, w.H, w.d), dtype=torch.float32, device=dev)
+    cbw, ngw = w.d * w.bits // 8, w.d // w.group
+
+    def step_attn(ev=None):
+        r0 = (T0 + state["t"]) * B
+        n = r0 + B
+        for l in range(L):
+            sl = slice(2 * l, 2 * l + 2)
+            rq.srftq_quantize(desc, new_tok[sl], signs[sl], lam[sl], codes[sl, r0:n],
+                              scales[sl, r0:n])
+            if ev is not None:
+                ev[l][0].record()
+            k, v = 2 * l, 2 * l + 1
+            rq.srftq_decode_attention(desc, q_dec, codes[k, :n], scales[k, :n], signs[k], lam[k],
+                                      codes[v, :n], scales[v, :n], signs[v], lam[v], n // B, B, 1,
+                                      1.0 / math.sqrt(w.d), att_out)
+            if ev is not None:
+                ev[l][1].record()
+        state["t"] += 1
+
+    for _ in range(2):
+        step_attn()
+    barrier()
+    eva = [[[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(L)]
+           for _ in range(K)]
+    s5, e5 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s5.record()
+    for k in range(K):
+        step_attn(eva[k])
+    e5.record()
+    barrier()
+    att_ms = _max_over_ranks(pg, dev, s5.elapsed_time(e5))
+    if rq.srftq_check_device() != 0:
+        raise RuntimeError("device guard fired during the fused-attention steps")
+    a_avg = statistics.mean(eva[k][l][0].elapsed_time(eva[k][l][1])
+                            for k in range(K) for l in range(L))
+    n_att = (T0 + state["t"]) * B
+    att_bytes = 2 * n_att * w.H * (cbw + 2 * ngw)   # K and V codes and scales read
+    fused = {"ms_per_step": att_ms / K,
+             "attention_ms_per_layer": a_avg,
+             "attention_GBps": att_bytes / (a_avg / 1e3) / 1e9,
+             "attention_frac_of_peak": att_bytes / (a_avg / 1e3) / 1e9 / read_peak()[0],
+             "step_over_fp16_read_time": (att_ms / K) / (fp16_ms / K),
+             "attention_over_fp16_read_per_layer": a_avg / (fp16_ms / K / L),
+             "step": "per layer: quantize 32 new K and V tokens, then one query per sequence "
+                     "and KV head attends over the layer's int4 K and V codes "
+                     "(srftq_decode_attention, rotated domain, float32 out)"}
+
     rotated = {"ms_per_step": rot_ms / K,
                "dequantize_rotated_ms_per_layer": r_avg,
                "dequantize_rotated_GBps": rot_bytes / (r_avg / 1e3) / 1e9,
@@ -741,6 +794,7 @@ def run_decode(args):
                              "shape, once per layer"},
         "int4_step_over_fp16_read_time": (ms / K) / (fp16_ms / K),
         "rotated_domain": rotated,
+        "fused_attention": fused,
         "int4_step_over_fp16_read_at_peak": (ms / K) / (fp16_bytes / K / (read_peak()[0] * 1e6)),
         "kernels": {"dequantize_ms_per_layer": d_avg,
                     "dequantize_GBps": achieved,

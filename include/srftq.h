@@ -182,6 +182,43 @@ int srftq_unrotate(const srftq_desc* desc, int64_t n_slices, int64_t n_rows, con
                    int64_t y_slice_stride_rows, const int8_t* signs, float* x,
                    int64_t x_slice_stride_rows, void* stream);
 
+/*
+ * srftq_decode_attention -- one decode step of attention, fused with
+ * dequantisation, for d = 128. For every sequence b < n_seq and KV head h,
+ * the q_per_kv (1, 2, 4 or 8) query heads h*q_per_kv + g attend over the
+ * n_ctx cached tokens of the quantised K and V caches:
+ *   out = sum_t softmax_t(softmax_scale * q . khat_t) vhat_t
+ * with khat, vhat what srftq_dequantize would return (before its fp16
+ * rounding). R is orthogonal ("When Quantization Is Free", Methodology 1),
+ * so the kernel rotates each query once with the K signs, reads only codes
+ * and scales, and undoes the V rotation once per output: it never writes a
+ * dequantised cache and runs no inverse transform per token.
+ *
+ *   q        [n_seq][heads*q_per_kv][d] fp16
+ *   k_codes, v_codes    rows of [heads][d*bits/8] uint8; k_scales, v_scales
+ *            rows of [heads][d/group] fp16; token t of sequence b is row
+ *            t*tok_stride_rows + b*seq_stride_rows (strides >= 0)
+ *   k_signs, v_signs [heads][d] int8; k_lambda, v_lambda [heads][d] float32
+ *            (the quantiser's, for the one slice each cache is)
+ *   out      [n_seq][heads*q_per_kv][d] float32, written; must not overlap
+ *            an input. It doubles as the call's scratch: the first of the
+ *            call's three kernels writes the rotated queries there, the
+ *            second overwrites them with the rotated-domain outputs and the
+ *            third unrotates those in place, so `out` holds the result only
+ *            once the call's work on `stream` is complete.
+ *
+ * Returns SRFTQ_ERR_UNSUPPORTED for d != 128 or another q_per_kv, and
+ * SRFTQ_ERR_INVALID_ARG for n_ctx < 1 or bad pointers and strides; every
+ * pointer must be 16-byte aligned (SRFTQ_ERR_MISALIGNED).
+ */
+int srftq_decode_attention(const srftq_desc* desc, int64_t n_seq, int64_t n_ctx, int32_t q_per_kv,
+                           const uint16_t* q, const uint8_t* k_codes, const uint16_t* k_scales,
+                           const int8_t* k_signs, const float* k_lambda, const uint8_t* v_codes,
+                           const uint16_t* v_scales, const int8_t* v_signs,
+                           const float* v_lambda, int64_t tok_stride_rows,
+                           int64_t seq_stride_rows, float softmax_scale, float* out,
+                           void* stream);
+
 /* Human-readable text for a status code (static storage, never NULL). */
 const char* srftq_status_string(int status);
 

@@ -31,6 +31,7 @@ from .srft_oracle import (  # noqa: F401
     SRHT,
     binary16_bits_to_float,
     calibrate_lambda,
+    decode_attention,
     dequantize,
     dequantize_rotated,
     float_to_binary16_bits,

@@ -355,6 +355,35 @@ def dequantize_rotated(codes: np.ndarray, scales: np.ndarray, lam: np.ndarray, d
     return {"bits": float_to_binary16_bits(yhat), "yhat": yhat}
 
 
+def decode_attention(q: np.ndarray, k_codes: np.ndarray, k_scales: np.ndarray,
+                     k_signs: np.ndarray, k_lam: np.ndarray, v_codes: np.ndarray,
+                     v_scales: np.ndarray, v_signs: np.ndarray, v_lam: np.ndarray, d: int,
+                     group: int, bits: int, kind: int, n_ctx: int, tok_stride_rows: int,
+                     seq_stride_rows: int, scale: float) -> np.ndarray:
+    """One decode step of attention over the quantised caches, float64:
+    out[b, h*Q + g] = sum_t softmax_t(scale * q[b, h*Q + g] . khat[t]) vhat[t]
+    with khat, vhat = ``dequantize`` of the rows t*tok_stride + b*seq_stride
+    (before the binary16 rounding). q [n_seq][H*Q][d]; caches [rows][H][...];
+    signs and lambda [H][d] (one slice)."""
+    q = np.asarray(q, dtype=np.float64)
+    n_seq, HQ, _ = q.shape
+    H = k_codes.shape[1]
+    Q = HQ // H
+    out = np.empty((n_seq, HQ, d), dtype=np.float64)
+    for b in range(n_seq):
+        rows = np.arange(n_ctx) * tok_stride_rows + b * seq_stride_rows
+        kx = dequantize(k_codes[None, rows], k_scales[None, rows], k_signs[None], k_lam[None],
+                        d, group, bits, kind)["xhat64"][0]
+        vx = dequantize(v_codes[None, rows], v_scales[None, rows], v_signs[None], v_lam[None],
+                        d, group, bits, kind)["xhat64"][0]
+        for h in range(H):
+            for g in range(Q):
+                s = scale * (kx[:, h, :] @ q[b, h * Q + g])
+                p = np.exp(s - s.max())
+                out[b, h * Q + g] = (p / p.sum()) @ vx[:, h, :]
+    return out
+
+
 def calibrate_lambda(x: np.ndarray, signs: np.ndarray, n_cal: int,
                      kind: int = SRFT) -> np.ndarray:
     """Per-channel lambda [S, H, d] (float64) from the first n_cal rows.

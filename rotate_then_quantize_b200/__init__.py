@@ -13,6 +13,7 @@ from .binding import (  # noqa: F401
     SrftqDesc,
     SrftqError,
     calibrate_lambda,
+    decode_attention,
     dequantize,
     dequantize_rotated,
     load_library,
@@ -21,6 +22,7 @@ from .binding import (  # noqa: F401
     rotate,
     srftq_calibrate_lambda,
     srftq_check_device,
+    srftq_decode_attention,
     srftq_dequantize,
     srftq_dequantize_rotated,
     srftq_probe_wait_timeout,

@@ -33,7 +33,8 @@ SRHT = 1
 
 # Every symbol include/srftq.h declares (checked by the CPU test suite).
 EXPORTED = ("srftq_quantize", "srftq_dequantize", "srftq_calibrate_lambda", "srftq_rotate",
-            "srftq_dequantize_rotated", "srftq_unrotate", "srftq_status_string",
+            "srftq_dequantize_rotated", "srftq_unrotate", "srftq_decode_attention",
+            "srftq_status_string",
             "srftq_check_device", "srftq_probe_wait_timeout", "srftq_version")
 
 
@@ -68,13 +69,16 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.srftq_rotate.argtypes = [D, I64, I64, P, I64, P, P, P, P]
     lib.srftq_dequantize_rotated.argtypes = [D, I64, I64, P, P, I64, P, P, I64, P]
     lib.srftq_unrotate.argtypes = [D, I64, I64, P, I64, P, P, I64, P]
+    lib.srftq_decode_attention.argtypes = [D, I64, I64, I32, P, P, P, P, P, P, P, P, P, I64, I64,
+                                           ctypes.c_float, P, P]
     lib.srftq_status_string.argtypes = [I32]
     lib.srftq_status_string.restype = ctypes.c_char_p
     lib.srftq_check_device.argtypes = [P]
     lib.srftq_probe_wait_timeout.argtypes = [ctypes.c_uint32, P]
     lib.srftq_version.argtypes = []
     for name in ("srftq_quantize", "srftq_dequantize", "srftq_calibrate_lambda", "srftq_rotate",
-                 "srftq_dequantize_rotated", "srftq_unrotate", "srftq_check_device",
+                 "srftq_dequantize_rotated", "srftq_unrotate", "srftq_decode_attention",
+                 "srftq_check_device",
                  "srftq_probe_wait_timeout", "srftq_version"):
         getattr(lib, name).restype = I32
     _lib = lib
@@ -202,6 +206,47 @@ def srftq_unrotate(desc: SrftqDesc, y, signs, x_out, stream=None) -> None:
     _check("srftq_unrotate", st)
 
 
+def _cache_rows(t, H: int, row_elems: int, name: str):
+    """(pointer, rows) of a contiguous [rows, H, e] cache tensor."""
+    if t.dim() != 3 or t.shape[1] != H or t.shape[2] != row_elems or not t.is_contiguous():
+        raise ValueError(f"{name}: expected contiguous [rows, {H}, {row_elems}], got "
+                         f"{tuple(t.shape)}")
+    return t.data_ptr(), t.shape[0]
+
+
+def srftq_decode_attention(desc: SrftqDesc, q, k_codes, k_scales, k_signs, k_lambda, v_codes,
+                           v_scales, v_signs, v_lambda, n_ctx: int, tok_stride_rows: int,
+                           seq_stride_rows: int, scale: float, out, stream=None) -> None:
+    """out [n_seq, H*q_per_kv, d] float32 = softmax(scale q . khat) vhat over n_ctx
+    tokens of the quantised K and V caches ([rows, H, ...] tensors; token t of
+    sequence b is row t*tok_stride_rows + b*seq_stride_rows)."""
+    lib = load_library()
+    H, d = desc.heads, desc.d
+    if q.dim() != 3 or q.shape[1] % H or q.shape[2] != d or not q.is_contiguous():
+        raise ValueError(f"q: expected contiguous [n_seq, {H}*q_per_kv, {d}]")
+    n_seq, q_per_kv = q.shape[0], q.shape[1] // H
+    if tuple(out.shape) != tuple(q.shape) or not out.is_contiguous():
+        raise ValueError("out must be a contiguous float32 tensor shaped like q")
+    cb, ng = d * desc.bits // 8, d // desc.group
+    pk, rk = _cache_rows(k_codes, H, cb, "k_codes")
+    pks, rks = _cache_rows(k_scales, H, ng, "k_scales")
+    pv, rv = _cache_rows(v_codes, H, cb, "v_codes")
+    pvs, rvs = _cache_rows(v_scales, H, ng, "v_scales")
+    need = (n_ctx - 1) * tok_stride_rows + (n_seq - 1) * seq_stride_rows + 1 if n_seq else 0
+    if min(rk, rks, rv, rvs) < need:
+        raise ValueError(f"the caches hold fewer than the {need} rows addressed")
+    for t, name in ((k_signs, "k_signs"), (v_signs, "v_signs"), (k_lambda, "k_lambda"),
+                    (v_lambda, "v_lambda")):
+        if tuple(t.shape) != (H, d) or not t.is_contiguous():
+            raise ValueError(f"{name}: expected contiguous [{H}, {d}]")
+    st = lib.srftq_decode_attention(ctypes.byref(desc), n_seq, int(n_ctx), q_per_kv, q.data_ptr(),
+                                    pk, pks, k_signs.data_ptr(), k_lambda.data_ptr(), pv, pvs,
+                                    v_signs.data_ptr(), v_lambda.data_ptr(), int(tok_stride_rows),
+                                    int(seq_stride_rows), float(scale), out.data_ptr(),
+                                    _stream_handle(stream))
+    _check("srftq_decode_attention", st)
+
+
 def srftq_probe_wait_timeout(polls: int, stream=None) -> int:
     """Launches the device-side timeout probe (see include/srftq.h); returns the status."""
     return int(load_library().srftq_probe_wait_timeout(int(polls), _stream_handle(stream)))
@@ -283,3 +328,29 @@ def unrotate(y, signs, rotation: int = SRFT, stream=None):
     x = torch.empty((S, N, H, d), dtype=torch.float32, device=y.device)
     srftq_unrotate(desc, y, signs, x, stream)
     return x
+
+
+def decode_attention(q, k_codes, k_scales, k_signs, k_lambda, v_codes, v_scales, v_signs,
+                     v_lambda, group: int = 16, bits: int = 4, rotation: int = SRFT,
+                     n_ctx: int = None, tok_stride_rows: int = None, seq_stride_rows: int = 1,
+                     scale: float = None, stream=None):
+    """Fused decode attention over quantised K/V caches (see srftq_decode_attention).
+    Defaults follow the decode layout row = token * n_seq + sequence."""
+    import math
+
+    import torch
+
+    n_seq, HQ, d = q.shape
+    H = k_codes.shape[1]
+    if tok_stride_rows is None:
+        tok_stride_rows = n_seq
+    if n_ctx is None:
+        n_ctx = k_codes.shape[0] // tok_stride_rows
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    desc = make_desc(d, H, group, bits, rotation)
+    out = torch.empty((n_seq, HQ, d), dtype=torch.float32, device=q.device)
+    srftq_decode_attention(desc, q, k_codes, k_scales, k_signs, k_lambda, v_codes, v_scales,
+                           v_signs, v_lambda, n_ctx, tok_stride_rows, seq_stride_rows, scale, out,
+                           stream)
+    return out

@@ -310,6 +310,47 @@ int srftq_unrotate(const srftq_desc* desc, int64_t n_slices, int64_t n_rows, con
   return by_d(desc->d, [&](auto d_) { return launch_unrotate<decltype(d_)::value>(c); });
 }
 
+int srftq_decode_attention(const srftq_desc* desc, int64_t n_seq, int64_t n_ctx, int32_t q_per_kv,
+                           const uint16_t* q, const uint8_t* k_codes, const uint16_t* k_scales,
+                           const int8_t* k_signs, const float* k_lambda, const uint8_t* v_codes,
+                           const uint16_t* v_scales, const int8_t* v_signs,
+                           const float* v_lambda, int64_t tok_stride_rows,
+                           int64_t seq_stride_rows, float softmax_scale, float* out,
+                           void* stream) {
+  int rc = check_desc(desc);
+  if (rc != SRFTQ_OK) return rc;
+  if (desc->d != 128) return SRFTQ_ERR_UNSUPPORTED;
+  if (q_per_kv != 1 && q_per_kv != 2 && q_per_kv != 4 && q_per_kv != 8)
+    return SRFTQ_ERR_UNSUPPORTED;
+  if (n_seq < 0 || n_ctx < 1 || tok_stride_rows < 0 || seq_stride_rows < 0)
+    return SRFTQ_ERR_INVALID_ARG;
+  if (n_seq == 0) return SRFTQ_OK;
+  if (!q || !k_codes || !k_scales || !k_signs || !k_lambda || !v_codes || !v_scales ||
+      !v_signs || !v_lambda || !out)
+    return SRFTQ_ERR_INVALID_ARG;
+  for (const void* p : {static_cast<const void*>(q), static_cast<const void*>(k_codes),
+                        static_cast<const void*>(k_scales), static_cast<const void*>(k_signs),
+                        static_cast<const void*>(k_lambda), static_cast<const void*>(v_codes),
+                        static_cast<const void*>(v_scales), static_cast<const void*>(v_signs),
+                        static_cast<const void*>(v_lambda), static_cast<const void*>(out)})
+    if (!aligned16(p)) return SRFTQ_ERR_MISALIGNED;
+  const int64_t d = desc->d, H = desc->heads;
+  const int64_t rows = (n_ctx - 1) * tok_stride_rows + (n_seq - 1) * seq_stride_rows + 1;
+  const int64_t cb = H * d * desc->bits / 8, sb = H * (d / desc->group) * 2;
+  const Range ro = extent(out, 1, 0, 1, n_seq * H * q_per_kv * d * 4);
+  const Range rq_ = extent(q, 1, 0, 1, n_seq * H * q_per_kv * d * 2);
+  for (Range in : {rq_, extent(k_codes, 1, 0, rows, cb), extent(k_scales, 1, 0, rows, sb),
+                   extent(v_codes, 1, 0, rows, cb), extent(v_scales, 1, 0, rows, sb),
+                   extent(k_signs, 1, 0, 1, H * d), extent(v_signs, 1, 0, 1, H * d),
+                   extent(k_lambda, 1, 0, 1, H * d * 4), extent(v_lambda, 1, 0, 1, H * d * 4)})
+    if (overlap(ro, in)) return SRFTQ_ERR_INVALID_ARG;
+  AttnCall c{desc->heads, desc->group, desc->bits, desc->rotation, q_per_kv, n_seq, n_ctx,
+             tok_stride_rows, seq_stride_rows, softmax_scale, q, k_codes, k_scales, k_signs,
+             k_lambda, v_codes, v_scales, v_signs, v_lambda, out,
+             static_cast<cudaStream_t>(stream)};
+  return launch_decode_attention_d128(c);
+}
+
 int srftq_probe_wait_timeout(uint32_t polls, void* stream) {
   if (polls == 0 || polls > srftq::kWaitLimit) return SRFTQ_ERR_INVALID_ARG;
   unsigned* guard = srftq::Runtime::guard_word();

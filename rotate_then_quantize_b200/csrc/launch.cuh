@@ -72,6 +72,23 @@ struct UnrotateCall {
   cudaStream_t stream;
 };
 
+struct AttnCall {
+  int32_t heads, group, bits, rotation, q_per_kv;
+  int64_t n_seq, n_ctx, tok_stride_rows, seq_stride_rows;
+  float scale;
+  const uint16_t* q;
+  const uint8_t* k_codes;
+  const uint16_t* k_scales;
+  const int8_t* k_signs;
+  const float* k_lambda;
+  const uint8_t* v_codes;
+  const uint16_t* v_scales;
+  const int8_t* v_signs;
+  const float* v_lambda;
+  float* out;
+  cudaStream_t stream;
+};
+
 struct CalibCall {
   int32_t heads, rotation;
   int64_t n_slices, n_cal;
@@ -98,6 +115,10 @@ template <int D> int launch_rotate(const RotateCall& c);
 template <int D> int launch_calibrate(const CalibCall& c);
 template <int D> int launch_dequantize_rotated(const RotDequantCall& c);
 template <int D> int launch_unrotate(const UnrotateCall& c);
+
+// Decode attention over the quantised cache in the rotated domain, d = 128
+// (launch_attention.cu).
+int launch_decode_attention_d128(const AttnCall& c);
 
 // d = 256 has its own kernels (two threads per vector; launch_d256.cu).
 template <> int launch_quantize<256>(const QuantCall& c);

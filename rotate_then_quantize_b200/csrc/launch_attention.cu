@@ -1,0 +1,41 @@
+// Launcher of the fused decode attention (d = 128; attention.cuh).
+#include "attention.cuh"
+#include "launch_impl.cuh"
+
+namespace srftq {
+
+int launch_decode_attention_d128(const AttnCall& c) {
+  if (c.n_seq == 0) return SRFTQ_OK;
+  const int64_t blocks = c.n_seq * c.heads * kAttnSplit;   // one cluster per (sequence, head)
+  if (blocks > INT_MAX) return SRFTQ_ERR_UNSUPPORTED;
+  AttnArgs a{c.n_seq,   c.n_ctx,    c.tok_stride_rows, c.seq_stride_rows, c.heads,
+             c.q_per_kv, c.scale,   c.q,               c.k_codes,         c.k_scales,
+             c.k_signs, c.k_lambda, c.v_codes,         c.v_scales,        c.v_signs,
+             c.v_lambda, c.out};
+  int rc = SRFTQ_ERR_UNSUPPORTED;
+  static_for<0, 2>([&](auto b_) {
+    constexpr int BITS = decltype(b_)::value == 0 ? 4 : 8;
+    static_for<3, 8>([&](auto lg_) {
+      constexpr int G = 1 << decltype(lg_)::value;
+      static_for<0, 2>([&](auto r_) {
+        constexpr int ROT = decltype(r_)::value;
+        static_for<0, 4>([&](auto n_) {
+          constexpr int NQ = 1 << decltype(n_)::value;
+          if (c.bits == BITS && c.group == G && c.rotation == ROT && c.q_per_kv == NQ) {
+            // queries rotated into `out`, attention over the codes, outputs unrotated
+            const int64_t nv = c.n_seq * c.heads * NQ;
+            const int64_t cap = int64_t(Runtime::num_sms()) * 16;
+            const int g1 = int((nv + 127) / 128 < cap ? (nv + 127) / 128 : cap);
+            attn_query_kernel<ROT, NQ><<<g1, 128, 0, c.stream>>>(a);
+            decode_attention_kernel<BITS, G, NQ><<<int(blocks), 128, 0, c.stream>>>(a);
+            attn_unrotate_kernel<ROT, NQ><<<g1, 128, 0, c.stream>>>(a);
+            rc = finish_launch();
+          }
+        });
+      });
+    });
+  });
+  return rc;
+}
+
+}  // namespace srftq

@@ -145,6 +145,25 @@ def test_rotated_domain_calls_validate_before_launching(lib):
     assert U(D, 1, 0, y, 8, sg, xh, 8, None) == b.SRFTQ_OK
 
 
+def test_decode_attention_validates_before_launching(lib):
+    c, s, sg, lam, xh, y = _addrs()
+    A = lib.srftq_decode_attention
+
+    def call(desc, n_seq=2, n_ctx=16, qpk=1, q=xh, kc=c, ks=s, ksg=sg, kl=lam, out=y, ts=2, ss=1):
+        return A(ctypes.byref(desc), n_seq, n_ctx, qpk, q, kc, ks, ksg, kl, kc + (1 << 28),
+                 ks + (1 << 28), ksg, kl, ts, ss, 0.1, out, None)
+
+    ok = rq.make_desc(128, 4, 16, 4, 0)
+    assert call(rq.make_desc(64, 4, 16, 4, 0)) == b.SRFTQ_ERR_UNSUPPORTED     # d = 128 only
+    assert call(ok, qpk=3) == b.SRFTQ_ERR_UNSUPPORTED
+    assert call(ok, n_ctx=0) == b.SRFTQ_ERR_INVALID_ARG
+    assert call(ok, ts=-1) == b.SRFTQ_ERR_INVALID_ARG
+    assert call(ok, q=0) == b.SRFTQ_ERR_INVALID_ARG
+    assert call(ok, out=y + 4) == b.SRFTQ_ERR_MISALIGNED
+    assert call(ok, out=xh) == b.SRFTQ_ERR_INVALID_ARG                         # out overlaps q
+    assert call(ok, n_seq=0) == b.SRFTQ_OK                                     # nothing to do
+
+
 def test_python_binding_rejects_bad_views():
     torch = pytest.importorskip("torch")
     x = torch.zeros((2, 8, 3, 64), dtype=torch.float16)

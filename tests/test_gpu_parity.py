@@ -507,3 +507,60 @@ def test_decode_attention_in_the_rotated_domain(rot):
         # data; 2e-3 only guards against gross disagreement
         err = np.abs(o[h] - o_ref) / np.maximum(1.0, np.abs(o_ref))
         assert err.max() < 2e-3, ("exact attention", h, float(err.max()))
+
+
+# ---------------------------------------------------------------------------
+# Fused decode attention over the quantised cache (rotated domain)
+# ---------------------------------------------------------------------------
+
+def _attn_case(rng, rows, H, d, group, bits, rot, outliers=0.0):
+    x = _x(rng, 1, rows, H, d, outlier_p=outliers)
+    s = _signs(rng, 1, H, d)
+    lam = oracle.calibrate_lambda(x, s, min(rows, 64), rot).astype(np.float32)
+    qz = oracle.quantize(x, s, lam, group, bits, rot)
+    return qz["codes"][0], qz["scales"][0], s[0], lam[0]
+
+
+@pytest.mark.parametrize("n_ctx", [1, 5, 128, 129, 1000])
+@pytest.mark.parametrize("q_per_kv", [1, 2, 8])
+@pytest.mark.parametrize("bits,group,rot", [(4, 16, 0), (8, 32, 1), (4, 128, 1)])
+def test_decode_attention_matches_oracle(n_ctx, q_per_kv, bits, group, rot):
+    """Token counts below the cluster's 8 CTAs (empty CTAs), ragged and
+    exact tiles; grouped queries; both rotations. The GPU path is float32
+    from codes to output (no fp16 cache), so it must agree with float64
+    attention over the dequantised cache to ~1e-5 relative."""
+    rng = np.random.default_rng(n_ctx * 31 + q_per_kv * 7 + bits + group + rot)
+    H, d, n_seq = 2, 128, 3
+    rows = n_ctx * n_seq
+    kc, ks, ksg, kl = _attn_case(rng, rows, H, d, group, bits, rot)
+    vc, vs, vsg, vl = _attn_case(rng, rows, H, d, group, bits, rot)
+    q = rng.standard_normal((n_seq, H * q_per_kv, d)).astype(np.float16)
+    scale = 1.0 / math.sqrt(d)
+    out = rq.decode_attention(_t(q), _t(kc), _t(ks.view(np.float16)), _t(ksg), _t(kl), _t(vc),
+                              _t(vs.view(np.float16)), _t(vsg), _t(vl), group, bits, rot,
+                              n_ctx=n_ctx, tok_stride_rows=n_seq, seq_stride_rows=1,
+                              scale=scale).cpu().numpy()
+    ref = oracle.decode_attention(q, kc, ks, ksg, kl, vc, vs, vsg, vl, d, group, bits, rot, n_ctx,
+                                  n_seq, 1, scale)
+    err = np.abs(out - ref) / np.maximum(1.0, np.abs(ref))
+    assert err.max() < 2e-5, float(err.max())
+
+
+def test_decode_attention_sequence_major_layout_and_outliers():
+    """Rows = sequence * n_ctx + token (the other common layout), and a
+    cache with x25 outliers, whose scores spread over a wide range."""
+    rng = np.random.default_rng(99)
+    H, d, n_seq, n_ctx, group, bits, rot = 4, 128, 2, 700, 16, 4, 0
+    rows = n_seq * n_ctx
+    kc, ks, ksg, kl = _attn_case(rng, rows, H, d, group, bits, rot, outliers=0.005)
+    vc, vs, vsg, vl = _attn_case(rng, rows, H, d, group, bits, rot, outliers=0.005)
+    q = _x(rng, 1, n_seq, H, d)[0]
+    scale = 1.0 / math.sqrt(d)
+    out = rq.decode_attention(_t(q), _t(kc), _t(ks.view(np.float16)), _t(ksg), _t(kl), _t(vc),
+                              _t(vs.view(np.float16)), _t(vsg), _t(vl), group, bits, rot,
+                              n_ctx=n_ctx, tok_stride_rows=1, seq_stride_rows=n_ctx,
+                              scale=scale).cpu().numpy()
+    ref = oracle.decode_attention(q, kc, ks, ksg, kl, vc, vs, vsg, vl, d, group, bits, rot, n_ctx,
+                                  1, n_ctx, scale)
+    err = np.abs(out - ref) / np.maximum(1.0, np.abs(ref))
+    assert err.max() < 1e-4, float(err.max())

@@ -398,3 +398,45 @@ def test_rotated_dequantisation_is_the_scaled_codes():
     lam = np.array([[[2.0, 4.0]]], dtype=np.float32)
     out = oracle.dequantize_rotated(codes, scales, lam, 2, 2, 4)
     np.testing.assert_array_equal(out["yhat"][0, 0, 0], [-7.0, 6.0])
+
+
+def _attn_cache(rng, rows, H, d, group, bits, kind):
+    x = rng.standard_normal((1, rows, H, d)).astype(np.float16)
+    s = np.where(rng.random((1, H, d)) < 0.5, -1, 1).astype(np.int8)
+    lam = np.exp(rng.uniform(-0.3, 0.3, (1, H, d))).astype(np.float32)
+    qz = oracle.quantize(x, s, lam, group, bits, kind)
+    return qz["codes"][0], qz["scales"][0], s[0], lam[0]
+
+
+@pytest.mark.parametrize("kind", [oracle.SRFT, oracle.SRHT])
+def test_decode_attention_special_cases(kind):
+    """Closed forms of the attention reference: one token gives that
+    token's dequantised value; a zero query weights every token equally (the
+    mean of the values); the two layouts of the same rows agree."""
+    rng = np.random.default_rng(17)
+    H, d, group, bits, n_seq = 2, 16, 8, 4, 3
+    kc, ks, ksg, kl = _attn_cache(rng, 12, H, d, group, bits, kind)
+    vc, vs, vsg, vl = _attn_cache(rng, 12, H, d, group, bits, kind)
+    q = rng.standard_normal((n_seq, 2 * H, d))
+    vx = oracle.dequantize(vc[None], vs[None], vsg[None], vl[None], d, group, bits,
+                           kind)["xhat64"][0]
+    one = oracle.decode_attention(q, kc, ks, ksg, kl, vc, vs, vsg, vl, d, group, bits, kind,
+                                  1, n_seq, 1, 0.25)
+    for b in range(n_seq):
+        for hq in range(2 * H):
+            np.testing.assert_allclose(one[b, hq], vx[b, hq // 2], rtol=1e-12, atol=1e-12)
+    zero = oracle.decode_attention(np.zeros_like(q), kc, ks, ksg, kl, vc, vs, vsg, vl, d, group,
+                                   bits, kind, 4, n_seq, 1, 0.25)
+    for b in range(n_seq):
+        rows = np.arange(4) * n_seq + b
+        for hq in range(2 * H):
+            np.testing.assert_allclose(zero[b, hq], vx[rows, hq // 2].mean(axis=0), rtol=1e-12,
+                                       atol=1e-12)
+    # sequence-major rows (row = b * 4 + t) hold the same tokens as token-major
+    # rows (row = t * 3 + b) after a permutation of the cache
+    perm = np.array([t * n_seq + b for b in range(n_seq) for t in range(4)])
+    a1 = oracle.decode_attention(q, kc, ks, ksg, kl, vc, vs, vsg, vl, d, group, bits, kind, 4,
+                                 n_seq, 1, 0.25)
+    a2 = oracle.decode_attention(q, kc[perm], ks[perm], ksg, kl, vc[perm], vs[perm], vsg, vl, d,
+                                 group, bits, kind, 4, 1, 4, 0.25)
+    np.testing.assert_allclose(a1, a2, rtol=1e-12, atol=1e-12)
