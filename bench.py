@@ -54,6 +54,9 @@ def parse_args(argv=None):
     ap.add_argument("--rotation", type=int, default=0, choices=[0, 1])
     ap.add_argument("--slices", type=int, default=None,
                     help="run the workload on its first SLICES slices only (smaller captures)")
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="decode_stream_d128: cached tokens per sequence (default 32768; "
+                         "smaller captures)")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -313,6 +316,10 @@ def workload(args):
         if not 1 <= args.slices <= w.S:
             raise SystemExit(f"--slices must be in 1..{w.S}")
         w = dataclasses.replace(w, S=args.slices)
+    if getattr(args, "tokens", None) is not None:
+        if args.workload != "decode_stream_d128" or not 512 <= args.tokens <= 32768:
+            raise SystemExit("--tokens applies to decode_stream_d128, 512..32768")
+        w = dataclasses.replace(w, N=args.tokens * 32)
     return w
 
 

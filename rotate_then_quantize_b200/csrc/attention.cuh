@@ -20,20 +20,21 @@
 //   attn_unrotate_kernel  one thread per output: s_V * R_V^T, in place.
 // The main kernel then carries no transform and stays small in registers.
 //
-// Main kernel: one cluster of kSplit CTAs per (b, h); CTA r takes the r-th
-// slice of the tokens. 128 threads per CTA, tokens in tiles of 128:
-//   scores  thread i takes token i of the tile: decodes its 128 key codes
-//           (fp16 magic-number decode, the scale applied by the same FMA)
-//           and dots them with the rotated, lambda- and scale-weighted
-//           queries held in shared memory;
-//   softmax running maximum and sum per query head (online softmax);
-//   values  thread (l, c) takes coordinates 8c .. 8c + 7 of the tile's
-//           tokens l, l + 8, ... and accumulates p_t sigma c_t;
-// then the 8 token lanes are summed, and rank 0 merges the kSplit partial
-// results in rank order through distributed shared memory (deterministic)
-// and scales by lambda_V / sum. Each tile's key codes are loaded during the
-// previous tile, and each thread issues all its value-code loads of a tile
-// before using any.
+// Main kernel: one cluster of kAttnSplit CTAs per (b, h); CTA r takes the
+// r-th slice of the tokens and each of its warps every kAttnWarps-th chunk
+// of 32 tokens. A warp streams its chunks through a kAttnStages-deep
+// cp.async ring in shared memory (codes and scales of K and V), so data in
+// flight holds no registers, and runs its own online softmax:
+//   scores  lane i takes token i: decodes its 128 key codes (fp16
+//           magic-number decode, the scale applied by the same FMA) and
+//           dots them with the staged queries in packed f32x2 FMAs;
+//   softmax a warp-uniform running maximum and per-lane running sums;
+//   values  lane (l, c) takes coordinates 8c .. 8c + 7 of the chunk's
+//           tokens l, l + 2, ..., the weights shuffled from the scoring
+//           lanes.
+// The warps merge in order in shared memory, then rank 0 merges the CTAs'
+// partial results in rank order through distributed shared memory
+// (deterministic) and scales by lambda_V / sum.
 #pragma once
 
 #include <cooperative_groups.h>
@@ -44,7 +45,11 @@
 namespace srftq {
 
 constexpr int kAttnSplit = 8;     // CTAs (one cluster) per (sequence, KV head)
-constexpr int kAttnTile = 128;    // tokens per tile
+constexpr int kAttnWarps = 4;     // warps per CTA, each with its own online softmax
+#ifndef SRFTQ_ATTN_STAGES
+#define SRFTQ_ATTN_STAGES 2
+#endif
+constexpr int kAttnStages = SRFTQ_ATTN_STAGES;   // 32-token chunks in flight per warp
 constexpr int kAttnMaxQ = 8;      // query heads per KV head, at most
 
 struct AttnArgs {
@@ -64,18 +69,29 @@ struct AttnArgs {
 };
 
 // sigma * code for the 8 codes of one code word (int4: one uint32; int8:
-// two) whose fp16 scale is the low half of sw. out[e] = coordinate 8m + e.
+// two) whose fp16 scale is the low half of sw. out[e] = coordinate 8m + e,
+// except that for int4 the odd coordinates come out as 16 * sigma * code:
+// their nibbles are taken where they lie (bits 4..7 of each 16-bit half,
+// the fp16 pair 1152 + 16 q), which saves the shifts, and the factor 16 is
+// folded, exactly, into what they are multiplied with or summed into.
 template <int BITS>
 __device__ __forceinline__ void decode8(const uint32_t* w, uint32_t sw, float (&out)[8]) {
   if constexpr (BITS == 4) {
-    // w >> 4t holds codes t and t + 4 in the low nibbles of its halves
-    const float off = -1032.0f * __half2float(__ushort_as_half(uint16_t(sw)));
-#pragma unroll
-    for (int t = 0; t < 4; ++t) {
-      const uint32_t hp = ((w[0] >> (4 * t)) & 0x000F000Fu) ^ 0x64086408u;   // 1032 + q
-      out[t] = fma_f16<0, 0>(hp, sw, off);
-      out[t + 4] = fma_f16<1, 0>(hp, sw, off);
-    }
+    const float sg = __half2float(__ushort_as_half(uint16_t(sw)));
+    const float off_e = -1032.0f * sg, off_o = -1152.0f * sg;
+    const uint32_t w8 = w[0] >> 8;   // codes 2, 3 and 6, 7 in the low bytes of the halves
+    const uint32_t h0 = (w[0] & 0x000F000Fu) ^ 0x64086408u;   // 1032 + q, codes 0 and 4
+    const uint32_t h1 = (w[0] & 0x00F000F0u) ^ 0x64806480u;   // 1152 + 16 q, codes 1 and 5
+    const uint32_t h2 = (w8 & 0x000F000Fu) ^ 0x64086408u;     // codes 2 and 6
+    const uint32_t h3 = (w8 & 0x00F000F0u) ^ 0x64806480u;     // codes 3 and 7
+    out[0] = fma_f16<0, 0>(h0, sw, off_e);
+    out[4] = fma_f16<1, 0>(h0, sw, off_e);
+    out[1] = fma_f16<0, 0>(h1, sw, off_o);
+    out[5] = fma_f16<1, 0>(h1, sw, off_o);
+    out[2] = fma_f16<0, 0>(h2, sw, off_e);
+    out[6] = fma_f16<1, 0>(h2, sw, off_e);
+    out[3] = fma_f16<0, 0>(h3, sw, off_o);
+    out[7] = fma_f16<1, 0>(h3, sw, off_o);
   } else {
     const float off = -1152.0f * __half2float(__ushort_as_half(uint16_t(sw)));
 #pragma unroll
@@ -148,246 +164,333 @@ __global__ void __launch_bounds__(128) attn_unrotate_kernel(const AttnArgs a) {
   }
 }
 
-// The key codes (CB bytes) and group scales (packed fp16 pairs) of one token.
-template <int BITS, int G>
-struct KeyRow {
-  static constexpr int CB = 128 * BITS / 8, NG = 128 / G;
-  uint32_t cw[CB / 4];
-  uint32_t sc[(NG + 1) / 2];
-  __device__ __forceinline__ void load(const uint8_t* codes, const uint16_t* scales,
-                                       int64_t vec) {
-    const uint4* cp = reinterpret_cast<const uint4*>(codes + vec * CB);
+// cp.async of 16 (L2 only), 8 or 4 bytes into shared memory, and its groups.
+template <int BYTES>
+__device__ __forceinline__ void cp_async(uint32_t dst, const void* src) {
+  if constexpr (BYTES == 16)
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+  else
+    asm volatile("cp.async.ca.shared.global [%0], [%1], %2;" ::"r"(dst), "l"(src), "n"(BYTES)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// The maximum and the sum over the 32 lanes of a warp.
+__device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
-    for (int i = 0; i < CB / 16; ++i) {
-      const uint4 u = cp[i];
-      cw[4 * i] = u.x;
-      cw[4 * i + 1] = u.y;
-      cw[4 * i + 2] = u.z;
-      cw[4 * i + 3] = u.w;
-    }
-    const uint16_t* sp = scales + vec * NG;
-    if constexpr (NG >= 8) {
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
-      for (int i = 0; i < NG / 8; ++i) {
-        const uint4 u = reinterpret_cast<const uint4*>(sp)[i];
-        sc[4 * i] = u.x;
-        sc[4 * i + 1] = u.y;
-        sc[4 * i + 2] = u.z;
-        sc[4 * i + 3] = u.w;
-      }
-    } else if constexpr (NG == 4) {
-      const uint2 u = *reinterpret_cast<const uint2*>(sp);
-      sc[0] = u.x;
-      sc[1] = u.y;
-    } else if constexpr (NG == 2) {
-      sc[0] = *reinterpret_cast<const uint32_t*>(sp);
-    } else {
-      sc[0] = sp[0];
-    }
-  }
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// Shared memory of the attention kernel. Each warp owns kAttnStages stages
+// of one 32-token chunk: key codes, value codes (32 rows of CB bytes, the
+// 16-byte pieces of row r stored at piece ^ swz(r) so that a lane reading
+// its own row and half-warps reading one row each are both conflict-free),
+// then key and value scales (32 rows of SBS bytes).
+template <int BITS, int G, int NQ>
+struct AttnLayout {
+  static constexpr int D = 128, CB = D * BITS / 8, NG = D / G;
+  static constexpr int SB = 2 * NG;                 // scale bytes per vector
+  static constexpr int SBS = SB >= 4 ? SB : 4;      // their row stride
+  static constexpr int PPT = CB / 16;               // 16-byte code pieces per row
+  static constexpr int KC = 0, VC = 32 * CB, KS = 64 * CB, VS = 64 * CB + 32 * SBS;
+  static constexpr int kStage = 64 * CB + 64 * SBS;
+  static constexpr int kQs = 0;                                     // float [NQ][D]
+  static constexpr int kAcc = kQs + NQ * D * 4;                     // float [NQ][D]
+  static constexpr int kMx = kAcc + NQ * D * 4;                     // float [NQ]
+  static constexpr int kSm = kMx + 4 * NQ;                          // float [NQ]
+  static constexpr int kWm = kSm + 4 * NQ;                          // float [NW][NQ]
+  static constexpr int kWl = kWm + 4 * NQ * kAttnWarps;             // float [NW][NQ]
+  static constexpr int kStages = (kWl + 4 * NQ * kAttnWarps + 127) / 128 * 128;
+  static constexpr int kBytes = kStages + kAttnWarps * kAttnStages * kStage;
+  static_assert(kStage >= NQ * D * 4, "a warp's partial sums fit in its first stage");
+  __device__ static constexpr int swz(int r) { return (r * CB / 128) % PPT; }
 };
 
+// CTAs per SM the register budget is sized for (128, 168 or 255 registers).
+template <int NQ>
+constexpr int attn_min_blocks() {
+  return NQ <= 2 ? 4 : NQ == 4 ? 3 : 2;
+}
+
 template <int BITS, int G, int NQ>
-__global__ void __cluster_dims__(kAttnSplit, 1, 1) __launch_bounds__(128)
-    decode_attention_kernel(const AttnArgs a) {
-  constexpr int D = 128;
-  constexpr int CB = D * BITS / 8;            // code bytes per vector
-  constexpr int NG = D / G;                   // scales per vector
-  constexpr int WPV = D / 8;                  // 8-code words per vector (16)
-  constexpr int WB = 8 * BITS / 8;            // bytes per 8-code word (4 or 8)
-  constexpr int VU = kAttnTile / 8;           // value tokens per thread and tile (16)
-  constexpr int VB = NQ >= 4 ? VU / 4 : VU;   // value loads in flight per batch
-  constexpr int VNB = VU / VB;
+__global__ void __cluster_dims__(kAttnSplit, 1, 1)
+    __launch_bounds__(kAttnWarps * 32, attn_min_blocks<NQ>()) decode_attention_kernel(const AttnArgs a) {
+  using L = AttnLayout<BITS, G, NQ>;
+  constexpr int D = 128, CB = L::CB, NG = L::NG, SB = L::SB, SBS = L::SBS, PPT = L::PPT;
+  constexpr int WB = BITS;                  // bytes per 8-code word (4 or 8)
+  constexpr int NW = kAttnWarps, NS = kAttnStages;
+  constexpr int VT = 16;                    // value tokens per lane and chunk
   namespace cg = cooperative_groups;
   cg::cluster_group cluster = cg::this_cluster();
+  extern __shared__ __align__(128) uint8_t smem[];
+  float* qs = reinterpret_cast<float*>(smem + L::kQs);
+  float* acc_out = reinterpret_cast<float*>(smem + L::kAcc);
+  float* mx = reinterpret_cast<float*>(smem + L::kMx);
+  float* sm = reinterpret_cast<float*>(smem + L::kSm);
+  float* wm = reinterpret_cast<float*>(smem + L::kWm);
+  float* wl = reinterpret_cast<float*>(smem + L::kWl);
   const int rank = static_cast<int>(cluster.block_rank());
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t bh = blockIdx.x / kAttnSplit;
   const int h = int(bh % a.heads);
   const int64_t b = bh / a.heads;
   float* qo = a.out + (b * a.heads * NQ + int64_t(h) * NQ) * D;   // queries in, result out
+  uint8_t* wst = smem + L::kStages + warp * NS * L::kStage;        // this warp's stages
+  const uint32_t wst_a = smem_addr(wst);
+  const uint32_t qs_a = smem_addr(qs);
 
-  __shared__ __align__(16) float qs[NQ][D];   // rotated queries * lambda_K * scale * log2 e
-  __shared__ float ps[NQ][kAttnTile];         // scores, then weights, of the tile
-  __shared__ float red[8][NQ][D];             // token-lane partial sums
-  __shared__ float mx[NQ], sm[NQ];            // running max (log2 units) and sum
-  __shared__ float wred[4][NQ];               // per-warp reductions
-  __shared__ float acc_out[NQ][D];            // this CTA's accumulated sum p sigma c
-
-  for (int i = tid; i < NQ * D; i += 128) qs[i / D][i % D] = qo[i];
-  if (tid < NQ) {
-    mx[tid] = -INFINITY;
-    sm[tid] = 0.0f;
-  }
+  // int4 keys decode their odd coordinates 16 times too large (decode8)
+  constexpr float kOdd = BITS == 4 ? 0.0625f : 1.0f;
+  for (int i = tid; i < NQ * D; i += NW * 32) qs[i] = (i & 1) ? qo[i] * kOdd : qo[i];
   __syncthreads();
 
-  // this CTA's tokens
+  // this CTA's tokens; warp w takes the 32-token chunks w, w + NW, ...
   const int64_t per = (a.n_ctx + kAttnSplit - 1) / kAttnSplit;
   const int64_t t_begin = rank * per;
   const int64_t t_end = t_begin + per < a.n_ctx ? t_begin + per : a.n_ctx;
-  const int lane_t = tid >> 4;       // value phase: token lane 0..7
-  const int wc = tid & 15;           // value phase: code word (coordinates 8 wc ..)
   const int64_t bs = b * a.seq_stride_rows;
   auto vec_of = [&](int64_t t) { return (t * a.tok_stride_rows + bs) * a.heads + h; };
-  float vacc[NQ][8];
-#pragma unroll
-  for (int g = 0; g < NQ; ++g)
-#pragma unroll
-    for (int e = 0; e < 8; ++e) vacc[g][e] = 0.0f;
+  const int64_t n_chunks =
+      t_end > t_begin + 32 * warp ? (t_end - t_begin - 32 * warp + 32 * NW - 1) / (32 * NW) : 0;
 
-  // With one or two query heads the next tile's key is loaded while this
-  // tile is scored; with more, the registers go to the accumulators.
-  constexpr bool kPrefetch = NQ <= 2;
-  KeyRow<BITS, G> kr;
-  if (kPrefetch && t_begin + tid < t_end) kr.load(a.k_codes, a.k_scales, vec_of(t_begin + tid));
-  for (int64_t t0 = t_begin; t0 < t_end; t0 += kAttnTile) {
-    const int nt = int(t_end - t0 < kAttnTile ? t_end - t0 : kAttnTile);
-    KeyRow<BITS, G> kn;
-    if constexpr (kPrefetch) {
-      if (t0 + kAttnTile + tid < t_end)
-        kn.load(a.k_codes, a.k_scales, vec_of(t0 + kAttnTile + tid));
-    } else {
-      if (tid < nt) kr.load(a.k_codes, a.k_scales, vec_of(t0 + tid));
-    }
-    // (2) scores of token t0 + tid
-    if (tid < nt) {
-      float s[NQ];
+  // Copies chunk c of this warp into stage c % NS (one cp.async group; an
+  // empty group past the last chunk keeps the group count uniform).
+  auto issue = [&](int64_t c) {
+    if (c < n_chunks) {
+      const int64_t t0 = t_begin + 32 * (warp + NW * c);
+      const int nt = int(t_end - t0 < 32 ? t_end - t0 : 32);
+      const uint32_t st = wst_a + uint32_t(c % NS) * L::kStage;
+      const int pc = lane % PPT;
 #pragma unroll
-      for (int g = 0; g < NQ; ++g) s[g] = 0.0f;
-#pragma unroll
-      for (int m = 0; m < WPV; ++m) {
-        float val[8];
-        const int g8 = (8 * m) / G;
-        decode8<BITS>(&kr.cw[m * WB / 4], (kr.sc[g8 / 2] >> (16 * (g8 & 1))) & 0xFFFFu, val);
-#pragma unroll
-        for (int g = 0; g < NQ; ++g) {
-          const float4 q0 = *reinterpret_cast<const float4*>(&qs[g][8 * m]);
-          const float4 q1 = *reinterpret_cast<const float4*>(&qs[g][8 * m + 4]);
-          s[g] = fmaf(val[0], q0.x, s[g]);
-          s[g] = fmaf(val[1], q0.y, s[g]);
-          s[g] = fmaf(val[2], q0.z, s[g]);
-          s[g] = fmaf(val[3], q0.w, s[g]);
-          s[g] = fmaf(val[4], q1.x, s[g]);
-          s[g] = fmaf(val[5], q1.y, s[g]);
-          s[g] = fmaf(val[6], q1.z, s[g]);
-          s[g] = fmaf(val[7], q1.w, s[g]);
+      for (int k = 0; k < PPT; ++k) {
+        const int r = lane / PPT + (32 / PPT) * k;
+        if (r < nt) {
+          const int64_t vec = vec_of(t0 + r);
+          const uint32_t o = uint32_t(r * CB + ((pc ^ L::swz(r)) * 16));
+          cp_async<16>(st + L::KC + o, a.k_codes + vec * CB + pc * 16);
+          cp_async<16>(st + L::VC + o, a.v_codes + vec * CB + pc * 16);
         }
       }
+      if (lane < nt) {
+        const int64_t vec = vec_of(t0 + lane);
+        const uint32_t o = uint32_t(lane * SBS);
+        const uint16_t* ks = a.k_scales + vec * NG;
+        const uint16_t* vs = a.v_scales + vec * NG;
+        if constexpr (SB >= 16) {
 #pragma unroll
-      for (int g = 0; g < NQ; ++g) ps[g][tid] = s[g];
-    }
-    // the value codes and scales of this thread's tokens, issued before use
-    // (in VNB batches of VB tokens, the first one before the softmax)
-    uint32_t vw[VB][WB / 4];
-    uint32_t vsw[VB];
-    auto load_values = [&](int ub) {
-#pragma unroll
-      for (int u = 0; u < VB; ++u) {
-        const int i = lane_t + 8 * (ub * VB + u);
-        if (i < nt) {
-          const int64_t vec = vec_of(t0 + i);
-          if constexpr (BITS == 4) {
-            vw[u][0] = *reinterpret_cast<const uint32_t*>(a.v_codes + vec * CB + wc * WB);
-          } else {
-            const uint2 w2 = *reinterpret_cast<const uint2*>(a.v_codes + vec * CB + wc * WB);
-            vw[u][0] = w2.x;
-            vw[u][WB / 4 - 1] = w2.y;
+          for (int q = 0; q < SB / 16; ++q) {
+            cp_async<16>(st + L::KS + o + 16 * q, ks + 8 * q);
+            cp_async<16>(st + L::VS + o + 16 * q, vs + 8 * q);
           }
-          vsw[u] = a.v_scales[vec * NG + (8 * wc) / G];
+        } else if constexpr (SB >= 4) {
+          cp_async<SB>(st + L::KS + o, ks);
+          cp_async<SB>(st + L::VS + o, vs);
+        } else {
+          // one scale per vector (2 bytes, below the smallest cp.async)
+          *reinterpret_cast<uint16_t*>(wst + (c % NS) * L::kStage + L::KS + o) = ks[0];
+          *reinterpret_cast<uint16_t*>(wst + (c % NS) * L::kStage + L::VS + o) = vs[0];
+        }
+      } else {
+        // past the end: value scale 0, so the stale codes there decode to 0
+        uint8_t* z = wst + (c % NS) * L::kStage + L::VS + lane * SBS;
+#pragma unroll
+        for (int q = 0; q < SBS / 4; ++q) reinterpret_cast<uint32_t*>(z)[q] = 0u;
+      }
+    }
+    cp_async_commit();
+  };
+
+  float m[NQ], l[NQ];          // running max (warp-uniform) and this lane's sum
+  float2 vacc[NQ][4];          // sum p sigma c, coordinates 8 vwi .. 8 vwi + 7
+#pragma unroll
+  for (int g = 0; g < NQ; ++g) {
+    m[g] = -INFINITY;
+    l[g] = 0.0f;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) vacc[g][e] = make_float2(0.0f, 0.0f);
+  }
+  const int vwi = lane & 15;   // value phase: code word (coordinates 8 vwi ..)
+  const int vt0 = lane >> 4;   // value phase: tokens vt0, vt0 + 2, ... of the chunk
+
+#pragma unroll
+  for (int c = 0; c < NS - 1; ++c) issue(c);
+  for (int64_t c = 0; c < n_chunks; ++c) {
+    issue(c + NS - 1);
+    cp_async_wait<NS - 1>();   // chunk c has landed (this lane's copies) ...
+    __syncwarp();              // ... and every lane's
+    const int64_t t0 = t_begin + 32 * (warp + NW * c);
+    const int nt = int(t_end - t0 < 32 ? t_end - t0 : 32);
+    const uint8_t* st = wst + (c % NS) * L::kStage;
+
+    // score of token t0 + lane (log2 units; -inf past the end)
+    float s[NQ];
+    if (lane < nt) {
+      uint32_t sw[(NG + 1) / 2];
+      const uint8_t* ksr = st + L::KS + lane * SBS;
+      if constexpr (SB >= 16) {
+#pragma unroll
+        for (int q = 0; q < SB / 16; ++q) {
+          const uint4 u = *reinterpret_cast<const uint4*>(ksr + 16 * q);
+          sw[4 * q] = u.x;
+          sw[4 * q + 1] = u.y;
+          sw[4 * q + 2] = u.z;
+          sw[4 * q + 3] = u.w;
+        }
+      } else if constexpr (SB == 8) {
+        const uint2 u = *reinterpret_cast<const uint2*>(ksr);
+        sw[0] = u.x;
+        sw[1] = u.y;
+      } else if constexpr (SB == 4) {
+        sw[0] = *reinterpret_cast<const uint32_t*>(ksr);
+      } else {
+        sw[0] = *reinterpret_cast<const uint16_t*>(ksr);
+      }
+      float2 s2[NQ];
+#pragma unroll
+      for (int g = 0; g < NQ; ++g) s2[g] = make_float2(0.0f, 0.0f);
+      const uint8_t* kr = st + L::KC + lane * CB;
+#pragma unroll
+      for (int pc = 0; pc < PPT; ++pc) {
+        const uint4 u = *reinterpret_cast<const uint4*>(kr + ((pc ^ L::swz(lane)) * 16));
+        const uint32_t uw[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int k = 0; k < 16 / WB; ++k) {
+          const int w8 = pc * (16 / WB) + k;   // coordinates 8 w8 .. 8 w8 + 7
+          const int g8 = (8 * w8) / G;
+          float val[8];
+          decode8<BITS>(&uw[k * WB / 4], (sw[g8 / 2] >> (16 * (g8 & 1))) & 0xFFFFu, val);
+#pragma unroll
+          for (int g = 0; g < NQ; ++g) {
+            const uint4 q0 = lds128(qs_a + uint32_t(g * D + 8 * w8) * 4u);
+            const uint4 q1 = lds128(qs_a + uint32_t(g * D + 8 * w8 + 4) * 4u);
+            s2[g] = fma2(make_float2(val[0], val[1]),
+                         make_float2(__uint_as_float(q0.x), __uint_as_float(q0.y)), s2[g]);
+            s2[g] = fma2(make_float2(val[2], val[3]),
+                         make_float2(__uint_as_float(q0.z), __uint_as_float(q0.w)), s2[g]);
+            s2[g] = fma2(make_float2(val[4], val[5]),
+                         make_float2(__uint_as_float(q1.x), __uint_as_float(q1.y)), s2[g]);
+            s2[g] = fma2(make_float2(val[6], val[7]),
+                         make_float2(__uint_as_float(q1.z), __uint_as_float(q1.w)), s2[g]);
+          }
         }
       }
-    };
-    load_values(0);
-    __syncthreads();
-
-    // (3) online softmax: tile maximum per query head, then the weights
+#pragma unroll
+      for (int g = 0; g < NQ; ++g) s[g] = s2[g].x + s2[g].y;
+    } else {
+#pragma unroll
+      for (int g = 0; g < NQ; ++g) s[g] = -INFINITY;
+    }
+    // online softmax over the chunk: lane 0 is always a token, so the new
+    // maximum is finite; alpha is 0 on the first chunk (m = -inf)
+    float p[NQ], alpha[NQ];
 #pragma unroll
     for (int g = 0; g < NQ; ++g) {
-      float m = tid < nt ? ps[g][tid] : -INFINITY;
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-      if ((tid & 31) == 0) wred[tid >> 5][g] = m;
+      const float mn = fmaxf(m[g], warp_max(s[g]));
+      alpha[g] = exp2f(m[g] - mn);
+      p[g] = exp2f(s[g] - mn);
+      l[g] = fmaf(l[g], alpha[g], p[g]);
+      m[g] = mn;
     }
-    __syncthreads();
-    float alpha[NQ], mnew[NQ], pown[NQ];
-#pragma unroll
-    for (int g = 0; g < NQ; ++g) {
-      const float tm = fmaxf(fmaxf(wred[0][g], wred[1][g]), fmaxf(wred[2][g], wred[3][g]));
-      mnew[g] = fmaxf(mx[g], tm);
-      alpha[g] = exp2f(mx[g] - mnew[g]);   // 0 on the first tile (mx = -inf)
-      pown[g] = tid < nt ? exp2f(ps[g][tid] - mnew[g]) : 0.0f;
-    }
-    float psum[NQ];
-#pragma unroll
-    for (int g = 0; g < NQ; ++g) {
-      psum[g] = pown[g];
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) psum[g] += __shfl_xor_sync(0xffffffffu, psum[g], o);
-    }
-    __syncthreads();   // everyone has read ps (scores), wred and mx
-#pragma unroll
-    for (int g = 0; g < NQ; ++g) {
-      ps[g][tid] = pown[g];
-      if ((tid & 31) == 0) wred[tid >> 5][g] = psum[g];
-    }
-    __syncthreads();
-    if (tid < NQ) {
-      const int g = tid;
-      sm[g] = sm[g] * alpha[g] + (wred[0][g] + wred[1][g] + wred[2][g] + wred[3][g]);
-      mx[g] = mnew[g];
-    }
-    // (4) values: rescale, then tokens lane_t, lane_t + 8, ... of the tile
+    // values: rescale, then p_i sigma c_i for tokens vt0, vt0 + 2, ... (a
+    // token past the end decodes with scale 0 and has p = 0)
 #pragma unroll
     for (int g = 0; g < NQ; ++g)
 #pragma unroll
-      for (int e = 0; e < 8; ++e) vacc[g][e] *= alpha[g];
+      for (int e = 0; e < 4; ++e) vacc[g][e] = mul2(vacc[g][e], splat(alpha[g]));
 #pragma unroll
-    for (int ub = 0; ub < VNB; ++ub) {
-      if (ub > 0) load_values(ub);
+    for (int u = 0; u < VT; ++u) {
+      const int i = vt0 + 2 * u;
+      const uint8_t* vr = st + L::VC + i * CB;
+      uint32_t w[WB / 4];
+      if constexpr (BITS == 4) {
+        w[0] = *reinterpret_cast<const uint32_t*>(
+            vr + (((vwi >> 2) ^ L::swz(i)) * 16) + (vwi & 3) * 4);
+      } else {
+        const uint2 w2 = *reinterpret_cast<const uint2*>(
+            vr + (((vwi >> 1) ^ L::swz(i)) * 16) + (vwi & 1) * 8);
+        w[0] = w2.x;
+        w[WB / 4 - 1] = w2.y;
+      }
+      const uint32_t vsc =
+          *reinterpret_cast<const uint16_t*>(st + L::VS + i * SBS + ((8 * vwi) / G) * 2);
+      float val[8];
+      decode8<BITS>(w, vsc, val);
 #pragma unroll
-      for (int u = 0; u < VB; ++u) {
-        const int i = lane_t + 8 * (ub * VB + u);
-        if (i < nt) {
-          float val[8];
-          decode8<BITS>(vw[u], vsw[u], val);
+      for (int g = 0; g < NQ; ++g) {
+        const float pi = __shfl_sync(0xffffffffu, p[g], i);
 #pragma unroll
-          for (int g = 0; g < NQ; ++g) {
-            const float p = ps[g][i];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) vacc[g][e] = fmaf(p, val[e], vacc[g][e]);
-          }
-        }
+        for (int e = 0; e < 4; ++e)
+          vacc[g][e] = fma2(splat(pi), make_float2(val[2 * e], val[2 * e + 1]), vacc[g][e]);
       }
     }
-    if constexpr (kPrefetch) {
-#pragma unroll
-      for (int i = 0; i < CB / 4; ++i) kr.cw[i] = kn.cw[i];
-#pragma unroll
-      for (int i = 0; i < (NG + 1) / 2; ++i) kr.sc[i] = kn.sc[i];
-    }
-    __syncthreads();   // ps and mx are rewritten by the next tile
+    __syncwarp();   // every lane is done with this stage before it is refilled
   }
+  cp_async_wait<0>();
+  __syncwarp();
 
-  // (5) sum the 8 token lanes: acc_out[g][j]
+  // warp totals: the lanes' sums, and lanes L and L + 16 (same coordinates),
+  // into the warp's first stage
+  float* wacc = reinterpret_cast<float*>(wst);
 #pragma unroll
-  for (int g = 0; g < NQ; ++g)
+  for (int g = 0; g < NQ; ++g) {
+    l[g] = warp_sum(l[g]);
 #pragma unroll
-    for (int e = 0; e < 8; ++e) red[lane_t][g][8 * wc + e] = vacc[g][e];
+    for (int e = 0; e < 4; ++e) {
+      vacc[g][e].x += __shfl_xor_sync(0xffffffffu, vacc[g][e].x, 16);
+      vacc[g][e].y += __shfl_xor_sync(0xffffffffu, vacc[g][e].y, 16);
+      vacc[g][e].y *= kOdd;   // int4: odd coordinates were summed 16 times too large
+    }
+    if (lane < 16) {
+      float4* dst = reinterpret_cast<float4*>(wacc + g * D + 8 * vwi);
+      dst[0] = make_float4(vacc[g][0].x, vacc[g][0].y, vacc[g][1].x, vacc[g][1].y);
+      dst[1] = make_float4(vacc[g][2].x, vacc[g][2].y, vacc[g][3].x, vacc[g][3].y);
+    }
+    if (lane == 0) {
+      wm[warp * NQ + g] = m[g];
+      wl[warp * NQ + g] = l[g];
+    }
+  }
   __syncthreads();
-  for (int idx = tid; idx < NQ * D; idx += 128) {
-    const int g = idx / D, j = idx % D;
-    float sacc = 0.0f;
+  // this CTA's (max, sum, accumulator), merging the warps in order
+  for (int idx = tid; idx < NQ * D; idx += NW * 32) {
+    const int g = idx / D;
+    float mt = -INFINITY;
 #pragma unroll
-    for (int l = 0; l < 8; ++l) sacc += red[l][g][j];
-    acc_out[g][j] = sacc;
+    for (int w = 0; w < NW; ++w) mt = fmaxf(mt, wm[w * NQ + g]);
+    float acc = 0.0f, lt = 0.0f;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) {
+      const float mw = wm[w * NQ + g];
+      const float cw = mw == -INFINITY ? 0.0f : exp2f(mw - mt);
+      const float* wa = reinterpret_cast<const float*>(smem + L::kStages + w * NS * L::kStage);
+      acc = fmaf(cw, wa[idx], acc);
+      lt = fmaf(cw, wl[w * NQ + g], lt);
+    }
+    acc_out[idx] = acc;
+    if (idx % D == 0) {
+      mx[g] = mt;
+      sm[g] = lt;
+    }
   }
   cluster.sync();
 
-  // (6) rank 0 merges the partial results in rank order: the rotated-domain
+  // rank 0 merges the partial results in rank order: the rotated-domain
   // output lambda_V * sum_t p_t sigma c_t / sum_t p_t, written over the
   // queries (the unrotation follows in attn_unrotate_kernel)
   if (rank == 0) {
-    for (int idx = tid; idx < NQ * D; idx += 128) {
+    for (int idx = tid; idx < NQ * D; idx += NW * 32) {
       const int g = idx / D, j = idx % D;
       float m_tot = -INFINITY;
       for (int r = 0; r < kAttnSplit; ++r)
@@ -395,9 +498,9 @@ __global__ void __cluster_dims__(kAttnSplit, 1, 1) __launch_bounds__(128)
       float l_tot = 0.0f, sacc = 0.0f;
       for (int r = 0; r < kAttnSplit; ++r) {
         const float mr = cluster.map_shared_rank(&mx[g], r)[0];
-        const float c = mr == -INFINITY ? 0.0f : exp2f(mr - m_tot);
-        l_tot += c * cluster.map_shared_rank(&sm[g], r)[0];
-        sacc += c * cluster.map_shared_rank(&acc_out[g][j], r)[0];
+        const float cr = mr == -INFINITY ? 0.0f : exp2f(mr - m_tot);
+        l_tot += cr * cluster.map_shared_rank(&sm[g], r)[0];
+        sacc += cr * cluster.map_shared_rank(&acc_out[idx], r)[0];
       }
       qo[idx] = sacc * a.v_lambda[int64_t(h) * D + j] / l_tot;
     }

@@ -26,8 +26,13 @@ int launch_decode_attention_d128(const AttnCall& c) {
             const int64_t nv = c.n_seq * c.heads * NQ;
             const int64_t cap = int64_t(Runtime::num_sms()) * 16;
             const int g1 = int((nv + 127) / 128 < cap ? (nv + 127) / 128 : cap);
+            constexpr auto K = decode_attention_kernel<BITS, G, NQ>;
+            constexpr int smem = AttnLayout<BITS, G, NQ>::kBytes;
+            int bps = 0;
+            rc = prepare_kernel<K>(smem, kAttnWarps * 32, &bps);
+            if (rc != SRFTQ_OK) return;
             attn_query_kernel<ROT, NQ><<<g1, 128, 0, c.stream>>>(a);
-            decode_attention_kernel<BITS, G, NQ><<<int(blocks), 128, 0, c.stream>>>(a);
+            K<<<int(blocks), kAttnWarps * 32, smem, c.stream>>>(a);
             attn_unrotate_kernel<ROT, NQ><<<g1, 128, 0, c.stream>>>(a);
             rc = finish_launch();
           }
