@@ -219,9 +219,12 @@ struct AttnLayout {
 };
 
 // CTAs per SM the register budget is sized for (128, 168 or 255 registers).
+#ifndef SRFTQ_ATTN_MINB
+#define SRFTQ_ATTN_MINB 4
+#endif
 template <int NQ>
 constexpr int attn_min_blocks() {
-  return NQ <= 2 ? 4 : NQ == 4 ? 3 : 2;
+  return NQ <= 2 ? SRFTQ_ATTN_MINB : NQ == 4 ? 3 : 2;
 }
 
 template <int BITS, int G, int NQ>
