@@ -234,7 +234,16 @@ __global__ void __cluster_dims__(kAttnSplit, 1, 1)
   constexpr int D = 128, CB = L::CB, NG = L::NG, SB = L::SB, SBS = L::SBS, PPT = L::PPT;
   constexpr int WB = BITS;                  // bytes per 8-code word (4 or 8)
   constexpr int NW = kAttnWarps, NS = kAttnStages;
-  constexpr int VT = 16;                    // value tokens per lane and chunk
+  // value phase: each lane takes VW consecutive code words (8 VW
+  // coordinates) of VT tokens; two words with one or two query heads (one
+  // scale conversion per 16 codes), one with more (registers)
+#ifndef SRFTQ_ATTN_VW
+#define SRFTQ_ATTN_VW 0
+#endif
+  constexpr int VW = SRFTQ_ATTN_VW > 0 ? SRFTQ_ATTN_VW : NQ <= 2 ? 2 : 1;
+  constexpr int LPT = 16 / VW;              // lanes per token row
+  constexpr int TPI = 32 / LPT;             // tokens per warp instruction
+  constexpr int VT = 32 / TPI;              // value tokens per lane and chunk
   namespace cg = cooperative_groups;
   cg::cluster_group cluster = cg::this_cluster();
   extern __shared__ __align__(128) uint8_t smem[];
@@ -316,16 +325,16 @@ __global__ void __cluster_dims__(kAttnSplit, 1, 1)
   };
 
   float m[NQ], l[NQ];          // running max (warp-uniform) and this lane's sum
-  float2 vacc[NQ][4];          // sum p sigma c, coordinates 8 vwi .. 8 vwi + 7
+  float2 vacc[NQ][4 * VW];     // sum p sigma c, coordinates 8 VW vwi ..
 #pragma unroll
   for (int g = 0; g < NQ; ++g) {
     m[g] = -INFINITY;
     l[g] = 0.0f;
 #pragma unroll
-    for (int e = 0; e < 4; ++e) vacc[g][e] = make_float2(0.0f, 0.0f);
+    for (int e = 0; e < 4 * VW; ++e) vacc[g][e] = make_float2(0.0f, 0.0f);
   }
-  const int vwi = lane & 15;   // value phase: code word (coordinates 8 vwi ..)
-  const int vt0 = lane >> 4;   // value phase: tokens vt0, vt0 + 2, ... of the chunk
+  const int vwi = lane % LPT;  // value phase: words VW vwi .. of the row
+  const int vt0 = lane / LPT;  // value phase: tokens vt0, vt0 + TPI, ... of the chunk
 
 #pragma unroll
   for (int c = 0; c < NS - 1; ++c) issue(c);
@@ -406,36 +415,49 @@ __global__ void __cluster_dims__(kAttnSplit, 1, 1)
       l[g] = fmaf(l[g], alpha[g], p[g]);
       m[g] = mn;
     }
-    // values: rescale, then p_i sigma c_i for tokens vt0, vt0 + 2, ... (a
-    // token past the end decodes with scale 0 and has p = 0)
+    // values: rescale, then p_i sigma c_i for tokens vt0, vt0 + TPI, ...
+    // (a token past the end decodes with scale 0 and has p = 0)
 #pragma unroll
     for (int g = 0; g < NQ; ++g)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) vacc[g][e] = mul2(vacc[g][e], splat(alpha[g]));
+      for (int e = 0; e < 4 * VW; ++e) vacc[g][e] = mul2(vacc[g][e], splat(alpha[g]));
 #pragma unroll
     for (int u = 0; u < VT; ++u) {
-      const int i = vt0 + 2 * u;
+      const int i = vt0 + TPI * u;
       const uint8_t* vr = st + L::VC + i * CB;
-      uint32_t w[WB / 4];
-      if constexpr (BITS == 4) {
-        w[0] = *reinterpret_cast<const uint32_t*>(
-            vr + (((vwi >> 2) ^ L::swz(i)) * 16) + (vwi & 3) * 4);
+      // VW * WB bytes at byte VW * WB * vwi of the row (inside one 16-byte piece)
+      constexpr int VB = VW * WB;
+      const uint8_t* src = vr + ((((VB * vwi) >> 4) ^ L::swz(i)) * 16) + ((VB * vwi) & 15);
+      uint32_t w[VB / 4];
+      if constexpr (VB == 4) {
+        w[0] = *reinterpret_cast<const uint32_t*>(src);
+      } else if constexpr (VB == 8) {
+        const uint2 u2 = *reinterpret_cast<const uint2*>(src);
+        w[0] = u2.x;
+        w[1] = u2.y;
       } else {
-        const uint2 w2 = *reinterpret_cast<const uint2*>(
-            vr + (((vwi >> 1) ^ L::swz(i)) * 16) + (vwi & 1) * 8);
-        w[0] = w2.x;
-        w[WB / 4 - 1] = w2.y;
+        const uint4 u4 = *reinterpret_cast<const uint4*>(src);
+        w[0] = u4.x;
+        w[1] = u4.y;
+        w[2] = u4.z;
+        w[3] = u4.w;
       }
-      const uint32_t vsc =
-          *reinterpret_cast<const uint16_t*>(st + L::VS + i * SBS + ((8 * vwi) / G) * 2);
-      float val[8];
-      decode8<BITS>(w, vsc, val);
+      float pi[NQ];
 #pragma unroll
-      for (int g = 0; g < NQ; ++g) {
-        const float pi = __shfl_sync(0xffffffffu, p[g], i);
+      for (int g = 0; g < NQ; ++g) pi[g] = __shfl_sync(0xffffffffu, p[g], i);
 #pragma unroll
-        for (int e = 0; e < 4; ++e)
-          vacc[g][e] = fma2(splat(pi), make_float2(val[2 * e], val[2 * e + 1]), vacc[g][e]);
+      for (int k = 0; k < VW; ++k) {
+        const int word = VW * vwi + k;   // coordinates 8 word .. 8 word + 7
+        const uint32_t vsc =
+            *reinterpret_cast<const uint16_t*>(st + L::VS + i * SBS + ((8 * word) / G) * 2);
+        float val[8];
+        decode8<BITS>(&w[k * WB / 4], vsc, val);
+#pragma unroll
+        for (int g = 0; g < NQ; ++g)
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            vacc[g][4 * k + e] =
+                fma2(splat(pi[g]), make_float2(val[2 * e], val[2 * e + 1]), vacc[g][4 * k + e]);
       }
     }
     __syncwarp();   // every lane is done with this stage before it is refilled
@@ -443,22 +465,27 @@ __global__ void __cluster_dims__(kAttnSplit, 1, 1)
   cp_async_wait<0>();
   __syncwarp();
 
-  // warp totals: the lanes' sums, and lanes L and L + 16 (same coordinates),
-  // into the warp's first stage
+  // warp totals: the lanes' sums, and the lanes vwi, vwi + LPT, ... (same
+  // coordinates), into the warp's first stage
   float* wacc = reinterpret_cast<float*>(wst);
 #pragma unroll
   for (int g = 0; g < NQ; ++g) {
     l[g] = warp_sum(l[g]);
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      vacc[g][e].x += __shfl_xor_sync(0xffffffffu, vacc[g][e].x, 16);
-      vacc[g][e].y += __shfl_xor_sync(0xffffffffu, vacc[g][e].y, 16);
+    for (int e = 0; e < 4 * VW; ++e) {
+#pragma unroll
+      for (int o = LPT; o < 32; o <<= 1) {
+        vacc[g][e].x += __shfl_xor_sync(0xffffffffu, vacc[g][e].x, o);
+        vacc[g][e].y += __shfl_xor_sync(0xffffffffu, vacc[g][e].y, o);
+      }
       vacc[g][e].y *= kOdd;   // int4: odd coordinates were summed 16 times too large
     }
-    if (lane < 16) {
-      float4* dst = reinterpret_cast<float4*>(wacc + g * D + 8 * vwi);
-      dst[0] = make_float4(vacc[g][0].x, vacc[g][0].y, vacc[g][1].x, vacc[g][1].y);
-      dst[1] = make_float4(vacc[g][2].x, vacc[g][2].y, vacc[g][3].x, vacc[g][3].y);
+    if (lane < LPT) {
+      float4* dst = reinterpret_cast<float4*>(wacc + g * D + 8 * VW * vwi);
+#pragma unroll
+      for (int e = 0; e < 2 * VW; ++e)
+        dst[e] = make_float4(vacc[g][2 * e].x, vacc[g][2 * e].y, vacc[g][2 * e + 1].x,
+                             vacc[g][2 * e + 1].y);
     }
     if (lane == 0) {
       wm[warp * NQ + g] = m[g];
