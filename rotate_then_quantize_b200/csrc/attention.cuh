@@ -46,11 +46,16 @@ namespace srftq {
 
 constexpr int kAttnSplit = 8;     // CTAs (one cluster) per (sequence, KV head)
 constexpr int kAttnWarps = 4;     // warps per CTA, each with its own online softmax
+// SRFTQ_ATTN_STAGES, SRFTQ_ATTN_MINB and SRFTQ_ATTN_VW can be set at build
+// time (-D) for measurement sweeps. The defaults are the measured best on the
+// decode-stream workload: 2 stages (3 took 0.457 against 0.407 ms per
+// layer), 4 CTAs per SM (5, at 96 registers, took 0.375 against 0.364 ms),
+// two value words per lane with one or two query heads (one took 0.365
+// against 0.357 ms).
 #ifndef SRFTQ_ATTN_STAGES
 #define SRFTQ_ATTN_STAGES 2
 #endif
 constexpr int kAttnStages = SRFTQ_ATTN_STAGES;   // 32-token chunks in flight per warp
-constexpr int kAttnMaxQ = 8;      // query heads per KV head, at most
 
 struct AttnArgs {
   int64_t n_seq, n_ctx, tok_stride_rows, seq_stride_rows;
