@@ -84,15 +84,17 @@ constexpr int kCalibCluster = 8;   // blocks (a thread-block cluster) per (slice
 
 // One cluster of kCalibCluster blocks per (slice, head); block r of the
 // cluster takes the batches of 64 rows starting at 64 (r + kCalibCluster b),
-// so n_cal = 512 is one batch per block. Threads 0..63 rotate one row each
-// and write y^2 to shared memory; thread j then adds column j over the
-// batch's rows, in row order, into a float64 accumulator. Rank 0 adds the
+// so n_cal = 512 is one batch per block. Each of the 64 threads rotates one
+// row and writes y^2 to shared memory; thread t then adds columns t, t + 64,
+// ... over the batch's rows, in row order, into float64 accumulators. Blocks
+// of 64 threads let 4 blocks share an SM at the transform's register count. Rank 0 adds the
 // blocks' partial sums in rank order, reading them from the other blocks'
 // shared memory (distributed shared memory of the cluster). Every addition
 // happens in a fixed order, so the result does not depend on scheduling.
 template <int D, int ROT>
-__global__ void __cluster_dims__(kCalibCluster, 1, 1) __launch_bounds__(128)
+__global__ void __cluster_dims__(kCalibCluster, 1, 1) __launch_bounds__(kCalibRows)
     calibrate_kernel(const CalibArgs a) {
+  constexpr int NC = (D + kCalibRows - 1) / kCalibRows;   // columns per thread
   __shared__ float sq[kCalibRows][D + 1];
   __shared__ double part[D];
   namespace cg = cooperative_groups;
@@ -102,41 +104,53 @@ __global__ void __cluster_dims__(kCalibCluster, 1, 1) __launch_bounds__(128)
   const int s = sh / a.heads;
   const int h = sh % a.heads;
   const int64_t tab = (int64_t(s) * a.heads + h) * D;
-  double acc = 0.0;
+  double acc[NC];   // columns threadIdx.x + kCalibRows c
+#pragma unroll
+  for (int c = 0; c < NC; ++c) acc[c] = 0.0;
   for (int64_t base = int64_t(kCalibRows) * rank; base < a.n_cal;
        base += int64_t(kCalibRows) * kCalibCluster) {
-    if (threadIdx.x < kCalibRows) {
-      const int64_t r = base + threadIdx.x;
-      if (r < a.n_cal) {
-        const uint16_t* xv = a.x + ((int64_t(s) * a.x_slice_stride_rows + r) * a.heads + h) * D;
-        uint32_t xw[D / 2], sgw[D / 2];
-        load_vector<D>(xv, a.signs + tab, xw, sgw);
-        float2 v[D / 2];
-        rotate_forward<ROT, D>(xw, sgw, v);
-        static_for<0, D / 2>([&](auto j_) {
-          constexpr int j = decltype(j_)::value;
-          const float y0 = v[j].x * gain_f<ROT, D>(2 * j);
-          const float y1 = v[j].y * gain_f<ROT, D>(2 * j + 1);
-          sq[threadIdx.x][2 * j] = y0 * y0;
-          sq[threadIdx.x][2 * j + 1] = y1 * y1;
-        });
-      } else {
-        for (int j = 0; j < D; ++j) sq[threadIdx.x][j] = 0.0f;
-      }
+    const int64_t r = base + threadIdx.x;   // one row per thread
+    if (r < a.n_cal) {
+      const uint16_t* xv = a.x + ((int64_t(s) * a.x_slice_stride_rows + r) * a.heads + h) * D;
+      uint32_t xw[D / 2], sgw[D / 2];
+      load_vector<D>(xv, a.signs + tab, xw, sgw);
+      float2 v[D / 2];
+      rotate_forward<ROT, D>(xw, sgw, v);
+      static_for<0, D / 2>([&](auto j_) {
+        constexpr int j = decltype(j_)::value;
+        const float y0 = v[j].x * gain_f<ROT, D>(2 * j);
+        const float y1 = v[j].y * gain_f<ROT, D>(2 * j + 1);
+        sq[threadIdx.x][2 * j] = y0 * y0;
+        sq[threadIdx.x][2 * j + 1] = y1 * y1;
+      });
+    } else {
+      for (int j = 0; j < D; ++j) sq[threadIdx.x][j] = 0.0f;
     }
     __syncthreads();
-    if (threadIdx.x < D) {
-      for (int i = 0; i < kCalibRows; ++i) acc += double(sq[i][threadIdx.x]);
+#pragma unroll
+    for (int c = 0; c < NC; ++c) {
+      const int j = threadIdx.x + kCalibRows * c;
+      if (j < D)
+        for (int i = 0; i < kCalibRows; ++i) acc[c] += double(sq[i][j]);
     }
     __syncthreads();
   }
-  if (threadIdx.x < D) part[threadIdx.x] = acc;
+#pragma unroll
+  for (int c = 0; c < NC; ++c) {
+    const int j = threadIdx.x + kCalibRows * c;
+    if (j < D) part[j] = acc[c];
+  }
   cluster.sync();
-  if (rank == 0 && threadIdx.x < D) {
-    double total = 0.0;
-    for (int r = 0; r < kCalibCluster; ++r) total += cluster.map_shared_rank(part, r)[threadIdx.x];
-    a.lambda_out[tab + threadIdx.x] =
-        total > 0.0 ? float(sqrt(total / double(a.n_cal))) : 1.0f;
+  if (rank == 0) {
+#pragma unroll
+    for (int c = 0; c < NC; ++c) {
+      const int j = threadIdx.x + kCalibRows * c;
+      if (j < D) {
+        double total = 0.0;
+        for (int q = 0; q < kCalibCluster; ++q) total += cluster.map_shared_rank(part, q)[j];
+        a.lambda_out[tab + j] = total > 0.0 ? float(sqrt(total / double(a.n_cal))) : 1.0f;
+      }
+    }
   }
   cluster.sync();   // the other blocks keep their shared memory until rank 0 is done
 }

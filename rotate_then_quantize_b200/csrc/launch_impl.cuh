@@ -266,9 +266,9 @@ int launch_calibrate(const CalibCall& c) {
   if (blocks > INT_MAX) return SRFTQ_ERR_UNSUPPORTED;
   CalibArgs a{c.n_cal, c.x_slice_stride_rows, c.heads, c.x, c.signs, c.lambda_out};
   if (c.rotation == kSRFT)
-    calibrate_kernel<D, kSRFT><<<int(blocks), 128, 0, c.stream>>>(a);
+    calibrate_kernel<D, kSRFT><<<int(blocks), kCalibRows, 0, c.stream>>>(a);
   else
-    calibrate_kernel<D, kSRHT><<<int(blocks), 128, 0, c.stream>>>(a);
+    calibrate_kernel<D, kSRHT><<<int(blocks), kCalibRows, 0, c.stream>>>(a);
   return finish_launch();
 }
 
