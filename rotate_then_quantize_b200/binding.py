@@ -219,7 +219,9 @@ def srftq_decode_attention(desc: SrftqDesc, q, k_codes, k_scales, k_signs, k_lam
                            seq_stride_rows: int, scale: float, out, stream=None) -> None:
     """out [n_seq, H*q_per_kv, d] float32 = softmax(scale q . khat) vhat over n_ctx
     tokens of the quantised K and V caches ([rows, H, ...] tensors; token t of
-    sequence b is row t*tok_stride_rows + b*seq_stride_rows)."""
+    sequence b is row t*tok_stride_rows + b*seq_stride_rows). The call makes
+    three launches on the stream and uses `out` as their scratch, so `out`
+    holds the result once that work is complete."""
     lib = load_library()
     H, d = desc.heads, desc.d
     if q.dim() != 3 or q.shape[1] % H or q.shape[2] != d or not q.is_contiguous():
