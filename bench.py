@@ -496,11 +496,45 @@ def run_e2e(args, rq, desc, w, x, signs, lam, codes, scales, xhat, barrier, pg, 
     ems = _max_over_ranks(pg, dev, s2.elapsed_time(e2))
     if rq.srftq_check_device() != 0:
         raise RuntimeError("device guard fired during the end-to-end steps")
+
+    # The bound of this path: the same host->device and device->host copies
+    # alone, concurrently on the copy streams, timed the same way (the data
+    # copied are the step's own buffers, so nothing changes).
+    def copy_step():
+        start_ev = torch.cuda.Event()
+        start_ev.record(main)
+        e_in, e_out = torch.cuda.Event(), torch.cuda.Event()
+        with torch.cuda.stream(s_in):
+            s_in.wait_event(start_ev)
+            x.copy_(x_host, non_blocking=True)
+            e_in.record(s_in)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(start_ev)
+            xhat_host.copy_(xhat, non_blocking=True)
+            e_out.record(s_out)
+        main.wait_event(e_in)
+        main.wait_event(e_out)
+
+    copy_step()
+    barrier()
+    s3, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s3.record(main)
+    for _ in range(args.e2e_steps):
+        copy_step()
+    e3.record(main)
+    barrier()
+    cms = _max_over_ranks(pg, dev, s3.elapsed_time(e3))
+    io_bytes = (x.numel() * x.element_size() + xhat.numel() * xhat.element_size())
     return {"value": step_bytes * args.e2e_steps * world / (ems / 1e3) / 1e9, "unit": "GB/s",
             "h2d_bytes_per_step": x.numel() * x.element_size(),
             "d2h_bytes_per_step": xhat.numel() * xhat.element_size(),
             "ms_per_step": ems / args.e2e_steps, "steps": args.e2e_steps,
             "chunks": len(chunks),
+            "copy_only": {"ms_per_step": cms / args.e2e_steps,
+                          "pcie_GBps": io_bytes * args.e2e_steps / (cms / 1e3) / 1e9,
+                          "frac": (cms / args.e2e_steps) / (ems / args.e2e_steps),
+                          "what": "the step's host->device and device->host copies alone, "
+                                  "concurrently; frac = copy-only time / end-to-end time"},
             "path": "pinned host -> device copy, srftq_calibrate_lambda + srftq_quantize + "
                     "srftq_dequantize, device -> pinned host copy of the dequantized cache; "
                     f"pipelined over {len(chunks)} chunks of slices on three streams"}
