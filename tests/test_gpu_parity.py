@@ -546,6 +546,59 @@ def test_decode_attention_matches_oracle(n_ctx, q_per_kv, bits, group, rot):
     assert err.max() < 2e-5, float(err.max())
 
 
+def test_decode_attention_full_decode_stream_size_sampled():
+    """The launch configuration the decode-stream bench times: 32 sequences x
+    8 KV heads (256 clusters) over 32,768 cached tokens, int4 G16, SRFT, one
+    query per KV head, rows = token * 32 + sequence. The cache is drawn on
+    the device (codes in [-7, 7], as the quantiser writes them, fp16 scales
+    in [0.01, 0.3], lambda in [0.5, 2]); three (sequence, head) outputs are
+    checked against float64 attention over the oracle's dequantisation of
+    the same rows. Each lane sums about 1,000 float32 products per
+    coordinate, so the bound is 1e-4 of max(1, |ref|) (the small cases
+    above meet 2e-5)."""
+    import torch
+    n_seq, H, d, n_ctx, group, bits, rot = 32, 8, 128, 32768, 16, 4, 0
+    rows = n_ctx * n_seq
+    gen = torch.Generator(device=DEV)
+    gen.manual_seed(2024)
+
+    def codes():
+        c = torch.randint(0, 256, (rows, H, d // 2), generator=gen, device=DEV,
+                          dtype=torch.int32).to(torch.uint8)
+        c ^= ((c & 0x0F) == 0x08).to(torch.uint8) * 0x08   # nibble -8 -> 0
+        c ^= ((c >> 4) == 0x08).to(torch.uint8) * 0x80
+        return c
+
+    def scales():
+        return (torch.rand((rows, H, d // group), generator=gen, device=DEV) * 0.29
+                + 0.01).to(torch.float16)
+
+    kc, ks, vc, vs = codes(), scales(), codes(), scales()
+    sgn = (torch.randint(0, 2, (2, H, d), generator=gen, device=DEV) * 2 - 1).to(torch.int8)
+    lam = torch.rand((2, H, d), generator=gen, device=DEV) * 1.5 + 0.5
+    q = torch.randn((n_seq, H, d), generator=gen, device=DEV).to(torch.float16)
+    scale = 1.0 / math.sqrt(d)
+    out = rq.decode_attention(q, kc, ks, sgn[0], lam[0], vc, vs, sgn[1], lam[1], group, bits,
+                              rot, n_ctx=n_ctx, tok_stride_rows=n_seq, seq_stride_rows=1,
+                              scale=scale)
+    torch.cuda.synchronize()
+    assert rq.srftq_check_device() == 0
+    out = out.cpu().numpy()
+    sg, lm = sgn.cpu().numpy(), lam.cpu().numpy()
+    for b, h in ((0, 0), (17, 5), (31, 7)):
+        idx = torch.arange(n_ctx, device=DEV) * n_seq + b
+
+        def rows_of(t):
+            return t.index_select(0, idx)[:, h:h + 1].cpu().numpy()
+
+        ref = oracle.decode_attention(
+            q[b:b + 1, h:h + 1].cpu().numpy(), rows_of(kc), rows_of(ks).view(np.uint16),
+            sg[0, h:h + 1], lm[0, h:h + 1], rows_of(vc), rows_of(vs).view(np.uint16),
+            sg[1, h:h + 1], lm[1, h:h + 1], d, group, bits, rot, n_ctx, 1, 0, scale)[0, 0]
+        err = np.abs(out[b, h] - ref) / np.maximum(1.0, np.abs(ref))
+        assert err.max() < 1e-4, (b, h, float(err.max()))
+
+
 def test_decode_attention_sequence_major_layout_and_outliers():
     """Rows = sequence * n_ctx + token (the other common layout), and a
     cache with x25 outliers, whose scores spread over a wide range."""
