@@ -435,6 +435,37 @@ def test_dequantize_rotated_matches_oracle(d, bits, group):
     assert torch.all(big[:, :4] == 7.0) and torch.all(big[:, 4 + N:] == 7.0)
 
 
+def test_dequantize_rotated_full_decode_stream_layer_sampled():
+    """One decode-stream layer as the bench dequantises it in the rotated
+    domain: 2 slices (K, V) x 1,048,576 rows (32,768 tokens x 32 sequences)
+    x 8 heads, int4 G16, in one launch (the grid walks the slices in y and a
+    slice's 134 M chunks in x). Codes in [-7, 7], fp16 scales in [0.01,
+    0.3] and lambda in [0.5, 2] are drawn on the device; 4096 sampled rows
+    are checked against the oracle."""
+    import torch
+    S, N, H, d, group, bits = 2, 32768 * 32, 8, 128, 16, 4
+    gen = torch.Generator(device=DEV)
+    gen.manual_seed(77)
+    codes = torch.randint(0, 256, (S, N, H, d // 2), generator=gen, device=DEV,
+                          dtype=torch.int32).to(torch.uint8)
+    codes ^= ((codes & 0x0F) == 0x08).to(torch.uint8) * 0x08
+    codes ^= ((codes >> 4) == 0x08).to(torch.uint8) * 0x80
+    scales = (torch.rand((S, N, H, d // group), generator=gen, device=DEV) * 0.29
+              + 0.01).to(torch.float16)
+    lam = torch.rand((S, H, d), generator=gen, device=DEV) * 1.5 + 0.5
+    out = rq.dequantize_rotated(codes, scales, lam, d, group, bits)
+    torch.cuda.synchronize()
+    rows = torch.randint(0, N, (4096,), generator=gen, device=DEV)
+    rows[0], rows[-1] = 0, N - 1
+    for s_ in range(S):
+        c = codes[s_].index_select(0, rows).cpu().numpy()[None]
+        sc = scales[s_].index_select(0, rows).cpu().numpy().view(np.uint16)[None]
+        want = oracle.dequantize_rotated(c, sc, lam[s_:s_ + 1].cpu().numpy(), d, group, bits)
+        got = out[s_].index_select(0, rows).cpu().numpy().view(np.uint16)[None]
+        parity.assert_clean(parity.check_dequant(got, want["bits"]),
+                            f"rotated dequant, full layer, slice {s_}")
+
+
 @pytest.mark.parametrize("d", [16, 32, 64, 128, 256])
 @pytest.mark.parametrize("rot", [0, 1])
 def test_unrotate_matches_oracle_and_inverts_rotate(d, rot):
