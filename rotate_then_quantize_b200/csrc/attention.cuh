@@ -55,6 +55,9 @@ constexpr int kAttnWarps = 4;     // warps per CTA, each with its own online sof
 #ifndef SRFTQ_ATTN_STAGES
 #define SRFTQ_ATTN_STAGES 2
 #endif
+#ifndef SRFTQ_ATTN_VW
+#define SRFTQ_ATTN_VW 0   // 0: two words with one or two query heads, one with more
+#endif
 constexpr int kAttnStages = SRFTQ_ATTN_STAGES;   // 32-token chunks in flight per warp
 
 struct AttnArgs {
@@ -242,9 +245,6 @@ __global__ void __cluster_dims__(kAttnSplit, 1, 1)
   // value phase: each lane takes VW consecutive code words (8 VW
   // coordinates) of VT tokens; two words with one or two query heads (one
   // scale conversion per 16 codes), one with more (registers)
-#ifndef SRFTQ_ATTN_VW
-#define SRFTQ_ATTN_VW 0
-#endif
   constexpr int VW = SRFTQ_ATTN_VW > 0 ? SRFTQ_ATTN_VW : NQ <= 2 ? 2 : 1;
   constexpr int LPT = 16 / VW;              // lanes per token row
   constexpr int TPI = 32 / LPT;             // tokens per warp instruction
