@@ -81,9 +81,14 @@ def test_reference_arm_runs_on_rank_zero_only(monkeypatch, capsys):
 
 
 def test_end_to_end_chunks_cover_every_slice_once():
-    for n in (1, 2, 3, 4, 7, 8, 9, 56, 64, 100):
-        chunks = bench.e2e_chunks(n)
-        assert 1 <= len(chunks) <= 8
-        covered = [s for a, b in chunks for s in range(a, b)]
-        assert covered == list(range(n))
-        assert all(b > a for a, b in chunks)
+    for target in (1, 8, 28, 56, 200):
+        for n in (1, 2, 3, 4, 7, 8, 9, 28, 56, 64, 100):
+            chunks = bench.e2e_chunks(n, target)
+            assert len(chunks) == min(target, n)
+            covered = [s for a, b in chunks for s in range(a, b)]
+            assert covered == list(range(n))
+            assert all(b > a for a, b in chunks)
+            sizes = [b - a for a, b in chunks]
+            assert max(sizes) - min(sizes) <= 1   # balanced
+    # the Qwen-shaped cache (56 slices) at the default: 28 chunks of 2 slices
+    assert bench.e2e_chunks(56, 28) == [(2 * i, 2 * i + 2) for i in range(28)]
