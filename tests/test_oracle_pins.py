@@ -408,6 +408,41 @@ def _attn_cache(rng, rows, H, d, group, bits, kind):
     return qz["codes"][0], qz["scales"][0], s[0], lam[0]
 
 
+@pytest.mark.parametrize("kind", [0, 1])
+def test_decode_attention_is_order_free_and_tends_to_the_argmax(kind):
+    """Two more properties of the attention reference. Attention is a sum
+    over tokens, so reversing the token order of the K and V rows together
+    leaves every output unchanged (a mismatched K/V row or a wrong stride
+    breaks this). With the softmax scale large, the weights concentrate on
+    the token of the largest score, and the output tends to that token's
+    dequantised value."""
+    rng = np.random.default_rng(23)
+    H, d, group, bits, n_seq, n_ctx = 2, 16, 8, 4, 2, 6
+    rows = n_ctx * n_seq
+    kc, ks, ksg, kl = _attn_cache(rng, rows, H, d, group, bits, kind)
+    vc, vs, vsg, vl = _attn_cache(rng, rows, H, d, group, bits, kind)
+    q = rng.standard_normal((n_seq, H, d))
+    a = oracle.decode_attention(q, kc, ks, ksg, kl, vc, vs, vsg, vl, d, group, bits, kind,
+                                n_ctx, n_seq, 1, 0.3)
+    rev = np.array([(n_ctx - 1 - t) * n_seq + b for t in range(n_ctx) for b in range(n_seq)])
+    a_rev = oracle.decode_attention(q, kc[rev], ks[rev], ksg, kl, vc[rev], vs[rev], vsg, vl, d,
+                                    group, bits, kind, n_ctx, n_seq, 1, 0.3)
+    np.testing.assert_allclose(a, a_rev, rtol=1e-12, atol=1e-12)
+    kx = oracle.dequantize(kc[None], ks[None], ksg[None], kl[None], d, group, bits,
+                           kind)["xhat64"][0]
+    vx = oracle.dequantize(vc[None], vs[None], vsg[None], vl[None], d, group, bits,
+                           kind)["xhat64"][0]
+    hard = oracle.decode_attention(q, kc, ks, ksg, kl, vc, vs, vsg, vl, d, group, bits, kind,
+                                   n_ctx, n_seq, 1, 1e4)
+    for b in range(n_seq):
+        r = np.arange(n_ctx) * n_seq + b
+        for h in range(H):
+            scores = kx[r, h] @ q[b, h]
+            top = np.argsort(scores)[-2:]
+            assert scores[top[1]] - scores[top[0]] > 1e-2   # a clear maximum here
+            np.testing.assert_allclose(hard[b, h], vx[r[top[1]], h], rtol=1e-9, atol=1e-9)
+
+
 @pytest.mark.parametrize("kind", [oracle.SRFT, oracle.SRHT])
 def test_decode_attention_special_cases(kind):
     """Closed forms of the attention reference: one token gives that
