@@ -12,6 +12,7 @@ import numpy as np
 import oracle
 from oracle import srft_oracle as so
 from test_oracle_pins import (
+    attention_pin_errors,
     brute_force_dft_error,
     golden_pack_mismatches,
     golden_quant_mismatches,
@@ -133,3 +134,53 @@ def test_lambda_multiplied_on_quantise_is_caught():
         return so.quantize(x, signs, 1.0 / np.asarray(lam, dtype=np.float32), group, bits, kind)
     code_err, _ = lossless_roundtrip_error(quantize, oracle.dequantize, oracle.SRFT)
     assert code_err > 0
+
+
+def _attention_variant(*, v_lambda=True, v_signs_of_k=False, v_shift=0, use_scale=True):
+    """decode_attention written out from the oracle's own steps, with one
+    plausible error switched on."""
+    def attn(q, k_codes, k_scales, k_signs, k_lam, v_codes, v_scales, v_signs, v_lam, d, group,
+             bits, kind, n_ctx, tok_stride_rows, seq_stride_rows, scale):
+        q = np.asarray(q, dtype=np.float64)
+        n_seq, HQ, _ = q.shape
+        H = k_codes.shape[1]
+        Q = HQ // H
+        out = np.empty((n_seq, HQ, d))
+        vs_used = k_signs if v_signs_of_k else v_signs
+        vl_used = v_lam if v_lambda else np.ones_like(v_lam)
+        for b in range(n_seq):
+            rows = np.arange(n_ctx) * tok_stride_rows + b * seq_stride_rows
+            vrows = rows[(np.arange(n_ctx) + v_shift) % n_ctx]
+            kx = oracle.dequantize(k_codes[None, rows], k_scales[None, rows], k_signs[None],
+                                   k_lam[None], d, group, bits, kind)["xhat64"][0]
+            vx = oracle.dequantize(v_codes[None, vrows], v_scales[None, vrows], vs_used[None],
+                                   vl_used[None], d, group, bits, kind)["xhat64"][0]
+            for h in range(H):
+                for g in range(Q):
+                    s_ = (scale if use_scale else 1.0) * (kx[:, h, :] @ q[b, h * Q + g])
+                    p = np.exp(s_ - s_.max())
+                    out[b, h * Q + g] = (p / p.sum()) @ vx[:, h, :]
+        return out
+    return attn
+
+
+def test_unchanged_attention_variant_passes_the_pins():
+    assert max(attention_pin_errors(_attention_variant()).values()) < 1e-9
+
+
+def test_attention_values_without_lambda_are_caught():
+    assert attention_pin_errors(_attention_variant(v_lambda=False))["one_token"] > 1e-3
+
+
+def test_attention_values_with_the_key_signs_are_caught():
+    assert attention_pin_errors(_attention_variant(v_signs_of_k=True))["one_token"] > 1e-3
+
+
+def test_attention_values_one_token_off_are_caught():
+    err = attention_pin_errors(_attention_variant(v_shift=1))
+    assert err["zero_query"] < 1e-9      # the same set of values, so the mean holds ...
+    assert err["order"] > 1e-3           # ... but the K/V pairing does not
+
+
+def test_attention_without_the_softmax_scale_is_caught():
+    assert attention_pin_errors(_attention_variant(use_scale=False))["argmax"] > 1e-3

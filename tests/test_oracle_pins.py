@@ -408,6 +408,48 @@ def _attn_cache(rng, rows, H, d, group, bits, kind):
     return qz["codes"][0], qz["scales"][0], s[0], lam[0]
 
 
+def attention_pin_errors(attn, kind: int = 0) -> dict:
+    """The attention pins as numbers, for any implementation `attn` with the
+    signature of ``oracle.decode_attention`` (the planted-mistake tests reuse
+    this): the error of the one-token closed form, of the zero-query mean, of
+    token-order invariance, and of the large-scale argmax limit."""
+    rng = np.random.default_rng(31 + kind)
+    H, d, group, bits, n_seq, n_ctx = 2, 16, 8, 4, 2, 6
+    rows = n_ctx * n_seq
+    kc, ks, ksg, kl = _attn_cache(rng, rows, H, d, group, bits, kind)
+    vc, vs, vsg, vl = _attn_cache(rng, rows, H, d, group, bits, kind)
+    q = rng.standard_normal((n_seq, H, d))
+    args = (d, group, bits, kind)
+    kx = oracle.dequantize(kc[None], ks[None], ksg[None], kl[None], *args)["xhat64"][0]
+    vx = oracle.dequantize(vc[None], vs[None], vsg[None], vl[None], *args)["xhat64"][0]
+    err = {}
+    one = attn(q, kc, ks, ksg, kl, vc, vs, vsg, vl, *args, 1, n_seq, 1, 0.3)
+    err["one_token"] = float(np.abs(one - vx[:n_seq]).max())
+    zero = attn(np.zeros_like(q), kc, ks, ksg, kl, vc, vs, vsg, vl, *args, n_ctx, n_seq, 1, 0.3)
+    mean = np.stack([vx[np.arange(n_ctx) * n_seq + b].mean(axis=0) for b in range(n_seq)])
+    err["zero_query"] = float(np.abs(zero - mean).max())
+    a = attn(q, kc, ks, ksg, kl, vc, vs, vsg, vl, *args, n_ctx, n_seq, 1, 0.3)
+    rev = np.array([(n_ctx - 1 - t) * n_seq + b for t in range(n_ctx) for b in range(n_seq)])
+    a_rev = attn(q, kc[rev], ks[rev], ksg, kl, vc[rev], vs[rev], vsg, vl, *args, n_ctx, n_seq,
+                 1, 0.3)
+    err["order"] = float(np.abs(a - a_rev).max())
+    hard = attn(q, kc, ks, ksg, kl, vc, vs, vsg, vl, *args, n_ctx, n_seq, 1, 1e4)
+    e = 0.0
+    for b in range(n_seq):
+        r = np.arange(n_ctx) * n_seq + b
+        for h in range(H):
+            top = int(np.argmax(kx[r, h] @ q[b, h]))
+            e = max(e, float(np.abs(hard[b, h] - vx[r[top], h]).max()))
+    err["argmax"] = e
+    return err
+
+
+@pytest.mark.parametrize("kind", [0, 1])
+def test_attention_pins_hold_for_the_oracle(kind):
+    err = attention_pin_errors(oracle.decode_attention, kind)
+    assert max(err.values()) < 1e-9, err
+
+
 @pytest.mark.parametrize("kind", [0, 1])
 def test_decode_attention_is_order_free_and_tends_to_the_argmax(kind):
     """Two more properties of the attention reference. Attention is a sum
