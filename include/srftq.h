@@ -223,10 +223,14 @@ int srftq_decode_attention(const srftq_desc* desc, int64_t n_seq, int64_t n_ctx,
 const char* srftq_status_string(int status);
 
 /*
- * srftq_check_device -- synchronise `stream`, then read and clear the
- * library-wide device guard word of the current device. Returns SRFTQ_OK
- * if no guard fired since the last check, SRFTQ_ERR_DEVICE_CHECK if one
- * did (a bounded wait gave up), SRFTQ_ERR_CUDA on a runtime error.
+ * srftq_check_device -- reads and clears, in one atomic step on `stream`,
+ * the library-wide device guard word of the current device, then
+ * synchronises `stream` and returns SRFTQ_OK if no guard fired since the
+ * last check, SRFTQ_ERR_DEVICE_CHECK if one did (a bounded wait gave up),
+ * SRFTQ_ERR_CUDA on a runtime error. The step is one one-thread kernel on
+ * `stream`: codec work still running on other streams cannot lose a bit
+ * (a bit set after the step is reported by the next check). Work on other
+ * streams is not waited for; synchronise them first to include it.
  */
 int srftq_check_device(void* stream);
 

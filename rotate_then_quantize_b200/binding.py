@@ -17,9 +17,7 @@ import ctypes
 import os
 
 PKG_DIR = os.path.dirname(os.path.abspath(__file__))
-# SRFTQ_LIB may point at another build of the same library (e.g. a variant
-# under evaluation); by default the in-tree build is loaded.
-LIB_PATH = os.environ.get("SRFTQ_LIB") or os.path.join(PKG_DIR, "libsrftq.so")
+LIB_PATH = os.path.join(PKG_DIR, "libsrftq.so")
 
 SRFTQ_OK = 0
 SRFTQ_ERR_INVALID_ARG = -1
@@ -106,34 +104,75 @@ def _stream_handle(stream) -> int:
     return int(stream.cuda_stream)
 
 
-def _rows_view(t, H: int, row_elems: int, name: str):
-    """(pointer, n_slices, n_rows, slice_stride_rows) of a [S, N, H, e] view."""
+def _rows_layout(t, H: int, row_elems: int, name: str):
+    """(pointer, n_slices, n_rows, slice_stride_rows) of a [S, N, H, e] view.
+
+    Each row's heads and elements must be contiguous; slices may sit further
+    apart than N rows (a window of a larger cache) but must not overlap, so a
+    view whose slice stride is below N rows (an expanded or overlapping
+    view) is refused before anything reaches the library."""
     if t.dim() != 4 or t.shape[2] != H or t.shape[3] != row_elems:
         raise ValueError(f"{name}: expected [S, N, {H}, {row_elems}], got {tuple(t.shape)}")
-    if t.stride(3) != 1 or t.stride(2) != row_elems or t.stride(1) != H * row_elems:
+    S, N = t.shape[0], t.shape[1]
+    if N > 1 and t.stride(1) != H * row_elems:
         raise ValueError(f"{name}: heads and elements of a row must be contiguous")
+    if t.stride(3) != 1 or t.stride(2) != row_elems:
+        raise ValueError(f"{name}: heads and elements of a row must be contiguous")
+    if S <= 1:
+        return t.data_ptr(), S, N, N
     if t.stride(0) % (H * row_elems) != 0:
         raise ValueError(f"{name}: slice stride must be a whole number of rows")
-    stride_rows = t.stride(0) // (H * row_elems) if t.shape[0] > 1 else t.shape[1]
-    return t.data_ptr(), t.shape[0], t.shape[1], max(stride_rows, t.shape[1])
+    stride_rows = t.stride(0) // (H * row_elems)
+    if stride_rows < N:
+        raise ValueError(f"{name}: slices overlap (slice stride {stride_rows} rows < {N} rows)")
+    return t.data_ptr(), S, N, stride_rows
 
 
-def _table(t, S: int, H: int, d: int, name: str):
+def _check_tensor(t, dtype, name: str):
+    """t must live on the current CUDA device and have the dtype the C ABI reads."""
+    import torch
+
+    if not isinstance(t, torch.Tensor):
+        raise ValueError(f"{name}: expected a torch tensor, got {type(t).__name__}")
+    if t.dtype != dtype:
+        raise ValueError(f"{name}: expected dtype {dtype}, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name}: expected a CUDA tensor, got one on {t.device}")
+    if t.device.index != torch.cuda.current_device():
+        raise ValueError(f"{name}: on {t.device}, but the current device is "
+                         f"cuda:{torch.cuda.current_device()}")
+
+
+def _rows_view(t, H: int, row_elems: int, name: str, dtype):
+    _check_tensor(t, dtype, name)
+    return _rows_layout(t, H, row_elems, name)
+
+
+def _table(t, S: int, H: int, d: int, name: str, dtype):
+    _check_tensor(t, dtype, name)
     if tuple(t.shape) != (S, H, d) or not t.is_contiguous():
         raise ValueError(f"{name}: expected contiguous [{S}, {H}, {d}], got {tuple(t.shape)}")
     return t.data_ptr()
 
 
+def _dtypes():
+    import torch
+
+    return torch.float16, torch.uint8, torch.int8, torch.float32
+
+
 def srftq_quantize(desc: SrftqDesc, x, signs, lam, codes, scales, stream=None) -> None:
     """x [S,N,H,d] fp16 -> codes [S,N,H,d*bits/8] uint8, scales [S,N,H,d/G] fp16."""
     lib = load_library()
-    px, S, N, xs = _rows_view(x, desc.heads, desc.d, "x")
-    pc, S2, N2, os_ = _rows_view(codes, desc.heads, desc.d * desc.bits // 8, "codes")
-    ps, S3, N3, os2 = _rows_view(scales, desc.heads, desc.d // desc.group, "scales")
+    F16, U8, I8, F32 = _dtypes()
+    H, d = desc.heads, desc.d
+    px, S, N, xs = _rows_view(x, H, d, "x", F16)
+    pc, S2, N2, os_ = _rows_view(codes, H, d * desc.bits // 8, "codes", U8)
+    ps, S3, N3, os2 = _rows_view(scales, H, d // desc.group, "scales", F16)
     if (S2, N2) != (S, N) or (S3, N3) != (S, N) or os2 != os_:
         raise ValueError("codes/scales must match x's slices and rows and share a slice stride")
-    st = lib.srftq_quantize(ctypes.byref(desc), S, N, px, xs, _table(signs, S, desc.heads, desc.d, "signs"),
-                            _table(lam, S, desc.heads, desc.d, "lambda"), pc, ps, os_,
+    st = lib.srftq_quantize(ctypes.byref(desc), S, N, px, xs, _table(signs, S, H, d, "signs", I8),
+                            _table(lam, S, H, d, "lambda", F32), pc, ps, os_,
                             _stream_handle(stream))
     _check("srftq_quantize", st)
 
@@ -141,14 +180,16 @@ def srftq_quantize(desc: SrftqDesc, x, signs, lam, codes, scales, stream=None) -
 def srftq_dequantize(desc: SrftqDesc, codes, scales, signs, lam, xhat, stream=None) -> None:
     """codes, scales -> xhat [S,N,H,d] fp16 (the inverse of srftq_quantize)."""
     lib = load_library()
-    pc, S, N, is_ = _rows_view(codes, desc.heads, desc.d * desc.bits // 8, "codes")
-    ps, S2, N2, is2 = _rows_view(scales, desc.heads, desc.d // desc.group, "scales")
-    px, S3, N3, os_ = _rows_view(xhat, desc.heads, desc.d, "xhat")
+    F16, U8, I8, F32 = _dtypes()
+    H, d = desc.heads, desc.d
+    pc, S, N, is_ = _rows_view(codes, H, d * desc.bits // 8, "codes", U8)
+    ps, S2, N2, is2 = _rows_view(scales, H, d // desc.group, "scales", F16)
+    px, S3, N3, os_ = _rows_view(xhat, H, d, "xhat", F16)
     if (S2, N2) != (S, N) or (S3, N3) != (S, N) or is2 != is_:
         raise ValueError("codes/scales/xhat shapes disagree")
     st = lib.srftq_dequantize(ctypes.byref(desc), S, N, pc, ps, is_,
-                              _table(signs, S, desc.heads, desc.d, "signs"),
-                              _table(lam, S, desc.heads, desc.d, "lambda"), px, os_,
+                              _table(signs, S, H, d, "signs", I8),
+                              _table(lam, S, H, d, "lambda", F32), px, os_,
                               _stream_handle(stream))
     _check("srftq_dequantize", st)
 
@@ -156,12 +197,14 @@ def srftq_dequantize(desc: SrftqDesc, codes, scales, signs, lam, xhat, stream=No
 def srftq_calibrate_lambda(desc: SrftqDesc, x, signs, lam_out, n_cal: int, stream=None) -> None:
     """lambda_out [S,H,d] float32 = RMS of the rotated first n_cal rows of x."""
     lib = load_library()
-    px, S, N, xs = _rows_view(x, desc.heads, desc.d, "x")
+    F16, U8, I8, F32 = _dtypes()
+    H, d = desc.heads, desc.d
+    px, S, N, xs = _rows_view(x, H, d, "x", F16)
     if n_cal > N:
         raise ValueError("n_cal exceeds the rows of x")
     st = lib.srftq_calibrate_lambda(ctypes.byref(desc), S, int(n_cal), px, xs,
-                                    _table(signs, S, desc.heads, desc.d, "signs"),
-                                    _table(lam_out, S, desc.heads, desc.d, "lambda_out"),
+                                    _table(signs, S, H, d, "signs", I8),
+                                    _table(lam_out, S, H, d, "lambda_out", F32),
                                     _stream_handle(stream))
     _check("srftq_calibrate_lambda", st)
 
@@ -169,26 +212,30 @@ def srftq_calibrate_lambda(desc: SrftqDesc, x, signs, lam_out, n_cal: int, strea
 def srftq_rotate(desc: SrftqDesc, x, signs, y_out, lam=None, stream=None) -> None:
     """y_out [S,N,H,d] float32 (contiguous) = R (s*x), divided by lambda if given."""
     lib = load_library()
-    px, S, N, xs = _rows_view(x, desc.heads, desc.d, "x")
-    if tuple(y_out.shape) != (S, N, desc.heads, desc.d) or not y_out.is_contiguous():
+    F16, U8, I8, F32 = _dtypes()
+    H, d = desc.heads, desc.d
+    px, S, N, xs = _rows_view(x, H, d, "x", F16)
+    _check_tensor(y_out, F32, "y_out")
+    if tuple(y_out.shape) != (S, N, H, d) or not y_out.is_contiguous():
         raise ValueError("y_out must be a contiguous [S, N, H, d] float32 tensor")
-    pl = _table(lam, S, desc.heads, desc.d, "lambda") if lam is not None else None
-    st = lib.srftq_rotate(ctypes.byref(desc), S, N, px, xs,
-                          _table(signs, S, desc.heads, desc.d, "signs"), pl, y_out.data_ptr(),
-                          _stream_handle(stream))
+    pl = _table(lam, S, H, d, "lambda", F32) if lam is not None else None
+    st = lib.srftq_rotate(ctypes.byref(desc), S, N, px, xs, _table(signs, S, H, d, "signs", I8),
+                          pl, y_out.data_ptr(), _stream_handle(stream))
     _check("srftq_rotate", st)
 
 
 def srftq_dequantize_rotated(desc: SrftqDesc, codes, scales, lam, out, stream=None) -> None:
     """codes, scales -> out [S,N,H,d] fp16 = lambda * sigma * q (the rotated domain)."""
     lib = load_library()
-    pc, S, N, is_ = _rows_view(codes, desc.heads, desc.d * desc.bits // 8, "codes")
-    ps, S2, N2, is2 = _rows_view(scales, desc.heads, desc.d // desc.group, "scales")
-    po, S3, N3, os_ = _rows_view(out, desc.heads, desc.d, "out")
+    F16, U8, I8, F32 = _dtypes()
+    H, d = desc.heads, desc.d
+    pc, S, N, is_ = _rows_view(codes, H, d * desc.bits // 8, "codes", U8)
+    ps, S2, N2, is2 = _rows_view(scales, H, d // desc.group, "scales", F16)
+    po, S3, N3, os_ = _rows_view(out, H, d, "out", F16)
     if (S2, N2) != (S, N) or (S3, N3) != (S, N) or is2 != is_:
         raise ValueError("codes/scales/out shapes disagree")
     st = lib.srftq_dequantize_rotated(ctypes.byref(desc), S, N, pc, ps, is_,
-                                      _table(lam, S, desc.heads, desc.d, "lambda"), po, os_,
+                                      _table(lam, S, H, d, "lambda", F32), po, os_,
                                       _stream_handle(stream))
     _check("srftq_dequantize_rotated", st)
 
@@ -196,18 +243,20 @@ def srftq_dequantize_rotated(desc: SrftqDesc, codes, scales, lam, out, stream=No
 def srftq_unrotate(desc: SrftqDesc, y, signs, x_out, stream=None) -> None:
     """x_out [S,N,H,d] float32 = s * R^T y for y [S,N,H,d] float32."""
     lib = load_library()
-    py, S, N, ys = _rows_view(y, desc.heads, desc.d, "y")
-    px, S2, N2, xs = _rows_view(x_out, desc.heads, desc.d, "x_out")
+    F16, U8, I8, F32 = _dtypes()
+    H, d = desc.heads, desc.d
+    py, S, N, ys = _rows_view(y, H, d, "y", F32)
+    px, S2, N2, xs = _rows_view(x_out, H, d, "x_out", F32)
     if (S2, N2) != (S, N):
         raise ValueError("y/x_out shapes disagree")
-    st = lib.srftq_unrotate(ctypes.byref(desc), S, N, py, ys,
-                            _table(signs, S, desc.heads, desc.d, "signs"), px, xs,
-                            _stream_handle(stream))
+    st = lib.srftq_unrotate(ctypes.byref(desc), S, N, py, ys, _table(signs, S, H, d, "signs", I8),
+                            px, xs, _stream_handle(stream))
     _check("srftq_unrotate", st)
 
 
-def _cache_rows(t, H: int, row_elems: int, name: str):
+def _cache_rows(t, H: int, row_elems: int, name: str, dtype):
     """(pointer, rows) of a contiguous [rows, H, e] cache tensor."""
+    _check_tensor(t, dtype, name)
     if t.dim() != 3 or t.shape[1] != H or t.shape[2] != row_elems or not t.is_contiguous():
         raise ValueError(f"{name}: expected contiguous [rows, {H}, {row_elems}], got "
                          f"{tuple(t.shape)}")
@@ -223,22 +272,26 @@ def srftq_decode_attention(desc: SrftqDesc, q, k_codes, k_scales, k_signs, k_lam
     three launches on the stream and uses `out` as their scratch, so `out`
     holds the result once that work is complete."""
     lib = load_library()
+    F16, U8, I8, F32 = _dtypes()
     H, d = desc.heads, desc.d
+    _check_tensor(q, F16, "q")
     if q.dim() != 3 or q.shape[1] % H or q.shape[2] != d or not q.is_contiguous():
         raise ValueError(f"q: expected contiguous [n_seq, {H}*q_per_kv, {d}]")
     n_seq, q_per_kv = q.shape[0], q.shape[1] // H
+    _check_tensor(out, F32, "out")
     if tuple(out.shape) != tuple(q.shape) or not out.is_contiguous():
         raise ValueError("out must be a contiguous float32 tensor shaped like q")
     cb, ng = d * desc.bits // 8, d // desc.group
-    pk, rk = _cache_rows(k_codes, H, cb, "k_codes")
-    pks, rks = _cache_rows(k_scales, H, ng, "k_scales")
-    pv, rv = _cache_rows(v_codes, H, cb, "v_codes")
-    pvs, rvs = _cache_rows(v_scales, H, ng, "v_scales")
+    pk, rk = _cache_rows(k_codes, H, cb, "k_codes", U8)
+    pks, rks = _cache_rows(k_scales, H, ng, "k_scales", F16)
+    pv, rv = _cache_rows(v_codes, H, cb, "v_codes", U8)
+    pvs, rvs = _cache_rows(v_scales, H, ng, "v_scales", F16)
     need = (n_ctx - 1) * tok_stride_rows + (n_seq - 1) * seq_stride_rows + 1 if n_seq else 0
     if min(rk, rks, rv, rvs) < need:
         raise ValueError(f"the caches hold fewer than the {need} rows addressed")
-    for t, name in ((k_signs, "k_signs"), (v_signs, "v_signs"), (k_lambda, "k_lambda"),
-                    (v_lambda, "v_lambda")):
+    for t, name, dt in ((k_signs, "k_signs", I8), (v_signs, "v_signs", I8),
+                        (k_lambda, "k_lambda", F32), (v_lambda, "v_lambda", F32)):
+        _check_tensor(t, dt, name)
         if tuple(t.shape) != (H, d) or not t.is_contiguous():
             raise ValueError(f"{name}: expected contiguous [{H}, {d}]")
     st = lib.srftq_decode_attention(ctypes.byref(desc), n_seq, int(n_ctx), q_per_kv, q.data_ptr(),

@@ -4,7 +4,8 @@ Each translation unit under csrc/ compiles in parallel to an object file in
 _build/ at the repository root; the objects are linked into
 rotate_then_quantize_b200/libsrftq.so. An object is rebuilt when it is older
 than its source or any header it may include (all of csrc/*.cuh and
-include/*.h). Usage: ``python -m rotate_then_quantize_b200.build [-j N] [--force]``.
+include/*.h). Usage:
+``python -m rotate_then_quantize_b200.build [-j N] [--force] [--debug]``.
 """
 
 from __future__ import annotations
@@ -21,6 +22,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libsrftq.so")
+LIB_DEBUG = os.path.join(PKG, "libsrftq_debug.so")
 
 NVCC = os.environ.get("NVCC", "nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -38,12 +40,12 @@ def _deps_mtime():
     return max(os.path.getmtime(p) for p in deps)
 
 
-def _compile(src: str, force: bool, verbose_ptxas: bool):
-    obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
+def _compile(src: str, force: bool, verbose_ptxas: bool, build_dir: str, flags: list):
+    obj = os.path.join(build_dir, os.path.basename(src)[:-3] + ".o")
     if (not force and os.path.exists(obj)
             and os.path.getmtime(obj) >= max(os.path.getmtime(src), _deps_mtime())):
         return obj, None
-    cmd = [NVCC, *ARCH, *FLAGS, "-c", src, "-o", obj]
+    cmd = [NVCC, *ARCH, *flags, "-c", src, "-o", obj]
     if verbose_ptxas:
         cmd.insert(1, "-Xptxas=-v")
     r = subprocess.run(cmd, capture_output=True, text=True)
@@ -53,43 +55,37 @@ def _compile(src: str, force: bool, verbose_ptxas: bool):
 
 
 def build(jobs: int | None = None, force: bool = False, verbose_ptxas: bool = False,
-          defines: tuple = (), out_dir: str | None = None, src_dir: str | None = None) -> str:
-    """Compiles every csrc/*.cu for sm_100a and links libsrftq.so; returns its path.
+          debug: bool = False) -> str:
+    """Compiles every csrc/*.cu for sm_100a and links the in-tree library; returns its path.
 
-    `defines` (NAME=VALUE strings), `src_dir` and `out_dir` build a variant
-    of the library in a separate directory instead of the in-tree one."""
-    global BUILD, LIB, CSRC
-    if src_dir:
-        if not out_dir:
-            raise ValueError("a build from other sources needs its own out_dir")
-        CSRC = os.path.abspath(src_dir)
-    if defines or out_dir:
-        if not out_dir:
-            raise ValueError("a variant build needs its own out_dir")
-        BUILD, LIB = os.path.join(out_dir, "obj"), os.path.join(out_dir, "libsrftq.so")
-        FLAGS.extend(f"-D{d}" for d in defines)
-    os.makedirs(BUILD, exist_ok=True)
+    debug=True builds libsrftq_debug.so instead (objects in _build/debug,
+    -DSRFTQ_DEBUG_CHECKS=1): the same kernels with index checks that record
+    an out-of-range access in the device guard word instead of making it."""
+    build_dir = os.path.join(BUILD, "debug") if debug else BUILD
+    lib = LIB_DEBUG if debug else LIB
+    flags = FLAGS + (["-DSRFTQ_DEBUG_CHECKS=1"] if debug else [])
+    os.makedirs(build_dir, exist_ok=True)
     srcs = _sources()
     jobs = jobs or min(len(srcs), os.cpu_count() or 4)
     logs = []
     with cf.ThreadPoolExecutor(max_workers=jobs) as ex:
-        futs = [ex.submit(_compile, s, force, verbose_ptxas) for s in srcs]
+        futs = [ex.submit(_compile, s, force, verbose_ptxas, build_dir, flags) for s in srcs]
         objs = []
         for f in futs:
             obj, log = f.result()
             objs.append(obj)
             if log:
                 logs.append(log)
-    if (force or not os.path.exists(LIB)
-            or os.path.getmtime(LIB) < max(os.path.getmtime(o) for o in objs)):
-        cmd = [NVCC, *ARCH, "-shared", "-o", LIB, *objs, "-lcudart"]
+    if (force or not os.path.exists(lib)
+            or os.path.getmtime(lib) < max(os.path.getmtime(o) for o in objs)):
+        cmd = [NVCC, *ARCH, "-shared", "-o", lib, *objs, "-lcudart"]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"link failed:\n{r.stderr[-8000:]}")
     if verbose_ptxas:
-        with open(os.path.join(BUILD, "ptxas.log"), "w") as f:
+        with open(os.path.join(build_dir, "ptxas.log"), "w") as f:
             f.write("\n".join(logs))
-    return LIB
+    return lib
 
 
 def main(argv=None):
@@ -98,14 +94,10 @@ def main(argv=None):
     ap.add_argument("--force", action="store_true")
     ap.add_argument("--ptxas-verbose", action="store_true",
                     help="write ptxas register/spill reports to _build/ptxas.log")
-    ap.add_argument("-D", dest="defines", action="append", default=[],
-                    help="extra preprocessor definition (variant builds)")
-    ap.add_argument("--out-dir", default=None, help="directory of a variant build")
-    ap.add_argument("--src", default=None, help="build these sources instead of csrc/")
+    ap.add_argument("--debug", action="store_true",
+                    help="build libsrftq_debug.so, the kernels with device-side index checks")
     args = ap.parse_args(argv)
-    path = build(args.jobs, args.force, args.ptxas_verbose, tuple(args.defines), args.out_dir,
-                 args.src)
-    print(path)
+    print(build(args.jobs, args.force, args.ptxas_verbose, args.debug))
 
 
 if __name__ == "__main__":

@@ -12,8 +12,10 @@
 #include "launch.cuh"
 #include "ptx.cuh"
 
-// Library-wide device guard word (one per device that loads the module).
+// Library-wide device guard word (one per device that loads the module), and
+// the word srftq_check_device reads it into.
 __device__ unsigned g_srftq_guard;
+__device__ unsigned g_srftq_guard_taken;
 
 namespace srftq {
 // One thread waits on a barrier that nothing arrives on, `polls` times at
@@ -25,6 +27,13 @@ __global__ void probe_wait_timeout_kernel(unsigned* guard, uint32_t polls) {
   for (uint32_t i = 0; i < polls; ++i)
     if (mbar_try_wait(&bar, 0)) return;
   atomicOr(guard, kGuardWaitTimeout);
+}
+
+// Reads and clears the guard word in one atomic step, so a bit that another
+// stream's kernel sets meanwhile is either reported now or kept for the next
+// check, never lost.
+__global__ void take_guard_kernel(unsigned* guard, unsigned* taken) {
+  *taken = atomicExch(guard, 0u);
 }
 }  // namespace srftq
 
@@ -256,13 +265,18 @@ const char* srftq_status_string(int status) {
 }
 
 int srftq_check_device(void* stream) {
-  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return SRFTQ_ERR_CUDA;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  unsigned* guard = srftq::Runtime::guard_word();
+  void* taken = nullptr;
+  if (!guard || cudaGetSymbolAddress(&taken, g_srftq_guard_taken) != cudaSuccess)
+    return SRFTQ_ERR_CUDA;
+  srftq::take_guard_kernel<<<1, 1, 0, st>>>(guard, static_cast<unsigned*>(taken));
+  if (cudaGetLastError() != cudaSuccess) return SRFTQ_ERR_CUDA;
   unsigned v = 0;
-  if (cudaMemcpyFromSymbol(&v, g_srftq_guard, sizeof(v)) != cudaSuccess) return SRFTQ_ERR_CUDA;
-  if (v == 0) return SRFTQ_OK;
-  const unsigned zero = 0;
-  if (cudaMemcpyToSymbol(g_srftq_guard, &zero, sizeof(zero)) != cudaSuccess) return SRFTQ_ERR_CUDA;
-  return SRFTQ_ERR_DEVICE_CHECK;
+  if (cudaMemcpyAsync(&v, taken, sizeof(v), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+      cudaStreamSynchronize(st) != cudaSuccess)
+    return SRFTQ_ERR_CUDA;
+  return v == 0 ? SRFTQ_OK : SRFTQ_ERR_DEVICE_CHECK;
 }
 
 int srftq_dequantize_rotated(const srftq_desc* desc, int64_t n_slices, int64_t n_rows,

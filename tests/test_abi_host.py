@@ -168,6 +168,66 @@ def test_python_binding_rejects_bad_views():
     torch = pytest.importorskip("torch")
     x = torch.zeros((2, 8, 3, 64), dtype=torch.float16)
     with pytest.raises(ValueError):
-        b._rows_view(x.transpose(1, 2), 3, 64, "x")
-    ptr, S, N, stride = b._rows_view(x[:, 2:6], 3, 64, "x")
+        b._rows_layout(x.transpose(1, 2), 3, 64, "x")
+    ptr, S, N, stride = b._rows_layout(x[:, 2:6], 3, 64, "x")
     assert (S, N, stride) == (2, 4, 8)
+
+
+def test_python_binding_refuses_overlapping_slices():
+    """An expanded view (slice stride 0) or any view whose slices sit closer
+    than N rows would make the library walk S * N rows of a smaller
+    allocation; the binding refuses it before the C ABI is called."""
+    torch = pytest.importorskip("torch")
+    x = torch.zeros((1, 8, 2, 64), dtype=torch.float16)
+    with pytest.raises(ValueError, match="overlap"):
+        b._rows_layout(x.expand(3, 8, 2, 64), 2, 64, "x")
+    big = torch.zeros((16, 2, 64), dtype=torch.float16)
+    overlapping = big.as_strided((2, 8, 2, 64), (4 * 128, 128, 64, 1))   # slice stride 4 < 8 rows
+    with pytest.raises(ValueError, match="overlap"):
+        b._rows_layout(overlapping, 2, 64, "x")
+    # one slice: the stride is irrelevant and the rows are passed as the stride
+    assert b._rows_layout(x.expand(1, 8, 2, 64), 2, 64, "x")[1:] == (1, 8, 8)
+    desc = rq.make_desc(64, 2, 16, 4)
+    codes = torch.zeros((1, 8, 2, 32), dtype=torch.uint8).expand(3, 8, 2, 32)
+    scales = torch.zeros((1, 8, 2, 4), dtype=torch.float16).expand(3, 8, 2, 4)
+    signs = torch.ones((3, 2, 64), dtype=torch.int8)
+    lam = torch.ones((3, 2, 64))
+    with pytest.raises(ValueError):
+        rq.srftq_quantize(desc, x.expand(3, 8, 2, 64), signs, lam, codes, scales)
+    with pytest.raises(ValueError):
+        rq.srftq_dequantize(desc, codes, scales, signs, lam, x.expand(3, 8, 2, 64))
+
+
+def test_python_binding_refuses_host_tensors_and_wrong_dtypes():
+    """The binding passes data pointers to device code, so a host tensor or a
+    tensor of another dtype (read as fp16, say) is refused with ValueError
+    before the library is called."""
+    torch = pytest.importorskip("torch")
+    desc = rq.make_desc(64, 2, 16, 4)
+    S, N, H, d = 2, 8, 2, 64
+    good = dict(x=torch.zeros((S, N, H, d), dtype=torch.float16),
+                signs=torch.ones((S, H, d), dtype=torch.int8),
+                lam=torch.ones((S, H, d), dtype=torch.float32),
+                codes=torch.zeros((S, N, H, d // 2), dtype=torch.uint8),
+                scales=torch.zeros((S, N, H, d // 16), dtype=torch.float16))
+    # host tensors of the right dtypes: refused for their device
+    with pytest.raises(ValueError, match="CUDA"):
+        rq.srftq_quantize(desc, **good)
+    for name, wrong in (("x", torch.float32), ("x", torch.bfloat16), ("signs", torch.uint8),
+                        ("lam", torch.float64), ("codes", torch.int8),
+                        ("scales", torch.float32)):
+        args = dict(good)
+        args[name] = good[name].to(wrong)
+        with pytest.raises(ValueError):
+            rq.srftq_quantize(desc, **args)
+        # the dtype is checked before the device
+        with pytest.raises(ValueError, match="dtype"):
+            b._check_tensor(args[name], good[name].dtype, name)
+    with pytest.raises(ValueError):
+        rq.srftq_dequantize(desc, good["codes"], good["scales"], good["signs"], good["lam"],
+                            good["x"].float())
+    with pytest.raises(ValueError):
+        rq.srftq_rotate(desc, good["x"], good["signs"], torch.zeros((S, N, H, d)))
+    with pytest.raises(ValueError):
+        rq.srftq_unrotate(desc, torch.zeros((S, N, H, d)), good["signs"],
+                          torch.zeros((S, N, H, d)))
