@@ -63,6 +63,9 @@ def parse_args(argv=None):
                          "(28 measured best on the Qwen-shaped step: 119 GB/s against 115 at 8)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-other-configs", action="store_true",
+                    help="skip the other_configs object (the other workloads' kernels, "
+                         "measured after the headline)")
     ap.add_argument("--cpu-sample", type=int, default=8192,
                     help="vectors per oracle step of the reference arm")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
@@ -422,6 +425,10 @@ def run_ours(args):
     }
     if e2e is not None:
         line["e2e"] = e2e
+    if world == 1 and not args.no_other_configs and args.slices is None:
+        del x, codes, scales, xhat
+        torch.cuda.empty_cache()
+        line["other_configs"] = other_configs(rq, dev)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, rot, args.cpu_seconds)
     if rank == 0:
@@ -430,6 +437,133 @@ def run_ours(args):
         pg.barrier()
         pg.destroy_process_group()
     return 0
+
+
+def _time_launches(fn, iters: int, warmup: int = 3) -> float:
+    """Mean CUDA-event duration (ms) of fn() on the current stream."""
+    import torch
+
+    for _ in range(warmup):
+        fn()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(iters)]
+    torch.cuda.synchronize()
+    for a, b in evs:
+        a.record()
+        fn()
+        b.record()
+    torch.cuda.synchronize()
+    return statistics.mean(a.elapsed_time(b) for a, b in evs)
+
+
+def _codec_figures(rq, w, rot, dev, iters):
+    """Quantise and dequantise GB/s of one workload at full size (one launch each)."""
+    import torch
+
+    x = kv_synth.make_x_torch(w, dev, seed=0)
+    signs = torch.from_numpy(kv_synth.rademacher_signs(w.S, w.H, w.d, seed=1)).to(dev)
+    desc = rq.make_desc(w.d, w.H, w.group, w.bits, rot)
+    lam = torch.empty((w.S, w.H, w.d), dtype=torch.float32, device=dev)
+    rq.srftq_calibrate_lambda(desc, x, signs, lam, w.n_cal)
+    codes = torch.empty((w.S, w.N, w.H, w.d * w.bits // 8), dtype=torch.uint8, device=dev)
+    scales = torch.empty((w.S, w.N, w.H, w.d // w.group), dtype=torch.float16, device=dev)
+    xhat = torch.empty_like(x)
+    q_ms = _time_launches(lambda: rq.srftq_quantize(desc, x, signs, lam, codes, scales), iters)
+    d_ms = _time_launches(lambda: rq.srftq_dequantize(desc, codes, scales, signs, lam, xhat),
+                          iters)
+    if rq.srftq_check_device() != 0:
+        raise RuntimeError(f"device guard fired in {w.name}")
+    peak = read_peak()[0]
+    b = w.vectors * w.bytes_per_vector()
+    out = {"rotation": "SRFT" if rot == 0 else "SRHT", "vectors": w.vectors,
+           "bytes_per_launch": b, "launches_timed": iters,
+           "quantize_ms": q_ms, "quantize_GBps": b / q_ms / 1e6,
+           "quantize_frac": b / q_ms / 1e6 / peak,
+           "dequantize_ms": d_ms, "dequantize_GBps": b / d_ms / 1e6,
+           "dequantize_frac": b / d_ms / 1e6 / peak,
+           "kernels": [codec_kernel("quantize", w.d), codec_kernel("dequantize", w.d)],
+           "rel_l2_error": round_trip_error(x, xhat)}
+    del x, codes, scales, xhat
+    torch.cuda.empty_cache()
+    return out
+
+
+def _attention_figures(rq, dev, iters):
+    """The fused decode attention on one decode-stream layer: 32 sequences x 8
+    KV heads over 32,768 cached int4 tokens (K and V), one query per KV head."""
+    import torch
+
+    w = kv_synth.WORKLOADS["decode_stream_d128"]
+    B = 32
+    n_ctx = w.N // B
+    x = kv_synth.make_x_torch(w, dev, seed=0, slices=range(2))
+    signs = torch.from_numpy(kv_synth.rademacher_signs(2, w.H, w.d, seed=1)).to(dev)
+    desc = rq.make_desc(w.d, w.H, w.group, w.bits, 0)
+    lam = torch.empty((2, w.H, w.d), dtype=torch.float32, device=dev)
+    rq.srftq_calibrate_lambda(desc, x, signs, lam, w.n_cal)
+    codes = torch.empty((2, w.N, w.H, w.d * w.bits // 8), dtype=torch.uint8, device=dev)
+    scales = torch.empty((2, w.N, w.H, w.d // w.group), dtype=torch.float16, device=dev)
+    rq.srftq_quantize(desc, x, signs, lam, codes, scales)
+    fp16_ms = _time_launches(lambda: torch.sum(x, dtype=torch.float32), iters)
+    del x
+    torch.cuda.empty_cache()
+    q = torch.randn((B, w.H, w.d), device=dev).to(torch.float16)
+    out = torch.empty((B, w.H, w.d), dtype=torch.float32, device=dev)
+    a_ms = _time_launches(lambda: rq.srftq_decode_attention(
+        desc, q, codes[0], scales[0], signs[0], lam[0], codes[1], scales[1], signs[1], lam[1],
+        n_ctx, B, 1, 1.0 / math.sqrt(w.d), out), iters)
+    if rq.srftq_check_device() != 0:
+        raise RuntimeError("device guard fired in the fused attention")
+    b = 2 * w.N * w.H * (w.d * w.bits // 8 + 2 * (w.d // w.group))
+    peak = read_peak()[0]
+    del codes, scales
+    torch.cuda.empty_cache()
+    return {"layer": "32 sequences x 8 KV heads x 32768 cached tokens, int4 G16 K and V, "
+                     "one query per KV head (srftq_decode_attention: 3 launches)",
+            "ms_per_layer": a_ms, "codes_and_scales_bytes": b, "GBps": b / a_ms / 1e6,
+            "frac": b / a_ms / 1e6 / peak, "launches_timed": iters,
+            "fp16_read_ms_per_layer": fp16_ms,
+            "over_fp16_read": a_ms / fp16_ms,
+            "fp16_read": "torch.sum over the layer's fp16 K and V (the same tokens)"}
+
+
+def parity_report():
+    """Counts from the committed full-data parity report (written by
+    tests/test_gpu_full_data.py), or None."""
+    p = os.path.join(ROOT, "profiles", "parity_full_data.json")
+    try:
+        with open(p) as f:
+            data = json.load(f)
+    except Exception:
+        return None
+    keep = ("vectors", "codes", "code_mismatch_in_band", "code_violations",
+            "scale_mismatch_in_band", "scale_violations", "zero_scale_groups",
+            "dequant_violations", "dequant_max_err_over_tol")
+    return {"source": "profiles/parity_full_data.json (tests/test_gpu_full_data.py, every "
+                      "vector against the oracle)",
+            **{k: {f: v[f] for f in keep if f in v} for k, v in data.items()
+               if isinstance(v, dict) and "vectors" in v}}
+
+
+def other_configs(rq, dev, iters=50):
+    """The other workloads' kernels at full size, measured after the headline
+    and outside its timed region: long-context int8 (SRFT and SRHT side by
+    side, with their round-trip errors), the Gemma-shaped d = 256 cache and
+    the fused decode attention of one decode-stream layer."""
+    out = {}
+    lc = kv_synth.WORKLOADS["longctx_int8_d128"]
+    srft = _codec_figures(rq, lc, 0, dev, iters)
+    srht = _codec_figures(rq, lc, 1, dev, iters)
+    out["longctx_int8_d128"] = {"SRFT": srft, "SRHT": srht,
+                                "rel_l2_mean_srft_vs_srht": [srft["rel_l2_error"]["rel_l2_mean"],
+                                                             srht["rel_l2_error"]["rel_l2_mean"]]}
+    out["gemma_like_d256"] = _codec_figures(rq, kv_synth.WORKLOADS["gemma_like_d256"], 0, dev,
+                                            iters)
+    out["decode_stream_d128_fused_attention"] = _attention_figures(rq, dev, iters)
+    rep = parity_report()
+    if rep is not None:
+        out["parity_full_data"] = rep
+    return out
 
 
 def e2e_chunks(n_slices: int, target: int = 8) -> list:

@@ -45,7 +45,12 @@ def check_rotation(y_gpu: np.ndarray, y_ref: np.ndarray) -> dict:
 
 def check_codes(ref: dict, codes_gpu: np.ndarray, scales_gpu: np.ndarray, bits: int,
                 group: int) -> dict:
-    """ref: output of oracle.quantize (or quantize_vectors + pack) on the same inputs."""
+    """ref: output of oracle.quantize (or quantize_vectors + pack) on the same inputs.
+
+    Groups whose oracle scale is zero (sigma = 0: the group's absmax rounds
+    to zero) must have all-zero codes on both sides; they are counted and any
+    nonzero code there is a violation. Every other group is compared as the
+    tolerances above say."""
     qmax = oracle.qmax_for(bits)
     q_gpu = oracle.unpack_codes(codes_gpu, bits)
     q_ref = ref["q"]
@@ -61,12 +66,16 @@ def check_codes(ref: dict, codes_gpu: np.ndarray, scales_gpu: np.ndarray, bits: 
     near_mid = np.abs(pre_s - mid) <= SCALE_BAND * np.maximum(np.abs(pre_s), 1e-30)
     scale_ok = (~smis) | (near_mid & (np.abs(s_ref - s_gpu) == 1))
     scale_viol = int(np.sum(~scale_ok))
-    # codes of groups whose scales agree
     qg_ref = q_ref.reshape(shape_g + (group,))
     qg_gpu = q_gpu.reshape(shape_g + (group,))
-    pre = np.abs(ref["pre"].reshape(shape_g + (group,)))
-    cmp = ~smis[..., None] & np.ones_like(qg_ref, dtype=bool)
+    # sigma = 0 groups (equal on both sides): every code must be zero
+    zero = (~smis) & (v_ref == 0)
+    zero_viol = int(np.sum(zero[..., None] & ((qg_gpu != 0) | (qg_ref != 0))))
+    # codes of the other groups whose scales agree
+    cmp = (~smis & ~zero)[..., None] & np.ones_like(qg_ref, dtype=bool)
     cmis = cmp & (qg_ref != qg_gpu)
+    pre = np.abs(ref["pre"].reshape(shape_g + (group,)))
+    pre = np.where(zero[..., None], 0.0, pre)    # w / 0 is not a rounding position
     frac = pre - np.floor(pre)
     near_half = np.abs(frac - 0.5) < CODE_BAND
     near_clamp = np.abs(pre - (qmax + 0.5)) < CODE_BAND
@@ -80,6 +89,8 @@ def check_codes(ref: dict, codes_gpu: np.ndarray, scales_gpu: np.ndarray, bits: 
         "scale_mismatch_in_band": int(np.sum(smis & scale_ok)),
         "scale_violations": scale_viol,
         "groups_excluded": int(np.sum(smis)),
+        "zero_scale_groups": int(np.sum(zero)),
+        "zero_scale_violations": zero_viol,
     }
 
 
