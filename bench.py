@@ -425,7 +425,8 @@ def run_ours(args):
     }
     if e2e is not None:
         line["e2e"] = e2e
-    if world == 1 and not args.no_other_configs and args.slices is None:
+    if (world == 1 and not args.no_other_configs and args.slices is None
+            and args.workload == "qwen_like_d128"):
         del x, codes, scales, xhat
         torch.cuda.empty_cache()
         line["other_configs"] = other_configs(rq, dev)

@@ -53,9 +53,9 @@
  * never a fault.
  *
  * Supported: d in {16, 32, 64, 128, 256}; group a power of two with
- * 8 <= group <= d, and group <= 64 at d = 256 (two threads share a d = 256
- * vector and a group must lie inside one thread's half); bits in {4, 8};
- * heads >= 1; rotation SRFT or SRHT.
+ * 8 <= group <= d (group = d is one scale per vector, the per-token
+ * scaling the pages compare against); bits in {4, 8}; heads >= 1; rotation
+ * SRFT or SRHT.
  */
 #ifndef SRFTQ_H
 #define SRFTQ_H

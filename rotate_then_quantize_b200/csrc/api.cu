@@ -72,9 +72,7 @@ int check_desc(const srftq_desc* d) {
   if (!(d->d == 16 || d->d == 32 || d->d == 64 || d->d == 128 || d->d == 256))
     return SRFTQ_ERR_UNSUPPORTED;
   if (d->bits != 4 && d->bits != 8) return SRFTQ_ERR_UNSUPPORTED;
-  // a group lies inside one thread's half of the vector at d = 256
-  const int gmax = d->d < 64 ? d->d : (d->d == 256 ? 64 : d->d);
-  if (!is_pow2(d->group) || d->group < 8 || d->group > gmax) return SRFTQ_ERR_UNSUPPORTED;
+  if (!is_pow2(d->group) || d->group < 8 || d->group > d->d) return SRFTQ_ERR_UNSUPPORTED;
   if (d->rotation != SRFTQ_ROT_SRFT && d->rotation != SRFTQ_ROT_SRHT) return SRFTQ_ERR_UNSUPPORTED;
   return SRFTQ_OK;
 }

@@ -29,7 +29,12 @@
 // exchange.
 //
 // Every group of 8..d/4 coordinates lies inside one warp's slots, so each
-// warp quantises its own groups. The dequantiser runs the steps backwards.
+// warp quantises its own groups. A group of d/2 or d coordinates spans both
+// warps' slots (SRFT d/2: each warp holds half of both groups; d: each warp
+// holds half of the one group) except SRHT d/2, where each warp holds one
+// whole group: the warps then swap their partial group absmaxes through
+// shared memory before the scales are formed, so both compute the same
+// scales. The dequantiser runs the steps backwards.
 // For SRFT it decodes one extra bin (X_{d/8}) in warp 0, so that both of its
 // inverse butterflies are local. Its even/odd outputs are swapped once more,
 // so that each warp writes whole fp16 words of one half of the row.
@@ -42,7 +47,7 @@ namespace srftq {
 template <int D, int BITS, int G>
 struct SplitShape {
   static_assert(D == 256, "split head dimension");
-  static_assert(G >= 8 && G <= D / 4 && (G & (G - 1)) == 0, "group (split kernels)");
+  static_assert(G >= 8 && G <= D && (G & (G - 1)) == 0, "group (split kernels)");
   static_assert(BITS == 4 || BITS == 8, "bits");
   static constexpr int TR = kTileRows;                   // vectors per tile
   static constexpr int DH = D / 2;                       // coordinates per role
@@ -56,12 +61,28 @@ struct SplitShape {
   static constexpr int SPC = 64 / BITS;                  // slots (pairs) per 16-byte chunk
   static constexpr int KR = NP / SPC;                    // code chunks per role
   static constexpr int CWR = 4 * KR;                     // code words per role
-  static constexpr int NG = D / G, NGR = DH / G;         // groups per vector / per role
+  static constexpr int NG = D / G;                       // groups per vector
+  static constexpr int NGR = G <= D / 4 ? DH / G : 1;    // groups per role (local groups)
   static constexpr int GS = G / 2;                       // slots per group
   static constexpr int QMAX = (1 << (BITS - 1)) - 1;
   // SRFT role 0's groups are the vector's first and last NGR / 2: scale
   // words (two consecutive groups) stay aligned when NGR / 2 is even
   static constexpr bool kScaleWords = NGR % 4 == 0;
+};
+
+// Groups of one role's NP slots. kLocal: every group lies inside one role
+// (G <= d/4; NGR groups of G/2 slots, mapped by split_group). Otherwise the
+// role's slots fall into LG local groups of LGS slots each: SRFT G = d/2,
+// the two slot halves belong to global groups 0 and 1 (in both roles); SRHT
+// G = d/2, all slots belong to global group R; G = d, all to group 0.
+// kCross: a global group has slots in both roles.
+template <int D, int G, int ROT>
+struct SplitGroups {
+  static constexpr int NP = D / 4;
+  static constexpr bool kLocal = G <= D / 4;
+  static constexpr int LGS = kLocal ? G / 2 : ((ROT == kSRFT && G == D / 2) ? NP / 2 : NP);
+  static constexpr int LG = NP / LGS;
+  static constexpr bool kCross = !kLocal && !(ROT == kSRHT && G == D / 2);
 };
 
 // Per-block shared-memory layout: the input stage (x tile for the quantiser,
@@ -85,7 +106,9 @@ struct SplitLayout {
   static constexpr int kTableOff = kXch2Off;
   static constexpr int kSignTabOff = kTableOff + 4 * kMaxHPT * kMultStride;
   static constexpr int kBarOff = align_up(kSignTabOff + 4 * kMaxHPT * kSignStride, 16);
-  static constexpr int kBytes = kBarOff + 16;
+  // partial group absmaxes of both roles (2 per lane), for groups wider than d/4
+  static constexpr int kAmxOff = kBarOff + 16;
+  static constexpr int kBytes = kAmxOff + (G > D / 4 ? 2 * 32 * 2 * 4 : 0);
 };
 
 // (role, slot) holding coordinate pair p, and whether the slot stores the
@@ -404,6 +427,7 @@ __global__ void __launch_bounds__(64, MINB)
                           const __grid_constant__ CUtensorMap tm_codes, const QuantArgs a) {
   using S = SplitShape<D, BITS, G>;
   using Lay = SplitLayout<D, BITS, G, true>;
+  using Grp = SplitGroups<D, G, ROT>;
   constexpr int NP = S::NP;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = smem_base_1024(smem_raw);
@@ -530,38 +554,56 @@ __global__ void __launch_bounds__(64, MINB)
       y[2 * ci] = mul2(y[2 * ci], make_float2(m4.x, m4.y));
       y[2 * ci + 1] = mul2(y[2 * ci + 1], make_float2(m4.z, m4.w));
     });
-    float am[S::NGR];
-    static_for<0, S::NGR>([&](auto g_) {
+    // local groups of LGS slots (every group of this role, or this role's
+    // part of a group that spans both roles)
+    constexpr int LG = Grp::kLocal ? S::NGR : Grp::LG;
+    constexpr int LGS = Grp::kLocal ? S::GS : Grp::LGS;
+    float am[LG];
+    static_for<0, LG>([&](auto g_) {
       constexpr int g = decltype(g_)::value;
-      constexpr int P0 = g * S::GS;
+      constexpr int P0 = g * LGS;
       float m = absmax3(0.0f, y[P0].x, y[P0].y);
-      static_for<1, S::GS>([&](auto p_) {
+      static_for<1, LGS>([&](auto p_) {
         constexpr int p = P0 + decltype(p_)::value;
         m = absmax3(m, y[p].x, y[p].y);
       });
       am[g] = m;
     });
+    if constexpr (Grp::kCross) {
+      // both roles hold part of every group: swap the partial absmaxes (the
+      // slots of this exchange were last read before this tile's first barrier)
+      float* amx = reinterpret_cast<float*>(smem + Lay::kAmxOff);
+      static_for<0, LG>([&](auto g_) {
+        constexpr int g = decltype(g_)::value;
+        amx[(role * 32 + lane) * 2 + g] = am[g];
+      });
+      bar_pair();
+      static_for<0, LG>([&](auto g_) {
+        constexpr int g = decltype(g_)::value;
+        am[g] = fmaxf(am[g], amx[((1 - role) * 32 + lane) * 2 + g]);
+      });
+    }
     float a_hi, a_lo;
     range_of(am, a_hi, a_lo);
     constexpr float kHi = 65504.0f * float(S::QMAX);
     constexpr float kLo = 6.103515625e-05f * float(S::QMAX);
-    uint32_t sw[(S::NGR + 1) / 2];
+    uint32_t sw[(LG + 1) / 2];
     uint32_t qb[2 * NP];
     if (a_hi <= kHi && a_lo >= kLo) {
-      float invs[S::NGR];
-      group_scales<S::NGR, S::QMAX, true>(am, sw, invs);
+      float invs[LG];
+      group_scales<LG, S::QMAX, true>(am, sw, invs);
       static_for<0, NP>([&](auto p_) {
         constexpr int p = decltype(p_)::value;
-        const float2 r = fma2(y[p], splat(invs[p / S::GS]), splat(kMagic));
+        const float2 r = fma2(y[p], splat(invs[p / LGS]), splat(kMagic));
         qb[2 * p] = __float_as_uint(r.x);
         qb[2 * p + 1] = __float_as_uint(r.y);
       });
     } else {
-      float invs[S::NGR];
-      group_scales<S::NGR, S::QMAX, false>(am, sw, invs);
+      float invs[LG];
+      group_scales<LG, S::QMAX, false>(am, sw, invs);
       static_for<0, NP>([&](auto p_) {
         constexpr int p = decltype(p_)::value;
-        const float inv = invs[p / S::GS];
+        const float inv = invs[p / LGS];
         const float q0 = fminf(fmaxf(y[p].x * inv, -float(S::QMAX)), float(S::QMAX));
         const float q1 = fminf(fmaxf(y[p].y * inv, -float(S::QMAX)), float(S::QMAX));
         qb[2 * p] = __float_as_uint(q0 + kMagic);
@@ -603,17 +645,29 @@ __global__ void __launch_bounds__(64, MINB)
       uint16_t* dst = a.scales +
           ((static_cast<size_t>(cur.s) * a.out_slice_stride_rows + row) * a.g.heads +
            cur.hb * hpt + hl) * S::NG;
-      constexpr bool kWords = ROT == kSRHT || S::kScaleWords;
-      static_for<0, S::NGR / 2>([&](auto k_) {
-        constexpr int k = decltype(k_)::value;
-        const int g0 = split_group<ROT, S::NGR>(2 * k, role);
-        if constexpr (kWords) {
-          *reinterpret_cast<uint32_t*>(dst + g0) = sw[k];
-        } else {
-          dst[g0] = static_cast<uint16_t>(sw[k] & 0xFFFFu);
-          dst[split_group<ROT, S::NGR>(2 * k + 1, role)] = static_cast<uint16_t>(sw[k] >> 16);
+      if constexpr (Grp::kLocal) {
+        constexpr bool kWords = ROT == kSRHT || S::kScaleWords;
+        static_for<0, S::NGR / 2>([&](auto k_) {
+          constexpr int k = decltype(k_)::value;
+          const int g0 = split_group<ROT, S::NGR>(2 * k, role);
+          if constexpr (kWords) {
+            *reinterpret_cast<uint32_t*>(dst + g0) = sw[k];
+          } else {
+            dst[g0] = static_cast<uint16_t>(sw[k] & 0xFFFFu);
+            dst[split_group<ROT, S::NGR>(2 * k + 1, role)] = static_cast<uint16_t>(sw[k] >> 16);
+          }
+        });
+      } else if constexpr (Grp::kCross) {
+        // both roles hold every scale of the vector (NG = 1 or 2); role 0 stores them
+        if (role == 0) {
+          if constexpr (S::NG == 2)
+            *reinterpret_cast<uint32_t*>(dst) = sw[0];
+          else
+            dst[0] = static_cast<uint16_t>(sw[0] & 0xFFFFu);
         }
-      });
+      } else {
+        dst[role] = static_cast<uint16_t>(sw[0] & 0xFFFFu);   // SRHT, G = d/2: group R
+      }
     }
     cur.advance(a.g);
   }
@@ -722,8 +776,11 @@ __global__ void __launch_bounds__(64, MINB)
 
   // The next tile's scales of this role's groups (as words: local groups 2k
   // and 2k + 1) and of the group of pair d/8 (SRFT: the extra bin), loaded
-  // one tile ahead.
-  constexpr int NSW = S::NGR / 2;
+  // one tile ahead. Groups wider than a role: word 0 holds the scales of the
+  // role's LG local groups (see SplitGroups).
+  using Grp = SplitGroups<D, G, ROT>;
+  constexpr int NSW = Grp::kLocal ? S::NGR / 2 : 1;
+  constexpr int LGS = Grp::kLocal ? S::GS : Grp::LGS;
   constexpr bool kWords = ROT == kSRHT || S::kScaleWords;
   auto load_scales = [&](const TileWalk& c, uint32_t (&rs)[NSW], uint32_t& ex) {
     const int row = c.rb * rpt + rl;
@@ -731,16 +788,24 @@ __global__ void __launch_bounds__(64, MINB)
       const uint16_t* src = a.scales +
           ((static_cast<size_t>(c.s) * a.in_slice_stride_rows + row) * a.g.heads + c.hb * hpt +
            hl) * S::NG;
-      static_for<0, NSW>([&](auto k_) {
-        constexpr int k = decltype(k_)::value;
-        const int g0 = split_group<ROT, S::NGR>(2 * k, role);
-        if constexpr (kWords) {
-          rs[k] = *reinterpret_cast<const uint32_t*>(src + g0);
-        } else {
-          rs[k] = uint32_t(src[g0]) |
-                  (uint32_t(src[split_group<ROT, S::NGR>(2 * k + 1, role)]) << 16);
-        }
-      });
+      if constexpr (Grp::kLocal) {
+        static_for<0, NSW>([&](auto k_) {
+          constexpr int k = decltype(k_)::value;
+          const int g0 = split_group<ROT, S::NGR>(2 * k, role);
+          if constexpr (kWords) {
+            rs[k] = *reinterpret_cast<const uint32_t*>(src + g0);
+          } else {
+            rs[k] = uint32_t(src[g0]) |
+                    (uint32_t(src[split_group<ROT, S::NGR>(2 * k + 1, role)]) << 16);
+          }
+        });
+      } else if constexpr (S::NG == 2) {
+        // SRFT: local halves 0 / 1 are global groups 0 / 1; SRHT: group R
+        const uint32_t w = *reinterpret_cast<const uint32_t*>(src);
+        rs[0] = ROT == kSRFT ? w : (role ? (w >> 16) : (w & 0xFFFFu));
+      } else {
+        rs[0] = src[0];
+      }
       if constexpr (ROT == kSRFT) ex = src[(D / 4) / G];
     } else {
       static_for<0, NSW>([&](auto k_) { rs[decltype(k_)::value] = 0u; });
@@ -787,7 +852,7 @@ __global__ void __launch_bounds__(64, MINB)
       static_for<0, 4>([&](auto q_) {
         constexpr int q = decltype(q_)::value;
         constexpr int j0 = k * S::SPC + q * (S::SPC / 4);   // first slot of the word
-        constexpr int lg = j0 / S::GS;                      // local group
+        constexpr int lg = j0 / LGS;                        // local group
         decode_split_word<BITS, lg & 1>(wd[q], rs[lg / 2], &y[j0]);
       });
     });

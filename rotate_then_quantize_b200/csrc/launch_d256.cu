@@ -1,5 +1,5 @@
 // Kernels and launchers for head dimension d = 256 (two role warps per block
-// for the codec; groups of 8 to 64 coordinates).
+// for the codec; groups of 8 to 256 coordinates).
 #include "aux256.cuh"
 #include "launch_split.cuh"
 
@@ -7,7 +7,7 @@ namespace srftq {
 
 template <>
 int launch_quantize<256>(const QuantCall& c) {
-  return dispatch_split<64>(c.bits, c.group, c.rotation, [&](auto b_, auto g_, auto r_) {
+  return dispatch_split<256>(c.bits, c.group, c.rotation, [&](auto b_, auto g_, auto r_) {
     return quantize_split_impl<256, decltype(b_)::value, decltype(g_)::value,
                                decltype(r_)::value>(c);
   });
@@ -15,7 +15,7 @@ int launch_quantize<256>(const QuantCall& c) {
 
 template <>
 int launch_dequantize<256>(const DequantCall& c) {
-  return dispatch_split<64>(c.bits, c.group, c.rotation, [&](auto b_, auto g_, auto r_) {
+  return dispatch_split<256>(c.bits, c.group, c.rotation, [&](auto b_, auto g_, auto r_) {
     return dequantize_split_impl<256, decltype(b_)::value, decltype(g_)::value,
                                  decltype(r_)::value>(c);
   });

@@ -82,8 +82,8 @@ def test_quantize_rejects_bad_descriptors(lib):
         (128, 2, 12, 4, 0, b.SRFTQ_ERR_UNSUPPORTED),   # group not a power of two
         (128, 2, 4, 4, 0, b.SRFTQ_ERR_UNSUPPORTED),    # group below 8
         (64, 2, 128, 4, 0, b.SRFTQ_ERR_UNSUPPORTED),   # group above d
-        (256, 2, 128, 4, 0, b.SRFTQ_ERR_UNSUPPORTED),  # group above 64 at d = 256
-        (256, 2, 256, 8, 1, b.SRFTQ_ERR_UNSUPPORTED),
+        (256, 2, 512, 4, 0, b.SRFTQ_ERR_UNSUPPORTED),  # group above d
+        (16, 2, 32, 8, 1, b.SRFTQ_ERR_UNSUPPORTED),
         (128, 2, 16, 3, 0, b.SRFTQ_ERR_UNSUPPORTED),   # bits
         (128, 2, 16, 4, 2, b.SRFTQ_ERR_UNSUPPORTED),   # rotation
     ]:

@@ -89,7 +89,7 @@ def _configs():
     for d in (16, 32, 64, 128, 256):
         for bits in (4, 8):
             g = 8
-            while g <= min(d, 64 if d == 256 else d):
+            while g <= d:
                 for rot in (rq.SRFT, rq.SRHT):
                     out.append((d, bits, g, rot))
                 g *= 2
@@ -122,7 +122,8 @@ def test_ragged_rows_and_heads(N, H):
 
 @pytest.mark.parametrize("H", [2, 4, 6, 8, 12, 16])
 @pytest.mark.parametrize("d,bits,group", [(64, 4, 16), (128, 4, 16), (128, 8, 32), (128, 4, 64),
-                                           (256, 4, 32), (256, 8, 64)])
+                                           (256, 4, 32), (256, 8, 64), (256, 4, 128),
+                                           (256, 8, 256)])
 def test_head_block_tiles(H, d, bits, group):
     """Tiles span up to 8 heads of 32 / heads-per-tile rows; cover every
     heads-per-tile value, several head blocks per slice and ragged rows."""
@@ -166,15 +167,22 @@ def test_ragged_rows_d128_d256(N, rot, d, group):
     run_and_check(x16, signs, lam, d, group, bits, rot, f"d{d} N{N} r{rot}")
 
 
-def test_unsupported_groups_d256():
-    """Groups wider than one thread's half of a d = 256 vector are refused."""
-    x = torch.zeros((1, 4, 1, 256), dtype=torch.float16, device=DEV)
-    st = torch.ones((1, 1, 256), dtype=torch.int8, device=DEV)
-    lt = torch.ones((1, 1, 256), device=DEV)
-    for group in (128, 256):
-        with pytest.raises(rq.SrftqError) as e:
-            rq.quantize(x, st, lt, group, 4)
-        assert e.value.status == rq.binding.SRFTQ_ERR_UNSUPPORTED
+@pytest.mark.parametrize("group", [128, 256])
+@pytest.mark.parametrize("rot", [0, 1])
+@pytest.mark.parametrize("N", [1, 7, 40])
+def test_groups_spanning_both_warps_d256(group, rot, N):
+    """At d = 256 the codec splits each vector over two warps. A group of
+    128 coordinates (SRFT) or 256 (either rotation; 256 is one scale per
+    vector, the per-token baseline) has coordinates in both warps, whose
+    partial absmaxes are combined before the scale is formed; an SRHT group
+    of 128 lies inside one warp. Ragged rows, several heads, outliers."""
+    rng = np.random.default_rng(N * 13 + group + rot)
+    d, H = 256, 3
+    x16 = _x(rng, 2, N, H, d, outlier_p=0.005, scale=25.0)
+    signs = _signs(rng, 2, H, d)
+    lam = np.exp(rng.uniform(-1, 1, (2, H, d))).astype(np.float32)
+    for bits in (4, 8):
+        run_and_check(x16, signs, lam, d, group, bits, rot, f"d256 g{group} r{rot} N{N} b{bits}")
 
 
 @pytest.mark.parametrize("d", [128, 256])
