@@ -97,6 +97,17 @@ def rademacher_signs(S: int, H: int, d: int, seed: int) -> np.ndarray:
     return out
 
 
+def householder_reflectors(S: int, H: int, k: int, d: int, seed: int) -> np.ndarray:
+    """float32 reflector vectors [S, H, k, d] drawn N(0, 1), one independent
+    set per (slice, head). The pages' reflectors are learned from data; these
+    stand in for them (they only need to be nonzero)."""
+    out = np.empty((S, H, k, d), dtype=np.float32)
+    for s in range(S):
+        for h in range(H):
+            out[s, h] = _rng(seed, s, h, 11).standard_normal((k, d))
+    return out
+
+
 def _values_numpy(w: Workload, s: int, seed: int, n_rows: int) -> np.ndarray:
     rng = _rng(seed, s)
     shape = (n_rows, w.H, w.d)

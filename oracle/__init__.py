@@ -19,6 +19,10 @@ Sources followed (cited by page title and section):
   with per-group absmax scaling over groups of 16.
 * "HyperQuant" (technical summary), Methodology 1: the randomized Hadamard
   transform RHT(x) = H D x, used for the SRHT variant.
+* "When Quantization Is Free", Methodology 3 (Householder rotations) and
+  Key Results (lossless regime): the codec with a rotation given as an
+  explicit matrix, in particular k Householder reflectors on top of the
+  SRFT base (``dense_oracle``).
 
 Every function is pinned by the ``-m "not gpu"`` tests in ``tests/`` against
 closed forms, library special cases, brute force and hand-worked examples.
@@ -45,4 +49,15 @@ from .srft_oracle import (  # noqa: F401
     srht_matrix,
     unpack_codes,
     unrotate,
+)
+from .dense_oracle import (  # noqa: F401,E402
+    calibrate_lambda_dense,
+    dequantize_dense,
+    householder_matrix,
+    householder_rotations,
+    quantize_dense,
+    reflector,
+    rotate_dense,
+    split_operand,
+    unrotate_dense,
 )
