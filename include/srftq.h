@@ -219,6 +219,78 @@ int srftq_decode_attention(const srftq_desc* desc, int64_t n_seq, int64_t n_ctx,
                            int64_t seq_stride_rows, float softmax_scale, float* out,
                            void* stream);
 
+/*
+ * Dense-rotation codec: the Householder variant of "When Quantization Is
+ * Free" (Methodology 3, Householder rotations: k = d/2 reflectors at
+ * d = 256 give practically lossless quantisation; Key Results, lossless
+ * regime), and any other orthogonal rotation given as a matrix. The codec
+ * after the rotation is the one above (lambda, group absmax, fp16 scale,
+ * rounding, packing; the dequantiser applies R^T). d in {64, 128, 256};
+ * desc->rotation selects the base of srftq_householder_rotation and is not
+ * read by the other dense calls. Same ownership, stream, error and
+ * alignment rules as above.
+ *
+ * Rotation matrices are float32 [S][H][d][d], row n giving output
+ * coordinate n (y = R x). The dense codec reads a rotation as an "operand":
+ * [S][H][2][d][d] fp16 bit patterns, part 0 = fp16_rn(R) ("hi"), part 1 =
+ * fp16_rn(R - hi) ("lo"), so hi + lo carries R to about 2^-22.
+ */
+
+/*
+ * srftq_householder_rotation -- R = H(v_1) H(v_2) ... H(v_k) B for every
+ * (slice, head), with H(v) = I - 2 v v^T / (v^T v) and B the signed base
+ * rotation of desc->rotation (SRFT or SRHT matrix times diag(s)): the
+ * learned reflectors act on top of the fixed SRFT base, H(v_k) first. k = 0
+ * gives B itself (the FFT / WHT rotation as a matrix). Computed in double,
+ * stored in float32. A reflector that is exactly zero is skipped.
+ *
+ *   reflectors   [S][H][k][d] float32 (may be NULL when k = 0)
+ *   signs        [S][H][d] int8
+ *   rotation_out [S][H][d][d] float32, written; must not overlap the inputs
+ * One launch (one block per (slice, head)). 0 <= k <= 65536.
+ */
+int srftq_householder_rotation(const srftq_desc* desc, int64_t n_slices, int32_t n_reflectors,
+                               const float* reflectors, const int8_t* signs,
+                               float* rotation_out, void* stream);
+
+/*
+ * srftq_dense_operand -- splits float32 rotations [S][H][d][d] into the
+ * fp16 operand [S][H][2][d][d] (hi, lo) the dense codec reads. One launch.
+ */
+int srftq_dense_operand(const srftq_desc* desc, int64_t n_slices, const float* rotation,
+                        uint16_t* operand_out, void* stream);
+
+/*
+ * srftq_calibrate_lambda_dense -- lambda_out[s][h][n] = sqrt(mean over rows
+ * r < n_cal of y_n^2), y = R x (R = hi + lo of the operand), 1 where the
+ * sum is zero; float64 sums in a fixed order (deterministic). One launch.
+ */
+int srftq_calibrate_lambda_dense(const srftq_desc* desc, int64_t n_slices, int64_t n_cal,
+                                 const uint16_t* x, int64_t x_slice_stride_rows,
+                                 const uint16_t* operand, float* lambda_out, void* stream);
+
+/*
+ * srftq_quantize_dense -- y = R x per vector, then the codec's quantiser:
+ * w = y / lambda, sigma = fp16(absmax / qmax), q = clamp(rne(w / sigma)).
+ * Arguments and layouts as srftq_quantize, with the operand in place of the
+ * signs. One launch.
+ */
+int srftq_quantize_dense(const srftq_desc* desc, int64_t n_slices, int64_t n_rows,
+                         const uint16_t* x, int64_t x_slice_stride_rows, const uint16_t* operand,
+                         const float* lambda, uint8_t* codes, uint16_t* scales,
+                         int64_t out_slice_stride_rows, void* stream);
+
+/*
+ * srftq_dequantize_dense -- xhat = R^T (lambda * sigma * q), rounded to
+ * fp16. Arguments and layouts as srftq_dequantize, with the operand in
+ * place of the signs. One launch.
+ */
+int srftq_dequantize_dense(const srftq_desc* desc, int64_t n_slices, int64_t n_rows,
+                           const uint8_t* codes, const uint16_t* scales,
+                           int64_t in_slice_stride_rows, const uint16_t* operand,
+                           const float* lambda, uint16_t* xhat, int64_t out_slice_stride_rows,
+                           void* stream);
+
 /* Human-readable text for a status code (static storage, never NULL). */
 const char* srftq_status_string(int status);
 

@@ -13,20 +13,30 @@ from .binding import (  # noqa: F401
     SrftqDesc,
     SrftqError,
     calibrate_lambda,
+    calibrate_lambda_dense,
     decode_attention,
+    dense_operand,
     dequantize,
+    dequantize_dense,
     dequantize_rotated,
+    householder_rotation,
     load_library,
     make_desc,
     quantize,
+    quantize_dense,
     rotate,
     srftq_calibrate_lambda,
+    srftq_calibrate_lambda_dense,
     srftq_check_device,
     srftq_decode_attention,
+    srftq_dense_operand,
     srftq_dequantize,
+    srftq_dequantize_dense,
     srftq_dequantize_rotated,
+    srftq_householder_rotation,
     srftq_probe_wait_timeout,
     srftq_quantize,
+    srftq_quantize_dense,
     srftq_rotate,
     srftq_unrotate,
     srftq_version,

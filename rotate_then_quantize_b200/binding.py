@@ -32,7 +32,8 @@ SRHT = 1
 # Every symbol include/srftq.h declares (checked by the CPU test suite).
 EXPORTED = ("srftq_quantize", "srftq_dequantize", "srftq_calibrate_lambda", "srftq_rotate",
             "srftq_dequantize_rotated", "srftq_unrotate", "srftq_decode_attention",
-            "srftq_status_string",
+            "srftq_householder_rotation", "srftq_dense_operand", "srftq_calibrate_lambda_dense",
+            "srftq_quantize_dense", "srftq_dequantize_dense", "srftq_status_string",
             "srftq_check_device", "srftq_probe_wait_timeout", "srftq_version")
 
 
@@ -69,16 +70,19 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.srftq_unrotate.argtypes = [D, I64, I64, P, I64, P, P, I64, P]
     lib.srftq_decode_attention.argtypes = [D, I64, I64, I32, P, P, P, P, P, P, P, P, P, I64, I64,
                                            ctypes.c_float, P, P]
+    lib.srftq_householder_rotation.argtypes = [D, I64, ctypes.c_int32, P, P, P, P]
+    lib.srftq_dense_operand.argtypes = [D, I64, P, P, P]
+    lib.srftq_calibrate_lambda_dense.argtypes = [D, I64, I64, P, I64, P, P, P]
+    lib.srftq_quantize_dense.argtypes = [D, I64, I64, P, I64, P, P, P, P, I64, P]
+    lib.srftq_dequantize_dense.argtypes = [D, I64, I64, P, P, I64, P, P, P, I64, P]
     lib.srftq_status_string.argtypes = [I32]
     lib.srftq_status_string.restype = ctypes.c_char_p
     lib.srftq_check_device.argtypes = [P]
     lib.srftq_probe_wait_timeout.argtypes = [ctypes.c_uint32, P]
     lib.srftq_version.argtypes = []
-    for name in ("srftq_quantize", "srftq_dequantize", "srftq_calibrate_lambda", "srftq_rotate",
-                 "srftq_dequantize_rotated", "srftq_unrotate", "srftq_decode_attention",
-                 "srftq_check_device",
-                 "srftq_probe_wait_timeout", "srftq_version"):
-        getattr(lib, name).restype = I32
+    for name in EXPORTED:
+        if name != "srftq_status_string":
+            getattr(lib, name).restype = I32
     _lib = lib
     return lib
 
@@ -302,6 +306,96 @@ def srftq_decode_attention(desc: SrftqDesc, q, k_codes, k_scales, k_signs, k_lam
     _check("srftq_decode_attention", st)
 
 
+def _matrices(t, S: int, H: int, shape: tuple, name: str, dtype):
+    _check_tensor(t, dtype, name)
+    if tuple(t.shape) != (S, H) + tuple(shape) or not t.is_contiguous():
+        raise ValueError(f"{name}: expected contiguous {(S, H) + tuple(shape)}, "
+                         f"got {tuple(t.shape)}")
+    return t.data_ptr()
+
+
+def srftq_householder_rotation(desc: SrftqDesc, reflectors, signs, rot_out, stream=None) -> None:
+    """rot_out [S,H,d,d] float32 = H(v_1) ... H(v_k) B (B the signed SRFT/SRHT
+    matrix of desc.rotation) for reflectors [S,H,k,d] float32 (None for k = 0)."""
+    lib = load_library()
+    F16, U8, I8, F32 = _dtypes()
+    S, H, d = rot_out.shape[0], desc.heads, desc.d
+    po = _matrices(rot_out, S, H, (d, d), "rot_out", F32)
+    ps = _table(signs, S, H, d, "signs", I8)
+    if reflectors is None:
+        k, pr = 0, None
+    else:
+        if reflectors.dim() != 4:
+            raise ValueError("reflectors: expected [S, H, k, d]")
+        k = reflectors.shape[2]
+        pr = _matrices(reflectors, S, H, (k, d), "reflectors", F32)
+    st = lib.srftq_householder_rotation(ctypes.byref(desc), S, int(k), pr, ps, po,
+                                        _stream_handle(stream))
+    _check("srftq_householder_rotation", st)
+
+
+def srftq_dense_operand(desc: SrftqDesc, rot, operand_out, stream=None) -> None:
+    """operand_out [S,H,2,d,d] fp16 = (fp16(R), fp16(R - hi)) of rot [S,H,d,d] float32."""
+    lib = load_library()
+    F16, U8, I8, F32 = _dtypes()
+    S, H, d = rot.shape[0], desc.heads, desc.d
+    pr = _matrices(rot, S, H, (d, d), "rot", F32)
+    po = _matrices(operand_out, S, H, (2, d, d), "operand_out", F16)
+    st = lib.srftq_dense_operand(ctypes.byref(desc), S, pr, po, _stream_handle(stream))
+    _check("srftq_dense_operand", st)
+
+
+def srftq_calibrate_lambda_dense(desc: SrftqDesc, x, operand, lam_out, n_cal: int,
+                                 stream=None) -> None:
+    """lam_out [S,H,d] float32 = RMS of R x over the first n_cal rows of x."""
+    lib = load_library()
+    F16, U8, I8, F32 = _dtypes()
+    H, d = desc.heads, desc.d
+    px, S, N, xs = _rows_view(x, H, d, "x", F16)
+    if n_cal > N:
+        raise ValueError("n_cal exceeds the rows of x")
+    st = lib.srftq_calibrate_lambda_dense(ctypes.byref(desc), S, int(n_cal), px, xs,
+                                          _matrices(operand, S, H, (2, d, d), "operand", F16),
+                                          _table(lam_out, S, H, d, "lambda_out", F32),
+                                          _stream_handle(stream))
+    _check("srftq_calibrate_lambda_dense", st)
+
+
+def srftq_quantize_dense(desc: SrftqDesc, x, operand, lam, codes, scales, stream=None) -> None:
+    """x [S,N,H,d] fp16 -> codes, scales with the dense rotation of `operand`."""
+    lib = load_library()
+    F16, U8, I8, F32 = _dtypes()
+    H, d = desc.heads, desc.d
+    px, S, N, xs = _rows_view(x, H, d, "x", F16)
+    pc, S2, N2, os_ = _rows_view(codes, H, d * desc.bits // 8, "codes", U8)
+    ps, S3, N3, os2 = _rows_view(scales, H, d // desc.group, "scales", F16)
+    if (S2, N2) != (S, N) or (S3, N3) != (S, N) or os2 != os_:
+        raise ValueError("codes/scales must match x's slices and rows and share a slice stride")
+    st = lib.srftq_quantize_dense(ctypes.byref(desc), S, N, px, xs,
+                                  _matrices(operand, S, H, (2, d, d), "operand", F16),
+                                  _table(lam, S, H, d, "lambda", F32), pc, ps, os_,
+                                  _stream_handle(stream))
+    _check("srftq_quantize_dense", st)
+
+
+def srftq_dequantize_dense(desc: SrftqDesc, codes, scales, operand, lam, xhat,
+                           stream=None) -> None:
+    """codes, scales -> xhat [S,N,H,d] fp16 = R^T (lambda sigma q)."""
+    lib = load_library()
+    F16, U8, I8, F32 = _dtypes()
+    H, d = desc.heads, desc.d
+    pc, S, N, is_ = _rows_view(codes, H, d * desc.bits // 8, "codes", U8)
+    ps, S2, N2, is2 = _rows_view(scales, H, d // desc.group, "scales", F16)
+    px, S3, N3, os_ = _rows_view(xhat, H, d, "xhat", F16)
+    if (S2, N2) != (S, N) or (S3, N3) != (S, N) or is2 != is_:
+        raise ValueError("codes/scales/xhat shapes disagree")
+    st = lib.srftq_dequantize_dense(ctypes.byref(desc), S, N, pc, ps, is_,
+                                    _matrices(operand, S, H, (2, d, d), "operand", F16),
+                                    _table(lam, S, H, d, "lambda", F32), px, os_,
+                                    _stream_handle(stream))
+    _check("srftq_dequantize_dense", st)
+
+
 def srftq_probe_wait_timeout(polls: int, stream=None) -> int:
     """Launches the device-side timeout probe (see include/srftq.h); returns the status."""
     return int(load_library().srftq_probe_wait_timeout(int(polls), _stream_handle(stream)))
@@ -409,3 +503,59 @@ def decode_attention(q, k_codes, k_scales, k_signs, k_lambda, v_codes, v_scales,
                            v_signs, v_lambda, n_ctx, tok_stride_rows, seq_stride_rows, scale, out,
                            stream)
     return out
+
+
+def householder_rotation(reflectors, signs, rotation: int = SRFT, stream=None):
+    """Returns R [S,H,d,d] float32 = H(v_1) ... H(v_k) B for reflectors
+    [S,H,k,d] float32 (or None) on top of the signed SRFT/SRHT base."""
+    import torch
+
+    S, H, d = signs.shape
+    desc = make_desc(d, H, 8, 4, rotation)
+    rot = torch.empty((S, H, d, d), dtype=torch.float32, device=signs.device)
+    srftq_householder_rotation(desc, reflectors, signs, rot, stream)
+    return rot
+
+
+def dense_operand(rot, stream=None):
+    """Returns the fp16 (hi, lo) operand [S,H,2,d,d] of rotations [S,H,d,d]."""
+    import torch
+
+    S, H, d, _ = rot.shape
+    desc = make_desc(d, H, 8, 4)
+    op = torch.empty((S, H, 2, d, d), dtype=torch.float16, device=rot.device)
+    srftq_dense_operand(desc, rot, op, stream)
+    return op
+
+
+def calibrate_lambda_dense(x, operand, n_cal: int = 512, stream=None):
+    import torch
+
+    S, N, H, d = x.shape
+    desc = make_desc(d, H, 8, 4)
+    lam = torch.empty((S, H, d), dtype=torch.float32, device=x.device)
+    srftq_calibrate_lambda_dense(desc, x, operand, lam, n_cal, stream)
+    return lam
+
+
+def quantize_dense(x, operand, lam, group: int = 16, bits: int = 4, stream=None):
+    """Returns (codes, scales) for x [S,N,H,d] fp16 with the dense rotation."""
+    import torch
+
+    S, N, H, d = x.shape
+    desc = make_desc(d, H, group, bits)
+    codes = torch.empty((S, N, H, d * bits // 8), dtype=torch.uint8, device=x.device)
+    scales = torch.empty((S, N, H, d // group), dtype=torch.float16, device=x.device)
+    srftq_quantize_dense(desc, x, operand, lam, codes, scales, stream)
+    return codes, scales
+
+
+def dequantize_dense(codes, scales, operand, lam, d: int, group: int = 16, bits: int = 4,
+                     stream=None):
+    import torch
+
+    S, N, H, _ = codes.shape
+    desc = make_desc(d, H, group, bits)
+    xhat = torch.empty((S, N, H, d), dtype=torch.float16, device=codes.device)
+    srftq_dequantize_dense(desc, codes, scales, operand, lam, xhat, stream)
+    return xhat

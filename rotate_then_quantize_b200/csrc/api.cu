@@ -77,6 +77,19 @@ int check_desc(const srftq_desc* d) {
   return SRFTQ_OK;
 }
 
+// The dense-rotation calls take d in {64, 128, 256}; the codec calls also
+// check the group and code width.
+int check_dense_shape(const srftq_desc* d, bool codec) {
+  if (!d) return SRFTQ_ERR_INVALID_ARG;
+  if (d->heads < 1) return SRFTQ_ERR_INVALID_ARG;
+  if (d->d != 64 && d->d != 128 && d->d != 256) return SRFTQ_ERR_UNSUPPORTED;
+  if (codec) {
+    if (d->bits != 4 && d->bits != 8) return SRFTQ_ERR_UNSUPPORTED;
+    if (!is_pow2(d->group) || d->group < 8 || d->group > d->d) return SRFTQ_ERR_UNSUPPORTED;
+  }
+  return SRFTQ_OK;
+}
+
 // Byte range [lo, hi) touched by rows 0..n_rows-1 of S slices with a stride
 // of `stride` rows of `row_bytes` each.
 struct Range {
@@ -361,6 +374,127 @@ int srftq_decode_attention(const srftq_desc* desc, int64_t n_seq, int64_t n_ctx,
              k_lambda, v_codes, v_scales, v_signs, v_lambda, out,
              static_cast<cudaStream_t>(stream)};
   return launch_decode_attention_d128(c);
+}
+
+// ---------------------------------------------------------------------------
+// Dense-rotation codec
+// ---------------------------------------------------------------------------
+
+int srftq_householder_rotation(const srftq_desc* desc, int64_t n_slices, int32_t n_reflectors,
+                               const float* reflectors, const int8_t* signs,
+                               float* rotation_out, void* stream) {
+  int rc = check_dense_shape(desc, false);
+  if (rc != SRFTQ_OK) return rc;
+  if (desc->rotation != SRFTQ_ROT_SRFT && desc->rotation != SRFTQ_ROT_SRHT)
+    return SRFTQ_ERR_UNSUPPORTED;
+  if (n_slices < 0 || n_reflectors < 0 || n_reflectors > 65536) return SRFTQ_ERR_INVALID_ARG;
+  if (n_slices == 0) return SRFTQ_OK;
+  if (!signs || !rotation_out || (n_reflectors > 0 && !reflectors)) return SRFTQ_ERR_INVALID_ARG;
+  if (!aligned16(signs) || !aligned16(rotation_out) || (reflectors && !aligned16(reflectors)))
+    return SRFTQ_ERR_MISALIGNED;
+  const int64_t d = desc->d, H = desc->heads;
+  const Range ro = extent(rotation_out, 1, 0, n_slices * H, d * d * 4);
+  if (overlap(ro, extent(signs, 1, 0, n_slices * H, d))) return SRFTQ_ERR_INVALID_ARG;
+  if (n_reflectors > 0 &&
+      overlap(ro, extent(reflectors, 1, 0, n_slices * H * n_reflectors, d * 4)))
+    return SRFTQ_ERR_INVALID_ARG;
+  HouseholderCall c{desc->d, desc->heads, desc->rotation, n_reflectors, n_slices, reflectors,
+                    signs, rotation_out, static_cast<cudaStream_t>(stream)};
+  return launch_householder(c);
+}
+
+int srftq_dense_operand(const srftq_desc* desc, int64_t n_slices, const float* rotation,
+                        uint16_t* operand_out, void* stream) {
+  int rc = check_dense_shape(desc, false);
+  if (rc != SRFTQ_OK) return rc;
+  if (n_slices < 0) return SRFTQ_ERR_INVALID_ARG;
+  if (n_slices == 0) return SRFTQ_OK;
+  if (!rotation || !operand_out) return SRFTQ_ERR_INVALID_ARG;
+  if (!aligned16(rotation) || !aligned16(operand_out)) return SRFTQ_ERR_MISALIGNED;
+  const int64_t d = desc->d, H = desc->heads;
+  if (overlap(extent(operand_out, 1, 0, n_slices * H, 2 * d * d * 2),
+              extent(rotation, 1, 0, n_slices * H, d * d * 4)))
+    return SRFTQ_ERR_INVALID_ARG;
+  OperandCall c{desc->d, desc->heads, n_slices, rotation, operand_out,
+                static_cast<cudaStream_t>(stream)};
+  return launch_dense_operand(c);
+}
+
+int srftq_calibrate_lambda_dense(const srftq_desc* desc, int64_t n_slices, int64_t n_cal,
+                                 const uint16_t* x, int64_t x_slice_stride_rows,
+                                 const uint16_t* operand, float* lambda_out, void* stream) {
+  int rc = check_dense_shape(desc, false);
+  if (rc != SRFTQ_OK) return rc;
+  if (n_slices < 0 || n_cal < 1) return SRFTQ_ERR_INVALID_ARG;
+  if (n_slices == 0) return SRFTQ_OK;
+  if (x_slice_stride_rows < n_cal) return SRFTQ_ERR_INVALID_ARG;
+  if (!x || !operand || !lambda_out) return SRFTQ_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(operand) || !aligned16(lambda_out)) return SRFTQ_ERR_MISALIGNED;
+  const int64_t d = desc->d, H = desc->heads;
+  const Range rl = extent(lambda_out, 1, 0, n_slices * H, d * 4);
+  if (overlap(rl, extent(x, n_slices, x_slice_stride_rows, n_cal, H * d * 2)) ||
+      overlap(rl, extent(operand, 1, 0, n_slices * H, 2 * d * d * 2)))
+    return SRFTQ_ERR_INVALID_ARG;
+  DenseCalibCall c{desc->d, desc->heads, n_slices, n_cal, x_slice_stride_rows, x, operand,
+                   lambda_out, static_cast<cudaStream_t>(stream)};
+  return launch_calibrate_dense(c);
+}
+
+int srftq_quantize_dense(const srftq_desc* desc, int64_t n_slices, int64_t n_rows,
+                         const uint16_t* x, int64_t x_slice_stride_rows, const uint16_t* operand,
+                         const float* lambda, uint8_t* codes, uint16_t* scales,
+                         int64_t out_slice_stride_rows, void* stream) {
+  int rc = check_dense_shape(desc, true);
+  if (rc != SRFTQ_OK) return rc;
+  if (n_slices < 0 || n_rows < 0) return SRFTQ_ERR_INVALID_ARG;
+  if (n_slices == 0 || n_rows == 0) return SRFTQ_OK;
+  if (x_slice_stride_rows < n_rows || out_slice_stride_rows < n_rows) return SRFTQ_ERR_INVALID_ARG;
+  if (!x || !operand || !lambda || !codes || !scales) return SRFTQ_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(operand) || !aligned16(lambda) || !aligned16(codes) ||
+      !aligned16(scales))
+    return SRFTQ_ERR_MISALIGNED;
+  const int64_t d = desc->d, H = desc->heads;
+  const Range rx = extent(x, n_slices, x_slice_stride_rows, n_rows, H * d * 2);
+  const Range rc_ = extent(codes, n_slices, out_slice_stride_rows, n_rows, H * d * desc->bits / 8);
+  const Range rs = extent(scales, n_slices, out_slice_stride_rows, n_rows, H * (d / desc->group) * 2);
+  const Range rop = extent(operand, 1, 0, n_slices * H, 2 * d * d * 2);
+  const Range rl = extent(lambda, 1, 0, n_slices * H, d * 4);
+  for (Range out : {rc_, rs})
+    for (Range in : {rx, rop, rl})
+      if (overlap(out, in)) return SRFTQ_ERR_INVALID_ARG;
+  if (overlap(rc_, rs)) return SRFTQ_ERR_INVALID_ARG;
+  DenseCall c{desc->d, desc->heads, desc->group, desc->bits, n_slices, n_rows,
+              x_slice_stride_rows, out_slice_stride_rows, x, nullptr, nullptr, codes, scales,
+              nullptr, operand, lambda, static_cast<cudaStream_t>(stream)};
+  return launch_quantize_dense(c);
+}
+
+int srftq_dequantize_dense(const srftq_desc* desc, int64_t n_slices, int64_t n_rows,
+                           const uint8_t* codes, const uint16_t* scales,
+                           int64_t in_slice_stride_rows, const uint16_t* operand,
+                           const float* lambda, uint16_t* xhat, int64_t out_slice_stride_rows,
+                           void* stream) {
+  int rc = check_dense_shape(desc, true);
+  if (rc != SRFTQ_OK) return rc;
+  if (n_slices < 0 || n_rows < 0) return SRFTQ_ERR_INVALID_ARG;
+  if (n_slices == 0 || n_rows == 0) return SRFTQ_OK;
+  if (in_slice_stride_rows < n_rows || out_slice_stride_rows < n_rows) return SRFTQ_ERR_INVALID_ARG;
+  if (!codes || !scales || !operand || !lambda || !xhat) return SRFTQ_ERR_INVALID_ARG;
+  if (!aligned16(codes) || !aligned16(scales) || !aligned16(operand) || !aligned16(lambda) ||
+      !aligned16(xhat))
+    return SRFTQ_ERR_MISALIGNED;
+  const int64_t d = desc->d, H = desc->heads;
+  const Range rx = extent(xhat, n_slices, out_slice_stride_rows, n_rows, H * d * 2);
+  for (Range in : {extent(codes, n_slices, in_slice_stride_rows, n_rows, H * d * desc->bits / 8),
+                   extent(scales, n_slices, in_slice_stride_rows, n_rows,
+                          H * (d / desc->group) * 2),
+                   extent(operand, 1, 0, n_slices * H, 2 * d * d * 2),
+                   extent(lambda, 1, 0, n_slices * H, d * 4)})
+    if (overlap(rx, in)) return SRFTQ_ERR_INVALID_ARG;
+  DenseCall c{desc->d, desc->heads, desc->group, desc->bits, n_slices, n_rows,
+              in_slice_stride_rows, out_slice_stride_rows, nullptr, codes, scales, nullptr,
+              nullptr, xhat, operand, lambda, static_cast<cudaStream_t>(stream)};
+  return launch_dequantize_dense(c);
 }
 
 int srftq_probe_wait_timeout(uint32_t polls, void* stream) {

@@ -1,0 +1,404 @@
+// The codec with a rotation given as a dense matrix: the Householder variant
+// of "When Quantization Is Free" (Methodology 3, Householder rotations: k
+// reflectors on top of the fixed SRFT base), or any orthogonal R.
+//
+//   householder_kernel     R = H(v_1) ... H(v_k) B, B the signed SRFT/SRHT
+//                          matrix, one block per (slice, head)
+//   operand_kernel         R (float32) -> fp16 pair (hi, lo), hi + lo = R to
+//                          about 2^-22; the layout every dense kernel reads
+//   dense_gemm_kernel      quantise (y = R x, then the codec's lambda, group
+//                          absmax, scale, rounding and packing) and
+//                          dequantise (xhat = R^T (lambda sigma q)), as a
+//                          register-tiled float32 product of 64-vector tiles
+//   dense_calibrate_kernel lambda = RMS of R x over the calibration rows
+//
+// Operand layout: [S][H][2][d][d] fp16, part 0 = hi, part 1 = lo, row n of a
+// part is output coordinate n (y_n = sum_k R[n][k] x_k).
+#pragma once
+
+#include <cuda_fp16.h>
+
+#include "codec.cuh"
+
+namespace srftq {
+
+// ---------------------------------------------------------------------------
+// Householder rotation and operand
+// ---------------------------------------------------------------------------
+
+struct HouseholderArgs {
+  int32_t heads, n_reflectors;
+  const float* reflectors;   // [S][H][k][d]
+  const int8_t* signs;       // [S][H][d]
+  float* rot;                // [S][H][d][d]
+};
+
+// Entry (n, j) of the unsigned base rotation, in double: SRFT rows
+// [X_0, X_{d/2}, sqrt2 Re X_k, sqrt2 Im X_k] of the unitary DFT (kernel
+// exp(-2 pi i k j / d)), SRHT (-1)^popcount(n & j) / sqrt(d).
+template <int D, int ROT>
+__device__ __forceinline__ double base_entry(int n, int j) {
+  const double c = inv_sqrt_pow2(D);
+  if constexpr (ROT == kSRHT) {
+    return (__popc(n & j) & 1) ? -c : c;
+  } else {
+    if (n == 0) return c;
+    if (n == 1) return (j & 1) ? -c : c;
+    const int k = n >> 1;
+    const int m = (k * j) & (D - 1);   // k j mod d: the angle 2 pi m / d is exact
+    double sn, cs;
+    sincospi(2.0 * double(m) / double(D), &sn, &cs);
+    const double r2 = 1.4142135623730950488 * c;
+    return (n & 1) ? -r2 * sn : r2 * cs;
+  }
+}
+
+// One block of D threads per (slice, head); thread j owns column j of R,
+// which lives in `rot` (each column is touched by its own thread only, so
+// only the reflector staged in shared memory needs barriers). Reflectors are
+// applied innermost first: R = H(v_1) (H(v_2) ( ... (H(v_k) B))). Dot
+// products and updates run in double; a zero reflector is skipped.
+template <int D, int ROT>
+__global__ void __launch_bounds__(D) householder_kernel(const HouseholderArgs a) {
+  __shared__ double v[D];
+  const int sh = blockIdx.x;                 // s * H + h
+  const int j = threadIdx.x;
+  float* R = a.rot + size_t(sh) * D * D;
+  const double sj = a.signs[size_t(sh) * D + j] < 0 ? -1.0 : 1.0;
+  for (int n = 0; n < D; ++n) R[size_t(n) * D + j] = float(base_entry<D, ROT>(n, j) * sj);
+  for (int i = a.n_reflectors - 1; i >= 0; --i) {
+    __syncthreads();   // every thread is done with the previous reflector
+    v[j] = double(a.reflectors[(size_t(sh) * a.n_reflectors + i) * D + j]);
+    __syncthreads();
+    double vv = 0.0, dot = 0.0;
+    for (int n = 0; n < D; ++n) {
+      vv = fma(v[n], v[n], vv);
+      dot = fma(v[n], double(R[size_t(n) * D + j]), dot);
+    }
+    if (vv == 0.0) continue;
+    const double f = 2.0 * dot / vv;
+    for (int n = 0; n < D; ++n) {
+      float* p = R + size_t(n) * D + j;
+      *p = float(double(*p) - f * v[n]);
+    }
+  }
+}
+
+// hi = fp16_rn(r), lo = fp16_rn(r - hi) (the difference is exact in float32).
+__global__ void __launch_bounds__(256) operand_kernel(const float* rot, uint16_t* op, int64_t mats,
+                                                     int dd) {
+  const int64_t total = mats * dd;
+  for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < total;
+       i += int64_t(gridDim.x) * blockDim.x) {
+    const float r = rot[i];
+    const __half hi = __float2half_rn(r);
+    const __half lo = __float2half_rn(r - __half2float(hi));
+    const int64_t m = i / dd, e = i - m * dd;
+    op[(2 * m) * dd + e] = __half_as_ushort(hi);
+    op[(2 * m + 1) * dd + e] = __half_as_ushort(lo);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Register-tiled float32 product of one 64-vector tile (CUDA cores)
+// ---------------------------------------------------------------------------
+
+constexpr int kDenseRows = 64;      // vectors per tile
+constexpr int kDenseThreads = 256;
+constexpr int kDenseKC = 32;        // K columns staged per step
+
+template <int D>
+struct DenseTile {
+  static constexpr int NT = D / 8;                 // threads along the outputs
+  static constexpr int TVG = kDenseThreads / NT;   // thread groups along the vectors
+  static constexpr int TV = kDenseRows / TVG;      // vectors per thread
+  static constexpr int AS = D + 4;                 // A / C row stride (floats)
+  static constexpr int BS = D + 4;                 // B row stride (floats)
+  static constexpr int kABytes = kDenseRows * AS * 4;
+  static constexpr int kBBytes = kDenseKC * BS * 4;
+  static constexpr int kBytes = kABytes + kBBytes;
+  static_assert(TV >= 1 && TVG * TV == kDenseRows, "tile shape");
+};
+
+// R[n][k] = hi + lo of the operand, as float32.
+__device__ __forceinline__ float op_value(const uint16_t* hi, const uint16_t* lo, size_t i) {
+  return __half2float(__ushort_as_half(hi[i])) + __half2float(__ushort_as_half(lo[i]));
+}
+
+// acc[i][c] += sum_k A[v_i][k] * Bt[k][n_c] over all K, where the staged
+// chunk Bt[kk][n] = R[n][k0 + kk] (TRANS = false: y = R x) or R[k0 + kk][n]
+// (TRANS = true: xhat = R^T y). A is already in shared memory.
+template <int D, bool TRANS>
+__device__ __forceinline__ void dense_product(const float* As, float* Bs, const uint16_t* hi,
+                                              const uint16_t* lo, int tid,
+                                              float (&acc)[DenseTile<D>::TV][8]) {
+  using T = DenseTile<D>;
+  const int tn = tid % T::NT, tv = tid / T::NT;
+#pragma unroll
+  for (int i = 0; i < T::TV; ++i)
+#pragma unroll
+    for (int c = 0; c < 8; ++c) acc[i][c] = 0.0f;
+  for (int k0 = 0; k0 < D; k0 += kDenseKC) {
+    __syncthreads();   // the previous chunk has been read
+    for (int idx = tid; idx < D * kDenseKC; idx += kDenseThreads) {
+      if constexpr (TRANS) {
+        const int kk = idx / D, n = idx % D;
+        Bs[kk * T::BS + n] = op_value(hi, lo, size_t(k0 + kk) * D + n);
+      } else {
+        const int n = idx / kDenseKC, kk = idx % kDenseKC;
+        Bs[kk * T::BS + n] = op_value(hi, lo, size_t(n) * D + k0 + kk);
+      }
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int kk = 0; kk < kDenseKC; ++kk) {
+      const float4 b0 = *reinterpret_cast<const float4*>(Bs + kk * T::BS + 8 * tn);
+      const float4 b1 = *reinterpret_cast<const float4*>(Bs + kk * T::BS + 8 * tn + 4);
+      const float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+      for (int i = 0; i < T::TV; ++i) {
+        const float av = As[(tv * T::TV + i) * T::AS + k0 + kk];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) acc[i][c] = fmaf(av, b[c], acc[i][c]);
+      }
+    }
+  }
+}
+
+struct DenseArgs {
+  int64_t n_slices, n_rows, in_stride_rows, out_stride_rows;
+  int32_t heads;
+  int64_t row_tiles;          // ceil(n_rows / 64)
+  const uint16_t* x;          // quantise input [S][T_in][H][d]
+  const uint8_t* codes_in;    // dequantise inputs [S][T_in][H][...]
+  const uint16_t* scales_in;
+  uint8_t* codes;             // quantise outputs [S][T_out][H][...]
+  uint16_t* scales;
+  uint16_t* xhat;             // dequantise output [S][T_out][H][d]
+  const uint16_t* operand;    // [S][H][2][d][d]
+  const float* lambda;        // [S][H][d]
+};
+
+// One block per (slice, head, 64-row tile).
+template <int D, int BITS, int G, bool QUANT>
+__global__ void __launch_bounds__(kDenseThreads) dense_gemm_kernel(const DenseArgs a) {
+  using T = DenseTile<D>;
+  constexpr int QMAX = (1 << (BITS - 1)) - 1;
+  constexpr int CB = D * BITS / 8, NG = D / G;
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  float* As = reinterpret_cast<float*>(smem_raw);
+  float* Bs = reinterpret_cast<float*>(smem_raw + T::kABytes);
+  const int tid = threadIdx.x;
+  const int64_t tile = blockIdx.x % a.row_tiles;
+  const int64_t sh = blockIdx.x / a.row_tiles;   // s * H + h
+  const int64_t s = sh / a.heads;
+  const int h = int(sh % a.heads);
+  const int64_t r0 = tile * kDenseRows;
+  const uint16_t* hi = a.operand + size_t(sh) * 2 * D * D;
+  const uint16_t* lo = hi + size_t(D) * D;
+  const float* lam = a.lambda + size_t(sh) * D;
+
+  // A tile: x (quantise) or lambda * sigma * q (dequantise), float32
+  for (int idx = tid; idx < kDenseRows * (D / 8); idx += kDenseThreads) {
+    const int v = idx / (D / 8), c8 = idx % (D / 8);
+    const int64_t r = r0 + v;
+    float f[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    if (r < a.n_rows) {
+      const size_t vec = size_t((s * a.in_stride_rows + r) * a.heads + h);
+      if constexpr (QUANT) {
+        const uint4 w = *reinterpret_cast<const uint4*>(a.x + vec * D + 8 * c8);
+        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 p = __half22float2(*reinterpret_cast<const __half2*>(&ww[e]));
+          f[2 * e] = p.x;
+          f[2 * e + 1] = p.y;
+        }
+      } else {
+        const float sg = __half2float(__ushort_as_half(a.scales_in[vec * NG + (8 * c8) / G]));
+        int q[8];
+        if constexpr (BITS == 4) {
+          const uint32_t w = *reinterpret_cast<const uint32_t*>(a.codes_in + vec * CB + 4 * c8);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) q[e] = int(int32_t(w << (28 - 4 * e)) >> 28);
+        } else {
+          const uint2 w = *reinterpret_cast<const uint2*>(a.codes_in + vec * CB + 8 * c8);
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            q[e] = int(int8_t(((e < 4 ? w.x : w.y) >> (8 * (e & 3))) & 0xFFu));
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) f[e] = (float(q[e]) * sg) * lam[8 * c8 + e];
+      }
+    }
+    float* dst = As + v * T::AS + 8 * c8;
+    *reinterpret_cast<float4*>(dst) = make_float4(f[0], f[1], f[2], f[3]);
+    *reinterpret_cast<float4*>(dst + 4) = make_float4(f[4], f[5], f[6], f[7]);
+  }
+
+  float acc[T::TV][8];
+  dense_product<D, !QUANT>(As, Bs, hi, lo, tid, acc);
+  const int tn = tid % T::NT, tv = tid / T::NT;
+
+  if constexpr (!QUANT) {
+    // xhat = R^T yhat, rounded to fp16: 8 consecutive outputs per vector
+#pragma unroll
+    for (int i = 0; i < T::TV; ++i) {
+      const int64_t r = r0 + tv * T::TV + i;
+      if (r >= a.n_rows) continue;
+      uint32_t w[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const __half2 h2 = __floats2half2_rn(acc[i][2 * e], acc[i][2 * e + 1]);
+        w[e] = *reinterpret_cast<const uint32_t*>(&h2);
+      }
+      const size_t vec = size_t((s * a.out_stride_rows + r) * a.heads + h);
+      *reinterpret_cast<uint4*>(a.xhat + vec * D + 8 * tn) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+  } else {
+    // y tile to shared memory (over A, which every thread has finished reading)
+    __syncthreads();
+    float* Cs = As;
+#pragma unroll
+    for (int i = 0; i < T::TV; ++i) {
+      float* dst = Cs + (tv * T::TV + i) * T::AS + 8 * tn;
+      *reinterpret_cast<float4*>(dst) = make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
+      *reinterpret_cast<float4*>(dst + 4) =
+          make_float4(acc[i][4], acc[i][5], acc[i][6], acc[i][7]);
+    }
+    __syncthreads();
+    // One warp per vector: lane l holds coordinates C l .. C l + C - 1, which
+    // lie in one group (G >= 8 >= C); a group spans LPG lanes.
+    constexpr int C = D / 32;
+    constexpr int LPG = G / C;
+    const int warp = tid >> 5, lane = tid & 31;
+    float lv[C];
+#pragma unroll
+    for (int c = 0; c < C; ++c) lv[c] = lam[C * lane + c];
+    for (int v = warp; v < kDenseRows; v += kDenseThreads / 32) {
+      const int64_t r = r0 + v;
+      if (r >= a.n_rows) break;   // warp-uniform: rows beyond N come last
+      float w[C];
+      float am = 0.0f;
+#pragma unroll
+      for (int c = 0; c < C; ++c) {
+        w[c] = __fdiv_rn(Cs[v * T::AS + C * lane + c], lv[c]);
+        am = fmaxf(am, fabsf(w[c]));
+      }
+#pragma unroll
+      for (int o = 1; o < LPG && o < 32; o <<= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
+      const float sf = fminf(div_by_const<QMAX>(am), 65504.0f);
+      const __half hs = __float2half_rn(sf);
+      const float sg = __half2float(hs);
+      uint32_t qb[C];
+#pragma unroll
+      for (int c = 0; c < C; ++c) {
+        float q = sg > 0.0f ? rintf(__fdiv_rn(w[c], sg)) : 0.0f;
+        q = fminf(fmaxf(q, -float(QMAX)), float(QMAX));
+        qb[c] = uint32_t(int32_t(q));
+      }
+      const size_t vec = size_t((s * a.out_stride_rows + r) * a.heads + h);
+      uint8_t* cdst = a.codes + vec * CB;
+      if constexpr (BITS == 4) {
+        // coordinates 2m (low nibble) and 2m + 1 (high nibble) share byte m
+        uint32_t word = 0;
+#pragma unroll
+        for (int c = 0; c < C; c += 2)
+          word |= ((qb[c] & 0xFu) | ((qb[c + 1] & 0xFu) << 4)) << (4 * c);
+        if constexpr (C == 8) {
+          reinterpret_cast<uint32_t*>(cdst)[lane] = word;
+        } else if constexpr (C == 4) {
+          reinterpret_cast<uint16_t*>(cdst)[lane] = uint16_t(word);
+        } else {
+          cdst[lane] = uint8_t(word);
+        }
+      } else {
+        uint32_t w0 = 0, w1 = 0;
+#pragma unroll
+        for (int c = 0; c < C; ++c) {
+          if (c < 4)
+            w0 |= (qb[c] & 0xFFu) << (8 * c);
+          else
+            w1 |= (qb[c] & 0xFFu) << (8 * (c - 4));
+        }
+        if constexpr (C == 8) {
+          reinterpret_cast<uint2*>(cdst)[lane] = make_uint2(w0, w1);
+        } else if constexpr (C == 4) {
+          reinterpret_cast<uint32_t*>(cdst)[lane] = w0;
+        } else {
+          reinterpret_cast<uint16_t*>(cdst)[lane] = uint16_t(w0);
+        }
+      }
+      if ((lane % LPG) == 0) a.scales[vec * NG + (C * lane) / G] = __half_as_ushort(hs);
+    }
+  }
+}
+
+// lambda[s][h][n] = sqrt(mean over the first n_cal rows of y_n^2), y = R x
+// (1 where the sum is 0). One block per (slice, head) walks the 64-row tiles
+// in order; each thread sums its own products in double in a fixed order,
+// then the vector groups are added in a fixed order: deterministic.
+struct DenseCalibArgs {
+  int64_t n_cal, x_stride_rows;
+  int32_t heads;
+  const uint16_t* x;
+  const uint16_t* operand;
+  float* lambda_out;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kDenseThreads) dense_calibrate_kernel(const DenseCalibArgs a) {
+  using T = DenseTile<D>;
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  float* As = reinterpret_cast<float*>(smem_raw);
+  float* Bs = reinterpret_cast<float*>(smem_raw + T::kABytes);
+  const int tid = threadIdx.x;
+  const int64_t sh = blockIdx.x;
+  const int64_t s = sh / a.heads;
+  const int h = int(sh % a.heads);
+  const uint16_t* hi = a.operand + size_t(sh) * 2 * D * D;
+  const uint16_t* lo = hi + size_t(D) * D;
+  const int tn = tid % T::NT, tv = tid / T::NT;
+  double ss[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  for (int64_t r0 = 0; r0 < a.n_cal; r0 += kDenseRows) {
+    __syncthreads();   // the previous tile's A has been read
+    for (int idx = tid; idx < kDenseRows * (D / 8); idx += kDenseThreads) {
+      const int v = idx / (D / 8), c8 = idx % (D / 8);
+      const int64_t r = r0 + v;
+      float f[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+      if (r < a.n_cal) {
+        const size_t vec = size_t((s * a.x_stride_rows + r) * a.heads + h);
+        const uint4 w = *reinterpret_cast<const uint4*>(a.x + vec * D + 8 * c8);
+        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 p = __half22float2(*reinterpret_cast<const __half2*>(&ww[e]));
+          f[2 * e] = p.x;
+          f[2 * e + 1] = p.y;
+        }
+      }
+      float* dst = As + v * T::AS + 8 * c8;
+      *reinterpret_cast<float4*>(dst) = make_float4(f[0], f[1], f[2], f[3]);
+      *reinterpret_cast<float4*>(dst + 4) = make_float4(f[4], f[5], f[6], f[7]);
+    }
+    float acc[T::TV][8];
+    dense_product<D, false>(As, Bs, hi, lo, tid, acc);
+#pragma unroll
+    for (int i = 0; i < T::TV; ++i)
+#pragma unroll
+      for (int c = 0; c < 8; ++c) ss[c] = fma(double(acc[i][c]), double(acc[i][c]), ss[c]);
+  }
+  // fixed-order sum over the TVG vector groups (the B stage is free now)
+  __syncthreads();
+  double* red = reinterpret_cast<double*>(smem_raw);
+#pragma unroll
+  for (int c = 0; c < 8; ++c) red[tv * D + 8 * tn + c] = ss[c];
+  __syncthreads();
+  for (int n = tid; n < D; n += kDenseThreads) {
+    double t = 0.0;
+    for (int g = 0; g < T::TVG; ++g) t += red[g * D + n];
+    a.lambda_out[size_t(sh) * D + n] = t == 0.0 ? 1.0f : float(sqrt(t / double(a.n_cal)));
+  }
+}
+
+}  // namespace srftq

@@ -99,6 +99,53 @@ struct CalibCall {
   cudaStream_t stream;
 };
 
+// Dense-rotation codec (launch_dense.cu).
+struct HouseholderCall {
+  int32_t d, heads, rotation, n_reflectors;
+  int64_t n_slices;
+  const float* reflectors;
+  const int8_t* signs;
+  float* rot;
+  cudaStream_t stream;
+};
+
+struct OperandCall {
+  int32_t d, heads;
+  int64_t n_slices;
+  const float* rot;
+  uint16_t* operand;
+  cudaStream_t stream;
+};
+
+struct DenseCall {
+  int32_t d, heads, group, bits;
+  int64_t n_slices, n_rows, in_stride_rows, out_stride_rows;
+  const uint16_t* x;
+  const uint8_t* codes_in;
+  const uint16_t* scales_in;
+  uint8_t* codes;
+  uint16_t* scales;
+  uint16_t* xhat;
+  const uint16_t* operand;
+  const float* lambda;
+  cudaStream_t stream;
+};
+
+struct DenseCalibCall {
+  int32_t d, heads;
+  int64_t n_slices, n_cal, x_stride_rows;
+  const uint16_t* x;
+  const uint16_t* operand;
+  float* lambda_out;
+  cudaStream_t stream;
+};
+
+int launch_householder(const HouseholderCall& c);
+int launch_dense_operand(const OperandCall& c);
+int launch_quantize_dense(const DenseCall& c);
+int launch_dequantize_dense(const DenseCall& c);
+int launch_calibrate_dense(const DenseCalibCall& c);
+
 // Services the per-d units get from the API unit.
 struct Runtime {
   // Encodes a rank-4 tiled tensor map; returns 0 on success.

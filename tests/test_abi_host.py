@@ -231,3 +231,39 @@ def test_python_binding_refuses_host_tensors_and_wrong_dtypes():
     with pytest.raises(ValueError):
         rq.srftq_unrotate(desc, torch.zeros((S, N, H, d)), good["signs"],
                           torch.zeros((S, N, H, d)))
+
+
+def test_dense_calls_validate_before_launching(lib):
+    c, s, sg, lam, xh, y = _addrs()
+    ok = rq.make_desc(256, 2, 32, 4, 0)
+    D = ctypes.byref(ok)
+    Hh = lib.srftq_householder_rotation
+    assert Hh(ctypes.byref(rq.make_desc(32, 2, 8, 4, 0)), 1, 4, y, sg, xh, None) == \
+        b.SRFTQ_ERR_UNSUPPORTED                                      # d = 64, 128, 256 only
+    assert Hh(ctypes.byref(rq.make_desc(256, 2, 8, 4, 5)), 1, 4, y, sg, xh, None) == \
+        b.SRFTQ_ERR_UNSUPPORTED                                      # base rotation
+    assert Hh(D, 1, -1, y, sg, xh, None) == b.SRFTQ_ERR_INVALID_ARG
+    assert Hh(D, 1, 4, 0, sg, xh, None) == b.SRFTQ_ERR_INVALID_ARG     # no reflectors
+    assert Hh(D, 1, 4, y, sg, y + 64, None) == b.SRFTQ_ERR_INVALID_ARG  # output over input
+    assert Hh(D, 1, 4, y, sg, xh + 8, None) == b.SRFTQ_ERR_MISALIGNED
+    assert Hh(D, 0, 4, y, sg, xh, None) == b.SRFTQ_OK
+    Op = lib.srftq_dense_operand
+    assert Op(D, 1, y, y + 16, None) == b.SRFTQ_ERR_INVALID_ARG
+    assert Op(D, 1, y, 0, None) == b.SRFTQ_ERR_INVALID_ARG
+    assert Op(D, 0, y, xh, None) == b.SRFTQ_OK
+    Q = lib.srftq_quantize_dense
+    assert Q(ctypes.byref(rq.make_desc(256, 2, 512, 4)), 1, 8, xh, 8, y, lam, c, s, 8, None) == \
+        b.SRFTQ_ERR_UNSUPPORTED
+    assert Q(D, 1, 8, xh, 8, y, lam, xh + 64, s, 8, None) == b.SRFTQ_ERR_INVALID_ARG  # in place
+    assert Q(D, 2, 8, xh, 4, y, lam, c, s, 8, None) == b.SRFTQ_ERR_INVALID_ARG       # stride < N
+    assert Q(D, 1, 8, xh, 8, y + 2, lam, c, s, 8, None) == b.SRFTQ_ERR_MISALIGNED
+    assert Q(D, 1, 0, xh, 8, y, lam, c, s, 8, None) == b.SRFTQ_OK
+    Dq = lib.srftq_dequantize_dense
+    assert Dq(D, 1, 8, c, s, 8, y, lam, c + 16, 8, None) == b.SRFTQ_ERR_INVALID_ARG
+    assert Dq(D, 1, 8, c, s, 8, None, lam, xh, 8, None) == b.SRFTQ_ERR_INVALID_ARG
+    assert Dq(D, 1, 0, c, s, 8, y, lam, xh, 8, None) == b.SRFTQ_OK
+    Cal = lib.srftq_calibrate_lambda_dense
+    assert Cal(D, 1, 0, xh, 8, y, lam, None) == b.SRFTQ_ERR_INVALID_ARG
+    assert Cal(D, 1, 9, xh, 8, y, lam, None) == b.SRFTQ_ERR_INVALID_ARG
+    assert Cal(D, 1, 4, xh, 8, y, xh, None) == b.SRFTQ_ERR_INVALID_ARG      # lambda over x
+    assert Cal(D, 0, 4, xh, 8, y, lam, None) == b.SRFTQ_OK

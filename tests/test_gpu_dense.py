@@ -1,0 +1,191 @@
+"""GPU parity of the dense-rotation codec (the Householder variant of "When
+Quantization Is Free", Methodology 3) against oracle/dense_oracle.py,
+through the C ABI.
+
+The rotation builder is compared with the oracle's float64 matrices (float32
+storage: 2e-6 absolute on entries of unit-norm rows); the operand split bit
+for bit; the codec stages with the same tolerances as the FFT codec
+(tests/parity.py), each stage fed the oracle's own inputs: the quantiser and
+the calibration get the operand of the oracle's matrix (rounded to float32),
+the dequantiser the oracle's codes.
+"""
+
+import numpy as np
+import pytest
+
+import kv_synth
+import oracle
+import parity
+
+torch = pytest.importorskip("torch")
+import rotate_then_quantize_b200 as rq  # noqa: E402
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+ROT_ENTRY_TOL = 2e-6
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    if not torch.cuda.is_available():
+        pytest.fail("no CUDA device")
+    rq.load_library()
+    yield
+    assert rq.srftq_check_device() == 0, "a device-side guard fired"
+
+
+def _t(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).to(DEV)
+
+
+def _np16(t):
+    return t.cpu().numpy().view(np.uint16)
+
+
+def _case(rng, S, N, H, d, k, kind, outlier_p=0.01, scale=20.0):
+    x = rng.standard_normal((S, N, H, d))
+    x = np.where(rng.random(x.shape) < outlier_p, x * scale, x).astype(np.float16)
+    signs = np.where(rng.random((S, H, d)) < 0.5, -1, 1).astype(np.int8)
+    V = rng.standard_normal((S, H, k, d)).astype(np.float32)
+    R = oracle.householder_rotations(V, signs, kind)
+    return x, signs, V, R
+
+
+@pytest.mark.parametrize("d", [64, 128, 256])
+@pytest.mark.parametrize("kind", [0, 1])
+@pytest.mark.parametrize("k_frac", [0, 1, 2])
+def test_householder_rotation_matches_oracle(d, kind, k_frac):
+    """k = 0 (the base matrix alone), one reflector, and k = d/2."""
+    k = {0: 0, 1: 1, 2: d // 2}[k_frac]
+    rng = np.random.default_rng(d + 10 * kind + k)
+    S, H = 2, 3
+    signs = np.where(rng.random((S, H, d)) < 0.5, -1, 1).astype(np.int8)
+    V = rng.standard_normal((S, H, k, d)).astype(np.float32)
+    R = oracle.householder_rotations(V, signs, kind)
+    got = rq.householder_rotation(_t(V) if k else None, _t(signs), rotation=kind).cpu().numpy()
+    err = np.abs(got - R).max()
+    assert err <= ROT_ENTRY_TOL, err
+    # and it is orthogonal to float32 accuracy
+    g = got.astype(np.float64)
+    assert np.abs(np.einsum("shij,shik->shjk", g, g) - np.eye(d)).max() < 1e-5
+
+
+def test_operand_split_is_bit_exact():
+    rng = np.random.default_rng(1)
+    R32 = (rng.standard_normal((2, 3, 128, 128)) / 11.3).astype(np.float32)
+    R32[0, 0, 0, :8] = [0.0, -0.0, 1e-9, -3e-6, 6.1e-5, 65504.0, 1.0, -1.0]  # zero, subnormals
+    op = rq.dense_operand(_t(R32)).cpu().numpy().view(np.uint16)
+    hi, lo = oracle.split_operand(R32)
+    assert np.array_equal(op[:, :, 0], hi)
+    assert np.array_equal(op[:, :, 1], lo)
+
+
+def _quant_check(x16, R, lam, d, group, bits, what):
+    op = rq.dense_operand(_t(R.astype(np.float32)))
+    lt = _t(lam)
+    codes, scales = rq.quantize_dense(_t(x16), op, lt, group, bits)
+    ref = oracle.quantize_dense(x16, R, lam, group, bits)
+    c_np, s_np = codes.cpu().numpy(), _np16(scales)
+    stats = parity.check_codes(ref, c_np, s_np, bits, group)
+    parity.assert_clean(stats, f"{what} codes")
+    # dequantiser on the oracle's codes, and the GPU round trip on its own codes
+    deq = oracle.dequantize_dense(ref["codes"], ref["scales"], R, lam, d, group, bits)
+    xhat = rq.dequantize_dense(_t(ref["codes"]), _t(ref["scales"].view(np.float16)), op, lt, d,
+                               group, bits)
+    parity.assert_clean(parity.check_dequant(_np16(xhat), deq["bits"]), f"{what} dequant")
+    xrt = rq.dequantize_dense(codes, scales, op, lt, d, group, bits)
+    deq_own = oracle.dequantize_dense(c_np, s_np, R, lam, d, group, bits)
+    parity.assert_clean(parity.check_dequant(_np16(xrt), deq_own["bits"]), f"{what} round trip")
+    return stats
+
+
+@pytest.mark.parametrize("d", [64, 128, 256])
+@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("kind", [0, 1])
+def test_dense_codec_matches_oracle(d, bits, kind):
+    """Every group size 8..d, ragged rows (several 64-row tiles and a partial
+    one), several slices and heads, k = d/2 reflectors."""
+    rng = np.random.default_rng(3 * d + bits + kind)
+    S, N, H = 2, 150, 3
+    x16, signs, V, R = _case(rng, S, N, H, d, d // 2, kind)
+    lam = oracle.calibrate_lambda_dense(x16, R, 64).astype(np.float32)
+    g = 8
+    while g <= d:
+        _quant_check(x16, R, lam, d, g, bits, f"d{d} b{bits} g{g} base{kind}")
+        g *= 2
+
+
+@pytest.mark.parametrize("d", [64, 256])
+@pytest.mark.parametrize("n_cal", [1, 63, 64, 200])
+def test_dense_calibration_matches_oracle(d, n_cal):
+    rng = np.random.default_rng(d + n_cal)
+    x16, signs, V, R = _case(rng, 2, max(n_cal, 8), 3, d, d // 2, 0)
+    op = rq.dense_operand(_t(R.astype(np.float32)))
+    lam = rq.calibrate_lambda_dense(_t(x16), op, n_cal).cpu().numpy()
+    parity.assert_clean(parity.check_lambda(lam, oracle.calibrate_lambda_dense(x16, R, n_cal)),
+                        f"dense lambda d{d} n_cal{n_cal}")
+
+
+def test_dense_codec_with_the_gpu_built_rotation():
+    """End to end on the GPU's own rotation (built from the same reflectors):
+    the codes agree with the oracle's within the boundary band, since the
+    two matrices differ only by float32 rounding."""
+    rng = np.random.default_rng(77)
+    d, group, bits = 256, 32, 4
+    x16, signs, V, R = _case(rng, 2, 100, 2, d, d // 2, 0, outlier_p=0.005, scale=25.0)
+    lam = oracle.calibrate_lambda_dense(x16, R, 64).astype(np.float32)
+    op = rq.dense_operand(rq.householder_rotation(_t(V), _t(signs)))
+    codes, scales = rq.quantize_dense(_t(x16), op, _t(lam), group, bits)
+    ref = oracle.quantize_dense(x16, R, lam, group, bits)
+    parity.assert_clean(parity.check_codes(ref, codes.cpu().numpy(), _np16(scales), bits, group),
+                        "gpu-built rotation")
+
+
+def test_dense_strided_windows_keep_their_guard_bands():
+    rng = np.random.default_rng(5)
+    d, group, bits, S, T, H, N, off = 128, 16, 4, 2, 90, 2, 37, 21
+    big = rng.standard_normal((S, T, H, d)).astype(np.float16)
+    signs = np.where(rng.random((S, H, d)) < 0.5, -1, 1).astype(np.int8)
+    R = oracle.householder_rotations(rng.standard_normal((S, H, 8, d)), signs, 0)
+    lam = np.exp(rng.uniform(-0.5, 0.5, (S, H, d))).astype(np.float32)
+    op, lt = rq.dense_operand(_t(R.astype(np.float32))), _t(lam)
+    codes = torch.full((S, T, H, d // 2), 0xAB, dtype=torch.uint8, device=DEV)
+    scales = torch.full((S, T, H, d // group), 7.0, dtype=torch.float16, device=DEV)
+    desc = rq.make_desc(d, H, group, bits)
+    rq.srftq_quantize_dense(desc, _t(big)[:, off:off + N], op, lt, codes[:, off:off + N],
+                            scales[:, off:off + N])
+    ref = oracle.quantize_dense(big[:, off:off + N], R, lam, group, bits)
+    c_np, s_np = codes.cpu().numpy(), _np16(scales)
+    parity.assert_clean(parity.check_codes(ref, c_np[:, off:off + N], s_np[:, off:off + N], bits,
+                                           group), "strided dense codes")
+    outside = np.ones(T, bool)
+    outside[off:off + N] = False
+    assert np.all(c_np[:, outside] == 0xAB)
+    assert np.all(s_np[:, outside] == np.float16(7.0).view(np.uint16))
+    xh = torch.full((S, T, H, d), -3.0, dtype=torch.float16, device=DEV)
+    rq.srftq_dequantize_dense(desc, codes[:, off:off + N], scales[:, off:off + N], op, lt,
+                              xh[:, off:off + N])
+    deq = oracle.dequantize_dense(c_np[:, off:off + N], s_np[:, off:off + N], R, lam, d, group,
+                                  bits)
+    xh_np = _np16(xh)
+    parity.assert_clean(parity.check_dequant(xh_np[:, off:off + N], deq["bits"]),
+                        "strided dense dequant")
+    assert np.all(xh_np[:, outside] == np.float16(-3.0).view(np.uint16))
+
+
+def test_dense_degenerate_values():
+    """Zero vectors (sigma = 0), tiny and huge values, extreme lambda."""
+    rng = np.random.default_rng(9)
+    d, group = 128, 16
+    x = rng.standard_normal((1, 64, 1, d))
+    x[:, 0] = 0.0
+    x[:, 1] = 1e-7 * rng.standard_normal(d)
+    x[:, 2] = 6e4 * np.sign(rng.standard_normal(d))
+    x16 = x.astype(np.float16)
+    signs = np.where(rng.random((1, 1, d)) < 0.5, -1, 1).astype(np.int8)
+    R = oracle.householder_rotations(rng.standard_normal((1, 1, 64, d)), signs, 0)
+    for lam_val in (1.0, 1e-3, 3e3):
+        lam = np.full((1, 1, d), lam_val, np.float32)
+        for bits in (4, 8):
+            _quant_check(x16, R, lam, d, group, bits, f"degenerate lam={lam_val} b{bits}")
