@@ -100,10 +100,52 @@ KERNEL_SOURCES = {
 }
 
 
-def codec_kernel(kind: str, d: int) -> str:
+def codec_kernel(kind: str, d: int, dense: bool = False) -> str:
     """Name of the kernel that runs `kind` ("quantize" / "dequantize") for a
-    head dimension: d = 256 runs on the two-warp kernels."""
+    head dimension: d = 256 runs on the two-warp kernels; a dense rotation
+    on the dense kernels."""
+    if dense:
+        return "dense_gemm_kernel"
     return f"{kind}{'_split' if d == 256 else ''}_kernel"
+
+
+def codec_calls(rq, w, desc, signs, seed, dev):
+    """(table, (calibrate, quantize, dequantize)) of a workload: the FFT/WHT
+    calls with the sign table, or, when the workload has Householder
+    reflectors, the dense calls with the operand of R = H(v_1)...H(v_k) B."""
+    import torch
+
+    if not w.reflectors:
+        return signs, (rq.srftq_calibrate_lambda, rq.srftq_quantize, rq.srftq_dequantize)
+    V = torch.from_numpy(kv_synth.householder_reflectors(w.S, w.H, w.reflectors, w.d,
+                                                         seed=seed)).to(dev)
+    op = rq.dense_operand(rq.householder_rotation(V, signs, rotation=desc.rotation))
+    return op, (rq.srftq_calibrate_lambda_dense, rq.srftq_quantize_dense,
+                rq.srftq_dequantize_dense)
+
+
+def fp32_alu_peak_tflops() -> float:
+    """FP32 FMA peak of the CUDA cores: 148 SMs x 128 lanes x 2 flops x the
+    measured maximum SM clock (MEASURED_PEAKS.json sm_max_mhz, else 1965 MHz)."""
+    mhz = 1965.0
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            mhz = float(json.load(f).get("sm_max_mhz", mhz))
+    except Exception:
+        pass
+    return 148 * 128 * 2 * mhz * 1e6 / 1e12
+
+
+def dense_roofline(w, kind, ms, kname):
+    """Roofline of a dense-rotation kernel: the contraction R x (or R^T y) is
+    2 d^2 flops per vector on the CUDA cores' float32 FMA pipe."""
+    flops = 2.0 * w.d * w.d * w.vectors
+    achieved = flops / (ms / 1e3) / 1e12
+    peak = fp32_alu_peak_tflops()
+    return {"bound": "alu", "kernel": kname, "launch": kind, "achieved": achieved,
+            "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+            "peak_source": "148 SMs x 128 FP32 lanes x 2 flops x max SM clock",
+            "algorithmic_flops_per_launch": flops, "traffic": None}
 
 
 def csrc_hash(kernel: str) -> str:
@@ -187,10 +229,19 @@ def _num(s):
 # ---------------------------------------------------------------------------
 
 def oracle_step(w, x16, signs, rot):
-    """One oracle pass on a sample: calibrate, quantize, dequantize."""
+    """One oracle pass on a sample: calibrate, quantize, dequantize (with the
+    workload's dense Householder rotation when it has reflectors)."""
     import oracle
 
-    lam = oracle.calibrate_lambda(x16, signs, min(w.n_cal, x16.shape[1]), rot).astype(np.float32)
+    n_cal = min(w.n_cal, x16.shape[1])
+    if w.reflectors:
+        V = kv_synth.householder_reflectors(1, w.H, w.reflectors, w.d, seed=1)
+        R = oracle.householder_rotations(V, signs, rot)
+        lam = oracle.calibrate_lambda_dense(x16, R, n_cal).astype(np.float32)
+        q = oracle.quantize_dense(x16, R, lam, w.group, w.bits)
+        oracle.dequantize_dense(q["codes"], q["scales"], R, lam, w.d, w.group, w.bits)
+        return
+    lam = oracle.calibrate_lambda(x16, signs, n_cal, rot).astype(np.float32)
     q = oracle.quantize(x16, signs, lam, w.group, w.bits, rot)
     oracle.dequantize(q["codes"], q["scales"], signs, lam, w.d, w.group, w.bits, rot)
 
@@ -346,15 +397,19 @@ def run_ours(args):
     scales = torch.empty((w.S, w.N, w.H, w.d // w.group), dtype=torch.float16, device=dev)
     xhat = torch.empty_like(x)
     desc = rq.make_desc(w.d, w.H, w.group, w.bits, rot)
+    # the per-(slice, head) table the calls read: the signs, or for a dense
+    # rotation the operand of R = H(v_1) ... H(v_k) B (built once, before timing)
+    table, fns = codec_calls(rq, w, desc, signs, sign_seed, dev)
+    f_cal, f_q, f_dq = fns
 
     def step(ev=None):
-        rq.srftq_calibrate_lambda(desc, x, signs, lam, w.n_cal)
+        f_cal(desc, x, table, lam, w.n_cal)
         if ev is not None:
             ev[0].record()
-        rq.srftq_quantize(desc, x, signs, lam, codes, scales)
+        f_q(desc, x, table, lam, codes, scales)
         if ev is not None:
             ev[1].record()
-        rq.srftq_dequantize(desc, codes, scales, signs, lam, xhat)
+        f_dq(desc, codes, scales, table, lam, xhat)
         if ev is not None:
             ev[2].record()
 
@@ -397,12 +452,20 @@ def run_ours(args):
     dom = "quantize" if q_avg >= d_avg else "dequantize"
     dom_ms = max(q_avg, d_avg)
     achieved = bytes_launch / (dom_ms / 1e3) / 1e9
-    kname = codec_kernel(dom, w.d)
+    kname = codec_kernel(dom, w.d, dense=w.reflectors > 0)
+    roof = {"bound": "hbm", "kernel": kname, "achieved": achieved, "peak": peak,
+            "unit": "GB/s", "frac": achieved / peak,
+            "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured"
+            else "fallback 6.65 TB/s",
+            "algorithmic_bytes_per_launch": bytes_launch,
+            "traffic": read_traffic(kname, w.name)}
+    if w.reflectors:
+        roof = dense_roofline(w, dom, dom_ms, kname)
 
     e2e = None
     if not args.no_e2e:
-        e2e = run_e2e(args, rq, desc, w, x, signs, lam, codes, scales, xhat, barrier, pg, dev,
-                      step_bytes, world)
+        e2e = run_e2e(args, rq, desc, w, x, table, lam, codes, scales, xhat, barrier, pg, dev,
+                      step_bytes, world, fns)
 
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": K,
@@ -414,11 +477,7 @@ def run_ours(args):
                     "quantize_GBps": bytes_launch / (q_avg / 1e3) / 1e9,
                     "dequantize_GBps": bytes_launch / (d_avg / 1e3) / 1e9,
                     "calibrate_ms_est": ms / K - q_avg - d_avg},
-        "roofline": {"bound": "hbm", "kernel": kname, "achieved": achieved, "peak": peak,
-                     "unit": "GB/s", "frac": achieved / peak,
-                     "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured" else "fallback 6.65 TB/s",
-                     "algorithmic_bytes_per_launch": bytes_launch,
-                     "traffic": read_traffic(kname, w.name)},
+        "roofline": roof,
         "gpu_launches": 3 * K,
         "clocks": clk,
         "quality": quality,
@@ -464,14 +523,14 @@ def _codec_figures(rq, w, rot, dev, iters):
     x = kv_synth.make_x_torch(w, dev, seed=0)
     signs = torch.from_numpy(kv_synth.rademacher_signs(w.S, w.H, w.d, seed=1)).to(dev)
     desc = rq.make_desc(w.d, w.H, w.group, w.bits, rot)
+    table, (f_cal, f_q, f_dq) = codec_calls(rq, w, desc, signs, 1, dev)
     lam = torch.empty((w.S, w.H, w.d), dtype=torch.float32, device=dev)
-    rq.srftq_calibrate_lambda(desc, x, signs, lam, w.n_cal)
+    f_cal(desc, x, table, lam, w.n_cal)
     codes = torch.empty((w.S, w.N, w.H, w.d * w.bits // 8), dtype=torch.uint8, device=dev)
     scales = torch.empty((w.S, w.N, w.H, w.d // w.group), dtype=torch.float16, device=dev)
     xhat = torch.empty_like(x)
-    q_ms = _time_launches(lambda: rq.srftq_quantize(desc, x, signs, lam, codes, scales), iters)
-    d_ms = _time_launches(lambda: rq.srftq_dequantize(desc, codes, scales, signs, lam, xhat),
-                          iters)
+    q_ms = _time_launches(lambda: f_q(desc, x, table, lam, codes, scales), iters)
+    d_ms = _time_launches(lambda: f_dq(desc, codes, scales, table, lam, xhat), iters)
     if rq.srftq_check_device() != 0:
         raise RuntimeError(f"device guard fired in {w.name}")
     peak = read_peak()[0]
@@ -482,7 +541,8 @@ def _codec_figures(rq, w, rot, dev, iters):
            "quantize_frac": b / q_ms / 1e6 / peak,
            "dequantize_ms": d_ms, "dequantize_GBps": b / d_ms / 1e6,
            "dequantize_frac": b / d_ms / 1e6 / peak,
-           "kernels": [codec_kernel("quantize", w.d), codec_kernel("dequantize", w.d)],
+           "kernels": [codec_kernel("quantize", w.d, w.reflectors > 0),
+                       codec_kernel("dequantize", w.d, w.reflectors > 0)],
            "rel_l2_error": round_trip_error(x, xhat)}
     del x, codes, scales, xhat
     torch.cuda.empty_cache()
@@ -560,6 +620,13 @@ def other_configs(rq, dev, iters=50):
                                                              srht["rel_l2_error"]["rel_l2_mean"]]}
     out["gemma_like_d256"] = _codec_figures(rq, kv_synth.WORKLOADS["gemma_like_d256"], 0, dev,
                                             iters)
+    hh = kv_synth.WORKLOADS["householder_d256"]
+    out["householder_d256"] = _codec_figures(rq, hh, 0, dev, iters)
+    q_flops = 2.0 * hh.d * hh.d * hh.vectors
+    for kind in ("quantize", "dequantize"):
+        out["householder_d256"][f"{kind}_TFLOPs"] = q_flops / out["householder_d256"][
+            f"{kind}_ms"] / 1e9
+    out["householder_d256"]["flops_per_launch"] = q_flops
     out["decode_stream_d128_fused_attention"] = _attention_figures(rq, dev, iters)
     rep = parity_report()
     if rep is not None:
@@ -577,7 +644,7 @@ def e2e_chunks(n_slices: int, target: int = 8) -> list:
 
 
 def run_e2e(args, rq, desc, w, x, signs, lam, codes, scales, xhat, barrier, pg, dev,
-            step_bytes, world) -> dict:
+            step_bytes, world, fns) -> dict:
     """The step end to end through the C ABI: the fp16 cache comes from pinned
     host memory and the dequantised cache goes back to it, every step. The
     step is pipelined over chunks of whole slices on three streams (copy in,
@@ -605,11 +672,10 @@ def run_e2e(args, rq, desc, w, x, signs, lam, codes, scales, xhat, barrier, pg, 
                 e_in.record(s_in)
             with torch.cuda.stream(s_cmp):
                 s_cmp.wait_event(e_in)
-                rq.srftq_calibrate_lambda(desc, x[a:b], signs[a:b], lam[a:b], w.n_cal, s_cmp)
-                rq.srftq_quantize(desc, x[a:b], signs[a:b], lam[a:b], codes[a:b], scales[a:b],
-                                  s_cmp)
-                rq.srftq_dequantize(desc, codes[a:b], scales[a:b], signs[a:b], lam[a:b],
-                                    xhat[a:b], s_cmp)
+                f_cal, f_q, f_dq = fns
+                f_cal(desc, x[a:b], signs[a:b], lam[a:b], w.n_cal, s_cmp)
+                f_q(desc, x[a:b], signs[a:b], lam[a:b], codes[a:b], scales[a:b], s_cmp)
+                f_dq(desc, codes[a:b], scales[a:b], signs[a:b], lam[a:b], xhat[a:b], s_cmp)
                 e_cmp.record(s_cmp)
             with torch.cuda.stream(s_out):
                 s_out.wait_event(e_cmp)

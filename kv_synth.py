@@ -42,6 +42,7 @@ class Workload:
     n_cal: int = 512
     rotations: tuple = (0,)
     note: str = ""
+    reflectors: int = 0   # Householder reflectors on the base rotation (dense codec)
 
     @property
     def vectors(self) -> int:
@@ -75,6 +76,12 @@ WORKLOADS = {
         outlier="coord", outlier_p=0.005, outlier_scale=25.0,
         note="2 layers x {K,V}, 4 KV heads, d=256, batch 4 x seq 8192 rows; N(0,1) "
              "with 0.5% of coordinates x25; int4 G32"),
+    "householder_d256": Workload(
+        "householder_d256", S=4, N=32768, H=4, d=256, bits=4, group=32, dist="normal",
+        outlier="coord", outlier_p=0.005, outlier_scale=25.0, reflectors=128,
+        note="the gemma_like_d256 shape with a dense rotation: k = d/2 = 128 Householder "
+             "reflectors (seeded N(0,1) vectors standing in for learned ones) on the SRFT "
+             "base; int4 G32"),
     "decode_stream_d128": Workload(
         "decode_stream_d128", S=64, N=32768 * 32, H=8, d=128, bits=4, group=16,
         dist="normal", outlier="none", outlier_p=0.0, outlier_scale=1.0,

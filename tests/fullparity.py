@@ -61,6 +61,25 @@ def check_chunk(job: tuple) -> dict:
     return out
 
 
+def check_chunk_dense(job: tuple) -> dict:
+    """Worker for the dense-rotation codec: as check_chunk, with the oracle's
+    rotation matrices R [1, H, d, d] in place of the sign rows."""
+    x16, R, lam, codes, scales, xhat, d, group, bits = job
+    with np.errstate(all="ignore"):
+        ref = oracle.quantize_dense(x16, R, lam, group, bits)
+        st = parity.check_codes(ref, codes, scales, bits, group, parity.DENSE_SCALE_BAND)
+        deq = oracle.dequantize_dense(codes, scales, R, lam, d, group, bits)
+        dq = parity.check_dequant(xhat, deq["bits"])
+    out = dict(st)
+    out["dequant_values"] = int(xhat.size)
+    out["dequant_violations"] = dq["violations"]
+    out["dequant_overflow_to_inf"] = dq["overflow_to_inf"]
+    out["dequant_max_abs_err"] = dq["max_abs_err"]
+    out["dequant_max_err_over_tol"] = dq["max_err_over_tol"]
+    out["vectors"] = int(np.prod(x16.shape[:3]))
+    return out
+
+
 def merge(total: dict, part: dict) -> dict:
     for k in _SUM_KEYS:
         total[k] = total.get(k, 0) + part.get(k, 0)
@@ -100,10 +119,10 @@ class Checker:
         self.total: dict = {}
         self.t0 = time.time()
 
-    def submit(self, job: tuple) -> None:
+    def submit(self, job: tuple, fn=check_chunk) -> None:
         while len(self.pending) >= 2 * self.n:
             self._drain_one()
-        self.pending.append(self.pool.apply_async(check_chunk, (job,)))
+        self.pending.append(self.pool.apply_async(fn, (job,)))
 
     def _drain_one(self) -> None:
         merge(self.total, self.pending.pop(0).get())

@@ -4,8 +4,8 @@ through the C ABI.
 
 The rotation builder is compared with the oracle's float64 matrices (float32
 storage: 2e-6 absolute on entries of unit-norm rows); the operand split bit
-for bit; the codec stages with the same tolerances as the FFT codec
-(tests/parity.py), each stage fed the oracle's own inputs: the quantiser and
+for bit; the codec stages with the tolerances of tests/parity.py (the scale
+band of the dense path: 1e-5), each stage fed the oracle's own inputs: the quantiser and
 the calibration get the operand of the oracle's matrix (rounded to float32),
 the dequantiser the oracle's codes.
 """
@@ -87,7 +87,7 @@ def _quant_check(x16, R, lam, d, group, bits, what):
     codes, scales = rq.quantize_dense(_t(x16), op, lt, group, bits)
     ref = oracle.quantize_dense(x16, R, lam, group, bits)
     c_np, s_np = codes.cpu().numpy(), _np16(scales)
-    stats = parity.check_codes(ref, c_np, s_np, bits, group)
+    stats = parity.check_codes(ref, c_np, s_np, bits, group, parity.DENSE_SCALE_BAND)
     parity.assert_clean(stats, f"{what} codes")
     # dequantiser on the oracle's codes, and the GPU round trip on its own codes
     deq = oracle.dequantize_dense(ref["codes"], ref["scales"], R, lam, d, group, bits)
@@ -138,8 +138,8 @@ def test_dense_codec_with_the_gpu_built_rotation():
     op = rq.dense_operand(rq.householder_rotation(_t(V), _t(signs)))
     codes, scales = rq.quantize_dense(_t(x16), op, _t(lam), group, bits)
     ref = oracle.quantize_dense(x16, R, lam, group, bits)
-    parity.assert_clean(parity.check_codes(ref, codes.cpu().numpy(), _np16(scales), bits, group),
-                        "gpu-built rotation")
+    parity.assert_clean(parity.check_codes(ref, codes.cpu().numpy(), _np16(scales), bits, group,
+                                           parity.DENSE_SCALE_BAND), "gpu-built rotation")
 
 
 def test_dense_strided_windows_keep_their_guard_bands():
@@ -158,7 +158,7 @@ def test_dense_strided_windows_keep_their_guard_bands():
     ref = oracle.quantize_dense(big[:, off:off + N], R, lam, group, bits)
     c_np, s_np = codes.cpu().numpy(), _np16(scales)
     parity.assert_clean(parity.check_codes(ref, c_np[:, off:off + N], s_np[:, off:off + N], bits,
-                                           group), "strided dense codes")
+                                           group, parity.DENSE_SCALE_BAND), "strided dense codes")
     outside = np.ones(T, bool)
     outside[off:off + N] = False
     assert np.all(c_np[:, outside] == 0xAB)

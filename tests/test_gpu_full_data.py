@@ -246,3 +246,54 @@ def test_full_data_decode_stream_slices_0_and_63(checker):
     assert stats["vectors"] == 2 * n * w.H
     del codes, scales, scratch
     torch.cuda.empty_cache()
+
+
+def test_full_data_householder_d256(checker):
+    """The dense-rotation codec at the Gemma-shaped size (4 slices x 32768
+    rows x 4 heads, d = 256, int4 G32) with k = 128 Householder reflectors
+    on the SRFT base ("When Quantization Is Free", Methodology 3), as the
+    benchmark launches it: every vector against the oracle, which uses its
+    own float64 rotation; the GPU reads the operand of that rotation rounded
+    to float32, and builds its own from the same reflectors for a second,
+    end-to-end pass."""
+    w = kv_synth.WORKLOADS["householder_d256"]
+    x = kv_synth.make_x_torch(w, DEV, seed=0)
+    signs = kv_synth.rademacher_signs(w.S, w.H, w.d, seed=1)
+    V = kv_synth.householder_reflectors(w.S, w.H, w.reflectors, w.d, seed=1)
+    R = oracle.householder_rotations(V, signs, 0)
+    lam64 = oracle.calibrate_lambda_dense(x[:, :w.n_cal].cpu().numpy(), R, w.n_cal)
+    lam = lam64.astype(np.float32)
+    lt = _t(lam)
+    op = rq.dense_operand(_t(R.astype(np.float32)))
+    lam_gpu = rq.calibrate_lambda_dense(x, op, w.n_cal).cpu().numpy()
+    lam_stats = parity.check_lambda(lam_gpu, lam64)
+    parity.assert_clean(lam_stats, "householder lambda")
+    codes, scales = rq.quantize_dense(x, op, lt, w.group, w.bits)
+    xhat = rq.dequantize_dense(codes, scales, op, lt, w.d, w.group, w.bits)
+    torch.cuda.synchronize()
+    step = max(1, VECTORS_PER_CHUNK // w.H)
+    for s in range(w.S):
+        for r0 in range(0, w.N, step):
+            r1 = min(w.N, r0 + step)
+            checker.submit((x[s:s + 1, r0:r1].cpu().numpy(), R[s:s + 1], lam[s:s + 1],
+                            codes[s:s + 1, r0:r1].cpu().numpy(), _bits16(scales[s:s + 1, r0:r1]),
+                            _bits16(xhat[s:s + 1, r0:r1]), w.d, w.group, w.bits),
+                           fullparity.check_chunk_dense)
+    quality = _rel_l2(x, xhat)
+    stats = checker.result()
+    # the GPU-built rotation end to end: codes within the band of the oracle's
+    op_gpu = rq.dense_operand(rq.householder_rotation(_t(V), _t(signs)))
+    codes2, scales2 = rq.quantize_dense(x[:1], op_gpu[:1], lt[:1], w.group, w.bits)
+    ref = oracle.quantize_dense(x[:1, :4096].cpu().numpy(), R[:1], lam[:1], w.group, w.bits)
+    gpu_built = parity.check_codes(ref, codes2[:, :4096].cpu().numpy(),
+                                   _bits16(scales2[:, :4096]), w.bits, w.group,
+                                   parity.DENSE_SCALE_BAND)
+    parity.assert_clean(gpu_built, "GPU-built rotation")
+    record = {"workload": w.name, "rotation": "Householder k=128 on SRFT",
+              "shape": [w.S, w.N, w.H, w.d], "bits": w.bits, "group": w.group,
+              "lambda_max_rel_err": lam_stats["max_rel_err"], "rel_l2_error": quality,
+              "gpu_built_rotation_first_4096_rows": gpu_built, **stats}
+    fullparity.write_report(f"{w.name}:householder", record)
+    print(record)
+    assert not fullparity.violations(stats), stats
+    assert stats["vectors"] == w.vectors
