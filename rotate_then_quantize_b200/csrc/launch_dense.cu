@@ -1,7 +1,9 @@
-// Launchers of the dense-rotation codec (dense.cuh): the Householder rotation
-// builder, the operand split, and the quantise / dequantise / calibration
-// products, for d in {64, 128, 256}.
+// Launchers of the dense-rotation codec: the Householder rotation builder,
+// the operand split and the dequantise / calibration products (dense.cuh,
+// CUDA cores), and the tensor-core quantiser (dense_mma.cuh), for d in
+// {64, 128, 256}.
 #include "dense.cuh"
+#include "dense_mma.cuh"
 #include "launch_impl.cuh"
 
 namespace srftq {
@@ -77,7 +79,69 @@ int launch_dense_codec(const DenseCall& c) {
   });
 }
 
-int launch_quantize_dense(const DenseCall& c) { return launch_dense_codec<true>(c); }
+constexpr int kDenseEpiGroups = 2;
+
+template <int D, int BITS, int G>
+int quantize_dense_mma(const DenseCall& c) {
+  using L = DenseMma<D, kDenseEpiGroups>;
+  const int64_t row_blocks = (c.n_rows + 127) / 128;
+  const int64_t total = c.n_slices * c.heads * row_blocks;
+  if (total > INT_MAX || c.n_rows > INT_MAX || c.n_slices * c.heads * 2 * D > INT_MAX)
+    return SRFTQ_ERR_UNSUPPORTED;
+  CUtensorMap tm_x, tm_op;
+  {
+    // x [S][T][H][d] fp16: boxes of 64 elements x 1 head x 128 rows
+    const uint64_t dims[4] = {uint64_t(D), uint64_t(c.heads), uint64_t(c.n_rows),
+                              uint64_t(c.n_slices)};
+    const uint64_t str[3] = {uint64_t(2 * D), uint64_t(c.heads) * 2 * D,
+                             uint64_t(c.in_stride_rows) * c.heads * 2 * D};
+    const uint32_t box[4] = {64u, 1u, 128u, 1u};
+    if (Runtime::encode_4d(&tm_x, CU_TENSOR_MAP_DATA_TYPE_UINT16, const_cast<uint16_t*>(c.x),
+                           dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B) != 0)
+      return SRFTQ_ERR_CUDA;
+  }
+  {
+    // operand [S][H][2][d][d] fp16 as a 2-D array of rows of d elements (a
+    // rank-4 map with two unit dimensions): boxes of 64 columns x d rows
+    const uint64_t dims[4] = {uint64_t(D), uint64_t(c.n_slices * c.heads * 2 * D), 1, 1};
+    const uint64_t str[3] = {uint64_t(2 * D), uint64_t(2 * D) * c.n_slices * c.heads * 2 * D,
+                             uint64_t(2 * D) * c.n_slices * c.heads * 2 * D};
+    const uint32_t box[4] = {64u, uint32_t(D), 1u, 1u};
+    if (Runtime::encode_4d(&tm_op, CU_TENSOR_MAP_DATA_TYPE_UINT16,
+                           const_cast<uint16_t*>(c.operand), dims, str, box,
+                           CU_TENSOR_MAP_SWIZZLE_128B) != 0)
+      return SRFTQ_ERR_CUDA;
+  }
+  unsigned* guard = Runtime::guard_word();
+  if (!guard) return SRFTQ_ERR_CUDA;
+  DenseMmaArgs a{c.n_rows, row_blocks, total, c.heads, c.codes, c.scales, c.out_stride_rows,
+                 c.lambda, guard};
+  constexpr auto K = quantize_dense_mma_kernel<D, BITS, G, kDenseEpiGroups>;
+  constexpr int smem = L::kBytes + kSmemSlack;
+  int bps = 0;
+  const int rc = prepare_kernel<K>(smem, L::kThreads, &bps);
+  if (rc != SRFTQ_OK) return rc;
+  const int64_t cap = int64_t(Runtime::num_sms()) * bps;
+  const int grid = int(total < cap ? total : cap);
+  K<<<grid, L::kThreads, smem, c.stream>>>(tm_x, tm_op, a);
+  return finish_launch();
+}
+
+int launch_quantize_dense(const DenseCall& c) {
+  if (c.n_slices == 0 || c.n_rows == 0) return SRFTQ_OK;
+  return by_dense_d(c.d, [&](auto d_) {
+    constexpr int D = decltype(d_)::value;
+    int rc = SRFTQ_ERR_UNSUPPORTED;
+    static_for<0, 2>([&](auto b_) {
+      constexpr int BITS = decltype(b_)::value == 0 ? 4 : 8;
+      static_for<3, ilog2(D) + 1>([&](auto lg_) {
+        constexpr int G = 1 << decltype(lg_)::value;
+        if (c.bits == BITS && c.group == G) rc = quantize_dense_mma<D, BITS, G>(c);
+      });
+    });
+    return rc;
+  });
+}
 int launch_dequantize_dense(const DenseCall& c) { return launch_dense_codec<false>(c); }
 
 int launch_calibrate_dense(const DenseCalibCall& c) {

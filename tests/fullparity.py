@@ -67,7 +67,8 @@ def check_chunk_dense(job: tuple) -> dict:
     x16, R, lam, codes, scales, xhat, d, group, bits = job
     with np.errstate(all="ignore"):
         ref = oracle.quantize_dense(x16, R, lam, group, bits)
-        st = parity.check_codes(ref, codes, scales, bits, group, parity.DENSE_SCALE_BAND)
+        st = parity.check_codes(ref, codes, scales, bits, group, parity.DENSE_SCALE_BAND,
+                                parity.dense_code_band(ref, lam, group))
         deq = oracle.dequantize_dense(codes, scales, R, lam, d, group, bits)
         dq = parity.check_dequant(xhat, deq["bits"])
     out = dict(st)

@@ -19,12 +19,16 @@ Tolerances (fixed before any kernel ran):
   values beyond the binary16 range round to the same infinity on both sides
   and count as equal.
 * lambda (calibration): relative 1e-5.
-* dense-rotation codec: the same, except the scale band, which is the
-  rotation tolerance (1e-5 relative) instead of 1e-6. Its rotation is a
-  float32 product summing d terms per coordinate (the FFT's rotated values
-  carry ~1e-7 relative error, the dense product's ~1e-6 at d = 256), and a
-  rotated value within the 1e-5 rotation tolerance can move absmax / qmax
-  across a binary16 midpoint only when it lies within 1e-5 of it.
+* dense-rotation codec: both bands follow from the rotation tolerance
+  instead. Its rotation is a float32 product summing d terms per coordinate
+  (on the tensor cores, d fp16 products per half of the operand): the FFT's
+  rotated values carry ~1e-7 relative error, the dense product's ~1e-6 at
+  d = 256. A rotated value within the 1e-5 rotation tolerance moves
+  absmax / qmax by at most 1e-5 relative (scale band 1e-5), and moves
+  w_j / sigma_g by at most 1e-5 max(|y_j|, rms(y)) / (lambda_j sigma_g)
+  code units (code band: that, or 1e-4 where it is smaller). The latter
+  matters for int8 (127 levels), whose code unit is 18 times finer than
+  int4's.
 """
 
 from __future__ import annotations
@@ -50,8 +54,21 @@ def check_rotation(y_gpu: np.ndarray, y_ref: np.ndarray) -> dict:
     return {"max_rel_err": float(err.max(initial=0.0)), "violations": bad}
 
 
+def dense_code_band(ref: dict, lam: np.ndarray, group: int) -> np.ndarray:
+    """Per-coordinate code band of the dense codec (see the module docstring):
+    max(1e-4, 1e-5 max(|y_j|, rms(y)) / (lambda_j sigma_g)) in code units,
+    from the oracle's rotated values y and scales; lam [S, H, d]."""
+    y = np.asarray(ref["y"], np.float64)
+    rms = np.sqrt(np.mean(y * y, axis=-1, keepdims=True))
+    sig = oracle.binary16_bits_to_float(ref["scale_bits"]).repeat(group, axis=-1)
+    lam_b = np.asarray(lam, np.float32).astype(np.float64)[:, None]
+    with np.errstate(divide="ignore", invalid="ignore"):
+        band = ROT_TOL * np.maximum(np.abs(y), rms) / (lam_b * sig)
+    return np.maximum(CODE_BAND, np.nan_to_num(band, nan=CODE_BAND, posinf=CODE_BAND))
+
+
 def check_codes(ref: dict, codes_gpu: np.ndarray, scales_gpu: np.ndarray, bits: int,
-                group: int, scale_band: float = SCALE_BAND) -> dict:
+                group: int, scale_band: float = SCALE_BAND, code_band=None) -> dict:
     """ref: output of oracle.quantize (or quantize_vectors + pack) on the same inputs.
 
     Groups whose oracle scale is zero (sigma = 0: the group's absmax rounds
@@ -84,8 +101,9 @@ def check_codes(ref: dict, codes_gpu: np.ndarray, scales_gpu: np.ndarray, bits: 
     pre = np.abs(ref["pre"].reshape(shape_g + (group,)))
     pre = np.where(zero[..., None], 0.0, pre)    # w / 0 is not a rounding position
     frac = pre - np.floor(pre)
-    near_half = np.abs(frac - 0.5) < CODE_BAND
-    near_clamp = np.abs(pre - (qmax + 0.5)) < CODE_BAND
+    cb = CODE_BAND if code_band is None else np.asarray(code_band).reshape(pre.shape)
+    near_half = np.abs(frac - 0.5) < cb
+    near_clamp = np.abs(pre - (qmax + 0.5)) < cb
     one_step = np.abs(qg_ref - qg_gpu) == 1
     allowed = (near_half | near_clamp) & one_step
     code_viol = int(np.sum(cmis & ~allowed))

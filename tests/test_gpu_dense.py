@@ -4,8 +4,8 @@ through the C ABI.
 
 The rotation builder is compared with the oracle's float64 matrices (float32
 storage: 2e-6 absolute on entries of unit-norm rows); the operand split bit
-for bit; the codec stages with the tolerances of tests/parity.py (the scale
-band of the dense path: 1e-5), each stage fed the oracle's own inputs: the quantiser and
+for bit; the codec stages with the tolerances of tests/parity.py (the dense
+path's bands follow from the rotation tolerance), each stage fed the oracle's own inputs: the quantiser and
 the calibration get the operand of the oracle's matrix (rounded to float32),
 the dequantiser the oracle's codes.
 """
@@ -87,7 +87,8 @@ def _quant_check(x16, R, lam, d, group, bits, what):
     codes, scales = rq.quantize_dense(_t(x16), op, lt, group, bits)
     ref = oracle.quantize_dense(x16, R, lam, group, bits)
     c_np, s_np = codes.cpu().numpy(), _np16(scales)
-    stats = parity.check_codes(ref, c_np, s_np, bits, group, parity.DENSE_SCALE_BAND)
+    stats = parity.check_codes(ref, c_np, s_np, bits, group, parity.DENSE_SCALE_BAND,
+                               parity.dense_code_band(ref, lam, group))
     parity.assert_clean(stats, f"{what} codes")
     # dequantiser on the oracle's codes, and the GPU round trip on its own codes
     deq = oracle.dequantize_dense(ref["codes"], ref["scales"], R, lam, d, group, bits)
@@ -139,7 +140,9 @@ def test_dense_codec_with_the_gpu_built_rotation():
     codes, scales = rq.quantize_dense(_t(x16), op, _t(lam), group, bits)
     ref = oracle.quantize_dense(x16, R, lam, group, bits)
     parity.assert_clean(parity.check_codes(ref, codes.cpu().numpy(), _np16(scales), bits, group,
-                                           parity.DENSE_SCALE_BAND), "gpu-built rotation")
+                                           parity.DENSE_SCALE_BAND,
+                                           parity.dense_code_band(ref, lam, group)),
+                        "gpu-built rotation")
 
 
 def test_dense_strided_windows_keep_their_guard_bands():
@@ -158,7 +161,9 @@ def test_dense_strided_windows_keep_their_guard_bands():
     ref = oracle.quantize_dense(big[:, off:off + N], R, lam, group, bits)
     c_np, s_np = codes.cpu().numpy(), _np16(scales)
     parity.assert_clean(parity.check_codes(ref, c_np[:, off:off + N], s_np[:, off:off + N], bits,
-                                           group, parity.DENSE_SCALE_BAND), "strided dense codes")
+                                           group, parity.DENSE_SCALE_BAND,
+                                           parity.dense_code_band(ref, lam, group)),
+                        "strided dense codes")
     outside = np.ones(T, bool)
     outside[off:off + N] = False
     assert np.all(c_np[:, outside] == 0xAB)
@@ -189,3 +194,26 @@ def test_dense_degenerate_values():
         lam = np.full((1, 1, d), lam_val, np.float32)
         for bits in (4, 8):
             _quant_check(x16, R, lam, d, group, bits, f"degenerate lam={lam_val} b{bits}")
+
+
+@pytest.mark.parametrize("d,group,bits", [(64, 16, 4), (128, 16, 4), (128, 128, 8),
+                                          (256, 32, 4), (256, 256, 4)])
+def test_dense_quantiser_ranges_cross_slices_and_heads(d, group, bits):
+    """More 128-row blocks than the GPU has SMs, so every CTA of the
+    quantiser takes a range of several blocks that crosses (slice, head)
+    boundaries: the operand is reloaded (d <= 128) or streamed (d = 256)
+    for each, and a partial last block per (slice, head). Every vector is
+    compared with the oracle."""
+    rng = np.random.default_rng(d + group + bits)
+    S, N, H = 3, 1000, 5                       # 8 blocks per (slice, head), 120 in all ...
+    if d < 256:
+        S, N = 4, 2600                         # ... or 21 x 20 = 420
+    x16, signs, V, R = _case(rng, S, N, H, d, d // 2, 0, outlier_p=0.005, scale=25.0)
+    lam = oracle.calibrate_lambda_dense(x16, R, 128).astype(np.float32)
+    op = rq.dense_operand(_t(R.astype(np.float32)))
+    codes, scales = rq.quantize_dense(_t(x16), op, _t(lam), group, bits)
+    ref = oracle.quantize_dense(x16, R, lam, group, bits)
+    parity.assert_clean(parity.check_codes(ref, codes.cpu().numpy(), _np16(scales), bits, group,
+                                           parity.DENSE_SCALE_BAND,
+                                           parity.dense_code_band(ref, lam, group)),
+                        f"d{d} g{group} b{bits} many blocks")

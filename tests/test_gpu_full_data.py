@@ -287,7 +287,8 @@ def test_full_data_householder_d256(checker):
     ref = oracle.quantize_dense(x[:1, :4096].cpu().numpy(), R[:1], lam[:1], w.group, w.bits)
     gpu_built = parity.check_codes(ref, codes2[:, :4096].cpu().numpy(),
                                    _bits16(scales2[:, :4096]), w.bits, w.group,
-                                   parity.DENSE_SCALE_BAND)
+                                   parity.DENSE_SCALE_BAND,
+                                   parity.dense_code_band(ref, lam[:1], w.group))
     parity.assert_clean(gpu_built, "GPU-built rotation")
     record = {"workload": w.name, "rotation": "Householder k=128 on SRFT",
               "shape": [w.S, w.N, w.H, w.d], "bits": w.bits, "group": w.group,

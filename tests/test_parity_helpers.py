@@ -121,3 +121,33 @@ def test_full_data_checker_runs_in_spawned_workers():
         c.close()
     assert clean["vectors"] == 80 and not fullparity.violations(clean)
     assert planted["code_violations"] == 1
+
+
+def test_dense_code_band_follows_the_rotation_tolerance():
+    """The dense codec's code band is max(1e-4, 1e-5 max(|y|, rms)/(lambda
+    sigma)): int8's finer code unit widens it, and a flip just outside 1e-4
+    but inside that band is counted, not failed; two steps never pass."""
+    rng = np.random.default_rng(12)
+    d, group = 64, 16
+    x16 = rng.standard_normal((1, 32, 1, d)).astype(np.float16)
+    R = oracle.householder_rotations(rng.standard_normal((1, 1, 8, d)), np.ones((1, 1, d), np.int8),
+                                     0)
+    lam = np.ones((1, 1, d), np.float32)
+    for bits, wider in ((4, False), (8, True)):
+        ref = oracle.quantize_dense(x16, R, lam, group, bits)
+        band = parity.dense_code_band(ref, lam, group)
+        assert band.min() >= parity.CODE_BAND
+        assert (band.max() > 2 * parity.CODE_BAND) == wider
+    ref = dict(ref)                                    # int8
+    band = parity.dense_code_band(ref, lam, group)
+    i = tuple(np.argwhere((band > 3e-4) & (np.abs(ref["q"]) < 100))[0])
+    pre, q = ref["pre"].copy(), ref["q"].copy()
+    pre[i] = q[i] + 0.5 + 2e-4 * (1 if q[i] >= 0 else -1)
+    ref["pre"] = pre
+    q_gpu = q.copy()
+    q_gpu[i] += 1 if q[i] >= 0 else -1
+    st = parity.check_codes(ref, oracle.pack_codes(q_gpu, 8), ref["scales"], 8, group,
+                            parity.DENSE_SCALE_BAND, band)
+    assert st["code_violations"] == 0 and st["code_mismatch_in_band"] == 1
+    st = parity.check_codes(ref, oracle.pack_codes(q_gpu, 8), ref["scales"], 8, group)
+    assert st["code_violations"] == 1                  # the fixed 1e-4 band would fail it
