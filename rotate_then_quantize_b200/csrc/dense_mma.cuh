@@ -11,9 +11,12 @@
 //
 // A *block* is 128 consecutive rows of one (slice, head): the MMA's M = 128
 // rows are 128 vectors, N = d outputs, K = d inputs (16 per instruction).
-// Blocks are numbered (slice, head, row block), row block fastest; every
-// CTA (one per SM) takes one contiguous range, so its (slice, head) and with
-// it the operand change only at the ends of a range.
+// CTA c (one per SM) serves head c % H, and the CTAs of one head split that
+// head's (slice, row block) sequence into contiguous ranges: the operand
+// changes only at slice boundaries, and the CTAs of all H heads walk the same
+// rows at about the same time, so every row of H heads that a DRAM page holds
+// is read while the page is open (one block reads only its head's d elements
+// of each row).
 //
 // Warp roles (128 + 128 E threads, E = 2):
 //   warp 0      A producer: TMA loads of x tiles (NST stages; 128-byte
@@ -72,7 +75,7 @@ struct DenseMma {
 };
 
 struct DenseMmaArgs {
-  int64_t n_rows, row_blocks, total_blocks;
+  int64_t n_rows, row_blocks, n_slices;
   int32_t heads;
   uint8_t* codes;         // [S][T_out][H][d*bits/8]
   uint16_t* scales;       // [S][T_out][H][d/G]
@@ -142,13 +145,16 @@ __global__ void __launch_bounds__(DenseMma<D, EPI>::kThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
 
-  // this CTA's contiguous range of blocks
-  const int64_t T = a.total_blocks;
-  const int64_t per = T / gridDim.x, rem = T % gridDim.x;
-  const int64_t b0 = blockIdx.x * per + (blockIdx.x < rem ? blockIdx.x : rem);
-  const int n = int(per + (blockIdx.x < rem ? 1 : 0));
+  // this CTA's head and contiguous range of (slice, row block) steps
+  const int hh = int(blockIdx.x % a.heads);
+  const int64_t j = blockIdx.x / a.heads, per_head = gridDim.x / a.heads;
+  const int64_t T = a.n_slices * a.row_blocks;
+  const int64_t per = T / per_head, rem = T % per_head;
+  const int64_t u0 = j * per + (j < rem ? j : rem);
+  const int n = int(per + (j < rem ? 1 : 0));
   if (n == 0) return;
-  auto sh_of = [&](int i) -> int64_t { return (b0 + i) / a.row_blocks; };
+  auto sh_of = [&](int i) -> int64_t { return ((u0 + i) / a.row_blocks) * a.heads + hh; };
+  auto rb_of = [&](int i) -> int64_t { return (u0 + i) % a.row_blocks; };
 
   if (tid == 0) {
     prefetch_tensormap(&tm_x);
@@ -189,8 +195,8 @@ __global__ void __launch_bounds__(DenseMma<D, EPI>::kThreads, 1)
         if (i >= L::kNST &&
             !wait_or_abort(&empty[st], ((i / L::kNST) & 1) ^ 1, abort_flag, a.guard))
           break;
-        const int64_t b = b0 + i, sh = b / a.row_blocks;
-        const int r0 = int((b % a.row_blocks) * 128);
+        const int64_t sh = sh_of(i);
+        const int r0 = int(rb_of(i) * 128);
         const int s = int(sh / a.heads), h = int(sh % a.heads);
         mbar_arrive_expect_tx(&full[st], L::kABytes);
 #pragma unroll
@@ -318,7 +324,7 @@ __global__ void __launch_bounds__(DenseMma<D, EPI>::kThreads, 1)
     int64_t tab_sh = -1;
     for (int i = grp; i < n; i += L::kEpi) {
       const int acc = i % L::kAcc;
-      const int64_t b = b0 + i, sh = b / a.row_blocks;
+      const int64_t sh = sh_of(i);
       if (sh != tab_sh) {
         __syncwarp();   // every lane is done reading the old table
         for (int j = lane; j < D; j += 32) rl[j] = __frcp_rn(a.lambda[sh * D + j]);
@@ -330,7 +336,7 @@ __global__ void __launch_bounds__(DenseMma<D, EPI>::kThreads, 1)
                                                  a.guard)))
         break;
       tc_fence_after();
-      const int64_t row = (b % a.row_blocks) * 128 + 32 * q + lane;
+      const int64_t row = rb_of(i) * 128 + 32 * q + lane;
       const bool valid = row < a.n_rows;
       const int64_t s = sh / a.heads, h = sh % a.heads;
       const size_t vec = size_t((s * a.out_stride_rows + row) * a.heads + h);

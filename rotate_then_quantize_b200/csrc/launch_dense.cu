@@ -114,15 +114,21 @@ int quantize_dense_mma(const DenseCall& c) {
   }
   unsigned* guard = Runtime::guard_word();
   if (!guard) return SRFTQ_ERR_CUDA;
-  DenseMmaArgs a{c.n_rows, row_blocks, total, c.heads, c.codes, c.scales, c.out_stride_rows,
-                 c.lambda, guard};
+  DenseMmaArgs a{c.n_rows, row_blocks, c.n_slices, c.heads, c.codes, c.scales,
+                 c.out_stride_rows, c.lambda, guard};
   constexpr auto K = quantize_dense_mma_kernel<D, BITS, G, kDenseEpiGroups>;
   constexpr int smem = L::kBytes + kSmemSlack;
   int bps = 0;
   const int rc = prepare_kernel<K>(smem, L::kThreads, &bps);
   if (rc != SRFTQ_OK) return rc;
+  // the same number of CTAs for every head (CTA c serves head c % H), at
+  // most one per (slice, row block) of a head
   const int64_t cap = int64_t(Runtime::num_sms()) * bps;
-  const int grid = int(total < cap ? total : cap);
+  const int64_t steps = c.n_slices * row_blocks;
+  int64_t per_head = cap / c.heads;
+  if (per_head < 1) per_head = 1;
+  if (per_head > steps) per_head = steps;
+  const int grid = int(per_head * c.heads);
   K<<<grid, L::kThreads, smem, c.stream>>>(tm_x, tm_op, a);
   return finish_launch();
 }
