@@ -54,6 +54,9 @@ def parse_args(argv=None):
     ap.add_argument("--rotation", type=int, default=0, choices=[0, 1])
     ap.add_argument("--slices", type=int, default=None,
                     help="run the workload on its first SLICES slices only (smaller captures)")
+    ap.add_argument("--reflectors", type=int, default=None,
+                    help="run the workload through the dense-rotation calls with this many "
+                         "(>= 1) Householder reflectors on its base rotation")
     ap.add_argument("--tokens", type=int, default=None,
                     help="decode_stream_d128: cached tokens per sequence (default 32768; "
                          "smaller captures)")
@@ -105,7 +108,7 @@ def codec_kernel(kind: str, d: int, dense: bool = False) -> str:
     head dimension: d = 256 runs on the two-warp kernels; a dense rotation
     on the dense kernels."""
     if dense:
-        return "dense_gemm_kernel"
+        return "quantize_dense_mma_kernel" if kind == "quantize" else "dense_gemm_kernel"
     return f"{kind}{'_split' if d == 256 else ''}_kernel"
 
 
@@ -137,14 +140,26 @@ def fp32_alu_peak_tflops() -> float:
 
 
 def dense_roofline(w, kind, ms, kname):
-    """Roofline of a dense-rotation kernel: the contraction R x (or R^T y) is
-    2 d^2 flops per vector on the CUDA cores' float32 FMA pipe."""
-    flops = 2.0 * w.d * w.d * w.vectors
+    """Roofline of a dense-rotation kernel. The quantiser runs R x on the
+    tensor cores as two fp16 products (the operand's hi and lo halves):
+    2 x 2 d^2 flops per vector against the measured dense fp16/bf16 peak.
+    The dequantiser runs R^T y on the CUDA cores: 2 d^2 flops per vector
+    against the float32 FMA peak."""
+    if kind == "quantize":
+        flops = 4.0 * w.d * w.d * w.vectors
+        peak, src = None, "measured (MEASURED_PEAKS.json bf16_tflops; fp16 runs at the same rate)"
+        try:
+            with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+                peak = float(json.load(f)["bf16_tflops"])
+        except Exception:
+            peak, src = 1590.0, "fallback 1.59 PFLOP/s"
+        bound = "tensor"
+    else:
+        flops = 2.0 * w.d * w.d * w.vectors
+        peak, src, bound = fp32_alu_peak_tflops(), "148 SMs x 128 FP32 lanes x 2 flops x max SM clock", "alu"
     achieved = flops / (ms / 1e3) / 1e12
-    peak = fp32_alu_peak_tflops()
-    return {"bound": "alu", "kernel": kname, "launch": kind, "achieved": achieved,
-            "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-            "peak_source": "148 SMs x 128 FP32 lanes x 2 flops x max SM clock",
+    return {"bound": bound, "kernel": kname, "launch": kind, "achieved": achieved,
+            "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak, "peak_source": src,
             "algorithmic_flops_per_launch": flops, "traffic": None}
 
 
@@ -373,6 +388,10 @@ def workload(args):
         if not 1 <= args.slices <= w.S:
             raise SystemExit(f"--slices must be in 1..{w.S}")
         w = dataclasses.replace(w, S=args.slices)
+    if getattr(args, "reflectors", None) is not None:
+        if args.workload == "decode_stream_d128" or w.d not in (64, 128, 256) or args.reflectors < 1:
+            raise SystemExit("--reflectors needs a codec workload with d in {64, 128, 256}")
+        w = dataclasses.replace(w, reflectors=args.reflectors, name=w.name + "+dense")
     if getattr(args, "tokens", None) is not None:
         if args.workload != "decode_stream_d128" or not 512 <= args.tokens <= 32768:
             raise SystemExit("--tokens applies to decode_stream_d128, 512..32768")
