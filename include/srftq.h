@@ -319,6 +319,27 @@ int srftq_check_device(void* stream);
  */
 int srftq_probe_wait_timeout(uint32_t polls, void* stream);
 
+/*
+ * srftq_debug_checks -- 1 if this library was built with the device-side
+ * index checks (SRFTQ_DEBUG_CHECKS; the in-tree libsrftq_debug.so), else 0.
+ * In that build every kernel checks each global-memory index it computes
+ * (vector slots, TMA tile coordinates) against the call's extents before the
+ * access; a failed check skips the access and records bit 1 of the guard
+ * word, which srftq_check_device reports as SRFTQ_ERR_DEVICE_CHECK. Nothing
+ * traps. The release build compiles the checks away.
+ */
+int srftq_debug_checks(void);
+
+/*
+ * srftq_probe_index_check -- exercises that check on the device: one thread
+ * checks `index` against [0, limit) as the kernels check theirs (no memory
+ * is accessed). In the debug build an index outside the range is recorded,
+ * and the next srftq_check_device on the stream returns
+ * SRFTQ_ERR_DEVICE_CHECK; in the release build nothing is recorded.
+ * Returns SRFTQ_ERR_CUDA if the launch fails, else SRFTQ_OK.
+ */
+int srftq_probe_index_check(int64_t index, int64_t limit, void* stream);
+
 /* Library version as 10000*major + 100*minor + patch. */
 int srftq_version(void);
 

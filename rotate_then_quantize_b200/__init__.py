@@ -14,6 +14,7 @@ from .binding import (  # noqa: F401
     SrftqError,
     calibrate_lambda,
     calibrate_lambda_dense,
+    debug_checks,
     decode_attention,
     dense_operand,
     dequantize,
@@ -34,6 +35,8 @@ from .binding import (  # noqa: F401
     srftq_dequantize_dense,
     srftq_dequantize_rotated,
     srftq_householder_rotation,
+    srftq_debug_checks,
+    srftq_probe_index_check,
     srftq_probe_wait_timeout,
     srftq_quantize,
     srftq_quantize_dense,

@@ -13,11 +13,14 @@ a [S, T, H, d] buffer) is passed through as the slice stride in rows.
 
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 
 PKG_DIR = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(PKG_DIR, "libsrftq.so")
+# the same library built with device-side index checks (SRFTQ_DEBUG_CHECKS)
+LIB_DEBUG_PATH = os.path.join(PKG_DIR, "libsrftq_debug.so")
 
 SRFTQ_OK = 0
 SRFTQ_ERR_INVALID_ARG = -1
@@ -34,7 +37,8 @@ EXPORTED = ("srftq_quantize", "srftq_dequantize", "srftq_calibrate_lambda", "srf
             "srftq_dequantize_rotated", "srftq_unrotate", "srftq_decode_attention",
             "srftq_householder_rotation", "srftq_dense_operand", "srftq_calibrate_lambda_dense",
             "srftq_quantize_dense", "srftq_dequantize_dense", "srftq_status_string",
-            "srftq_check_device", "srftq_probe_wait_timeout", "srftq_version")
+            "srftq_check_device", "srftq_probe_wait_timeout", "srftq_probe_index_check",
+            "srftq_debug_checks", "srftq_version")
 
 
 class SrftqDesc(ctypes.Structure):
@@ -48,17 +52,22 @@ class SrftqError(RuntimeError):
         self.status = status
 
 
-_lib = None
+_libs = {}            # path -> loaded library
+_use_debug = False    # set inside debug_checks()
 
 
-def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
-    """Loads libsrftq.so once; raises if it is missing (no CPU fallback exists)."""
-    global _lib
-    if _lib is not None:
-        return _lib
+def load_library(path: str | None = None) -> ctypes.CDLL:
+    """Loads the in-tree libsrftq.so once (or, inside `debug_checks()`, the
+    in-tree libsrftq_debug.so); raises if it is missing (no CPU fallback
+    exists)."""
+    if path is None:
+        path = LIB_DEBUG_PATH if _use_debug else LIB_PATH
+    if path in _libs:
+        return _libs[path]
     if not os.path.exists(path):
+        flag = " --debug" if path == LIB_DEBUG_PATH else ""
         raise FileNotFoundError(
-            f"{path} not found: build it with `python -m rotate_then_quantize_b200.build`")
+            f"{path} not found: build it with `python -m rotate_then_quantize_b200.build{flag}`")
     lib = ctypes.CDLL(path)
     P, I64, I32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
     D = ctypes.POINTER(SrftqDesc)
@@ -79,12 +88,31 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.srftq_status_string.restype = ctypes.c_char_p
     lib.srftq_check_device.argtypes = [P]
     lib.srftq_probe_wait_timeout.argtypes = [ctypes.c_uint32, P]
+    lib.srftq_probe_index_check.argtypes = [I64, I64, P]
+    lib.srftq_debug_checks.argtypes = []
     lib.srftq_version.argtypes = []
     for name in EXPORTED:
         if name != "srftq_status_string":
             getattr(lib, name).restype = I32
-    _lib = lib
+    _libs[path] = lib
     return lib
+
+
+@contextlib.contextmanager
+def debug_checks():
+    """Within the block every srftq_* call of this module goes to the in-tree
+    debug build (libsrftq_debug.so, `python -m rotate_then_quantize_b200.build
+    --debug`), whose kernels check every global-memory index against the
+    call's extents and record a failure in the device guard word
+    (srftq_check_device) instead of making the access."""
+    global _use_debug
+    load_library(LIB_DEBUG_PATH)
+    prev = _use_debug
+    _use_debug = True
+    try:
+        yield
+    finally:
+        _use_debug = prev
 
 
 def status_string(status: int) -> str:
@@ -399,6 +427,17 @@ def srftq_dequantize_dense(desc: SrftqDesc, codes, scales, operand, lam, xhat,
 def srftq_probe_wait_timeout(polls: int, stream=None) -> int:
     """Launches the device-side timeout probe (see include/srftq.h); returns the status."""
     return int(load_library().srftq_probe_wait_timeout(int(polls), _stream_handle(stream)))
+
+
+def srftq_probe_index_check(index: int, limit: int, stream=None) -> int:
+    """Launches the device-side index-check probe (see include/srftq.h); returns the status."""
+    return int(load_library().srftq_probe_index_check(int(index), int(limit),
+                                                      _stream_handle(stream)))
+
+
+def srftq_debug_checks() -> bool:
+    """Whether the active library was built with the device-side index checks."""
+    return bool(load_library().srftq_debug_checks())
 
 
 def srftq_check_device(stream=None) -> int:

@@ -26,8 +26,14 @@ LIB_DEBUG = os.path.join(PKG, "libsrftq_debug.so")
 
 NVCC = os.environ.get("NVCC", "nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
+# -fno-gnu-unique and -Bsymbolic keep every function-local static (the
+# per-kernel attribute and occupancy caches) private to its library: a
+# process may load libsrftq.so and libsrftq_debug.so side by side, and GCC
+# would otherwise emit those statics as STB_GNU_UNIQUE symbols, which the
+# dynamic linker merges across libraries even when they are loaded locally.
 FLAGS = ["-std=c++17", "-O3", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-O2",
-         "-I", os.path.join(ROOT, "include")]
+         "-Xcompiler", "-fno-gnu-unique", "-I", os.path.join(ROOT, "include")]
+LINK_FLAGS = ["-Xlinker", "-Bsymbolic"]
 
 
 def _sources():
@@ -78,7 +84,7 @@ def build(jobs: int | None = None, force: bool = False, verbose_ptxas: bool = Fa
                 logs.append(log)
     if (force or not os.path.exists(lib)
             or os.path.getmtime(lib) < max(os.path.getmtime(o) for o in objs)):
-        cmd = [NVCC, *ARCH, "-shared", "-o", lib, *objs, "-lcudart"]
+        cmd = [NVCC, *ARCH, "-shared", *LINK_FLAGS, "-o", lib, *objs, "-lcudart"]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"link failed:\n{r.stderr[-8000:]}")

@@ -29,6 +29,12 @@ __global__ void probe_wait_timeout_kernel(unsigned* guard, uint32_t polls) {
   atomicOr(guard, kGuardWaitTimeout);
 }
 
+// The index check of the debug build, on a given index: records kGuardIndex
+// when index is outside [0, limit) (the access it guards is never made).
+__global__ void probe_index_check_kernel(unsigned* guard, int64_t index, int64_t limit) {
+  (void)dbg_ok(index >= 0 && index < limit, guard);
+}
+
 // Reads and clears the guard word in one atomic step, so a bit that another
 // stream's kernel sets meanwhile is either reported now or kept for the next
 // check, never lost.
@@ -505,6 +511,16 @@ int srftq_probe_wait_timeout(uint32_t polls, void* stream) {
   return cudaGetLastError() == cudaSuccess ? SRFTQ_OK : SRFTQ_ERR_CUDA;
 }
 
-int srftq_version(void) { return 100; }
+int srftq_probe_index_check(int64_t index, int64_t limit, void* stream) {
+  unsigned* guard = srftq::Runtime::guard_word();
+  if (!guard) return SRFTQ_ERR_CUDA;
+  srftq::probe_index_check_kernel<<<1, 1, 0, static_cast<cudaStream_t>(stream)>>>(guard, index,
+                                                                                 limit);
+  return cudaGetLastError() == cudaSuccess ? SRFTQ_OK : SRFTQ_ERR_CUDA;
+}
+
+int srftq_debug_checks(void) { return srftq::kDebugChecks ? 1 : 0; }
+
+int srftq_version(void) { return 200; }
 
 }  // extern "C"

@@ -74,6 +74,8 @@ struct AttnArgs {
   const int8_t* v_signs;
   const float* v_lambda;
   float* out;                 // [n_seq][heads * q_per_kv][d] float32
+  int64_t rows;               // rows the caches hold (debug-build index checks)
+  unsigned* guard;
 };
 
 // sigma * code for the 8 codes of one code word (int4: one uint32; int8:
@@ -293,15 +295,16 @@ __global__ void __cluster_dims__(kAttnSplit, 1, 1)
 #pragma unroll
       for (int k = 0; k < PPT; ++k) {
         const int r = lane / PPT + (32 / PPT) * k;
-        if (r < nt) {
-          const int64_t vec = vec_of(t0 + r);
+        const int64_t vec = vec_of(t0 + r);
+        if (r < nt && dbg_ok(vec < a.rows * a.heads, a.guard)) {
           const uint32_t o = uint32_t(r * CB + ((pc ^ L::swz(r)) * 16));
           cp_async<16>(st + L::KC + o, a.k_codes + vec * CB + pc * 16);
           cp_async<16>(st + L::VC + o, a.v_codes + vec * CB + pc * 16);
         }
       }
-      if (lane < nt) {
-        const int64_t vec = vec_of(t0 + lane);
+      const int64_t svec = vec_of(t0 + lane);
+      if (lane < nt && dbg_ok(svec < a.rows * a.heads, a.guard)) {
+        const int64_t vec = svec;
         const uint32_t o = uint32_t(lane * SBS);
         const uint16_t* ks = a.k_scales + vec * NG;
         const uint16_t* vs = a.v_scales + vec * NG;

@@ -37,6 +37,7 @@ struct RotateArgs {
   const int8_t* signs;
   const float* lambda;  // may be null
   float* y;
+  unsigned* guard;      // debug-build index checks
 };
 
 // y = R (s * x) [/ lambda], one thread per vector, grid-stride.
@@ -49,12 +50,16 @@ __global__ void __launch_bounds__(128) rotate_kernel(const RotateArgs a) {
     const int64_t sr = v_id / a.heads;
     const int64_t r = sr % a.n_rows;
     const int64_t s = sr / a.n_rows;
-    const uint16_t* xv = a.x + ((s * a.x_slice_stride_rows + r) * a.heads + h) * D;
+    int64_t vx = (s * a.x_slice_stride_rows + r) * a.heads + h;
+    if (!dbg_ok(vx < vec_limit(a.n_slices, a.x_slice_stride_rows, a.n_rows, a.heads), a.guard))
+      vx = 0;   // debug build: recorded, read vector 0 instead
+    const uint16_t* xv = a.x + vx * D;
     const int64_t tab = (s * a.heads + h) * D;
     uint32_t xw[D / 2], sgw[D / 2];
     load_vector<D>(xv, a.signs + tab, xw, sgw);
     float2 v[D / 2];
     rotate_forward<ROT, D>(xw, sgw, v);
+    if (!dbg_ok(v_id < a.n_slices * a.n_rows * a.heads, a.guard)) continue;
     float* yv = a.y + v_id * D;
     static_for<0, D / 4>([&](auto c_) {
       constexpr int ci = decltype(c_)::value;
@@ -77,6 +82,8 @@ struct CalibArgs {
   const uint16_t* x;
   const int8_t* signs;
   float* lambda_out;
+  int64_t n_slices;     // debug-build index checks
+  unsigned* guard;
 };
 
 constexpr int kCalibRows = 64;     // rows rotated per batch
@@ -111,7 +118,10 @@ __global__ void __cluster_dims__(kCalibCluster, 1, 1) __launch_bounds__(kCalibRo
        base += int64_t(kCalibRows) * kCalibCluster) {
     const int64_t r = base + threadIdx.x;   // one row per thread
     if (r < a.n_cal) {
-      const uint16_t* xv = a.x + ((int64_t(s) * a.x_slice_stride_rows + r) * a.heads + h) * D;
+      int64_t vx = (int64_t(s) * a.x_slice_stride_rows + r) * a.heads + h;
+      if (!dbg_ok(vx < vec_limit(a.n_slices, a.x_slice_stride_rows, a.n_cal, a.heads), a.guard))
+        vx = 0;   // debug build: recorded, read vector 0 instead
+      const uint16_t* xv = a.x + vx * D;
       uint32_t xw[D / 2], sgw[D / 2];
       load_vector<D>(xv, a.signs + tab, xw, sgw);
       float2 v[D / 2];
@@ -148,7 +158,8 @@ __global__ void __cluster_dims__(kCalibCluster, 1, 1) __launch_bounds__(kCalibRo
       if (j < D) {
         double total = 0.0;
         for (int q = 0; q < kCalibCluster; ++q) total += cluster.map_shared_rank(part, q)[j];
-        a.lambda_out[tab + j] = total > 0.0 ? float(sqrt(total / double(a.n_cal))) : 1.0f;
+        if (dbg_ok(tab + j < a.n_slices * a.heads * D, a.guard))
+          a.lambda_out[tab + j] = total > 0.0 ? float(sqrt(total / double(a.n_cal))) : 1.0f;
       }
     }
   }

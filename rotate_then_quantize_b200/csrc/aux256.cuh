@@ -81,11 +81,14 @@ __global__ void __launch_bounds__(128) rotate256_kernel(const RotateArgs a) {
     const int64_t sr = v_id / a.heads;
     const int64_t rr = sr % a.n_rows;
     const int64_t s = sr / a.n_rows;
-    const uint16_t* xv = a.x + ((s * a.x_slice_stride_rows + rr) * a.heads + h) * 256;
+    int64_t vx = (s * a.x_slice_stride_rows + rr) * a.heads + h;
+    if (!dbg_ok(vx < vec_limit(a.n_slices, a.x_slice_stride_rows, a.n_rows, a.heads), a.guard))
+      vx = 0;   // debug build: recorded, read vector 0 instead
+    const uint16_t* xv = a.x + vx * 256;
     const int64_t tab = (s * a.heads + h) * 256;
     float2 v[64];
     rotate256_lane<ROT>(xv, a.signs + tab, p, v);
-    if (valid) {
+    if (valid && dbg_ok(v_id < total, a.guard)) {
       float* yv = a.y + v_id * 256;
       static_for<0, 64>([&](auto j_) {
         constexpr int j = decltype(j_)::value;
@@ -123,7 +126,10 @@ __global__ void __cluster_dims__(kCalibCluster, 1, 1) __launch_bounds__(128)
     const int64_t rr = b + rl;
     const bool valid = rr < a.n_cal;
     const int64_t rc = valid ? rr : 0;
-    const uint16_t* xv = a.x + ((int64_t(s) * a.x_slice_stride_rows + rc) * a.heads + h) * 256;
+    int64_t vx = (int64_t(s) * a.x_slice_stride_rows + rc) * a.heads + h;
+    if (!dbg_ok(vx < vec_limit(a.n_slices, a.x_slice_stride_rows, a.n_cal, a.heads), a.guard))
+      vx = 0;   // debug build: recorded, read vector 0 instead
+    const uint16_t* xv = a.x + vx * 256;
     float2 v[64];
     rotate256_lane<ROT>(xv, a.signs + tab, p, v);
     // two passes of 32 rows each through a 32 x 256 shared tile
@@ -156,8 +162,11 @@ __global__ void __cluster_dims__(kCalibCluster, 1, 1) __launch_bounds__(128)
       t0 += q[threadIdx.x];
       t1 += q[threadIdx.x + 128];
     }
-    a.lambda_out[tab + threadIdx.x] = t0 > 0.0 ? float(sqrt(t0 / double(a.n_cal))) : 1.0f;
-    a.lambda_out[tab + threadIdx.x + 128] = t1 > 0.0 ? float(sqrt(t1 / double(a.n_cal))) : 1.0f;
+    if (dbg_ok(tab + threadIdx.x + 128 < a.n_slices * a.heads * 256, a.guard)) {
+      a.lambda_out[tab + threadIdx.x] = t0 > 0.0 ? float(sqrt(t0 / double(a.n_cal))) : 1.0f;
+      a.lambda_out[tab + threadIdx.x + 128] =
+          t1 > 0.0 ? float(sqrt(t1 / double(a.n_cal))) : 1.0f;
+    }
   }
   cluster.sync();   // the other blocks keep their shared memory until rank 0 is done
 }

@@ -109,6 +109,18 @@ __device__ __forceinline__ uint8_t* smem_base_1024(uint8_t* raw) {
   return raw + ((0u - a) & 1023u);
 }
 
+// Number of vector slots rows 0..N-1 of S slices with a stride of `stride`
+// rows span: the bound of every vector index a call may touch (debug checks).
+__device__ __forceinline__ int64_t vec_limit(int64_t S, int64_t stride, int64_t N, int64_t H) {
+  return ((S - 1) * stride + N) * H;
+}
+
+// The tile a TMA copy addresses lies inside the call's extents (debug checks).
+__device__ __forceinline__ bool tile_in_range(const TileWalk& c, const TileGeom& g) {
+  return c.s >= 0 && c.s < g.n_slices && c.hb >= 0 && c.hb < g.head_blocks && c.rb >= 0 &&
+         c.rb < g.row_blocks;
+}
+
 struct QuantArgs {
   TileGeom g;
   const int8_t* signs;    // [S][H][d]
@@ -513,6 +525,10 @@ __global__ void __launch_bounds__(WPC * 32, MINB)
 
   auto issue = [&](const TileWalk& c, int st) {
     uint8_t* sb = ws + st * Lay::kInBytes;
+    if (!dbg_ok(tile_in_range(c, a.g), a.guard)) {
+      mbar_arrive(&bars[st]);   // debug build: no copy, the phase completes empty
+      return;
+    }
     mbar_arrive_expect_tx(&bars[st], Lay::kStageTx);
 #pragma unroll
     for (int p = 0; p < S::X_PIECES; ++p)
@@ -520,10 +536,12 @@ __global__ void __launch_bounds__(WPC * 32, MINB)
                   c.hb * hpt, c.rb * rpt, c.s);
   };
   auto store_codes = [&](const TileWalk& c) {
+    if (dbg_ok(tile_in_range(c, a.g), a.guard)) {
 #pragma unroll
-    for (int p = 0; p < S::C_PIECES; ++p)
-      tma_store_4d(&tm_codes, ob + p * (S::TR * S::C_SPAN), p * S::C_SPAN, c.hb * hpt,
-                   c.rb * rpt, c.s);
+      for (int p = 0; p < S::C_PIECES; ++p)
+        tma_store_4d(&tm_codes, ob + p * (S::TR * S::C_SPAN), p * S::C_SPAN, c.hb * hpt,
+                     c.rb * rpt, c.s);
+    }
     bulk_commit();
   };
 
@@ -616,9 +634,13 @@ __global__ void __launch_bounds__(WPC * 32, MINB)
     quantize_codes<D, BITS, G>(v, sw, words);
 
     const int row = cur.rb * rpt + rl;
-    const bool valid = row < a.g.n_rows;
     const size_t vec = (static_cast<size_t>(cur.s) * a.out_slice_stride_rows + row) * a.g.heads +
                        cur.hb * hpt + hl;
+    const bool valid =
+        row < a.g.n_rows &&
+        dbg_ok(int64_t(vec) < vec_limit(a.g.n_slices, a.out_slice_stride_rows, a.g.n_rows,
+                                        a.g.heads),
+               a.guard);
 
     // (f) codes: swizzled staging tile, stored by TMA at the next convergence
     // (rows past N are clipped by TMA). The store issued at this tile's start
@@ -733,6 +755,10 @@ __global__ void __launch_bounds__(WPC * 32, MINB)
 
   auto issue = [&](const TileWalk& c, int st) {
     uint8_t* sb = ws + st * Lay::kInBytes;
+    if (!dbg_ok(tile_in_range(c, a.g), a.guard)) {
+      mbar_arrive(&bars[st]);   // debug build: no copy, the phase completes empty
+      return;
+    }
     if constexpr (S::CODES_TMA) {
       mbar_arrive_expect_tx(&bars[st], Lay::kStageTx);
 #pragma unroll
@@ -744,10 +770,12 @@ __global__ void __launch_bounds__(WPC * 32, MINB)
     }
   };
   auto store_xhat = [&](const TileWalk& c) {
+    if (dbg_ok(tile_in_range(c, a.g), a.guard)) {
 #pragma unroll
-    for (int p = 0; p < S::X_PIECES; ++p)
-      tma_store_4d(&tm_xhat, ob + p * (S::TR * S::X_SPAN), p * (S::X_SPAN / 2), c.hb * hpt,
-                   c.rb * rpt, c.s);
+      for (int p = 0; p < S::X_PIECES; ++p)
+        tma_store_4d(&tm_xhat, ob + p * (S::TR * S::X_SPAN), p * (S::X_SPAN / 2), c.hb * hpt,
+                     c.rb * rpt, c.s);
+    }
     bulk_commit();
   };
 
@@ -764,9 +792,12 @@ __global__ void __launch_bounds__(WPC * 32, MINB)
   // the next tile's scales are loaded one tile ahead, into registers
   auto load_scales = [&](const TileWalk& c, uint32_t (&sw)[S::SW]) {
     const int row = c.rb * rpt + rl;
-    if (row < a.g.n_rows) {
-      const size_t vec = (static_cast<size_t>(c.s) * a.in_slice_stride_rows + row) * a.g.heads +
-                         c.hb * hpt + hl;
+    const size_t vec = (static_cast<size_t>(c.s) * a.in_slice_stride_rows + row) * a.g.heads +
+                       c.hb * hpt + hl;
+    if (row < a.g.n_rows &&
+        dbg_ok(int64_t(vec) < vec_limit(a.g.n_slices, a.in_slice_stride_rows, a.g.n_rows,
+                                        a.g.heads),
+               a.guard)) {
       const uint16_t* src = a.scales + vec * S::NG;
       if constexpr (S::NG == 1) {
         sw[0] = src[0];
@@ -802,7 +833,12 @@ __global__ void __launch_bounds__(WPC * 32, MINB)
     const uint32_t parity = (it / NST) & 1;
     const uint8_t* sb = ws + st * Lay::kInBytes;
     const int row = cur.rb * rpt + rl;
-    const bool valid = row < a.g.n_rows;
+    const bool valid =
+        row < a.g.n_rows &&
+        dbg_ok(int64_t((static_cast<size_t>(cur.s) * a.in_slice_stride_rows + row) * a.g.heads +
+                       cur.hb * hpt + hl) <
+                   vec_limit(a.g.n_slices, a.in_slice_stride_rows, a.g.n_rows, a.g.heads),
+               a.guard);
 
     uint32_t sw[S::SW];
     static_for<0, S::SW>([&](auto k_) { sw[decltype(k_)::value] = sw_next[decltype(k_)::value]; });

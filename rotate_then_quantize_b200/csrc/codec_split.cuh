@@ -468,6 +468,10 @@ __global__ void __launch_bounds__(64, MINB)
   __syncthreads();
 
   auto issue = [&](const TileWalk& c) {
+    if (!dbg_ok(tile_in_range(c, a.g), a.guard)) {
+      mbar_arrive(bar);   // debug build: no copy, the phase completes empty
+      return;
+    }
     mbar_arrive_expect_tx(bar, S::X_TILE);
 #pragma unroll
     for (int pc = 0; pc < S::X_PIECES; ++pc)
@@ -475,10 +479,12 @@ __global__ void __launch_bounds__(64, MINB)
                   c.s);
   };
   auto store_codes = [&](const TileWalk& c) {
+    if (dbg_ok(tile_in_range(c, a.g), a.guard)) {
 #pragma unroll
-    for (int pc = 0; pc < S::C_PIECES; ++pc)
-      tma_store_4d(&tm_codes, ob + pc * (S::TR * S::C_SPAN), pc * S::C_SPAN, c.hb * hpt,
-                   c.rb * rpt, c.s);
+      for (int pc = 0; pc < S::C_PIECES; ++pc)
+        tma_store_4d(&tm_codes, ob + pc * (S::TR * S::C_SPAN), pc * S::C_SPAN, c.hb * hpt,
+                     c.rb * rpt, c.s);
+    }
     bulk_commit();
   };
 
@@ -641,10 +647,13 @@ __global__ void __launch_bounds__(64, MINB)
 
     // (f) this role's scales; consecutive global groups go out as words
     const int row = cur.rb * rpt + rl;
-    if (row < a.g.n_rows) {
-      uint16_t* dst = a.scales +
-          ((static_cast<size_t>(cur.s) * a.out_slice_stride_rows + row) * a.g.heads +
-           cur.hb * hpt + hl) * S::NG;
+    const size_t svec = (static_cast<size_t>(cur.s) * a.out_slice_stride_rows + row) *
+                            a.g.heads + cur.hb * hpt + hl;
+    if (row < a.g.n_rows &&
+        dbg_ok(int64_t(svec) < vec_limit(a.g.n_slices, a.out_slice_stride_rows, a.g.n_rows,
+                                         a.g.heads),
+               a.guard)) {
+      uint16_t* dst = a.scales + svec * S::NG;
       if constexpr (Grp::kLocal) {
         constexpr bool kWords = ROT == kSRHT || S::kScaleWords;
         static_for<0, S::NGR / 2>([&](auto k_) {
@@ -754,6 +763,10 @@ __global__ void __launch_bounds__(64, MINB)
   __syncthreads();
 
   auto issue = [&](const TileWalk& c) {
+    if (!dbg_ok(tile_in_range(c, a.g), a.guard)) {
+      mbar_arrive(bar);   // debug build: no copy, the phase completes empty
+      return;
+    }
     mbar_arrive_expect_tx(bar, S::C_TILE);
 #pragma unroll
     for (int pc = 0; pc < S::C_PIECES; ++pc)
@@ -761,10 +774,12 @@ __global__ void __launch_bounds__(64, MINB)
                   c.rb * rpt, c.s);
   };
   auto store_xhat = [&](const TileWalk& c) {
+    if (dbg_ok(tile_in_range(c, a.g), a.guard)) {
 #pragma unroll
-    for (int pc = 0; pc < S::X_PIECES; ++pc)
-      tma_store_4d(&tm_xhat, ob + pc * (S::TR * S::X_SPAN), pc * 64, c.hb * hpt, c.rb * rpt,
-                   c.s);
+      for (int pc = 0; pc < S::X_PIECES; ++pc)
+        tma_store_4d(&tm_xhat, ob + pc * (S::TR * S::X_SPAN), pc * 64, c.hb * hpt, c.rb * rpt,
+                     c.s);
+    }
     bulk_commit();
   };
 
@@ -784,10 +799,13 @@ __global__ void __launch_bounds__(64, MINB)
   constexpr bool kWords = ROT == kSRHT || S::kScaleWords;
   auto load_scales = [&](const TileWalk& c, uint32_t (&rs)[NSW], uint32_t& ex) {
     const int row = c.rb * rpt + rl;
-    if (row < a.g.n_rows) {
-      const uint16_t* src = a.scales +
-          ((static_cast<size_t>(c.s) * a.in_slice_stride_rows + row) * a.g.heads + c.hb * hpt +
-           hl) * S::NG;
+    const size_t svec = (static_cast<size_t>(c.s) * a.in_slice_stride_rows + row) * a.g.heads +
+                        c.hb * hpt + hl;
+    if (row < a.g.n_rows &&
+        dbg_ok(int64_t(svec) < vec_limit(a.g.n_slices, a.in_slice_stride_rows, a.g.n_rows,
+                                         a.g.heads),
+               a.guard)) {
+      const uint16_t* src = a.scales + svec * S::NG;
       if constexpr (Grp::kLocal) {
         static_for<0, NSW>([&](auto k_) {
           constexpr int k = decltype(k_)::value;

@@ -31,6 +31,8 @@ struct HouseholderArgs {
   const float* reflectors;   // [S][H][k][d]
   const int8_t* signs;       // [S][H][d]
   float* rot;                // [S][H][d][d]
+  int64_t n_slices;          // debug-build index checks
+  unsigned* guard;
 };
 
 // Entry (n, j) of the unsigned base rotation, in double: SRFT rows
@@ -63,6 +65,7 @@ __global__ void __launch_bounds__(D) householder_kernel(const HouseholderArgs a)
   __shared__ double v[D];
   const int sh = blockIdx.x;                 // s * H + h
   const int j = threadIdx.x;
+  if (!dbg_ok(sh < a.n_slices * a.heads, a.guard)) return;   // block-uniform
   float* R = a.rot + size_t(sh) * D * D;
   const double sj = a.signs[size_t(sh) * D + j] < 0 ? -1.0 : 1.0;
   for (int n = 0; n < D; ++n) R[size_t(n) * D + j] = float(base_entry<D, ROT>(n, j) * sj);
@@ -177,6 +180,7 @@ struct DenseArgs {
   uint16_t* xhat;             // dequantise output [S][T_out][H][d]
   const uint16_t* operand;    // [S][H][2][d][d]
   const float* lambda;        // [S][H][d]
+  unsigned* guard;            // debug-build index checks
 };
 
 // One block per (slice, head, 64-row tile).
@@ -203,8 +207,10 @@ __global__ void __launch_bounds__(kDenseThreads) dense_gemm_kernel(const DenseAr
     const int v = idx / (D / 8), c8 = idx % (D / 8);
     const int64_t r = r0 + v;
     float f[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-    if (r < a.n_rows) {
-      const size_t vec = size_t((s * a.in_stride_rows + r) * a.heads + h);
+    const size_t vec = size_t((s * a.in_stride_rows + r) * a.heads + h);
+    if (r < a.n_rows &&
+        dbg_ok(int64_t(vec) < vec_limit(a.n_slices, a.in_stride_rows, a.n_rows, a.heads),
+               a.guard)) {
       if constexpr (QUANT) {
         const uint4 w = *reinterpret_cast<const uint4*>(a.x + vec * D + 8 * c8);
         const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
@@ -246,6 +252,10 @@ __global__ void __launch_bounds__(kDenseThreads) dense_gemm_kernel(const DenseAr
     for (int i = 0; i < T::TV; ++i) {
       const int64_t r = r0 + tv * T::TV + i;
       if (r >= a.n_rows) continue;
+      if (!dbg_ok((s * a.out_stride_rows + r) * a.heads + h <
+                      vec_limit(a.n_slices, a.out_stride_rows, a.n_rows, a.heads),
+                  a.guard))
+        continue;
       uint32_t w[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
@@ -298,6 +308,9 @@ __global__ void __launch_bounds__(kDenseThreads) dense_gemm_kernel(const DenseAr
         qb[c] = uint32_t(int32_t(q));
       }
       const size_t vec = size_t((s * a.out_stride_rows + r) * a.heads + h);
+      if (!dbg_ok(int64_t(vec) < vec_limit(a.n_slices, a.out_stride_rows, a.n_rows, a.heads),
+                  a.guard))
+        continue;   // warp-uniform: every lane holds the same vector
       uint8_t* cdst = a.codes + vec * CB;
       if constexpr (BITS == 4) {
         // coordinates 2m (low nibble) and 2m + 1 (high nibble) share byte m
@@ -344,6 +357,8 @@ struct DenseCalibArgs {
   const uint16_t* x;
   const uint16_t* operand;
   float* lambda_out;
+  int64_t n_slices;           // debug-build index checks
+  unsigned* guard;
 };
 
 template <int D>
@@ -366,8 +381,10 @@ __global__ void __launch_bounds__(kDenseThreads) dense_calibrate_kernel(const De
       const int v = idx / (D / 8), c8 = idx % (D / 8);
       const int64_t r = r0 + v;
       float f[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-      if (r < a.n_cal) {
-        const size_t vec = size_t((s * a.x_stride_rows + r) * a.heads + h);
+      const size_t vec = size_t((s * a.x_stride_rows + r) * a.heads + h);
+      if (r < a.n_cal &&
+          dbg_ok(int64_t(vec) < vec_limit(a.n_slices, a.x_stride_rows, a.n_cal, a.heads),
+                 a.guard)) {
         const uint4 w = *reinterpret_cast<const uint4*>(a.x + vec * D + 8 * c8);
         const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
@@ -397,7 +414,8 @@ __global__ void __launch_bounds__(kDenseThreads) dense_calibrate_kernel(const De
   for (int n = tid; n < D; n += kDenseThreads) {
     double t = 0.0;
     for (int g = 0; g < T::TVG; ++g) t += red[g * D + n];
-    a.lambda_out[size_t(sh) * D + n] = t == 0.0 ? 1.0f : float(sqrt(t / double(a.n_cal)));
+    if (dbg_ok(sh < a.n_slices * a.heads, a.guard))
+      a.lambda_out[size_t(sh) * D + n] = t == 0.0 ? 1.0f : float(sqrt(t / double(a.n_cal)));
   }
 }
 

@@ -198,6 +198,10 @@ __global__ void __launch_bounds__(DenseMma<D, EPI>::kThreads, 1)
         const int64_t sh = sh_of(i);
         const int r0 = int(rb_of(i) * 128);
         const int s = int(sh / a.heads), h = int(sh % a.heads);
+        if (!dbg_ok(s < a.n_slices && r0 < a.n_rows, a.guard)) {
+          mbar_arrive(&full[st]);   // debug build: no copy, the phase completes empty
+          continue;
+        }
         mbar_arrive_expect_tx(&full[st], L::kABytes);
 #pragma unroll
         for (int p = 0; p < L::kPieces; ++p)
@@ -337,9 +341,12 @@ __global__ void __launch_bounds__(DenseMma<D, EPI>::kThreads, 1)
         break;
       tc_fence_after();
       const int64_t row = rb_of(i) * 128 + 32 * q + lane;
-      const bool valid = row < a.n_rows;
       const int64_t s = sh / a.heads, h = sh % a.heads;
       const size_t vec = size_t((s * a.out_stride_rows + row) * a.heads + h);
+      const bool valid =
+          row < a.n_rows &&
+          dbg_ok(int64_t(vec) < vec_limit(a.n_slices, a.out_stride_rows, a.n_rows, a.heads),
+                 a.guard);
       const uint32_t taddr = tmem_base + (uint32_t(32 * q) << 16) + uint32_t(acc) * uint32_t(D);
       if constexpr (G <= 64) {
         // every group lies inside one 64-column chunk

@@ -8,10 +8,13 @@ int launch_decode_attention_d128(const AttnCall& c) {
   if (c.n_seq == 0) return SRFTQ_OK;
   const int64_t blocks = c.n_seq * c.heads * kAttnSplit;   // one cluster per (sequence, head)
   if (blocks > INT_MAX) return SRFTQ_ERR_UNSUPPORTED;
+  unsigned* guard = Runtime::guard_word();
+  if (!guard) return SRFTQ_ERR_CUDA;
+  const int64_t rows = (c.n_ctx - 1) * c.tok_stride_rows + (c.n_seq - 1) * c.seq_stride_rows + 1;
   AttnArgs a{c.n_seq,   c.n_ctx,    c.tok_stride_rows, c.seq_stride_rows, c.heads,
              c.q_per_kv, c.scale,   c.q,               c.k_codes,         c.k_scales,
              c.k_signs, c.k_lambda, c.v_codes,         c.v_scales,        c.v_signs,
-             c.v_lambda, c.out};
+             c.v_lambda, c.out,     rows,              guard};
   int rc = SRFTQ_ERR_UNSUPPORTED;
   static_for<0, 2>([&](auto b_) {
     constexpr int BITS = decltype(b_)::value == 0 ? 4 : 8;

@@ -25,7 +25,10 @@ template <>
 int launch_rotate<256>(const RotateCall& c) {
   const int64_t total = c.n_slices * c.n_rows * c.heads;
   if (total == 0) return SRFTQ_OK;
-  RotateArgs a{c.n_slices, c.n_rows, c.x_slice_stride_rows, c.heads, c.x, c.signs, c.lambda, c.y};
+  unsigned* guard = Runtime::guard_word();
+  if (!guard) return SRFTQ_ERR_CUDA;
+  RotateArgs a{c.n_slices, c.n_rows, c.x_slice_stride_rows, c.heads, c.x, c.signs, c.lambda, c.y,
+               guard};
   const int64_t want = (2 * total + 127) / 128;
   const int64_t cap = int64_t(Runtime::num_sms()) * 16;
   const int grid = int(want < cap ? want : cap);
@@ -41,7 +44,10 @@ int launch_calibrate<256>(const CalibCall& c) {
   const int64_t blocks = c.n_slices * c.heads * kCalibCluster;   // one cluster per (slice, head)
   if (blocks == 0) return SRFTQ_OK;
   if (blocks > INT_MAX) return SRFTQ_ERR_UNSUPPORTED;
-  CalibArgs a{c.n_cal, c.x_slice_stride_rows, c.heads, c.x, c.signs, c.lambda_out};
+  unsigned* guard = Runtime::guard_word();
+  if (!guard) return SRFTQ_ERR_CUDA;
+  CalibArgs a{c.n_cal, c.x_slice_stride_rows, c.heads, c.x, c.signs, c.lambda_out, c.n_slices,
+              guard};
   if (c.rotation == kSRFT)
     calibrate256_kernel<kSRFT><<<int(blocks), 128, 0, c.stream>>>(a);
   else
@@ -53,8 +59,10 @@ template <>
 int launch_unrotate<256>(const UnrotateCall& c) {
   const int64_t total = c.n_slices * c.n_rows * c.heads;
   if (total == 0) return SRFTQ_OK;
+  unsigned* guard = Runtime::guard_word();
+  if (!guard) return SRFTQ_ERR_CUDA;
   UnrotateArgs a{c.n_slices, c.n_rows, c.y_slice_stride_rows, c.x_slice_stride_rows, c.heads,
-                 c.y, c.signs, c.x};
+                 c.y, c.signs, c.x, guard};
   const int64_t want = (2 * total + 127) / 128;
   const int64_t cap = int64_t(Runtime::num_sms()) * 16;
   const int grid = int(want < cap ? want : cap);

@@ -26,7 +26,9 @@ int launch_householder(const HouseholderCall& c) {
   if (c.n_slices == 0) return SRFTQ_OK;
   const int64_t blocks = c.n_slices * c.heads;
   if (blocks > INT_MAX) return SRFTQ_ERR_UNSUPPORTED;
-  HouseholderArgs a{c.heads, c.n_reflectors, c.reflectors, c.signs, c.rot};
+  unsigned* guard = Runtime::guard_word();
+  if (!guard) return SRFTQ_ERR_CUDA;
+  HouseholderArgs a{c.heads, c.n_reflectors, c.reflectors, c.signs, c.rot, c.n_slices, guard};
   return by_dense_d(c.d, [&](auto d_) {
     constexpr int D = decltype(d_)::value;
     if (c.rotation == kSRFT)
@@ -54,9 +56,11 @@ int launch_dense_codec(const DenseCall& c) {
   const int64_t tiles = (c.n_rows + kDenseRows - 1) / kDenseRows;
   const int64_t blocks = c.n_slices * c.heads * tiles;
   if (blocks > INT_MAX) return SRFTQ_ERR_UNSUPPORTED;
+  unsigned* guard = Runtime::guard_word();
+  if (!guard) return SRFTQ_ERR_CUDA;
   DenseArgs a{c.n_slices, c.n_rows, c.in_stride_rows, c.out_stride_rows, c.heads, tiles,
               c.x,        c.codes_in, c.scales_in,  c.codes,           c.scales, c.xhat,
-              c.operand,  c.lambda};
+              c.operand,  c.lambda,   guard};
   return by_dense_d(c.d, [&](auto d_) {
     constexpr int D = decltype(d_)::value;
     int rc = SRFTQ_ERR_UNSUPPORTED;
@@ -154,7 +158,10 @@ int launch_calibrate_dense(const DenseCalibCall& c) {
   const int64_t blocks = c.n_slices * c.heads;
   if (blocks == 0) return SRFTQ_OK;
   if (blocks > INT_MAX) return SRFTQ_ERR_UNSUPPORTED;
-  DenseCalibArgs a{c.n_cal, c.x_stride_rows, c.heads, c.x, c.operand, c.lambda_out};
+  unsigned* guard = Runtime::guard_word();
+  if (!guard) return SRFTQ_ERR_CUDA;
+  DenseCalibArgs a{c.n_cal, c.x_stride_rows, c.heads, c.x, c.operand, c.lambda_out, c.n_slices,
+                   guard};
   return by_dense_d(c.d, [&](auto d_) {
     constexpr int D = decltype(d_)::value;
     constexpr auto K = dense_calibrate_kernel<D>;

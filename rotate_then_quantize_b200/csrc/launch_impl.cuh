@@ -248,7 +248,10 @@ template <int D>
 int launch_rotate(const RotateCall& c) {
   const int64_t total = c.n_slices * c.n_rows * c.heads;
   if (total == 0) return SRFTQ_OK;
-  RotateArgs a{c.n_slices, c.n_rows, c.x_slice_stride_rows, c.heads, c.x, c.signs, c.lambda, c.y};
+  unsigned* guard = Runtime::guard_word();
+  if (!guard) return SRFTQ_ERR_CUDA;
+  RotateArgs a{c.n_slices, c.n_rows, c.x_slice_stride_rows, c.heads, c.x, c.signs, c.lambda, c.y,
+               guard};
   const int64_t want = (total + 127) / 128;
   const int64_t cap = int64_t(Runtime::num_sms()) * 16;
   const int grid = int(want < cap ? want : cap);
@@ -264,7 +267,10 @@ int launch_calibrate(const CalibCall& c) {
   const int64_t blocks = c.n_slices * c.heads * kCalibCluster;   // one cluster per (slice, head)
   if (blocks == 0) return SRFTQ_OK;
   if (blocks > INT_MAX) return SRFTQ_ERR_UNSUPPORTED;
-  CalibArgs a{c.n_cal, c.x_slice_stride_rows, c.heads, c.x, c.signs, c.lambda_out};
+  unsigned* guard = Runtime::guard_word();
+  if (!guard) return SRFTQ_ERR_CUDA;
+  CalibArgs a{c.n_cal, c.x_slice_stride_rows, c.heads, c.x, c.signs, c.lambda_out, c.n_slices,
+              guard};
   if (c.rotation == kSRFT)
     calibrate_kernel<D, kSRFT><<<int(blocks), kCalibRows, 0, c.stream>>>(a);
   else
@@ -277,8 +283,10 @@ int launch_dequantize_rotated(const RotDequantCall& c) {
   const int64_t per_slice = c.n_rows * c.heads * (D / 8);
   if (per_slice == 0 || c.n_slices == 0) return SRFTQ_OK;
   if (per_slice >= (int64_t(1) << 32)) return SRFTQ_ERR_UNSUPPORTED;   // 32-bit in-slice index
+  unsigned* guard = Runtime::guard_word();
+  if (!guard) return SRFTQ_ERR_CUDA;
   RotDequantArgs a{c.n_slices, c.n_rows, c.in_slice_stride_rows, c.out_slice_stride_rows,
-                   c.heads, c.codes, c.scales, c.lambda, c.out};
+                   c.heads, c.codes, c.scales, c.lambda, c.out, guard};
   // y walks the slices; x covers a slice, about 8 blocks of 256 per SM in all
   const int64_t gy = c.n_slices < 65535 ? c.n_slices : 65535;
   const int64_t cap_x = (int64_t(Runtime::num_sms()) * 8 + gy - 1) / gy;
@@ -302,8 +310,10 @@ template <int D>
 int launch_unrotate(const UnrotateCall& c) {
   const int64_t total = c.n_slices * c.n_rows * c.heads;
   if (total == 0) return SRFTQ_OK;
+  unsigned* guard = Runtime::guard_word();
+  if (!guard) return SRFTQ_ERR_CUDA;
   UnrotateArgs a{c.n_slices, c.n_rows, c.y_slice_stride_rows, c.x_slice_stride_rows, c.heads,
-                 c.y, c.signs, c.x};
+                 c.y, c.signs, c.x, guard};
   const int64_t want = (total + 127) / 128;
   const int64_t cap = int64_t(Runtime::num_sms()) * 16;
   const int grid = int(want < cap ? want : cap);

@@ -8,8 +8,29 @@
 
 namespace srftq {
 
-// Device guard word: bit 0 = a bounded mbarrier wait gave up.
+// Device guard word: bit 0 = a bounded mbarrier wait gave up; bit 1 = an
+// index check of the debug build (SRFTQ_DEBUG_CHECKS) failed.
 constexpr unsigned kGuardWaitTimeout = 1u;
+constexpr unsigned kGuardIndex = 2u;
+
+#ifdef SRFTQ_DEBUG_CHECKS
+constexpr bool kDebugChecks = true;
+#else
+constexpr bool kDebugChecks = false;
+#endif
+
+// Index check of the debug build: returns whether an access may go ahead.
+// In the debug build a failed check records kGuardIndex in the guard word
+// (the access is then skipped by the caller); nothing traps. In the release
+// build it is the constant true and compiles away.
+__device__ __forceinline__ bool dbg_ok(bool ok, unsigned* guard) {
+  if constexpr (kDebugChecks) {
+    if (!ok) atomicOr(guard, kGuardIndex);
+    return ok;
+  } else {
+    return true;
+  }
+}
 
 // try_wait polls suspend the thread for a hardware-defined slice (well under
 // a microsecond each); 1 << 22 of them bound a wait to a few seconds at most.

@@ -28,6 +28,7 @@ struct RotDequantArgs {
   const uint16_t* scales;   // [S][T_in][H][d / G] fp16
   const float* lambda;      // [S][H][d]
   uint16_t* out;            // [S][T_out][H][d] fp16
+  unsigned* guard;          // debug-build index checks
 };
 
 // One thread per 8 coordinates (one 16-byte output chunk) of a slice; the
@@ -59,7 +60,9 @@ __global__ void __launch_bounds__(256) dequantize_rotated_kernel(const RotDequan
         const uint32_t c = base + 256u * u;
         if (c < per_slice) {
           const uint32_t k = c % CPV, vh = c / CPV;   // chunk, (row, head) of the slice
-          const int64_t vin = in_base + vh;
+          int64_t vin = in_base + vh;
+          if (!dbg_ok(vin < vec_limit(a.n_slices, a.in_slice_stride_rows, a.n_rows, H), a.guard))
+            vin = 0;   // debug build: recorded, read vector 0 instead
           const int j0 = 8 * int(k);
           w[u] = *reinterpret_cast<const CodeT*>(a.codes + vin * (D * BITS / 8) + j0 * BITS / 8);
           sw[u] = a.scales[vin * (D / G) + j0 / G];
@@ -104,8 +107,9 @@ __global__ void __launch_bounds__(256) dequantize_rotated_kernel(const RotDequan
         for (int e = 0; e < 4; ++e)
           o[e] = pack_f16x2(q[2 * e] * lv[2 * e], q[2 * e + 1] * lv[2 * e + 1]);
         const int64_t vout = out_base + c / CPV;
-        *reinterpret_cast<uint4*>(a.out + vout * D + 8 * (c % CPV)) =
-            make_uint4(o[0], o[1], o[2], o[3]);
+        if (dbg_ok(vout < vec_limit(a.n_slices, a.out_slice_stride_rows, a.n_rows, H), a.guard))
+          *reinterpret_cast<uint4*>(a.out + vout * D + 8 * (c % CPV)) =
+              make_uint4(o[0], o[1], o[2], o[3]);
       }
     }
   }
@@ -117,6 +121,7 @@ struct UnrotateArgs {
   const float* y;         // [S][T_y][H][d] float32, rotated-domain vectors
   const int8_t* signs;    // [S][H][d]
   float* x;               // [S][T_x][H][d] float32
+  unsigned* guard;        // debug-build index checks
 };
 
 // x = s * R^T y for d <= 128, one thread per vector.
@@ -129,7 +134,10 @@ __global__ void __launch_bounds__(128) unrotate_kernel(const UnrotateArgs a) {
     const int64_t sr = v_id / a.heads;
     const int64_t r = sr % a.n_rows;
     const int64_t s = sr / a.n_rows;
-    const float* yv = a.y + ((s * a.y_slice_stride_rows + r) * a.heads + h) * D;
+    int64_t vy = (s * a.y_slice_stride_rows + r) * a.heads + h;
+    if (!dbg_ok(vy < vec_limit(a.n_slices, a.y_slice_stride_rows, a.n_rows, a.heads), a.guard))
+      vy = 0;   // debug build: recorded, read vector 0 instead
+    const float* yv = a.y + vy * D;
     const int8_t* sg = a.signs + (s * a.heads + h) * D;
     float2 v[D / 2];
     // inverse input: coordinate gain times y (transform.cuh, rotate_inverse)
@@ -141,7 +149,10 @@ __global__ void __launch_bounds__(128) unrotate_kernel(const UnrotateArgs a) {
           make_float2(y4.z * gain_f<ROT, D>(4 * ci + 2), y4.w * gain_f<ROT, D>(4 * ci + 3));
     });
     rotate_inverse<ROT, D>(v);
-    float* xv = a.x + ((s * a.x_slice_stride_rows + r) * a.heads + h) * D;
+    const int64_t vxo = (s * a.x_slice_stride_rows + r) * a.heads + h;
+    if (!dbg_ok(vxo < vec_limit(a.n_slices, a.x_slice_stride_rows, a.n_rows, a.heads), a.guard))
+      continue;
+    float* xv = a.x + vxo * D;
     static_for<0, D / 4>([&](auto c_) {
       constexpr int ci = decltype(c_)::value;
       const char4 s4 = reinterpret_cast<const char4*>(sg)[ci];
@@ -170,7 +181,10 @@ __global__ void __launch_bounds__(128) unrotate256_kernel(const UnrotateArgs a) 
     const int64_t sr = v_id / a.heads;
     const int64_t r = sr % a.n_rows;
     const int64_t s = sr / a.n_rows;
-    const float* yv = a.y + ((s * a.y_slice_stride_rows + r) * a.heads + h) * 256;
+    int64_t vy = (s * a.y_slice_stride_rows + r) * a.heads + h;
+    if (!dbg_ok(vy < vec_limit(a.n_slices, a.y_slice_stride_rows, a.n_rows, a.heads), a.guard))
+      vy = 0;   // debug build: recorded, read vector 0 instead
+    const float* yv = a.y + vy * 256;
     const int8_t* sg = a.signs + (s * a.heads + h) * 256;
     float2 v[64];
     static_for<0, 64>([&](auto j_) {
@@ -180,9 +194,13 @@ __global__ void __launch_bounds__(128) unrotate256_kernel(const UnrotateArgs a) 
       const float2 y2 = reinterpret_cast<const float2*>(yv)[pair];
       v[j] = make_float2(y2.x * g, y2.y * g);
     });
-    float* xv = a.x + ((s * a.x_slice_stride_rows + r) * a.heads + h) * 256;
+    const int64_t vxo = (s * a.x_slice_stride_rows + r) * a.heads + h;
+    const bool out_ok = valid && dbg_ok(vxo < vec_limit(a.n_slices, a.x_slice_stride_rows,
+                                                        a.n_rows, a.heads),
+                                        a.guard);
+    float* xv = a.x + vxo * 256;
     auto put = [&](int n, float val) {   // element n, sign applied
-      if (valid) xv[n] = sg[n] < 0 ? -val : val;
+      if (out_ok) xv[n] = sg[n] < 0 ? -val : val;
     };
     if constexpr (ROT == kSRFT) {
       float2 us[64];

@@ -267,3 +267,32 @@ def test_dense_calls_validate_before_launching(lib):
     assert Cal(D, 1, 9, xh, 8, y, lam, None) == b.SRFTQ_ERR_INVALID_ARG
     assert Cal(D, 1, 4, xh, 8, y, xh, None) == b.SRFTQ_ERR_INVALID_ARG      # lambda over x
     assert Cal(D, 0, 4, xh, 8, y, lam, None) == b.SRFTQ_OK
+
+
+def test_debug_library_exports_the_boundary_and_reports_its_checks(lib):
+    """The index-checking build (libsrftq_debug.so) exports every declared
+    symbol too; srftq_debug_checks tells the two builds apart without a GPU."""
+    if not os.path.exists(b.LIB_DEBUG_PATH):
+        pytest.fail("libsrftq_debug.so is not built; run python -m rotate_then_quantize_b200.build "
+                    "--debug")
+    out = subprocess.run(["nm", "-D", "--defined-only", b.LIB_DEBUG_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (srftq_\w+)", out))
+    for name in _declared():
+        assert name in exported, name
+    assert rq.load_library(b.LIB_DEBUG_PATH).srftq_debug_checks() == 1
+    assert lib.srftq_debug_checks() == 0
+
+
+def test_no_symbol_is_merged_across_libraries(lib):
+    """libsrftq.so and libsrftq_debug.so may share a process. A symbol of
+    type STB_GNU_UNIQUE (nm: "u"), as GCC emits for the local statics of
+    template functions, would be merged between them by the dynamic linker
+    even when both are loaded locally, and one library's kernel-attribute
+    cache would then stand for the other's kernels."""
+    for path in (b.LIB_PATH, b.LIB_DEBUG_PATH):
+        if not os.path.exists(path):
+            continue
+        out = subprocess.run(["nm", "-D", path], capture_output=True, text=True, check=True).stdout
+        unique = [ln for ln in out.splitlines() if " u " in ln]
+        assert not unique, (path, unique[:5])
