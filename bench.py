@@ -100,6 +100,13 @@ KERNEL_SOURCES = {
     "dequantize_split_kernel": ("codec_split.cuh", "codec.cuh", "transform.cuh", "common.cuh",
                                 "ptx.cuh", "launch.cuh", "launch_impl.cuh", "launch_split.cuh",
                                 "launch_d256.cu"),
+    "quantize_dense_mma_kernel": ("dense_mma.cuh", "tc.cuh", "codec.cuh", "transform.cuh",
+                                  "common.cuh", "ptx.cuh", "launch.cuh", "launch_impl.cuh",
+                                  "launch_dense.cu", "dense.cuh", "dense_mma_dequant.cuh"),
+    "dequantize_dense_mma_kernel": ("dense_mma_dequant.cuh", "tc.cuh", "codec.cuh",
+                                    "transform.cuh", "common.cuh", "ptx.cuh", "launch.cuh",
+                                    "launch_impl.cuh", "launch_dense.cu", "dense.cuh",
+                                    "dense_mma.cuh"),
 }
 
 
@@ -108,7 +115,7 @@ def codec_kernel(kind: str, d: int, dense: bool = False) -> str:
     head dimension: d = 256 runs on the two-warp kernels; a dense rotation
     on the dense kernels."""
     if dense:
-        return "quantize_dense_mma_kernel" if kind == "quantize" else "dense_gemm_kernel"
+        return f"{kind}_dense_mma_kernel"
     return f"{kind}{'_split' if d == 256 else ''}_kernel"
 
 
@@ -127,40 +134,46 @@ def codec_calls(rq, w, desc, signs, seed, dev):
                 rq.srftq_dequantize_dense)
 
 
-def fp32_alu_peak_tflops() -> float:
-    """FP32 FMA peak of the CUDA cores: 148 SMs x 128 lanes x 2 flops x the
-    measured maximum SM clock (MEASURED_PEAKS.json sm_max_mhz, else 1965 MHz)."""
-    mhz = 1965.0
+def dense_flops_per_vector(kind: str, d: int) -> float:
+    """Tensor-core flops per vector of the dense-rotation kernels: the
+    quantiser computes R x as two fp16 products (x exact, R = hi + lo); the
+    dequantiser computes R^T a as three (a = a_hi + a_lo: a_hi hi, a_lo hi,
+    a_hi lo)."""
+    return (4.0 if kind == "quantize" else 6.0) * d * d
+
+
+def read_tensor_peak():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
-            mhz = float(json.load(f).get("sm_max_mhz", mhz))
+            return (float(json.load(f)["bf16_tflops"]),
+                    "measured (MEASURED_PEAKS.json bf16_tflops; fp16 runs at the same rate)")
     except Exception:
-        pass
-    return 148 * 128 * 2 * mhz * 1e6 / 1e12
+        return 1590.0, "fallback 1.59 PFLOP/s"
 
 
 def dense_roofline(w, kind, ms, kname):
-    """Roofline of a dense-rotation kernel. The quantiser runs R x on the
-    tensor cores as two fp16 products (the operand's hi and lo halves):
-    2 x 2 d^2 flops per vector against the measured dense fp16/bf16 peak.
-    The dequantiser runs R^T y on the CUDA cores: 2 d^2 flops per vector
-    against the float32 FMA peak."""
-    if kind == "quantize":
-        flops = 4.0 * w.d * w.d * w.vectors
-        peak, src = None, "measured (MEASURED_PEAKS.json bf16_tflops; fp16 runs at the same rate)"
-        try:
-            with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
-                peak = float(json.load(f)["bf16_tflops"])
-        except Exception:
-            peak, src = 1590.0, "fallback 1.59 PFLOP/s"
-        bound = "tensor"
-    else:
-        flops = 2.0 * w.d * w.d * w.vectors
-        peak, src, bound = fp32_alu_peak_tflops(), "148 SMs x 128 FP32 lanes x 2 flops x max SM clock", "alu"
-    achieved = flops / (ms / 1e3) / 1e12
-    return {"bound": bound, "kernel": kname, "launch": kind, "achieved": achieved,
-            "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak, "peak_source": src,
-            "algorithmic_flops_per_launch": flops, "traffic": None}
+    """Roofline of a dense-rotation kernel: whichever of the tensor-core time
+    (flops / measured dense fp16 peak) and the HBM time (algorithmic bytes /
+    measured copy bandwidth) is longer bounds it; the other is reported
+    beside it."""
+    flops = dense_flops_per_vector(kind, w.d) * w.vectors
+    nbytes = w.vectors * w.bytes_per_vector()
+    tpeak, tsrc = read_tensor_peak()
+    hpeak, hsrc = read_peak()
+    t_tc, t_hbm = flops / (tpeak * 1e12), nbytes / (hpeak * 1e9)
+    tc = {"bound": "tensor", "achieved": flops / (ms / 1e3) / 1e12, "peak": tpeak,
+          "unit": "TFLOP/s", "peak_source": tsrc, "algorithmic_flops_per_launch": flops}
+    hb = {"bound": "hbm", "achieved": nbytes / (ms / 1e3) / 1e9, "peak": hpeak, "unit": "GB/s",
+          "peak_source": f"{hsrc} (MEASURED_PEAKS.json hbm_gbs)" if hsrc == "measured"
+          else "fallback 6.65 TB/s", "algorithmic_bytes_per_launch": nbytes}
+    for r in (tc, hb):
+        r["frac"] = r["achieved"] / r["peak"]
+    main, other = (tc, hb) if t_tc >= t_hbm else (hb, tc)
+    out = {"bound": main["bound"], "kernel": kname, "launch": kind}
+    out.update({k: v for k, v in main.items() if k != "bound"})
+    out["traffic"] = read_traffic(kname, w.name)
+    out["other_bound"] = other
+    return out
 
 
 def csrc_hash(kernel: str) -> str:
@@ -641,11 +654,10 @@ def other_configs(rq, dev, iters=50):
                                             iters)
     hh = kv_synth.WORKLOADS["householder_d256"]
     out["householder_d256"] = _codec_figures(rq, hh, 0, dev, iters)
-    q_flops = 2.0 * hh.d * hh.d * hh.vectors
-    for kind in ("quantize", "dequantize"):
-        out["householder_d256"][f"{kind}_TFLOPs"] = q_flops / out["householder_d256"][
-            f"{kind}_ms"] / 1e9
-    out["householder_d256"]["flops_per_launch"] = q_flops
+    flops = {k: dense_flops_per_vector(k, hh.d) * hh.vectors for k in ("quantize", "dequantize")}
+    for kind, f in flops.items():
+        out["householder_d256"][f"{kind}_TFLOPs"] = f / out["householder_d256"][f"{kind}_ms"] / 1e9
+    out["householder_d256"]["flops_per_launch"] = flops
     out["decode_stream_d128_fused_attention"] = _attention_figures(rq, dev, iters)
     rep = parity_report()
     if rep is not None:

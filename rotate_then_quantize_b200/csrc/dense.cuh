@@ -6,11 +6,12 @@
 //                          matrix, one block per (slice, head)
 //   operand_kernel         R (float32) -> fp16 pair (hi, lo), hi + lo = R to
 //                          about 2^-22; the layout every dense kernel reads
-//   dense_gemm_kernel      quantise (y = R x, then the codec's lambda, group
-//                          absmax, scale, rounding and packing) and
-//                          dequantise (xhat = R^T (lambda sigma q)), as a
-//                          register-tiled float32 product of 64-vector tiles
-//   dense_calibrate_kernel lambda = RMS of R x over the calibration rows
+//   dense_calibrate_kernel lambda = RMS of R x over the calibration rows, as
+//                          a register-tiled float32 product of 64-vector
+//                          tiles (CUDA cores)
+//
+// The quantiser and dequantiser run on the tensor cores (dense_mma.cuh,
+// dense_mma_dequant.cuh).
 //
 // Operand layout: [S][H][2][d][d] fp16, part 0 = hi, part 1 = lo, row n of a
 // part is output coordinate n (y_n = sum_k R[n][k] x_k).
@@ -128,10 +129,9 @@ __device__ __forceinline__ float op_value(const uint16_t* hi, const uint16_t* lo
   return __half2float(__ushort_as_half(hi[i])) + __half2float(__ushort_as_half(lo[i]));
 }
 
-// acc[i][c] += sum_k A[v_i][k] * Bt[k][n_c] over all K, where the staged
-// chunk Bt[kk][n] = R[n][k0 + kk] (TRANS = false: y = R x) or R[k0 + kk][n]
-// (TRANS = true: xhat = R^T y). A is already in shared memory.
-template <int D, bool TRANS>
+// acc[i][c] = sum_k A[v_i][k] * Bt[k][n_c] over all K (y = R x), where the
+// staged chunk Bt[kk][n] = R[n][k0 + kk]. A is already in shared memory.
+template <int D>
 __device__ __forceinline__ void dense_product(const float* As, float* Bs, const uint16_t* hi,
                                               const uint16_t* lo, int tid,
                                               float (&acc)[DenseTile<D>::TV][8]) {
@@ -144,13 +144,8 @@ __device__ __forceinline__ void dense_product(const float* As, float* Bs, const 
   for (int k0 = 0; k0 < D; k0 += kDenseKC) {
     __syncthreads();   // the previous chunk has been read
     for (int idx = tid; idx < D * kDenseKC; idx += kDenseThreads) {
-      if constexpr (TRANS) {
-        const int kk = idx / D, n = idx % D;
-        Bs[kk * T::BS + n] = op_value(hi, lo, size_t(k0 + kk) * D + n);
-      } else {
-        const int n = idx / kDenseKC, kk = idx % kDenseKC;
-        Bs[kk * T::BS + n] = op_value(hi, lo, size_t(n) * D + k0 + kk);
-      }
+      const int n = idx / kDenseKC, kk = idx % kDenseKC;
+      Bs[kk * T::BS + n] = op_value(hi, lo, size_t(n) * D + k0 + kk);
     }
     __syncthreads();
 #pragma unroll 4
@@ -164,185 +159,6 @@ __device__ __forceinline__ void dense_product(const float* As, float* Bs, const 
 #pragma unroll
         for (int c = 0; c < 8; ++c) acc[i][c] = fmaf(av, b[c], acc[i][c]);
       }
-    }
-  }
-}
-
-struct DenseArgs {
-  int64_t n_slices, n_rows, in_stride_rows, out_stride_rows;
-  int32_t heads;
-  int64_t row_tiles;          // ceil(n_rows / 64)
-  const uint16_t* x;          // quantise input [S][T_in][H][d]
-  const uint8_t* codes_in;    // dequantise inputs [S][T_in][H][...]
-  const uint16_t* scales_in;
-  uint8_t* codes;             // quantise outputs [S][T_out][H][...]
-  uint16_t* scales;
-  uint16_t* xhat;             // dequantise output [S][T_out][H][d]
-  const uint16_t* operand;    // [S][H][2][d][d]
-  const float* lambda;        // [S][H][d]
-  unsigned* guard;            // debug-build index checks
-};
-
-// One block per (slice, head, 64-row tile).
-template <int D, int BITS, int G, bool QUANT>
-__global__ void __launch_bounds__(kDenseThreads) dense_gemm_kernel(const DenseArgs a) {
-  using T = DenseTile<D>;
-  constexpr int QMAX = (1 << (BITS - 1)) - 1;
-  constexpr int CB = D * BITS / 8, NG = D / G;
-  extern __shared__ __align__(16) uint8_t smem_raw[];
-  float* As = reinterpret_cast<float*>(smem_raw);
-  float* Bs = reinterpret_cast<float*>(smem_raw + T::kABytes);
-  const int tid = threadIdx.x;
-  const int64_t tile = blockIdx.x % a.row_tiles;
-  const int64_t sh = blockIdx.x / a.row_tiles;   // s * H + h
-  const int64_t s = sh / a.heads;
-  const int h = int(sh % a.heads);
-  const int64_t r0 = tile * kDenseRows;
-  const uint16_t* hi = a.operand + size_t(sh) * 2 * D * D;
-  const uint16_t* lo = hi + size_t(D) * D;
-  const float* lam = a.lambda + size_t(sh) * D;
-
-  // A tile: x (quantise) or lambda * sigma * q (dequantise), float32
-  for (int idx = tid; idx < kDenseRows * (D / 8); idx += kDenseThreads) {
-    const int v = idx / (D / 8), c8 = idx % (D / 8);
-    const int64_t r = r0 + v;
-    float f[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-    const size_t vec = size_t((s * a.in_stride_rows + r) * a.heads + h);
-    if (r < a.n_rows &&
-        dbg_ok(int64_t(vec) < vec_limit(a.n_slices, a.in_stride_rows, a.n_rows, a.heads),
-               a.guard)) {
-      if constexpr (QUANT) {
-        const uint4 w = *reinterpret_cast<const uint4*>(a.x + vec * D + 8 * c8);
-        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 p = __half22float2(*reinterpret_cast<const __half2*>(&ww[e]));
-          f[2 * e] = p.x;
-          f[2 * e + 1] = p.y;
-        }
-      } else {
-        const float sg = __half2float(__ushort_as_half(a.scales_in[vec * NG + (8 * c8) / G]));
-        int q[8];
-        if constexpr (BITS == 4) {
-          const uint32_t w = *reinterpret_cast<const uint32_t*>(a.codes_in + vec * CB + 4 * c8);
-#pragma unroll
-          for (int e = 0; e < 8; ++e) q[e] = int(int32_t(w << (28 - 4 * e)) >> 28);
-        } else {
-          const uint2 w = *reinterpret_cast<const uint2*>(a.codes_in + vec * CB + 8 * c8);
-#pragma unroll
-          for (int e = 0; e < 8; ++e)
-            q[e] = int(int8_t(((e < 4 ? w.x : w.y) >> (8 * (e & 3))) & 0xFFu));
-        }
-#pragma unroll
-        for (int e = 0; e < 8; ++e) f[e] = (float(q[e]) * sg) * lam[8 * c8 + e];
-      }
-    }
-    float* dst = As + v * T::AS + 8 * c8;
-    *reinterpret_cast<float4*>(dst) = make_float4(f[0], f[1], f[2], f[3]);
-    *reinterpret_cast<float4*>(dst + 4) = make_float4(f[4], f[5], f[6], f[7]);
-  }
-
-  float acc[T::TV][8];
-  dense_product<D, !QUANT>(As, Bs, hi, lo, tid, acc);
-  const int tn = tid % T::NT, tv = tid / T::NT;
-
-  if constexpr (!QUANT) {
-    // xhat = R^T yhat, rounded to fp16: 8 consecutive outputs per vector
-#pragma unroll
-    for (int i = 0; i < T::TV; ++i) {
-      const int64_t r = r0 + tv * T::TV + i;
-      if (r >= a.n_rows) continue;
-      if (!dbg_ok((s * a.out_stride_rows + r) * a.heads + h <
-                      vec_limit(a.n_slices, a.out_stride_rows, a.n_rows, a.heads),
-                  a.guard))
-        continue;
-      uint32_t w[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const __half2 h2 = __floats2half2_rn(acc[i][2 * e], acc[i][2 * e + 1]);
-        w[e] = *reinterpret_cast<const uint32_t*>(&h2);
-      }
-      const size_t vec = size_t((s * a.out_stride_rows + r) * a.heads + h);
-      *reinterpret_cast<uint4*>(a.xhat + vec * D + 8 * tn) = make_uint4(w[0], w[1], w[2], w[3]);
-    }
-  } else {
-    // y tile to shared memory (over A, which every thread has finished reading)
-    __syncthreads();
-    float* Cs = As;
-#pragma unroll
-    for (int i = 0; i < T::TV; ++i) {
-      float* dst = Cs + (tv * T::TV + i) * T::AS + 8 * tn;
-      *reinterpret_cast<float4*>(dst) = make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
-      *reinterpret_cast<float4*>(dst + 4) =
-          make_float4(acc[i][4], acc[i][5], acc[i][6], acc[i][7]);
-    }
-    __syncthreads();
-    // One warp per vector: lane l holds coordinates C l .. C l + C - 1, which
-    // lie in one group (G >= 8 >= C); a group spans LPG lanes.
-    constexpr int C = D / 32;
-    constexpr int LPG = G / C;
-    const int warp = tid >> 5, lane = tid & 31;
-    float lv[C];
-#pragma unroll
-    for (int c = 0; c < C; ++c) lv[c] = lam[C * lane + c];
-    for (int v = warp; v < kDenseRows; v += kDenseThreads / 32) {
-      const int64_t r = r0 + v;
-      if (r >= a.n_rows) break;   // warp-uniform: rows beyond N come last
-      float w[C];
-      float am = 0.0f;
-#pragma unroll
-      for (int c = 0; c < C; ++c) {
-        w[c] = __fdiv_rn(Cs[v * T::AS + C * lane + c], lv[c]);
-        am = fmaxf(am, fabsf(w[c]));
-      }
-#pragma unroll
-      for (int o = 1; o < LPG && o < 32; o <<= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
-      const float sf = fminf(div_by_const<QMAX>(am), 65504.0f);
-      const __half hs = __float2half_rn(sf);
-      const float sg = __half2float(hs);
-      uint32_t qb[C];
-#pragma unroll
-      for (int c = 0; c < C; ++c) {
-        float q = sg > 0.0f ? rintf(__fdiv_rn(w[c], sg)) : 0.0f;
-        q = fminf(fmaxf(q, -float(QMAX)), float(QMAX));
-        qb[c] = uint32_t(int32_t(q));
-      }
-      const size_t vec = size_t((s * a.out_stride_rows + r) * a.heads + h);
-      if (!dbg_ok(int64_t(vec) < vec_limit(a.n_slices, a.out_stride_rows, a.n_rows, a.heads),
-                  a.guard))
-        continue;   // warp-uniform: every lane holds the same vector
-      uint8_t* cdst = a.codes + vec * CB;
-      if constexpr (BITS == 4) {
-        // coordinates 2m (low nibble) and 2m + 1 (high nibble) share byte m
-        uint32_t word = 0;
-#pragma unroll
-        for (int c = 0; c < C; c += 2)
-          word |= ((qb[c] & 0xFu) | ((qb[c + 1] & 0xFu) << 4)) << (4 * c);
-        if constexpr (C == 8) {
-          reinterpret_cast<uint32_t*>(cdst)[lane] = word;
-        } else if constexpr (C == 4) {
-          reinterpret_cast<uint16_t*>(cdst)[lane] = uint16_t(word);
-        } else {
-          cdst[lane] = uint8_t(word);
-        }
-      } else {
-        uint32_t w0 = 0, w1 = 0;
-#pragma unroll
-        for (int c = 0; c < C; ++c) {
-          if (c < 4)
-            w0 |= (qb[c] & 0xFFu) << (8 * c);
-          else
-            w1 |= (qb[c] & 0xFFu) << (8 * (c - 4));
-        }
-        if constexpr (C == 8) {
-          reinterpret_cast<uint2*>(cdst)[lane] = make_uint2(w0, w1);
-        } else if constexpr (C == 4) {
-          reinterpret_cast<uint32_t*>(cdst)[lane] = w0;
-        } else {
-          reinterpret_cast<uint16_t*>(cdst)[lane] = uint16_t(w0);
-        }
-      }
-      if ((lane % LPG) == 0) a.scales[vec * NG + (C * lane) / G] = __half_as_ushort(hs);
     }
   }
 }
@@ -399,7 +215,7 @@ __global__ void __launch_bounds__(kDenseThreads) dense_calibrate_kernel(const De
       *reinterpret_cast<float4*>(dst + 4) = make_float4(f[4], f[5], f[6], f[7]);
     }
     float acc[T::TV][8];
-    dense_product<D, false>(As, Bs, hi, lo, tid, acc);
+    dense_product<D>(As, Bs, hi, lo, tid, acc);
 #pragma unroll
     for (int i = 0; i < T::TV; ++i)
 #pragma unroll

@@ -94,6 +94,17 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
          (uint64_t(1) << 46) | (uint64_t(2) << 61);
 }
 
+// Shared-memory matrix descriptor of an MN-major operand stored as TMA boxes
+// of rows of 64 fp16 (128 bytes) with the 128-byte swizzle: 64 contiguous MN
+// elements per row, 8-row K groups 1024 bytes apart (stride offset), and
+// successive 64-element MN blocks `lbo` bytes apart (leading offset).
+// Successive K steps of 16 rows advance the start address by 2048 bytes (two
+// whole swizzle atoms).
+__device__ __forceinline__ uint64_t sw128_mn_desc(uint32_t saddr, uint32_t lbo) {
+  return uint64_t((saddr >> 4) & 0x3FFFu) | (uint64_t((lbo >> 4) & 0x3FFFu) << 16) |
+         (uint64_t(1024 >> 4) << 32) | (uint64_t(1) << 46) | (uint64_t(2) << 61);
+}
+
 // Instruction descriptor of kind::f16: fp32 accumulator (bits 4-5 = 1), fp16
 // A and B (bits 7-9, 10-12 = 0), both K-major (bits 15, 16 = 0), N >> 3 in
 // bits 17-22, M >> 4 in bits 24-28.

@@ -217,3 +217,87 @@ def test_dense_quantiser_ranges_cross_slices_and_heads(d, group, bits):
                                            parity.DENSE_SCALE_BAND,
                                            parity.dense_code_band(ref, lam, group)),
                         f"d{d} g{group} b{bits} many blocks")
+
+
+def _random_codes(rng, S, N, H, d, group, bits, lo_exp, hi_exp):
+    """Arbitrary code bytes (every nibble / byte value, the quantiser's unused
+    -8 and -128 included) and fp16 scales log-uniform over 2^lo_exp ..
+    2^hi_exp, so that the rows of one block span several binades."""
+    codes = rng.integers(0, 256, (S, N, H, d * bits // 8), dtype=np.uint8)
+    sig = np.exp2(rng.uniform(lo_exp, hi_exp, (S, N, H, d // group)))
+    scales = np.minimum(sig, 65504.0).astype(np.float16).view(np.uint16)
+    return codes, scales
+
+
+def _assert_dequant_scale_free(gpu_bits, xhat64, what):
+    """The dequantiser against the oracle's float64 xhat, at any magnitude:
+    each finite output within one binary16 ulp of the exact value (its own
+    rounding) plus 1e-5 of the vector's largest |xhat| (the float32
+    accumulation of 3 d tensor-core products, for an output that cancels);
+    an infinite output only where the exact value is at the overflow
+    threshold (65520) within that same error, with its sign."""
+    a = oracle.binary16_bits_to_float(np.asarray(gpu_bits).view(np.uint16))
+    r = np.asarray(xhat64, np.float64)
+    vmax = np.max(np.abs(r), axis=-1, keepdims=True)
+    band = 1e-5 * vmax
+    mag = np.abs(r)
+    ulp = np.where(mag < 2.0 ** -14, 2.0 ** -24,
+                   np.exp2(np.floor(np.log2(np.maximum(mag, 2.0 ** -14))) - 10))
+    ulp = np.minimum(ulp, 32.0)
+    fin = np.isfinite(a)
+    ok_f = fin & (np.abs(np.where(fin, a, 0.0) - r) <= ulp + band)
+    ok_i = np.isinf(a) & (np.sign(a) == np.sign(r)) & (mag >= 65520.0 - band)
+    ok = ok_f | ok_i
+    assert ok.all(), (f"{what}: {int((~ok).sum())} of {ok.size} outputs off, "
+                      f"{int(np.isnan(a).sum())} NaN")
+
+
+@pytest.mark.parametrize("d,group,bits", [(64, 8, 8), (128, 16, 4), (128, 128, 8),
+                                          (256, 32, 4), (256, 8, 8), (256, 256, 4)])
+def test_dense_dequantiser_ranges_cross_slices_and_heads(d, group, bits):
+    """The tensor-core dequantiser with more 128-row blocks than SMs: every
+    CTA walks a range that crosses (slice, head) boundaries (operand
+    reloaded for d <= 128, streamed for d = 256), with a partial last block
+    per (slice, head); codes are arbitrary bytes and the scales of a vector
+    span 2^-7 .. 2^-3, so each row takes its own power-of-two range scale.
+    Every output is compared with the oracle."""
+    rng = np.random.default_rng(7 * d + group + bits)
+    S, N, H = 3, 1000, 5
+    if d < 256:
+        S, N = 4, 2600
+    signs = np.where(rng.random((S, H, d)) < 0.5, -1, 1).astype(np.int8)
+    R = oracle.householder_rotations(rng.standard_normal((S, H, 16, d)), signs, 1)
+    lam = np.exp(rng.uniform(-2.0, 2.0, (S, H, d))).astype(np.float32)
+    codes, scales = _random_codes(rng, S, N, H, d, group, bits, -7.0, -3.0)
+    op = rq.dense_operand(_t(R.astype(np.float32)))
+    xhat = rq.dequantize_dense(_t(codes), _t(scales.view(np.float16)), op, _t(lam), d, group,
+                               bits)
+    deq = oracle.dequantize_dense(codes, scales, R, lam, d, group, bits)
+    what = f"d{d} g{group} b{bits} many blocks dequant"
+    parity.assert_clean(parity.check_dequant(_np16(xhat), deq["bits"]), what)
+    _assert_dequant_scale_free(_np16(xhat), deq["xhat64"], what)
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+def test_dense_dequantiser_extreme_magnitudes(bits):
+    """lambda sigma q far outside fp16's range in both directions: sigma up
+    to 65504 with lambda up to 1e4 (|a| ~ 1e10: outputs overflow to inf),
+    fp16-subnormal sigma with lambda down to 1e-6 (outputs far below fp16's
+    normal range), and vectors mixing both. The row scale keeps every A
+    element inside fp16 before the split, so the outputs stay within the
+    scale-free bound of the exact values."""
+    rng = np.random.default_rng(11 + bits)
+    d, group, S, N, H = 128, 16, 2, 300, 2
+    signs = np.where(rng.random((S, H, d)) < 0.5, -1, 1).astype(np.int8)
+    R = oracle.householder_rotations(rng.standard_normal((S, H, 8, d)), signs, 0)
+    op = rq.dense_operand(_t(R.astype(np.float32)))
+    for lam_lo, lam_hi, e_lo, e_hi in ((1e2, 1e4, 8.0, 15.9), (1e-6, 1e-4, -24.0, -14.0),
+                                       (1e-3, 1e3, -24.0, 15.9)):
+        lam = np.exp(rng.uniform(np.log(lam_lo), np.log(lam_hi), (S, H, d))).astype(np.float32)
+        codes, scales = _random_codes(rng, S, N, H, d, group, bits, e_lo, e_hi)
+        xhat = rq.dequantize_dense(_t(codes), _t(scales.view(np.float16)), op, _t(lam), d, group,
+                                   bits)
+        deq = oracle.dequantize_dense(codes, scales, R, lam, d, group, bits)
+        _assert_dequant_scale_free(
+            _np16(xhat), deq["xhat64"],
+            f"b{bits} lambda {lam_lo:g}..{lam_hi:g} sigma 2^{e_lo:g}..2^{e_hi:g}")
