@@ -131,14 +131,6 @@ __device__ __forceinline__ void split_pair_slot(int p, int& r, int& j, bool& con
 // Block barrier of the two warps (named barrier 1).
 __device__ __forceinline__ void bar_pair() { asm volatile("bar.sync 1, 64;" ::: "memory"); }
 
-__device__ __forceinline__ uint2 lds64(uint32_t addr) {
-  uint2 v;
-  asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
-  return v;
-}
-__device__ __forceinline__ void sts64(uint32_t addr, uint2 v) {
-  asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(addr), "r"(v.x), "r"(v.y) : "memory");
-}
 __device__ __forceinline__ float2 u2f2(uint2 u) {
   return make_float2(__uint_as_float(u.x), __uint_as_float(u.y));
 }

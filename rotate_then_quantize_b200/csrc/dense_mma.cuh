@@ -153,8 +153,7 @@ __global__ void __launch_bounds__(DenseMma<D, EPI>::kThreads, 1)
   const int64_t u0 = j * per + (j < rem ? j : rem);
   const int n = int(per + (j < rem ? 1 : 0));
   if (n == 0) return;
-  auto sh_of = [&](int i) -> int64_t { return ((u0 + i) / a.row_blocks) * a.heads + hh; };
-  auto rb_of = [&](int i) -> int64_t { return (u0 + i) % a.row_blocks; };
+  const BlockWalk w0(u0, a.row_blocks, a.heads, hh);
 
   if (tid == 0) {
     prefetch_tensormap(&tm_x);
@@ -190,14 +189,14 @@ __global__ void __launch_bounds__(DenseMma<D, EPI>::kThreads, 1)
     // ---------------- A producer ----------------
     if (lane == 0) {
       int i = 0;
-      for (; i < n; ++i) {
+      BlockWalk w = w0;
+      for (; i < n; ++i, w.next()) {
         const int st = i % L::kNST;
         if (i >= L::kNST &&
             !wait_or_abort(&empty[st], ((i / L::kNST) & 1) ^ 1, abort_flag, a.guard))
           break;
-        const int64_t sh = sh_of(i);
-        const int r0 = int(rb_of(i) * 128);
-        const int s = int(sh / a.heads), h = int(sh % a.heads);
+        const int r0 = int(w.rb * 128);
+        const int s = int(w.s), h = hh;
         if (!dbg_ok(s < a.n_slices && r0 < a.n_rows, a.guard)) {
           mbar_arrive(&full[st]);   // debug build: no copy, the phase completes empty
           continue;
@@ -217,8 +216,9 @@ __global__ void __launch_bounds__(DenseMma<D, EPI>::kThreads, 1)
       if constexpr (!L::kStreamB) {
         int run = -1;
         int64_t prev = -1;
-        for (int i = 0; i < n; ++i) {
-          const int64_t sh = sh_of(i);
+        BlockWalk w = w0;
+        for (int i = 0; i < n; ++i, w.next()) {
+          const int64_t sh = w.sh();
           if (sh == prev) continue;
           if (run >= 0 && !wait_or_abort(&bempty[0], run & 1, abort_flag, a.guard)) break;
           ++run;
@@ -235,8 +235,9 @@ __global__ void __launch_bounds__(DenseMma<D, EPI>::kThreads, 1)
       } else {
         int c = 0;
         bool ok = true;
-        for (int i = 0; i < n && ok; ++i) {
-          const int64_t sh = sh_of(i);
+        BlockWalk w = w0;
+        for (int i = 0; i < n && ok; ++i, w.next()) {
+          const int64_t sh = w.sh();
           for (int q = 0; q < 2 && ok; ++q)
             for (int p = 0; p < L::kPieces; ++p) {
               const int slot = c % L::kBSlots;
@@ -262,9 +263,10 @@ __global__ void __launch_bounds__(DenseMma<D, EPI>::kThreads, 1)
       int run = -1, c = 0, i = 0;
       int64_t prev = -1;
       bool ok = true;
-      for (; i < n && ok; ++i) {
+      BlockWalk w = w0;
+      for (; i < n && ok; ++i, w.next()) {
         const int st = i % L::kNST, acc = i % L::kAcc;
-        const int64_t sh = sh_of(i);
+        const int64_t sh = w.sh();
         if (!wait_or_abort(&full[st], (i / L::kNST) & 1, abort_flag, a.guard)) break;
         if (i >= L::kAcc &&
             !wait_or_abort(&tempty[acc], ((i / L::kAcc) & 1) ^ 1, abort_flag, a.guard))
@@ -311,7 +313,7 @@ __global__ void __launch_bounds__(DenseMma<D, EPI>::kThreads, 1)
         tc_commit(&empty[st]);
         tc_commit(&tfull[acc]);
         if constexpr (!L::kStreamB) {
-          if (i + 1 == n || sh_of(i + 1) != sh) tc_commit(&bempty[0]);
+          if (i + 1 == n || w.last_of_slice()) tc_commit(&bempty[0]);
         }
       }
       // drain: every MMA issued (a block cut short by an abort included)
@@ -326,9 +328,11 @@ __global__ void __launch_bounds__(DenseMma<D, EPI>::kThreads, 1)
     // this warp's own 1 / lambda table (no barrier across warps)
     float* rl = reinterpret_cast<float*>(smem + L::kTabOff) + (warp - 4) * D;
     int64_t tab_sh = -1;
+    BlockWalk w = w0;
+    for (int k = 0; k < grp; ++k) w.next();
     for (int i = grp; i < n; i += L::kEpi) {
       const int acc = i % L::kAcc;
-      const int64_t sh = sh_of(i);
+      const int64_t sh = w.sh();
       if (sh != tab_sh) {
         __syncwarp();   // every lane is done reading the old table
         for (int j = lane; j < D; j += 32) rl[j] = __frcp_rn(a.lambda[sh * D + j]);
@@ -340,8 +344,9 @@ __global__ void __launch_bounds__(DenseMma<D, EPI>::kThreads, 1)
                                                  a.guard)))
         break;
       tc_fence_after();
-      const int64_t row = rb_of(i) * 128 + 32 * q + lane;
-      const int64_t s = sh / a.heads, h = sh % a.heads;
+      const int64_t row = int64_t(w.rb) * 128 + 32 * q + lane;
+      const int64_t s = w.s, h = hh;
+      for (int k = 0; k < L::kEpi; ++k) w.next();   // this group's next block
       const size_t vec = size_t((s * a.out_stride_rows + row) * a.heads + h);
       const bool valid =
           row < a.n_rows &&

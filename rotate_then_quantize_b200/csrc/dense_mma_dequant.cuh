@@ -11,10 +11,13 @@
 // (R = hi + lo, fp16) serves unchanged.
 //
 // Precision. a_j is not exact in fp16 (q has up to 7 bits, sigma 11, lambda
-// 24), so A is split like B: a = a_hi + a_lo, a_hi = fp16(a), a_lo =
-// fp16(a - a_hi) (the residual a - a_hi is exact in float32). The product
-// sums a_hi hi + a_lo hi + a_hi lo into one float32 accumulator; the dropped
-// a_lo lo term is below 2^-24 of |a R|.
+// 24), so A is split like B: a = a_hi + a_lo, a_hi = a with its low 13
+// mantissa bits cleared (exact in fp16 inside its normal range), a_lo =
+// fp16(a - a_hi) (the residual is exact in float32; |a_lo| < 2^-10 |a|).
+// The product sums a_hi hi + a_lo hi + a_hi lo into one float32
+// accumulator; the dropped a_lo lo term is below 2^-22 of |a R|. (The split
+// by truncation costs two float-to-half conversions per pair of values
+// instead of four for a rounded one.)
 // Range. Each row (vector) is scaled by an exact power of two 2^-e before the
 // split, so that |a_j 2^-e| < 2^15 stays inside fp16's normal range whatever
 // the data's magnitude: e comes from the row's largest |sigma| and the
@@ -26,7 +29,7 @@
 // in the quantiser (CTA c serves head c % H, contiguous (slice, row block)
 // ranges).
 //
-// Warp roles (512 threads):
+// Warp roles (768 threads):
 //   warp 0      B producer: TMA loads of the operand in chunks of 64 rows of R
 //               (64 values of j) x d columns, as boxes of 64 x 64 fp16 with
 //               the 128-byte swizzle. d <= 128: the whole operand (hi and
@@ -37,11 +40,14 @@
 //   warp 2      codes producer: one TMA load (two for 256-byte rows) of the
 //               block's 128 x d*bits/8 code bytes per stage, swizzled
 //   warp 3      idle
-//   warps 4-11  A producers: warp 4 + w serves rows 32 (w % 4) .. + 31 and
-//               half w / 4 of every 64-wide K piece; it turns codes, scales
-//               and lambda into the hi / lo fp16 rows of A in the 128-byte
-//               swizzled K-major layout, then hands the piece to the MMA
-//   warps 12-15 epilogue: warp 12 + q reads TMEM lanes 32q .. 32q + 31 (rows),
+//   warps 4-19  A producers: warp 4 + w serves rows 32 (w % 4) .. + 31 and
+//               the 16 coordinates 16 (w / 4) .. + 15 of every 64-wide K
+//               piece; it turns codes, scales and lambda (its columns'
+//               values, kept in its own shared-memory table) into the hi / lo
+//               fp16 rows of A in the 128-byte swizzled K-major layout, then
+//               hands the piece to the MMA (sixteen warps, so that four per
+//               scheduler hide each other's latency)
+//   warps 20-23 epilogue: warp 20 + q reads TMEM lanes 32q .. 32q + 31 (rows),
 //               scales by 2^e, rounds to fp16 and stores the row
 // Every wait is bounded. A wait that gives up raises the guard word and a
 // shared abort flag that ends every role's loop; the roles drain what they
@@ -70,13 +76,19 @@ struct DenseDeq {
   static constexpr int kCStages = 2;
   static constexpr int kAcc = D == 256 ? 2 : 4;         // TMEM accumulators
   static constexpr uint32_t kTmemCols = kAcc * D <= 256 ? 256u : 512u;
-  static constexpr int kProdWarps = 8;
+  static constexpr int kParts = 4;                      // column parts of a piece
+  static constexpr int kEW = 64 / kParts;               // coordinates per thread per piece
+  static constexpr int kSub = kEW / 8;                  // 16-byte A chunks per thread
+  static constexpr int kCW = kEW * BITS / 32;           // code words per thread per piece
+  static constexpr int kProdWarps = 4 * kParts;
   static constexpr int kEpiWarp0 = 4 + kProdWarps;
   static constexpr int kThreads = 32 * kEpiWarp0 + 128;
   static constexpr int kAOff = 0;
   static constexpr int kBOff = kAOff + kASlots * kASlot;
   static constexpr int kCOff = kBOff + kBSlots * kBChunk;
-  static constexpr int kBarOff = kCOff + kCStages * kCTile;
+  static constexpr int kLamOff = kCOff + kCStages * kCTile;   // lambda, per producer warp
+  static constexpr int kLamWarp = kPieces * kEW;              // floats per producer warp
+  static constexpr int kBarOff = kLamOff + kProdWarps * kLamWarp * 4;
   // cfull, cempty per code stage; afull, aempty per A slot; bfull, bempty
   // per B slot; tfull, tempty per accumulator; the MMA role's final drain
   static constexpr int kNumBars = 2 * kCStages + 2 * kASlots + 2 * kBSlots + 2 * kAcc + 1;
@@ -225,8 +237,7 @@ __global__ void __launch_bounds__(DenseDeq<D, BITS>::kThreads, 1)
   const int64_t u0 = jc * per + (jc < rem ? jc : rem);
   const int n = int(per + (jc < rem ? 1 : 0));
   if (n == 0) return;
-  auto sh_of = [&](int i) -> int64_t { return ((u0 + i) / a.row_blocks) * a.heads + hh; };
-  auto rb_of = [&](int i) -> int64_t { return (u0 + i) % a.row_blocks; };
+  const BlockWalk w0(u0, a.row_blocks, a.heads, hh);
 
   if (tid == 0) {
     prefetch_tensormap(&tm_c);
@@ -277,8 +288,9 @@ __global__ void __launch_bounds__(DenseDeq<D, BITS>::kThreads, 1)
       if constexpr (!L::kStreamB) {
         int run = -1;
         int64_t prev = -1;
-        for (int i = 0; i < n; ++i) {
-          const int64_t sh = sh_of(i);
+        BlockWalk w = w0;
+        for (int i = 0; i < n; ++i, w.next()) {
+          const int64_t sh = w.sh();
           if (sh == prev) continue;
           if (run >= 0 && !wait_or_abort(&bempty[0], run & 1, abort_flag, a.guard)) break;
           ++run;
@@ -292,8 +304,9 @@ __global__ void __launch_bounds__(DenseDeq<D, BITS>::kThreads, 1)
       } else {
         int c = 0;
         bool ok = true;
-        for (int i = 0; i < n && ok; ++i) {
-          const int64_t sh = sh_of(i);
+        BlockWalk w = w0;
+        for (int i = 0; i < n && ok; ++i, w.next()) {
+          const int64_t sh = w.sh();
           for (int kc = 0; kc < L::kPieces && ok; ++kc)
             for (int q = 0; q < 2; ++q) {
               const int slot = c % L::kBSlots;
@@ -316,14 +329,14 @@ __global__ void __launch_bounds__(DenseDeq<D, BITS>::kThreads, 1)
     // ---------------- codes producer ----------------
     if (lane == 0) {
       int i = 0;
-      for (; i < n; ++i) {
+      BlockWalk w = w0;
+      for (; i < n; ++i, w.next()) {
         const int st = i % L::kCStages;
         if (i >= L::kCStages &&
             !wait_or_abort(&cempty[st], ((i / L::kCStages) & 1) ^ 1, abort_flag, a.guard))
           break;
-        const int64_t sh = sh_of(i);
-        const int r0 = int(rb_of(i) * 128);
-        const int s = int(sh / a.heads), h = int(sh % a.heads);
+        const int r0 = int(w.rb * 128);
+        const int s = int(w.s), h = hh;
         if (!dbg_ok(s < a.n_slices && r0 < a.n_rows, a.guard)) {
           mbar_arrive(&cfull[st]);   // debug build: no copy, the phase completes empty
           continue;
@@ -343,9 +356,10 @@ __global__ void __launch_bounds__(DenseDeq<D, BITS>::kThreads, 1)
       int run = -1, ca = 0, cb = 0;
       int64_t prev = -1;
       bool ok = true;
-      for (int i = 0; i < n && ok; ++i) {
+      BlockWalk w = w0;
+      for (int i = 0; i < n && ok; ++i, w.next()) {
         const int acc = i % L::kAcc;
-        const int64_t sh = sh_of(i);
+        const int64_t sh = w.sh();
         if (i >= L::kAcc &&
             !wait_or_abort(&tempty[acc], ((i / L::kAcc) & 1) ^ 1, abort_flag, a.guard))
           break;
@@ -399,7 +413,7 @@ __global__ void __launch_bounds__(DenseDeq<D, BITS>::kThreads, 1)
         if (!ok) break;
         tc_commit(&tfull[acc]);
         if constexpr (!L::kStreamB) {
-          if (i + 1 == n || sh_of(i + 1) != sh) tc_commit(&bempty[0]);
+          if (i + 1 == n || w.last_of_slice()) tc_commit(&bempty[0]);
         }
       }
       // drain: every MMA issued (a block cut short by an abort included)
@@ -409,139 +423,176 @@ __global__ void __launch_bounds__(DenseDeq<D, BITS>::kThreads, 1)
     }
   } else if (warp >= 4 && warp < L::kEpiWarp0) {
     // ---------------- A producers ----------------
+    constexpr int EW = L::kEW, SUB = L::kSub, CW = L::kCW;
     const int pw = warp - 4;
     const int r = 32 * (pw & 3) + lane;   // row of the block
-    auto produce = [&](auto half_) {
-      constexpr int HF = decltype(half_)::value;   // half of each 64-wide piece
-      float lmax = 0.0f;
-      int64_t lam_sh = -1;
-      auto scales_of = [&](int i, uint32_t (&sw)[SW]) {
-        const int64_t sh = sh_of(i);
-        const int64_t row = rb_of(i) * 128 + r;
-        const size_t vec =
-            size_t(((sh / a.heads) * a.in_stride_rows + row) * a.heads + sh % a.heads);
-        const bool valid =
-            row < a.n_rows &&
-            dbg_ok(int64_t(vec) < vec_limit(a.n_slices, a.in_stride_rows, a.n_rows, a.heads),
-                   a.guard);
-        dense_load_scales<NG>(a.scales + vec * NG, valid, sw);
-      };
-      uint32_t sw_next[SW];
-      scales_of(0, sw_next);
-      int ca = 0;
-      bool ok = true;
-      for (int i = 0; i < n && ok; ++i) {
-        uint32_t sw[SW];
+    const int part = pw >> 2;             // coordinates EW part .. + EW - 1 of each piece
+    // lambda_j of this warp's columns: ltab[EW p + c] = lambda[64 p + EW part + c]
+    float* ltab = reinterpret_cast<float*>(smem + L::kLamOff) + pw * L::kLamWarp;
+    float lmax = 0.0f;
+    int64_t lam_sh = -1;
+    auto scales_of = [&](const BlockWalk& ww, uint32_t (&sw)[SW]) {
+      const int64_t row = int64_t(ww.rb) * 128 + r;
+      const size_t vec = size_t((ww.s * a.in_stride_rows + row) * a.heads + hh);
+      const bool valid =
+          row < a.n_rows &&
+          dbg_ok(int64_t(vec) < vec_limit(a.n_slices, a.in_stride_rows, a.n_rows, a.heads),
+                 a.guard);
+      dense_load_scales<NG>(a.scales + vec * NG, valid, sw);
+    };
+    BlockWalk w = w0, wn = w0;
+    uint32_t sw_next[SW];
+    scales_of(wn, sw_next);
+    wn.next();
+    int ca = 0;
+    bool ok = true;
+    for (int i = 0; i < n && ok; ++i, w.next()) {
+      uint32_t sw[SW];
 #pragma unroll
-        for (int k = 0; k < SW; ++k) sw[k] = sw_next[k];
-        if (i + 1 < n) scales_of(i + 1, sw_next);   // one block ahead
-        const int64_t sh = sh_of(i);
-        if (sh != lam_sh) {
-          lmax = dense_lambda_max<D>(a.lambda + sh * D, lane);
-          lam_sh = sh;
-        }
-        const float down = exp2_int(-dense_row_exponent<QMAX>(dense_sigma_max<NG>(sw), lmax));
-        const float* lam = a.lambda + sh * D;
-        const int st = i % L::kCStages;
-        if (!__all_sync(0xffffffffu, wait_or_abort(&cfull[st], (i / L::kCStages) & 1,
+      for (int k = 0; k < SW; ++k) sw[k] = sw_next[k];
+      if (i + 1 < n) {   // one block ahead
+        scales_of(wn, sw_next);
+        wn.next();
+      }
+      const int64_t sh = w.sh();
+      if (sh != lam_sh) {
+        lmax = dense_lambda_max<D>(a.lambda + sh * D, lane);
+        __syncwarp();   // every lane is done reading the old table
+        for (int t = lane; t < L::kLamWarp; t += 32)
+          ltab[t] = __ldg(a.lambda + sh * D + 64 * (t / EW) + EW * part + t % EW);
+        __syncwarp();
+        lam_sh = sh;
+      }
+      const float down = exp2_int(-dense_row_exponent<QMAX>(dense_sigma_max<NG>(sw), lmax));
+      const int st = i % L::kCStages;
+      if (!__all_sync(0xffffffffu, wait_or_abort(&cfull[st], (i / L::kCStages) & 1,
+                                                 abort_flag, a.guard))) {
+        ok = false;
+        break;
+      }
+      const uint32_t ctile = smem_addr(Cs + st * L::kCTile);
+      static_for<0, L::kPieces>([&](auto p_) {
+        constexpr int p = decltype(p_)::value;
+        if (!ok) return;
+        const int as = ca % L::kASlots;
+        if (ca >= L::kASlots &&
+            !__all_sync(0xffffffffu, wait_or_abort(&aempty[as], ((ca / L::kASlots) & 1) ^ 1,
                                                    abort_flag, a.guard))) {
           ok = false;
-          break;
+          return;
         }
-        const uint32_t ctile = smem_addr(Cs + st * L::kCTile);
-        static_for<0, L::kPieces>([&](auto p_) {
-          constexpr int p = decltype(p_)::value;
-          if (!ok) return;
-          const int as = ca % L::kASlots;
-          if (ca >= L::kASlots &&
-              !__all_sync(0xffffffffu, wait_or_abort(&aempty[as], ((ca / L::kASlots) & 1) ^ 1,
-                                                     abort_flag, a.guard))) {
-            ok = false;
-            return;
-          }
-          // this thread's 32 codes: elements 64 p + 32 HF .. + 31 of row r
-          constexpr int kOff = (64 * p + 32 * HF) * BITS / 8;    // byte offset in the row
-          constexpr int kBox = kOff / L::kCSpan;
-          constexpr int kChunk = (kOff % L::kCSpan) / 16;
-          const uint32_t rowa =
-              swz_row<L::kCSpan>(ctile + uint32_t(kBox * 128 * L::kCSpan), uint32_t(r));
-          uint32_t cw[BITS];
-          {
-            const uint4 v = lds128(swz_chunk<L::kCSpan>(rowa, kChunk));
-            cw[0] = v.x;
-            cw[1] = v.y;
-            cw[2] = v.z;
-            cw[3] = v.w;
-          }
-          if constexpr (BITS == 8) {
-            const uint4 v = lds128(swz_chunk<L::kCSpan>(rowa, kChunk + 1));
-            cw[4] = v.x;
-            cw[5] = v.y;
-            cw[6] = v.z;
-            cw[7] = v.w;
-          }
-          const uint32_t arow = smem_addr(As + as * L::kASlot) + uint32_t(r) * 128u;
-          static_for<0, 4>([&](auto k_) {
-            constexpr int k = decltype(k_)::value;
-            constexpr int j0 = 64 * p + 32 * HF + 8 * k;   // first coordinate
-            constexpr int g = j0 / G;
-            const float sg =
-                __half2float(__ushort_as_half(uint16_t(sw[g / 2] >> (16 * (g % 2))))) * down;
-            const float4 l0 = __ldg(reinterpret_cast<const float4*>(lam + j0));
-            const float4 l1 = __ldg(reinterpret_cast<const float4*>(lam + j0 + 4));
-            const float lv[8] = {l0.x, l0.y, l0.z, l0.w, l1.x, l1.y, l1.z, l1.w};
-            float f[8];
-            dense_codes8<BITS>(cw + k * (BITS / 4), f);
-            uint32_t hw[4], lw[4];
-#pragma unroll
-            for (int m = 0; m < 4; ++m) {
-              const float2 qv = add2(make_float2(f[2 * m], f[2 * m + 1]), splat(-kBias));
-              const float2 sv = mul2(splat(sg), make_float2(lv[2 * m], lv[2 * m + 1]));
-              const float2 x = mul2(qv, sv);
-              const __half2 hi = __floats2half2_rn(x.x, x.y);
-              const float2 hf = __half22float2(hi);
-              const __half2 lo = __floats2half2_rn(x.x - hf.x, x.y - hf.y);
-              hw[m] = *reinterpret_cast<const uint32_t*>(&hi);
-              lw[m] = *reinterpret_cast<const uint32_t*>(&lo);
-            }
-            const uint32_t pos = uint32_t(((4 * HF + k) ^ (r & 7)) << 4);
-            sts128(arow + pos, make_uint4(hw[0], hw[1], hw[2], hw[3]));
-            sts128(arow + uint32_t(L::kAPiece) + pos, make_uint4(lw[0], lw[1], lw[2], lw[3]));
+        // this thread's EW codes: coordinates 64 p + EW part .. of row r.
+        // All loads first, then the arithmetic, then the stores (the stores
+        // are ordered asm, so a load placed after one could not move ahead).
+        const int off = (64 * p + EW * part) * BITS / 8;   // byte offset in the row
+        const uint32_t rowa = swz_row<L::kCSpan>(
+            ctile + uint32_t((off / L::kCSpan) * 128 * L::kCSpan), uint32_t(r));
+        const uint32_t caddr =
+            swz_chunk<L::kCSpan>(rowa, uint32_t((off % L::kCSpan) / 16)) + uint32_t(off % 16);
+        uint32_t cw[CW];
+        if constexpr (CW == 2) {
+          const uint2 v = lds64(caddr);
+          cw[0] = v.x;
+          cw[1] = v.y;
+        } else {
+          static_for<0, CW / 4>([&](auto c_) {
+            constexpr int c = decltype(c_)::value;
+            const uint4 v = lds128(c == 0 ? caddr : swz_chunk<L::kCSpan>(rowa, uint32_t(
+                                                        (off % L::kCSpan) / 16 + c)));
+            cw[4 * c] = v.x;
+            cw[4 * c + 1] = v.y;
+            cw[4 * c + 2] = v.z;
+            cw[4 * c + 3] = v.w;
           });
-          fence_proxy_async_smem();   // generic writes -> the MMA's async-proxy reads
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&afull[as]);
-          ++ca;
+        }
+        float2 lv[EW / 2];
+        {
+          const uint32_t lp = smem_addr(ltab + EW * p);
+#pragma unroll
+          for (int m = 0; m < EW / 4; ++m) {
+            const uint4 t = lds128(lp + 16u * m);
+            lv[2 * m] = make_float2(__uint_as_float(t.x), __uint_as_float(t.y));
+            lv[2 * m + 1] = make_float2(__uint_as_float(t.z), __uint_as_float(t.w));
+          }
+        }
+        uint32_t hw[EW / 2], lw[EW / 2];
+        static_for<0, SUB>([&](auto k_) {
+          constexpr int k = decltype(k_)::value;
+          // sigma 2^-e of the group of this 8-coordinate chunk
+          uint32_t hb = 0u;
+          static_for<0, L::kParts>([&](auto t_) {
+            constexpr int t = decltype(t_)::value;
+            constexpr int g = (64 * p + EW * t + 8 * k) / G;
+            if (part == t) hb = (sw[g / 2] >> (16 * (g % 2))) & 0xFFFFu;
+          });
+          const float2 s2 = splat(__half2float(__ushort_as_half(uint16_t(hb))) * down);
+          float f[8];
+          dense_codes8<BITS>(cw + k * (BITS / 4), f);
+#pragma unroll
+          for (int m = 0; m < 4; ++m) {
+            const float2 x = mul2(add2(make_float2(f[2 * m], f[2 * m + 1]), splat(-kBias)),
+                                  mul2(s2, lv[4 * k + m]));
+            // a_hi: a with the low 13 mantissa bits cleared (exact in fp16);
+            // a_lo: the exact float32 residual, rounded to fp16 once
+            const float2 ht = make_float2(__uint_as_float(__float_as_uint(x.x) & 0xFFFFE000u),
+                                          __uint_as_float(__float_as_uint(x.y) & 0xFFFFE000u));
+            const float2 res = add2(x, make_float2(-ht.x, -ht.y));
+            const __half2 hi = __floats2half2_rn(ht.x, ht.y);
+            const __half2 lo = __floats2half2_rn(res.x, res.y);
+            hw[4 * k + m] = *reinterpret_cast<const uint32_t*>(&hi);
+            lw[4 * k + m] = *reinterpret_cast<const uint32_t*>(&lo);
+          }
         });
+        const uint32_t arow = smem_addr(As + as * L::kASlot) + uint32_t(r) * 128u;
+        static_for<0, SUB>([&](auto k_) {
+          constexpr int k = decltype(k_)::value;
+          const uint32_t pos = uint32_t(((SUB * part + k) ^ (r & 7)) << 4);
+          sts128(arow + pos, make_uint4(hw[4 * k], hw[4 * k + 1], hw[4 * k + 2], hw[4 * k + 3]));
+          sts128(arow + uint32_t(L::kAPiece) + pos,
+                 make_uint4(lw[4 * k], lw[4 * k + 1], lw[4 * k + 2], lw[4 * k + 3]));
+        });
+        fence_proxy_async_smem();   // generic writes -> the MMA's async-proxy reads
         __syncwarp();
-        if (lane == 0) mbar_arrive(&cempty[st]);   // this warp is done with the codes
-      }
-    };
-    if (pw < 4)
-      produce(Int<0>{});
-    else
-      produce(Int<1>{});
+        if (lane == 0) mbar_arrive(&afull[as]);
+        ++ca;
+      });
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&cempty[st]);   // this warp is done with the codes
+    }
   } else if (warp >= L::kEpiWarp0) {
     // ---------------- epilogue ----------------
     const int q = warp & 3;   // TMEM lane quarter
     float lmax = 0.0f;
     int64_t lam_sh = -1;
-    for (int i = 0; i < n; ++i) {
-      const int acc = i % L::kAcc;
-      const int64_t sh = sh_of(i);
-      if (sh != lam_sh) {
-        lmax = dense_lambda_max<D>(a.lambda + sh * D, lane);
-        lam_sh = sh;
-      }
-      const int64_t row = rb_of(i) * 128 + 32 * q + lane;
-      const int64_t s = sh / a.heads, h = sh % a.heads;
-      const size_t vin = size_t((s * a.in_stride_rows + row) * a.heads + h);
+    auto scales_of = [&](const BlockWalk& ww, uint32_t (&sw)[SW]) {
+      const int64_t row = int64_t(ww.rb) * 128 + 32 * q + lane;
+      const size_t vin = size_t((ww.s * a.in_stride_rows + row) * a.heads + hh);
       const bool in_ok =
           row < a.n_rows &&
           dbg_ok(int64_t(vin) < vec_limit(a.n_slices, a.in_stride_rows, a.n_rows, a.heads),
                  a.guard);
-      uint32_t sw[SW];
       dense_load_scales<NG>(a.scales + vin * NG, in_ok, sw);
+    };
+    BlockWalk w = w0, wn = w0;
+    uint32_t sw_next[SW];
+    scales_of(wn, sw_next);
+    wn.next();
+    for (int i = 0; i < n; ++i, w.next()) {
+      const int acc = i % L::kAcc;
+      const int64_t sh = w.sh();
+      if (sh != lam_sh) {
+        lmax = dense_lambda_max<D>(a.lambda + sh * D, lane);
+        lam_sh = sh;
+      }
+      const int64_t row = int64_t(w.rb) * 128 + 32 * q + lane;
+      const int64_t s = w.s, h = hh;
+      uint32_t sw[SW];
+#pragma unroll
+      for (int k = 0; k < SW; ++k) sw[k] = sw_next[k];
+      if (i + 1 < n) {   // one block ahead
+        scales_of(wn, sw_next);
+        wn.next();
+      }
       const float up = exp2_int(dense_row_exponent<QMAX>(dense_sigma_max<NG>(sw), lmax));
       // warp-uniform outcome: the TMEM loads below are warp-collective
       if (!__all_sync(0xffffffffu, wait_or_abort(&tfull[acc], (i / L::kAcc) & 1, abort_flag,
@@ -554,34 +605,29 @@ __global__ void __launch_bounds__(DenseDeq<D, BITS>::kThreads, 1)
           dbg_ok(int64_t(vout) < vec_limit(a.n_slices, a.out_stride_rows, a.n_rows, a.heads),
                  a.guard);
       const uint32_t taddr = tmem_base + (uint32_t(32 * q) << 16) + uint32_t(acc) * uint32_t(D);
-      static_for<0, D / 64>([&](auto c_) {
+      static_for<0, D / 32>([&](auto c_) {
         constexpr int cc = decltype(c_)::value;
-        uint32_t r0[32], r1[32];
-        tmem_ld32(taddr + uint32_t(64 * cc), r0);
-        tmem_ld32(taddr + uint32_t(64 * cc + 32), r1);
-        tmem_wait_ld(r0, r1);
-        if constexpr (cc == D / 64 - 1) {
+        uint32_t r0[32];
+        tmem_ld32(taddr + uint32_t(32 * cc), r0);
+        tmem_wait_ld1(r0);
+        if constexpr (cc == D / 32 - 1) {
           tc_fence_before();   // this warp is done with the accumulator
           __syncwarp();
           if (lane == 0) mbar_arrive(&tempty[acc]);
         }
-        uint32_t w[32];
+        uint32_t wv[16];
 #pragma unroll
         for (int m = 0; m < 16; ++m) {
-          const float2 v0 = mul2(
+          const float2 v = mul2(
               make_float2(__uint_as_float(r0[2 * m]), __uint_as_float(r0[2 * m + 1])), splat(up));
-          const float2 v1 = mul2(
-              make_float2(__uint_as_float(r1[2 * m]), __uint_as_float(r1[2 * m + 1])), splat(up));
-          const __half2 h0 = __floats2half2_rn(v0.x, v0.y);
-          const __half2 h1 = __floats2half2_rn(v1.x, v1.y);
-          w[m] = *reinterpret_cast<const uint32_t*>(&h0);
-          w[16 + m] = *reinterpret_cast<const uint32_t*>(&h1);
+          const __half2 h2 = __floats2half2_rn(v.x, v.y);
+          wv[m] = *reinterpret_cast<const uint32_t*>(&h2);
         }
         if (valid) {
-          uint4* dst = reinterpret_cast<uint4*>(a.xhat + vout * D + 64 * cc);
+          uint4* dst = reinterpret_cast<uint4*>(a.xhat + vout * D + 32 * cc);
 #pragma unroll
-          for (int k = 0; k < 8; ++k)
-            dst[k] = make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+          for (int k = 0; k < 4; ++k)
+            dst[k] = make_uint4(wv[4 * k], wv[4 * k + 1], wv[4 * k + 2], wv[4 * k + 3]);
         }
       });
     }

@@ -167,6 +167,16 @@ __device__ __forceinline__ void sts128(uint32_t addr, uint4 v) {
                : "memory");
 }
 
+// 8-byte shared-memory load / store at a 32-bit shared address.
+__device__ __forceinline__ uint2 lds64(uint32_t addr) {
+  uint2 v;
+  asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ void sts64(uint32_t addr, uint2 v) {
+  asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(addr), "r"(v.x), "r"(v.y) : "memory");
+}
+
 // Row r of a swizzled TMA box of rows of SPAN bytes: the 16-byte chunk c of
 // the row sits at  base + r * SPAN + ((c ^ (r' & mask)) << 4), r' = the
 // 128-byte line index of the row. For a row whose offset has no bits inside

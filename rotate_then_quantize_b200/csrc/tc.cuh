@@ -82,6 +82,19 @@ __device__ __forceinline__ void tmem_wait_ld(uint32_t (&a)[32], uint32_t (&b)[32
       : "memory");
 }
 
+__device__ __forceinline__ void tmem_wait_ld1(uint32_t (&a)[32]) {
+  asm volatile(
+      "tcgen05.wait::ld.sync.aligned;"
+      : "+r"(a[0]), "+r"(a[1]), "+r"(a[2]), "+r"(a[3]), "+r"(a[4]), "+r"(a[5]), "+r"(a[6]),
+        "+r"(a[7]), "+r"(a[8]), "+r"(a[9]), "+r"(a[10]), "+r"(a[11]), "+r"(a[12]),
+        "+r"(a[13]), "+r"(a[14]), "+r"(a[15]), "+r"(a[16]), "+r"(a[17]), "+r"(a[18]),
+        "+r"(a[19]), "+r"(a[20]), "+r"(a[21]), "+r"(a[22]), "+r"(a[23]), "+r"(a[24]),
+        "+r"(a[25]), "+r"(a[26]), "+r"(a[27]), "+r"(a[28]), "+r"(a[29]), "+r"(a[30]),
+        "+r"(a[31])
+      :
+      : "memory");
+}
+
 // Shared-memory matrix descriptor of a K-major operand stored as rows of 128
 // bytes (64 fp16) with the 128-byte swizzle, 8-row groups 1024 bytes apart
 // (the layout TMA writes for a box 128 bytes wide): start address >> 4 in
@@ -113,6 +126,26 @@ constexpr uint32_t f16_idesc() {
   static_assert(M == 128 && N % 16 == 0 && N >= 16 && N <= 256, "MMA shape");
   return (1u << 4) | (uint32_t(N >> 3) << 17) | (uint32_t(M >> 4) << 24);
 }
+
+// A CTA's contiguous range of one head's (slice, row block) sequence, walked
+// one block at a time without a division per step (64-bit division and
+// remainder are long instruction sequences on the GPU).
+// (The launchers keep slices x row blocks, and slices x heads x d, below
+// 2^31, so every field fits 32 bits.)
+struct BlockWalk {
+  int32_t s, rb, row_blocks, heads, h;
+  __device__ BlockWalk(int64_t u, int64_t row_blocks_, int32_t heads_, int32_t h_)
+      : s(int32_t(u / row_blocks_)), rb(int32_t(u % row_blocks_)),
+        row_blocks(int32_t(row_blocks_)), heads(heads_), h(h_) {}
+  __device__ int64_t sh() const { return int64_t(s) * heads + h; }   // slice * H + head
+  __device__ bool last_of_slice() const { return rb + 1 == row_blocks; }
+  __device__ void next() {
+    if (++rb == row_blocks) {
+      rb = 0;
+      ++s;
+    }
+  }
+};
 
 // Bounded wait that also gives up as soon as another role has aborted; the
 // first role to give up raises the guard word and the abort flag.
