@@ -17,6 +17,7 @@
 // part is output coordinate n (y_n = sum_k R[n][k] x_k).
 #pragma once
 
+#include <cooperative_groups.h>
 #include <cuda_fp16.h>
 
 #include "codec.cuh"
@@ -164,9 +165,12 @@ __device__ __forceinline__ void dense_product(const float* As, float* Bs, const 
 }
 
 // lambda[s][h][n] = sqrt(mean over the first n_cal rows of y_n^2), y = R x
-// (1 where the sum is 0). One block per (slice, head) walks the 64-row tiles
-// in order; each thread sums its own products in double in a fixed order,
-// then the vector groups are added in a fixed order: deterministic.
+// (1 where the sum is 0). One cluster of kDenseCalibCluster blocks per
+// (slice, head); block r of the cluster takes the 64-row tiles r, r + 8, ...
+// Each thread sums its own products in double in a fixed order, the vector
+// groups of a block are then added in a fixed order, and rank 0 adds the
+// blocks' partial sums in rank order, reading them from the other blocks'
+// shared memory (distributed shared memory of the cluster): deterministic.
 struct DenseCalibArgs {
   int64_t n_cal, x_stride_rows;
   int32_t heads;
@@ -177,21 +181,29 @@ struct DenseCalibArgs {
   unsigned* guard;
 };
 
+constexpr int kDenseCalibCluster = 8;
+
 template <int D>
-__global__ void __launch_bounds__(kDenseThreads) dense_calibrate_kernel(const DenseCalibArgs a) {
+__global__ void __cluster_dims__(kDenseCalibCluster, 1, 1) __launch_bounds__(kDenseThreads)
+    dense_calibrate_kernel(const DenseCalibArgs a) {
   using T = DenseTile<D>;
   extern __shared__ __align__(16) uint8_t smem_raw[];
+  __shared__ double part[D];   // this block's column sums
   float* As = reinterpret_cast<float*>(smem_raw);
   float* Bs = reinterpret_cast<float*>(smem_raw + T::kABytes);
+  namespace cg = cooperative_groups;
+  cg::cluster_group cluster = cg::this_cluster();
+  const int rank = static_cast<int>(cluster.block_rank());
   const int tid = threadIdx.x;
-  const int64_t sh = blockIdx.x;
+  const int64_t sh = blockIdx.x / kDenseCalibCluster;
   const int64_t s = sh / a.heads;
   const int h = int(sh % a.heads);
   const uint16_t* hi = a.operand + size_t(sh) * 2 * D * D;
   const uint16_t* lo = hi + size_t(D) * D;
   const int tn = tid % T::NT, tv = tid / T::NT;
   double ss[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-  for (int64_t r0 = 0; r0 < a.n_cal; r0 += kDenseRows) {
+  for (int64_t r0 = int64_t(kDenseRows) * rank; r0 < a.n_cal;
+       r0 += int64_t(kDenseRows) * kDenseCalibCluster) {
     __syncthreads();   // the previous tile's A has been read
     for (int idx = tid; idx < kDenseRows * (D / 8); idx += kDenseThreads) {
       const int v = idx / (D / 8), c8 = idx % (D / 8);
@@ -230,9 +242,18 @@ __global__ void __launch_bounds__(kDenseThreads) dense_calibrate_kernel(const De
   for (int n = tid; n < D; n += kDenseThreads) {
     double t = 0.0;
     for (int g = 0; g < T::TVG; ++g) t += red[g * D + n];
-    if (dbg_ok(sh < a.n_slices * a.heads, a.guard))
-      a.lambda_out[size_t(sh) * D + n] = t == 0.0 ? 1.0f : float(sqrt(t / double(a.n_cal)));
+    part[n] = t;
   }
+  cluster.sync();
+  if (rank == 0) {
+    for (int n = tid; n < D; n += kDenseThreads) {
+      double t = 0.0;
+      for (int q = 0; q < kDenseCalibCluster; ++q) t += cluster.map_shared_rank(part, q)[n];
+      if (dbg_ok(sh < a.n_slices * a.heads, a.guard))
+        a.lambda_out[size_t(sh) * D + n] = t == 0.0 ? 1.0f : float(sqrt(t / double(a.n_cal)));
+    }
+  }
+  cluster.sync();   // the other blocks keep their shared memory until rank 0 is done
 }
 
 }  // namespace srftq

@@ -188,7 +188,8 @@ int launch_dequantize_dense(const DenseCall& c) {
 }
 
 int launch_calibrate_dense(const DenseCalibCall& c) {
-  const int64_t blocks = c.n_slices * c.heads;
+  // one cluster of kDenseCalibCluster blocks per (slice, head)
+  const int64_t blocks = c.n_slices * c.heads * kDenseCalibCluster;
   if (blocks == 0) return SRFTQ_OK;
   if (blocks > INT_MAX) return SRFTQ_ERR_UNSUPPORTED;
   unsigned* guard = Runtime::guard_word();
@@ -199,8 +200,7 @@ int launch_calibrate_dense(const DenseCalibCall& c) {
     constexpr int D = decltype(d_)::value;
     constexpr auto K = dense_calibrate_kernel<D>;
     constexpr int smem = DenseTile<D>::kBytes;
-    int bps = 0;
-    const int rc = prepare_kernel<K>(smem, kDenseThreads, &bps);
+    const int rc = prepare_smem<K>(smem);
     if (rc != SRFTQ_OK) return rc;
     K<<<int(blocks), kDenseThreads, smem, c.stream>>>(a);
     return finish_launch();

@@ -84,6 +84,24 @@ int prepare_kernel(int smem_bytes, int threads, int* blocks_per_sm) {
   return SRFTQ_OK;
 }
 
+// The dynamic shared-memory opt-in alone (for cluster kernels, whose
+// occupancy is not a per-SM block count).
+template <auto K>
+int prepare_smem(int smem_bytes) {
+  static std::atomic<uint64_t> attr_done{0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SRFTQ_ERR_CUDA;
+  const uint64_t bit = 1ull << (dev & 63);
+  if (!(attr_done.load(std::memory_order_acquire) & bit)) {
+    if (smem_bytes > 48 * 1024 &&
+        cudaFuncSetAttribute(K, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes) !=
+            cudaSuccess)
+      return SRFTQ_ERR_CUDA;
+    attr_done.fetch_or(bit, std::memory_order_acq_rel);
+  }
+  return SRFTQ_OK;
+}
+
 // Calls f(Int<BITS>, Int<G>, Int<ROT>) for the run-time configuration.
 template <int D, typename F>
 int dispatch_config(int bits, int group, int rot, F&& f) {
