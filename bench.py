@@ -23,6 +23,7 @@ cpu_baseline  the float64 CPU oracle, as it stands, on a bounded sample.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import math
@@ -57,6 +58,9 @@ def parse_args(argv=None):
     ap.add_argument("--reflectors", type=int, default=None,
                     help="run the workload through the dense-rotation calls with this many "
                          "(>= 1) Householder reflectors on its base rotation")
+    ap.add_argument("--dense", action="store_true",
+                    help="run the workload's base rotation itself (the SRFT / SRHT matrix, "
+                         "no reflectors) through the dense tensor-core calls")
     ap.add_argument("--tokens", type=int, default=None,
                     help="decode_stream_d128: cached tokens per sequence (default 32768; "
                          "smaller captures)")
@@ -121,14 +125,16 @@ def codec_kernel(kind: str, d: int, dense: bool = False) -> str:
 
 def codec_calls(rq, w, desc, signs, seed, dev):
     """(table, (calibrate, quantize, dequantize)) of a workload: the FFT/WHT
-    calls with the sign table, or, when the workload has Householder
-    reflectors, the dense calls with the operand of R = H(v_1)...H(v_k) B."""
+    calls with the sign table, or, when the workload runs dense, the dense
+    calls with the operand of R = H(v_1)...H(v_k) B (k = 0: B itself)."""
     import torch
 
-    if not w.reflectors:
+    if not w.dense:
         return signs, (rq.srftq_calibrate_lambda, rq.srftq_quantize, rq.srftq_dequantize)
-    V = torch.from_numpy(kv_synth.householder_reflectors(w.S, w.H, w.reflectors, w.d,
-                                                         seed=seed)).to(dev)
+    V = None
+    if w.reflectors:
+        V = torch.from_numpy(kv_synth.householder_reflectors(w.S, w.H, w.reflectors, w.d,
+                                                             seed=seed)).to(dev)
     op = rq.dense_operand(rq.householder_rotation(V, signs, rotation=desc.rotation))
     return op, (rq.srftq_calibrate_lambda_dense, rq.srftq_quantize_dense,
                 rq.srftq_dequantize_dense)
@@ -258,11 +264,11 @@ def _num(s):
 
 def oracle_step(w, x16, signs, rot):
     """One oracle pass on a sample: calibrate, quantize, dequantize (with the
-    workload's dense Householder rotation when it has reflectors)."""
+    workload's dense rotation, reflectors or none, when it runs dense)."""
     import oracle
 
     n_cal = min(w.n_cal, x16.shape[1])
-    if w.reflectors:
+    if w.dense:
         V = kv_synth.householder_reflectors(1, w.H, w.reflectors, w.d, seed=1)
         R = oracle.householder_rotations(V, signs, rot)
         lam = oracle.calibrate_lambda_dense(x16, R, n_cal).astype(np.float32)
@@ -394,7 +400,6 @@ def _max_over_ranks(pg, dev, ms):
 
 def workload(args):
     """The named workload, cut to its first --slices slices if given."""
-    import dataclasses
 
     w = kv_synth.WORKLOADS[args.workload]
     if args.slices is not None:
@@ -405,6 +410,11 @@ def workload(args):
         if args.workload == "decode_stream_d128" or w.d not in (64, 128, 256) or args.reflectors < 1:
             raise SystemExit("--reflectors needs a codec workload with d in {64, 128, 256}")
         w = dataclasses.replace(w, reflectors=args.reflectors, name=w.name + "+dense")
+    if getattr(args, "dense", False):
+        if args.workload == "decode_stream_d128" or w.d not in (64, 128, 256) or w.reflectors:
+            raise SystemExit("--dense needs a codec workload with d in {64, 128, 256} and no "
+                             "reflectors")
+        w = dataclasses.replace(w, dense_base=True, name=w.name + "+dense0")
     if getattr(args, "tokens", None) is not None:
         if args.workload != "decode_stream_d128" or not 512 <= args.tokens <= 32768:
             raise SystemExit("--tokens applies to decode_stream_d128, 512..32768")
@@ -484,14 +494,14 @@ def run_ours(args):
     dom = "quantize" if q_avg >= d_avg else "dequantize"
     dom_ms = max(q_avg, d_avg)
     achieved = bytes_launch / (dom_ms / 1e3) / 1e9
-    kname = codec_kernel(dom, w.d, dense=w.reflectors > 0)
+    kname = codec_kernel(dom, w.d, dense=w.dense)
     roof = {"bound": "hbm", "kernel": kname, "achieved": achieved, "peak": peak,
             "unit": "GB/s", "frac": achieved / peak,
             "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured"
             else "fallback 6.65 TB/s",
             "algorithmic_bytes_per_launch": bytes_launch,
             "traffic": read_traffic(kname, w.name)}
-    if w.reflectors:
+    if w.dense:
         roof = dense_roofline(w, dom, dom_ms, kname)
 
     e2e = None
@@ -573,8 +583,8 @@ def _codec_figures(rq, w, rot, dev, iters):
            "quantize_frac": b / q_ms / 1e6 / peak,
            "dequantize_ms": d_ms, "dequantize_GBps": b / d_ms / 1e6,
            "dequantize_frac": b / d_ms / 1e6 / peak,
-           "kernels": [codec_kernel("quantize", w.d, w.reflectors > 0),
-                       codec_kernel("dequantize", w.d, w.reflectors > 0)],
+           "kernels": [codec_kernel("quantize", w.d, w.dense),
+                       codec_kernel("dequantize", w.d, w.dense)],
            "rel_l2_error": round_trip_error(x, xhat)}
     del x, codes, scales, xhat
     torch.cuda.empty_cache()
@@ -641,7 +651,9 @@ def parity_report():
 def other_configs(rq, dev, iters=50):
     """The other workloads' kernels at full size, measured after the headline
     and outside its timed region: long-context int8 (SRFT and SRHT side by
-    side, with their round-trip errors), the Gemma-shaped d = 256 cache and
+    side, with their round-trip errors), the Gemma-shaped d = 256 cache, the
+    Householder workload, the headline shape's SRFT as a dense tensor-core
+    product (the matrix itself, beside the FFT kernels of the headline) and
     the fused decode attention of one decode-stream layer."""
     out = {}
     lc = kv_synth.WORKLOADS["longctx_int8_d128"]
@@ -658,6 +670,9 @@ def other_configs(rq, dev, iters=50):
     for kind, f in flops.items():
         out["householder_d256"][f"{kind}_TFLOPs"] = f / out["householder_d256"][f"{kind}_ms"] / 1e9
     out["householder_d256"]["flops_per_launch"] = flops
+    qd = dataclasses.replace(kv_synth.WORKLOADS["qwen_like_d128"], dense_base=True,
+                             name="qwen_like_d128+dense0")
+    out["qwen_like_d128_srft_tensor_core"] = _codec_figures(rq, qd, 0, dev, iters)
     out["decode_stream_d128_fused_attention"] = _attention_figures(rq, dev, iters)
     rep = parity_report()
     if rep is not None:

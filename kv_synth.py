@@ -43,6 +43,14 @@ class Workload:
     rotations: tuple = (0,)
     note: str = ""
     reflectors: int = 0   # Householder reflectors on the base rotation (dense codec)
+    dense_base: bool = False   # the base rotation itself as a dense product (k = 0)
+
+    @property
+    def dense(self) -> bool:
+        """The rotation runs as a dense d x d product (the tensor-core codec):
+        always with reflectors, and for the plain SRFT / SRHT matrix when
+        dense_base is set."""
+        return self.reflectors > 0 or self.dense_base
 
     @property
     def vectors(self) -> int:

@@ -301,3 +301,29 @@ def test_dense_dequantiser_extreme_magnitudes(bits):
         _assert_dequant_scale_free(
             _np16(xhat), deq["xhat64"],
             f"b{bits} lambda {lam_lo:g}..{lam_hi:g} sigma 2^{e_lo:g}..2^{e_hi:g}")
+
+
+@pytest.mark.parametrize("d,bits,group,kind", [(128, 4, 16, 0), (128, 8, 16, 1), (256, 4, 32, 0),
+                                               (64, 4, 8, 0)])
+def test_dense_form_of_the_base_rotation_is_the_fft_codec(d, bits, group, kind):
+    """The tensor-core codec run with the signed SRFT / SRHT matrix itself
+    (k = 0, built on the GPU) against the FFT codec's oracle
+    (oracle.quantize / dequantize, which rotate by the transform): the same
+    codes and scales within the dense bands, and the oracle's dequantised
+    values from the oracle's codes."""
+    rng = np.random.default_rng(d + bits + kind)
+    S, N, H = 2, 300, 3
+    x16, signs, _, _ = _case(rng, S, N, H, d, 1, kind)
+    lam = oracle.calibrate_lambda(x16, signs, 64, kind).astype(np.float32)
+    op = rq.dense_operand(rq.householder_rotation(None, _t(signs), rotation=kind))
+    codes, scales = rq.quantize_dense(_t(x16), op, _t(lam), group, bits)
+    ref = oracle.quantize(x16, signs, lam, group, bits, kind)
+    parity.assert_clean(parity.check_codes(ref, codes.cpu().numpy(), _np16(scales), bits, group,
+                                           parity.DENSE_SCALE_BAND,
+                                           parity.dense_code_band(ref, lam, group)),
+                        f"dense base d{d} b{bits} rot{kind}")
+    xhat = rq.dequantize_dense(_t(ref["codes"]), _t(ref["scales"].view(np.float16)), op, _t(lam),
+                               d, group, bits)
+    deq = oracle.dequantize(ref["codes"], ref["scales"], signs, lam, d, group, bits, kind)
+    parity.assert_clean(parity.check_dequant(_np16(xhat), deq["bits"]),
+                        f"dense base d{d} b{bits} rot{kind} dequant")
