@@ -117,9 +117,12 @@ def test_dense_codec_matches_oracle(d, bits, kind):
         g *= 2
 
 
-@pytest.mark.parametrize("d", [64, 256])
-@pytest.mark.parametrize("n_cal", [1, 63, 64, 200])
+@pytest.mark.parametrize("d", [64, 128, 256])
+@pytest.mark.parametrize("n_cal", [1, 63, 64, 200, 1100])
 def test_dense_calibration_matches_oracle(d, n_cal):
+    """One cluster per (slice, head) whose blocks take every 8th 64-row
+    tile: fewer rows than blocks, a partial tile, and (1100 rows) more tiles
+    than blocks."""
     rng = np.random.default_rng(d + n_cal)
     x16, signs, V, R = _case(rng, 2, max(n_cal, 8), 3, d, d // 2, 0)
     op = rq.dense_operand(_t(R.astype(np.float32)))
