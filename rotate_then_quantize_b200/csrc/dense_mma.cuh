@@ -19,15 +19,18 @@
 // of each row).
 //
 // Warp roles (128 + 128 E threads, E = 2):
-//   warp 0      A producer: TMA loads of x tiles (NST stages; 128-byte
-//               swizzled K-major rows, rows past N zero-filled)
+//   warp 0      A producer: TMA loads of x tiles (128-byte swizzled K-major
+//               rows, rows past N zero-filled): whole 128-row blocks in NST
+//               stages for d <= 128, 64-wide K pieces through a ring of
+//               NST piece slots for d = 256
 //   warp 1      tensor-memory allocation and the MMA issue (one lane)
 //   warp 2      B producer: TMA loads of the operand. d <= 128: the whole
 //               operand (hi and lo) stays resident and is reloaded when the
 //               (slice, head) changes, after the MMAs that read the old one
 //               have completed. d = 256 (256 KB of operand): streamed from
 //               L2 in chunks of one 64-wide K piece of hi or lo, through a
-//               ring of slots, in the order the MMAs read them.
+//               ring of five slots, in the order the MMAs read them (piece
+//               by piece, hi then lo).
 //   warp 3      idle
 //   warps 4..   epilogue, E groups of four warps; group g takes the blocks
 //               g, g + E, ... of the range; warp 4 + 4g + q reads TMEM lanes
@@ -50,17 +53,20 @@ struct DenseMma {
   static constexpr int kPieces = D / 64;                    // 128-byte K pieces
   static constexpr int kAPiece = 128 * 128;                 // 128 rows x 128 B
   static constexpr int kABytes = kPieces * kAPiece;         // one A stage
-  static constexpr int kNST = D == 256 ? 2 : (D == 128 ? 3 : 4);
+  // A stages: whole blocks (d <= 128), or single K pieces of a block when
+  // the operand is streamed (d = 256), which leaves room for a deeper ring
+  static constexpr int kNST = kStreamB ? 3 : (D == 128 ? 3 : 4);
+  static constexpr int kAStage = kStreamB ? kAPiece : kABytes;
   static constexpr int kBPiece = D * 128;                   // d rows x 128 B
   static constexpr int kBChunks = 2 * kPieces;              // (part, piece) chunks
-  static constexpr int kBSlots = kStreamB ? 2 : kBChunks;
+  static constexpr int kBSlots = kStreamB ? 5 : kBChunks;
   static constexpr int kBBytes = kBSlots * kBPiece;
   static constexpr int kAcc = D == 256 ? 2 : 4;             // TMEM accumulators
   static constexpr uint32_t kTmemCols = kAcc * D <= 256 ? 256u : 512u;
   static constexpr int kEpi = EPI;
   static constexpr int kThreads = 128 + 128 * EPI;
   static constexpr int kAOff = 0;
-  static constexpr int kBOff = kNST * kABytes;
+  static constexpr int kBOff = kNST * kAStage;
   static constexpr int kTabOff = kBOff + kBBytes;           // 1 / lambda, per epilogue warp
   static constexpr int kBarOff = kTabOff + 4 * EPI * D * 4;
   // full, empty per A stage; bfull, bempty per B slot; tfull, tempty per
@@ -188,26 +194,39 @@ __global__ void __launch_bounds__(DenseMma<D, EPI>::kThreads, 1)
   if (warp == 0) {
     // ---------------- A producer ----------------
     if (lane == 0) {
-      int i = 0;
+      // stage u = block u (whole blocks) or piece u of the CTA's sequence
+      int u = 0;
+      bool ok = true;
       BlockWalk w = w0;
-      for (; i < n; ++i, w.next()) {
-        const int st = i % L::kNST;
-        if (i >= L::kNST &&
-            !wait_or_abort(&empty[st], ((i / L::kNST) & 1) ^ 1, abort_flag, a.guard))
-          break;
+      for (int i = 0; i < n && ok; ++i, w.next()) {
         const int r0 = int(w.rb * 128);
         const int s = int(w.s), h = hh;
-        if (!dbg_ok(s < a.n_slices && r0 < a.n_rows, a.guard)) {
-          mbar_arrive(&full[st]);   // debug build: no copy, the phase completes empty
-          continue;
-        }
-        mbar_arrive_expect_tx(&full[st], L::kABytes);
+        const bool in = dbg_ok(s < a.n_slices && r0 < a.n_rows, a.guard);
+        for (int p0 = 0; p0 < L::kPieces; p0 += L::kStreamB ? 1 : L::kPieces) {
+          const int st = u % L::kNST;
+          if (u >= L::kNST &&
+              !wait_or_abort(&empty[st], ((u / L::kNST) & 1) ^ 1, abort_flag, a.guard)) {
+            ok = false;
+            break;
+          }
+          ++u;
+          if (!in) {
+            mbar_arrive(&full[st]);   // debug build: no copy, the phase completes empty
+            continue;
+          }
+          mbar_arrive_expect_tx(&full[st], L::kAStage);
+          if constexpr (L::kStreamB) {
+            tma_load_4d(As + st * L::kAStage, &tm_x, &full[st], 64 * p0, h, r0, s);
+          } else {
 #pragma unroll
-        for (int p = 0; p < L::kPieces; ++p)
-          tma_load_4d(As + st * L::kABytes + p * L::kAPiece, &tm_x, &full[st], 64 * p, h, r0, s);
+            for (int p = 0; p < L::kPieces; ++p)
+              tma_load_4d(As + st * L::kAStage + p * L::kAPiece, &tm_x, &full[st], 64 * p, h,
+                          r0, s);
+          }
+        }
       }
       // drain: every issued stage lands before the CTA can exit
-      for (int k = (i > L::kNST ? i - L::kNST : 0); k < i; ++k)
+      for (int k = (u > L::kNST ? u - L::kNST : 0); k < u; ++k)
         (void)mbar_wait_bounded(&full[k % L::kNST], (k / L::kNST) & 1);
     }
   } else if (warp == 2) {
@@ -238,8 +257,8 @@ __global__ void __launch_bounds__(DenseMma<D, EPI>::kThreads, 1)
         BlockWalk w = w0;
         for (int i = 0; i < n && ok; ++i, w.next()) {
           const int64_t sh = w.sh();
-          for (int q = 0; q < 2 && ok; ++q)
-            for (int p = 0; p < L::kPieces; ++p) {
+          for (int p = 0; p < L::kPieces && ok; ++p)
+            for (int q = 0; q < 2; ++q) {
               const int slot = c % L::kBSlots;
               if (c >= L::kBSlots &&
                   !wait_or_abort(&bempty[slot], ((c / L::kBSlots) & 1) ^ 1, abort_flag,
@@ -260,17 +279,55 @@ __global__ void __launch_bounds__(DenseMma<D, EPI>::kThreads, 1)
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
-      int run = -1, c = 0, i = 0;
+      int run = -1, c = 0, i = 0, u = 0;
       int64_t prev = -1;
       bool ok = true;
       BlockWalk w = w0;
       for (; i < n && ok; ++i, w.next()) {
-        const int st = i % L::kNST, acc = i % L::kAcc;
+        const int acc = i % L::kAcc;
         const int64_t sh = w.sh();
-        if (!wait_or_abort(&full[st], (i / L::kNST) & 1, abort_flag, a.guard)) break;
         if (i >= L::kAcc &&
             !wait_or_abort(&tempty[acc], ((i / L::kAcc) & 1) ^ 1, abort_flag, a.guard))
           break;
+        const uint32_t d = tmem_base + uint32_t(acc) * uint32_t(D);
+        if constexpr (L::kStreamB) {
+          // piece by piece: A piece p with the hi and lo chunks of piece p
+          int k = 0;
+          for (int p = 0; p < L::kPieces && ok; ++p) {
+            const int st = u % L::kNST;
+            if (!wait_or_abort(&full[st], (u / L::kNST) & 1, abort_flag, a.guard)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t sa = smem_addr(As + st * L::kAStage);
+            for (int q = 0; q < 2; ++q) {
+              const int slot = c % L::kBSlots;
+              if (!wait_or_abort(&bfull[slot], (c / L::kBSlots) & 1, abort_flag, a.guard)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              const uint32_t sb = smem_addr(Bs + slot * L::kBPiece);
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                tc_mma_f16(d, sw128_desc(sa + 32 * j), sw128_desc(sb + 32 * j), L::kIdesc,
+                           k > 0 ? 1u : 0u);
+                ++k;
+              }
+              tc_commit(&bempty[slot]);
+              ++c;
+            }
+            if (!ok) break;
+            tc_commit(&empty[st]);
+            ++u;
+          }
+          if (!ok) break;
+          tc_commit(&tfull[acc]);
+          continue;
+        }
+        const int st = i % L::kNST;
+        if (!wait_or_abort(&full[st], (i / L::kNST) & 1, abort_flag, a.guard)) break;
         if constexpr (!L::kStreamB) {
           if (sh != prev) {
             ++run;
@@ -279,24 +336,11 @@ __global__ void __launch_bounds__(DenseMma<D, EPI>::kThreads, 1)
           }
         }
         tc_fence_after();
-        const uint32_t sa = smem_addr(As + st * L::kABytes);
-        const uint32_t d = tmem_base + uint32_t(acc) * uint32_t(D);
+        const uint32_t sa = smem_addr(As + st * L::kAStage);
         int k = 0;
-        for (int q = 0; q < 2 && ok; ++q)
+        for (int q = 0; q < 2; ++q)
           for (int p = 0; p < L::kPieces; ++p) {
-            uint32_t sb;
-            int slot = 0;
-            if constexpr (L::kStreamB) {
-              slot = c % L::kBSlots;
-              if (!wait_or_abort(&bfull[slot], (c / L::kBSlots) & 1, abort_flag, a.guard)) {
-                ok = false;
-                break;
-              }
-              tc_fence_after();
-              sb = smem_addr(Bs + slot * L::kBPiece);
-            } else {
-              sb = smem_addr(Bs + (q * L::kPieces + p) * L::kBPiece);
-            }
+            const uint32_t sb = smem_addr(Bs + (q * L::kPieces + p) * L::kBPiece);
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
               const uint64_t ad = sw128_desc(sa + p * L::kAPiece + 32 * j);
@@ -304,17 +348,10 @@ __global__ void __launch_bounds__(DenseMma<D, EPI>::kThreads, 1)
               tc_mma_f16(d, ad, bd, L::kIdesc, k > 0 ? 1u : 0u);
               ++k;
             }
-            if constexpr (L::kStreamB) {
-              tc_commit(&bempty[slot]);
-              ++c;
-            }
           }
-        if (!ok) break;
         tc_commit(&empty[st]);
         tc_commit(&tfull[acc]);
-        if constexpr (!L::kStreamB) {
-          if (i + 1 == n || w.last_of_slice()) tc_commit(&bempty[0]);
-        }
+        if (i + 1 == n || w.last_of_slice()) tc_commit(&bempty[0]);
       }
       // drain: every MMA issued (a block cut short by an abort included)
       // completes before TMEM is freed
