@@ -125,11 +125,6 @@ struct DenseTile {
   static_assert(TV >= 1 && TVG * TV == kDenseRows, "tile shape");
 };
 
-// R[n][k] = hi + lo of the operand, as float32.
-__device__ __forceinline__ float op_value(const uint16_t* hi, const uint16_t* lo, size_t i) {
-  return __half2float(__ushort_as_half(hi[i])) + __half2float(__ushort_as_half(lo[i]));
-}
-
 // acc[i][c] = sum_k A[v_i][k] * Bt[k][n_c] over all K (y = R x), where the
 // staged chunk Bt[kk][n] = R[n][k0 + kk]. A is already in shared memory.
 template <int D>
@@ -143,10 +138,33 @@ __device__ __forceinline__ void dense_product(const float* As, float* Bs, const 
 #pragma unroll
     for (int c = 0; c < 8; ++c) acc[i][c] = 0.0f;
   for (int k0 = 0; k0 < D; k0 += kDenseKC) {
+    // 16-byte loads of 8 consecutive K values of one row of hi and of lo,
+    // all issued before any is used (each thread has D / 64 of them per
+    // part), then R = hi + lo stored transposed
+    constexpr int kPer = D * (kDenseKC / 8) / kDenseThreads;
+    static_assert(kPer >= 1 && kPer * kDenseThreads == D * (kDenseKC / 8), "staging split");
+    uint4 wh[kPer], wl[kPer];
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      const int t = tid + u * kDenseThreads;
+      const size_t off = size_t(t / (kDenseKC / 8)) * D + k0 + 8 * (t % (kDenseKC / 8));
+      wh[u] = *reinterpret_cast<const uint4*>(hi + off);
+      wl[u] = *reinterpret_cast<const uint4*>(lo + off);
+    }
     __syncthreads();   // the previous chunk has been read
-    for (int idx = tid; idx < D * kDenseKC; idx += kDenseThreads) {
-      const int n = idx / kDenseKC, kk = idx % kDenseKC;
-      Bs[kk * T::BS + n] = op_value(hi, lo, size_t(n) * D + k0 + kk);
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      const int t = tid + u * kDenseThreads;
+      const int n = t / (kDenseKC / 8), c = t % (kDenseKC / 8);
+      const uint32_t hw[4] = {wh[u].x, wh[u].y, wh[u].z, wh[u].w};
+      const uint32_t lw[4] = {wl[u].x, wl[u].y, wl[u].z, wl[u].w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 h2 = __half22float2(*reinterpret_cast<const __half2*>(&hw[e]));
+        const float2 l2 = __half22float2(*reinterpret_cast<const __half2*>(&lw[e]));
+        Bs[(8 * c + 2 * e) * T::BS + n] = h2.x + l2.x;
+        Bs[(8 * c + 2 * e + 1) * T::BS + n] = h2.y + l2.y;
+      }
     }
     __syncthreads();
 #pragma unroll 4
@@ -205,6 +223,7 @@ __global__ void __cluster_dims__(kDenseCalibCluster, 1, 1) __launch_bounds__(kDe
   for (int64_t r0 = int64_t(kDenseRows) * rank; r0 < a.n_cal;
        r0 += int64_t(kDenseRows) * kDenseCalibCluster) {
     __syncthreads();   // the previous tile's A has been read
+#pragma unroll
     for (int idx = tid; idx < kDenseRows * (D / 8); idx += kDenseThreads) {
       const int v = idx / (D / 8), c8 = idx % (D / 8);
       const int64_t r = r0 + v;
