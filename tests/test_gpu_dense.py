@@ -330,3 +330,21 @@ def test_dense_form_of_the_base_rotation_is_the_fft_codec(d, bits, group, kind):
     deq = oracle.dequantize(ref["codes"], ref["scales"], signs, lam, d, group, bits, kind)
     parity.assert_clean(parity.check_dequant(_np16(xhat), deq["bits"]),
                         f"dense base d{d} b{bits} rot{kind} dequant")
+
+
+@pytest.mark.parametrize("d,bits,group,kind", [(128, 4, 16, 0), (256, 4, 32, 1)])
+def test_dense_base_codes_decode_with_the_fft_dequantiser(d, bits, group, kind):
+    """The tensor-core quantiser run with the SRFT / SRHT matrix itself and the
+    FFT / WHT dequantiser implement one codec: codes and scales from the first
+    decode with the second to the oracle's dequantisation of those codes."""
+    rng = np.random.default_rng(5 * d + bits + kind)
+    S, N, H = 2, 200, 2
+    x16, signs, _, _ = _case(rng, S, N, H, d, 1, kind)
+    lam = oracle.calibrate_lambda(x16, signs, 64, kind).astype(np.float32)
+    op = rq.dense_operand(rq.householder_rotation(None, _t(signs), rotation=kind))
+    codes, scales = rq.quantize_dense(_t(x16), op, _t(lam), group, bits)
+    xhat = rq.dequantize(codes, scales, _t(signs), _t(lam), d, group=group, bits=bits,
+                         rotation=kind)
+    deq = oracle.dequantize(codes.cpu().numpy(), _np16(scales), signs, lam, d, group, bits, kind)
+    parity.assert_clean(parity.check_dequant(_np16(xhat), deq["bits"]),
+                        f"dense-quantised, FFT-dequantised d{d} rot{kind}")
