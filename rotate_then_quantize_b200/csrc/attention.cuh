@@ -222,11 +222,62 @@ struct AttnLayout {
   static constexpr int kSm = kMx + 4 * NQ;                          // float [NQ]
   static constexpr int kWm = kSm + 4 * NQ;                          // float [NW][NQ]
   static constexpr int kWl = kWm + 4 * NQ * kAttnWarps;             // float [NW][NQ]
-  static constexpr int kStages = (kWl + 4 * NQ * kAttnWarps + 127) / 128 * 128;
+  static constexpr int kQe = kWl + 4 * NQ * kAttnWarps;             // int [8]: piece exponents
+  static constexpr int kQm = kQe + 4 * 8;                           // float [8]: 2^-(E + 16)
+  static constexpr int kQsum = kQm + 4 * 8;                         // int [3][8]: piece sums
+  static constexpr int kStages = (kQsum + 4 * 24 + 127) / 128 * 128;
   static constexpr int kBytes = kStages + kAttnWarps * kAttnStages * kStage;
   static_assert(kStage >= NQ * D * 4, "a warp's partial sums fit in its first stage");
   __device__ static constexpr int swz(int r) { return (r * CB / 128) % PPT; }
 };
+
+// Integer tensor-core scores (int4 keys, one query per KV head, G >= 16).
+//
+// score_t = sum_j sigma_{t,g(j)} q_j c_{t,j} is a contraction over the 128
+// coordinates, with sigma constant on each group. Each 16-coordinate
+// sub-group m of the query gets its own exponent E_m (|q_j| 2^E_m < 64 on
+// it) and the integer Q_j = rint(q_j 2^(E_m + 16)) = B0 2^16 + B1 2^8 + B2
+// in balanced base-256 digits (each a signed byte). A warp-level
+// mma.m16n8k32 (u8 x s8 -> s32) then gives, for 16 tokens at a time, the
+// exact integers D_p[t][m] = sum_{j in m} c_{t,j} B_p[j]: the codes enter
+// as offset-binary bytes u = c + 8 (one AND-XOR per four codes), and the
+// accumulator starts at -8 sum_{j in m} B_p[j], which removes the offset
+// exactly. Column m of n-tile p holds digit p on sub-group m only (a
+// block-diagonal B), so every (token, sub-group) partial lands in one
+// register of one lane. D_0 2^16 + D_1 2^8 + D_2 = sum c Q fits in int32
+// (|c| <= 8, |B0| <= 65, |B1|, |B2| <= 128 over 16 coordinates), is
+// converted once, and is scaled by sigma 2^-(E_m + 16). The query's
+// representation error is at most 2^-22 of its sub-group maximum; the
+// products and sums are exact until that one conversion.
+
+// k-order of the fragments: for k-step ks, lane (row group g, thread t)
+// holds word 4t + ks of its token rows; the low nibbles of the word's
+// bytes (coordinates 8w + 2i) are k = 4t + i, the high nibbles
+// (coordinates 8w + 2i + 1) are k = 4t + 16 + i.
+__device__ __forceinline__ void imma_u8s8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                          uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%0, %1, %2, %3};"
+      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Q = rint(q 2^(e + 16)) split into balanced base-256 digits B0 2^16 + B1 2^8 + B2.
+__device__ __forceinline__ void query_digits(float q, int e, int (&b)[3]) {
+  const int Q = __float2int_rn(ldexpf(q, e + 16));
+  b[2] = ((Q + 128) & 255) - 128;
+  const int q1 = (Q - b[2]) >> 8;
+  b[1] = ((q1 + 128) & 255) - 128;
+  b[0] = (q1 - b[1]) >> 8;
+}
+
+#ifndef SRFTQ_ATTN_INT_SCORES
+#define SRFTQ_ATTN_INT_SCORES 1   // 0: every case on the per-lane float32 scores
+#endif
+template <int BITS, int G, int NQ>
+__host__ __device__ constexpr bool attn_int_scores() {
+  return SRFTQ_ATTN_INT_SCORES && BITS == 4 && NQ == 1 && G >= 16;
+}
 
 // CTAs per SM the register budget is sized for (128, 168 or 255 registers).
 #ifndef SRFTQ_ATTN_MINB
@@ -270,10 +321,73 @@ __global__ void __cluster_dims__(kAttnSplit, 1, 1)
   const uint32_t wst_a = smem_addr(wst);
   const uint32_t qs_a = smem_addr(qs);
 
-  // int4 keys decode their odd coordinates 16 times too large (decode8)
+  // int4 keys decode their odd coordinates 16 times too large (decode8);
+  // the integer scores take the codes exactly
+  constexpr bool kInt = attn_int_scores<BITS, G, NQ>();
   constexpr float kOdd = BITS == 4 ? 0.0625f : 1.0f;
-  for (int i = tid; i < NQ * D; i += NW * 32) qs[i] = (i & 1) ? qo[i] * kOdd : qo[i];
+  for (int i = tid; i < NQ * D; i += NW * 32) qs[i] = (!kInt && (i & 1)) ? qo[i] * kOdd : qo[i];
   __syncthreads();
+
+  // integer scores: per sub-group exponent, multiplier and digit sums, then
+  // this lane's B fragments (bq[ks][p]: digit p, k-step ks) and the
+  // accumulator start -8 sum B_p for its columns 2t, 2t + 1
+  const int gq = lane >> 2, tq = lane & 3;
+  uint32_t bq[kInt ? 4 : 1][3][2];
+  int cinit[3][2];
+  float qmul[2];
+  if constexpr (kInt) {
+    int* qe = reinterpret_cast<int*>(smem + L::kQe);
+    float* qm = reinterpret_cast<float*>(smem + L::kQm);
+    int* qsum = reinterpret_cast<int*>(smem + L::kQsum);
+    if (tid < 8) {
+      float amax = 0.0f;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) amax = fmaxf(amax, fabsf(qs[16 * tid + j]));
+      // a non-finite query gives NaN scores, as float32 arithmetic would
+      const bool fin = amax <= 3.402823466e38f;
+      const int e = (amax > 0.0f && fin) ? 5 - ilogbf(amax) : 0;
+      int sum[3] = {0, 0, 0};
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        int b[3];
+        query_digits(fin ? qs[16 * tid + j] : 0.0f, e, b);
+        sum[0] += b[0];
+        sum[1] += b[1];
+        sum[2] += b[2];
+      }
+      qe[tid] = e;
+      qm[tid] = fin ? ldexpf(1.0f, -(e + 16)) : __int_as_float(0x7fc00000);
+#pragma unroll
+      for (int p = 0; p < 3; ++p) qsum[8 * p + tid] = sum[p];
+    }
+    __syncthreads();
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks) {
+      const int w = 4 * tq + ks;          // code word (8 coordinates) of this k-step
+      const bool on = (w >> 1) == gq;     // column gq is sub-group w / 2
+      const int e = qe[w >> 1];
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t r[3] = {0u, 0u, 0u};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          int b[3];
+          const float qv = qs[8 * w + 2 * i + hh];
+          query_digits(on && qv == qv && fabsf(qv) <= 3.402823466e38f ? qv : 0.0f, e, b);
+#pragma unroll
+          for (int p = 0; p < 3; ++p) r[p] |= uint32_t(b[p] & 255) << (8 * i);
+        }
+#pragma unroll
+        for (int p = 0; p < 3; ++p) bq[ks][p][hh] = r[p];
+      }
+    }
+#pragma unroll
+    for (int p = 0; p < 3; ++p)
+#pragma unroll
+      for (int jj = 0; jj < 2; ++jj) cinit[p][jj] = -8 * qsum[8 * p + 2 * tq + jj];
+    qmul[0] = qm[2 * tq];
+    qmul[1] = qm[2 * tq + 1];
+  }
 
   // this CTA's tokens; warp w takes the 32-token chunks w, w + NW, ...
   const int64_t per = (a.n_ctx + kAttnSplit - 1) / kAttnSplit;
@@ -354,9 +468,67 @@ __global__ void __cluster_dims__(kAttnSplit, 1, 1)
     const int nt = int(t_end - t0 < 32 ? t_end - t0 : 32);
     const uint8_t* st = wst + (c % NS) * L::kStage;
 
-    // score of token t0 + lane (log2 units; -inf past the end)
+    // score of token t0 + lane (log2 units; -inf past the end); with integer
+    // scores, of this lane's own token 16 (t >> 1) + 8 (t & 1) + g
     float s[NQ];
-    if (lane < nt) {
+    if constexpr (kInt) {
+      float srow[2][2];   // [16-token tile][row g, row g + 8]
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt) {
+        int acc[3][4];
+#pragma unroll
+        for (int p = 0; p < 3; ++p) {
+          acc[p][0] = cinit[p][0];
+          acc[p][1] = cinit[p][1];
+          acc[p][2] = cinit[p][0];
+          acc[p][3] = cinit[p][1];
+        }
+        const int r0 = 16 * mt + gq, r1 = r0 + 8;
+        const uint4 u0 =
+            *reinterpret_cast<const uint4*>(st + L::KC + r0 * CB + ((tq ^ L::swz(r0)) * 16));
+        const uint4 u1 =
+            *reinterpret_cast<const uint4*>(st + L::KC + r1 * CB + ((tq ^ L::swz(r1)) * 16));
+        const uint32_t w0[4] = {u0.x, u0.y, u0.z, u0.w}, w1[4] = {u1.x, u1.y, u1.z, u1.w};
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+          const uint32_t a0 = (w0[ks] & 0x0F0F0F0Fu) ^ 0x08080808u;
+          const uint32_t a1 = (w1[ks] & 0x0F0F0F0Fu) ^ 0x08080808u;
+          const uint32_t a2 = ((w0[ks] >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u;
+          const uint32_t a3 = ((w1[ks] >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u;
+#pragma unroll
+          for (int p = 0; p < 3; ++p)
+            imma_u8s8(acc[p], a0, a1, a2, a3, bq[ks][p][0], bq[ks][p][1]);
+        }
+#pragma unroll
+        for (int hr = 0; hr < 2; ++hr) {
+          const uint8_t* ksr = st + L::KS + (r0 + 8 * hr) * SBS;
+          float sa, sb;
+          if constexpr (G == 16) {
+            const uint32_t sp = *reinterpret_cast<const uint32_t*>(ksr + 4 * tq);
+            sa = __half2float(__ushort_as_half(uint16_t(sp)));
+            sb = __half2float(__ushort_as_half(uint16_t(sp >> 16)));
+          } else {
+            sa = sb = __half2float(*reinterpret_cast<const __half*>(ksr + 2 * ((32 * tq) / G)));
+          }
+          float f[2];
+#pragma unroll
+          for (int jj = 0; jj < 2; ++jj)
+            f[jj] = float(acc[0][2 * hr + jj] * 65536 + acc[1][2 * hr + jj] * 256 +
+                          acc[2][2 * hr + jj]) * qmul[jj];
+          srow[mt][hr] = fmaf(sa, f[0], sb * f[1]);
+        }
+      }
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+        for (int hr = 0; hr < 2; ++hr) {
+          srow[mt][hr] += __shfl_xor_sync(0xffffffffu, srow[mt][hr], 1);
+          srow[mt][hr] += __shfl_xor_sync(0xffffffffu, srow[mt][hr], 2);
+        }
+      const float own = (tq >> 1) ? ((tq & 1) ? srow[1][1] : srow[1][0])
+                                  : ((tq & 1) ? srow[0][1] : srow[0][0]);
+      s[0] = 16 * (tq >> 1) + 8 * (tq & 1) + gq < nt ? own : -INFINITY;
+    } else if (lane < nt) {
       uint32_t sw[(NG + 1) / 2];
       const uint8_t* ksr = st + L::KS + lane * SBS;
       if constexpr (SB >= 16) {
@@ -423,6 +595,9 @@ __global__ void __cluster_dims__(kAttnSplit, 1, 1)
       l[g] = fmaf(l[g], alpha[g], p[g]);
       m[g] = mn;
     }
+    // integer scores: token i's weight moves to lane i, where the value
+    // phase takes it from
+    if constexpr (kInt) p[0] = __shfl_sync(0xffffffffu, p[0], 4 * (lane & 7) + (lane >> 3));
     // values: rescale, then p_i sigma c_i for tokens vt0, vt0 + TPI, ...
     // (a token past the end decodes with scale 0 and has p = 0)
 #pragma unroll

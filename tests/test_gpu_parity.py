@@ -562,7 +562,8 @@ def _attn_case(rng, rows, H, d, group, bits, rot, outliers=0.0):
 
 @pytest.mark.parametrize("n_ctx", [1, 5, 128, 129, 1000])
 @pytest.mark.parametrize("q_per_kv", [1, 2, 8])
-@pytest.mark.parametrize("bits,group,rot", [(4, 16, 0), (8, 32, 1), (4, 128, 1)])
+@pytest.mark.parametrize("bits,group,rot", [(4, 16, 0), (8, 32, 1), (4, 128, 1), (4, 32, 0),
+                                            (4, 64, 1)])
 def test_decode_attention_matches_oracle(n_ctx, q_per_kv, bits, group, rot):
     """Token counts below the cluster's 8 CTAs (empty CTAs), ragged and
     exact tiles; grouped queries; both rotations. The GPU path is float32
