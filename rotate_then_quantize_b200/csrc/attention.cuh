@@ -225,7 +225,8 @@ struct AttnLayout {
   static constexpr int kQe = kWl + 4 * NQ * kAttnWarps;             // int [8]: piece exponents
   static constexpr int kQm = kQe + 4 * 8;                           // float [8]: 2^-(E + 16)
   static constexpr int kQsum = kQm + 4 * 8;                         // int [3][8]: piece sums
-  static constexpr int kStages = (kQsum + 4 * 24 + 127) / 128 * 128;
+  static constexpr int kBtab = (kQsum + 4 * 24 + 15) / 16 * 16;     // uint2 [4][3][32]: B fragments
+  static constexpr int kStages = (kBtab + 8 * 4 * 3 * 32 + 127) / 128 * 128;
   static constexpr int kBytes = kStages + kAttnWarps * kAttnStages * kStage;
   static_assert(kStage >= NQ * D * 4, "a warp's partial sums fit in its first stage");
   __device__ static constexpr int swz(int r) { return (r * CB / 128) % PPT; }
@@ -329,10 +330,11 @@ __global__ void __cluster_dims__(kAttnSplit, 1, 1)
   __syncthreads();
 
   // integer scores: per sub-group exponent, multiplier and digit sums, then
-  // this lane's B fragments (bq[ks][p]: digit p, k-step ks) and the
-  // accumulator start -8 sum B_p for its columns 2t, 2t + 1
+  // the CTA's table of B fragments (one uint2 per k-step, digit and lane,
+  // read back per chunk) and this lane's accumulator start -8 sum B_p for
+  // its columns 2t, 2t + 1
   const int gq = lane >> 2, tq = lane & 3;
-  uint32_t bq[kInt ? 4 : 1][3][2];
+  const uint32_t btab_a = smem_addr(smem + L::kBtab) + 8u * uint32_t(lane);
   int cinit[3][2];
   float qmul[2];
   if constexpr (kInt) {
@@ -361,25 +363,26 @@ __global__ void __cluster_dims__(kAttnSplit, 1, 1)
       for (int p = 0; p < 3; ++p) qsum[8 * p + tid] = sum[p];
     }
     __syncthreads();
-#pragma unroll
-    for (int ks = 0; ks < 4; ++ks) {
-      const int w = 4 * tq + ks;          // code word (8 coordinates) of this k-step
-      const bool on = (w >> 1) == gq;     // column gq is sub-group w / 2
+    // entry (ks, lane l, half hh): lane l = (row group g, thread t) holds, in
+    // byte i, digit p of coordinate 8 w + 2 i + hh of word w = 4 t + ks when
+    // column g is that word's sub-group w / 2, else 0
+    uint32_t* btab = reinterpret_cast<uint32_t*>(smem + L::kBtab);
+    for (int idx = tid; idx < 4 * 32 * 2; idx += NW * 32) {
+      const int hh = idx & 1, l = (idx >> 1) & 31, ks = idx >> 6;
+      const int w = 4 * (l & 3) + ks;
+      const bool on = (w >> 1) == (l >> 2);
       const int e = qe[w >> 1];
+      uint32_t r[3] = {0u, 0u, 0u};
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        uint32_t r[3] = {0u, 0u, 0u};
+      for (int i = 0; i < 4; ++i) {
+        int b[3];
+        const float qv = qs[8 * w + 2 * i + hh];
+        query_digits(on && qv == qv && fabsf(qv) <= 3.402823466e38f ? qv : 0.0f, e, b);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          int b[3];
-          const float qv = qs[8 * w + 2 * i + hh];
-          query_digits(on && qv == qv && fabsf(qv) <= 3.402823466e38f ? qv : 0.0f, e, b);
-#pragma unroll
-          for (int p = 0; p < 3; ++p) r[p] |= uint32_t(b[p] & 255) << (8 * i);
-        }
-#pragma unroll
-        for (int p = 0; p < 3; ++p) bq[ks][p][hh] = r[p];
+        for (int p = 0; p < 3; ++p) r[p] |= uint32_t(b[p] & 255) << (8 * i);
       }
+#pragma unroll
+      for (int p = 0; p < 3; ++p) btab[2 * (32 * (3 * ks + p) + l) + hh] = r[p];
     }
 #pragma unroll
     for (int p = 0; p < 3; ++p)
@@ -387,6 +390,7 @@ __global__ void __cluster_dims__(kAttnSplit, 1, 1)
       for (int jj = 0; jj < 2; ++jj) cinit[p][jj] = -8 * qsum[8 * p + 2 * tq + jj];
     qmul[0] = qm[2 * tq];
     qmul[1] = qm[2 * tq + 1];
+    __syncthreads();
   }
 
   // this CTA's tokens; warp w takes the 32-token chunks w, w + NW, ...
@@ -472,6 +476,15 @@ __global__ void __cluster_dims__(kAttnSplit, 1, 1)
     // scores, of this lane's own token 16 (t >> 1) + 8 (t & 1) + g
     float s[NQ];
     if constexpr (kInt) {
+      uint32_t bq[4][3][2];   // this lane's B fragments, held for the chunk's two tiles
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks)
+#pragma unroll
+        for (int p = 0; p < 3; ++p) {
+          const uint2 b = lds64(btab_a + uint32_t(256 * (3 * ks + p)));
+          bq[ks][p][0] = b.x;
+          bq[ks][p][1] = b.y;
+        }
       float srow[2][2];   // [16-token tile][row g, row g + 8]
 #pragma unroll
       for (int mt = 0; mt < 2; ++mt) {
