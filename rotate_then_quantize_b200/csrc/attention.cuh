@@ -25,7 +25,11 @@
 // of 32 tokens. A warp streams its chunks through a kAttnStages-deep
 // cp.async ring in shared memory (codes and scales of K and V), so data in
 // flight holds no registers, and runs its own online softmax:
-//   scores  lane i takes token i: decodes its 128 key codes (fp16
+//   scores  int4 keys with one query per KV head and groups of 16 or more:
+//           integer tensor-core products over 16 tokens at a time
+//           (mma.m16n8k32, u8 codes x s8 query digits, see below), one
+//           conversion per (token, 16-coordinate sub-group); otherwise
+//           lane i takes token i, decodes its 128 key codes (fp16
 //           magic-number decode, the scale applied by the same FMA) and
 //           dots them with the staged queries in packed f32x2 FMAs;
 //   softmax a warp-uniform running maximum and per-lane running sums;
