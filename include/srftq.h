@@ -192,7 +192,11 @@ int srftq_unrotate(const srftq_desc* desc, int64_t n_slices, int64_t n_rows, con
  * rounding). R is orthogonal ("When Quantization Is Free", Methodology 1),
  * so the kernel rotates each query once with the K signs, reads only codes
  * and scales, and undoes the V rotation once per output: it never writes a
- * dequantised cache and runs no inverse transform per token.
+ * dequantised cache and runs no inverse transform per token. Arithmetic is
+ * float32, except the key scores for int4 codes with q_per_kv = 1 and
+ * group >= 16. There the rotated query is held as integers, exact to 2^-22
+ * of its largest value in each run of 16 coordinates, and multiplied with
+ * the codes on the integer tensor cores.
  *
  *   q        [n_seq][heads*q_per_kv][d] fp16
  *   k_codes, v_codes    rows of [heads][d*bits/8] uint8; k_scales, v_scales
