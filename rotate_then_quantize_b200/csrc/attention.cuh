@@ -62,6 +62,9 @@ constexpr int kAttnWarps = 4;     // warps per CTA, each with its own online sof
 #ifndef SRFTQ_ATTN_VW
 #define SRFTQ_ATTN_VW 0   // 0: two words with one or two query heads, one with more
 #endif
+#ifndef SRFTQ_ATTN_PDL
+#define SRFTQ_ATTN_PDL 1  // programmatic launches of the attention and unrotation grids
+#endif
 constexpr int kAttnStages = SRFTQ_ATTN_STAGES;   // 32-token chunks in flight per warp
 
 struct AttnArgs {
@@ -125,6 +128,7 @@ template <int ROT, int NQ>
 __global__ void __launch_bounds__(128) attn_query_kernel(const AttnArgs a) {
   constexpr int D = 128;
   constexpr float kLog2e = 1.4426950408889634f;
+  asm volatile("griddepcontrol.launch_dependents;");   // the attention grid waits for this one
   const int64_t total = a.n_seq * a.heads * NQ;
   for (int64_t v_id = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; v_id < total;
        v_id += int64_t(gridDim.x) * blockDim.x) {
@@ -152,6 +156,7 @@ __global__ void __launch_bounds__(128) attn_query_kernel(const AttnArgs a) {
 template <int ROT, int NQ>
 __global__ void __launch_bounds__(128) attn_unrotate_kernel(const AttnArgs a) {
   constexpr int D = 128;
+  asm volatile("griddepcontrol.wait;" ::: "memory");   // the attention grid's outputs
   const int64_t total = a.n_seq * a.heads * NQ;
   for (int64_t v_id = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; v_id < total;
        v_id += int64_t(gridDim.x) * blockDim.x) {
@@ -326,6 +331,70 @@ __global__ void __cluster_dims__(kAttnSplit, 1, 1)
   const uint32_t wst_a = smem_addr(wst);
   const uint32_t qs_a = smem_addr(qs);
 
+  // this CTA's tokens; warp w takes the 32-token chunks w, w + NW, ...
+  const int64_t per = (a.n_ctx + kAttnSplit - 1) / kAttnSplit;
+  const int64_t t_begin = rank * per;
+  const int64_t t_end = t_begin + per < a.n_ctx ? t_begin + per : a.n_ctx;
+  const int64_t bs = b * a.seq_stride_rows;
+  auto vec_of = [&](int64_t t) { return (t * a.tok_stride_rows + bs) * a.heads + h; };
+  const int64_t n_chunks =
+      t_end > t_begin + 32 * warp ? (t_end - t_begin - 32 * warp + 32 * NW - 1) / (32 * NW) : 0;
+
+  // Copies chunk c of this warp into stage c % NS (one cp.async group; an
+  // empty group past the last chunk keeps the group count uniform).
+  auto issue = [&](int64_t c) {
+    if (c < n_chunks) {
+      const int64_t t0 = t_begin + 32 * (warp + NW * c);
+      const int nt = int(t_end - t0 < 32 ? t_end - t0 : 32);
+      const uint32_t st = wst_a + uint32_t(c % NS) * L::kStage;
+      const int pc = lane % PPT;
+#pragma unroll
+      for (int k = 0; k < PPT; ++k) {
+        const int r = lane / PPT + (32 / PPT) * k;
+        const int64_t vec = vec_of(t0 + r);
+        if (r < nt && dbg_ok(vec < a.rows * a.heads, a.guard)) {
+          const uint32_t o = uint32_t(r * CB + ((pc ^ L::swz(r)) * 16));
+          cp_async<16>(st + L::KC + o, a.k_codes + vec * CB + pc * 16);
+          cp_async<16>(st + L::VC + o, a.v_codes + vec * CB + pc * 16);
+        }
+      }
+      const int64_t svec = vec_of(t0 + lane);
+      if (lane < nt && dbg_ok(svec < a.rows * a.heads, a.guard)) {
+        const int64_t vec = svec;
+        const uint32_t o = uint32_t(lane * SBS);
+        const uint16_t* ks = a.k_scales + vec * NG;
+        const uint16_t* vs = a.v_scales + vec * NG;
+        if constexpr (SB >= 16) {
+#pragma unroll
+          for (int q = 0; q < SB / 16; ++q) {
+            cp_async<16>(st + L::KS + o + 16 * q, ks + 8 * q);
+            cp_async<16>(st + L::VS + o + 16 * q, vs + 8 * q);
+          }
+        } else if constexpr (SB >= 4) {
+          cp_async<SB>(st + L::KS + o, ks);
+          cp_async<SB>(st + L::VS + o, vs);
+        } else {
+          // one scale per vector (2 bytes, below the smallest cp.async)
+          *reinterpret_cast<uint16_t*>(wst + (c % NS) * L::kStage + L::KS + o) = ks[0];
+          *reinterpret_cast<uint16_t*>(wst + (c % NS) * L::kStage + L::VS + o) = vs[0];
+        }
+      } else {
+        // past the end: value scale 0, so the stale codes there decode to 0
+        uint8_t* z = wst + (c % NS) * L::kStage + L::VS + lane * SBS;
+#pragma unroll
+        for (int q = 0; q < SBS / 4; ++q) reinterpret_cast<uint32_t*>(z)[q] = 0u;
+      }
+    }
+    cp_async_commit();
+  };
+
+  // the first chunks' copies read only the caches, so they start before the
+  // queries are ready; with a programmatic launch the queries come from the
+  // grid launched just before, which this waits for (a no-op otherwise)
+#pragma unroll
+  for (int c = 0; c < NS - 1; ++c) issue(c);
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+
   // int4 keys decode their odd coordinates 16 times too large (decode8);
   // the integer scores take the codes exactly
   constexpr bool kInt = attn_int_scores<BITS, G, NQ>();
@@ -397,63 +466,6 @@ __global__ void __cluster_dims__(kAttnSplit, 1, 1)
     __syncthreads();
   }
 
-  // this CTA's tokens; warp w takes the 32-token chunks w, w + NW, ...
-  const int64_t per = (a.n_ctx + kAttnSplit - 1) / kAttnSplit;
-  const int64_t t_begin = rank * per;
-  const int64_t t_end = t_begin + per < a.n_ctx ? t_begin + per : a.n_ctx;
-  const int64_t bs = b * a.seq_stride_rows;
-  auto vec_of = [&](int64_t t) { return (t * a.tok_stride_rows + bs) * a.heads + h; };
-  const int64_t n_chunks =
-      t_end > t_begin + 32 * warp ? (t_end - t_begin - 32 * warp + 32 * NW - 1) / (32 * NW) : 0;
-
-  // Copies chunk c of this warp into stage c % NS (one cp.async group; an
-  // empty group past the last chunk keeps the group count uniform).
-  auto issue = [&](int64_t c) {
-    if (c < n_chunks) {
-      const int64_t t0 = t_begin + 32 * (warp + NW * c);
-      const int nt = int(t_end - t0 < 32 ? t_end - t0 : 32);
-      const uint32_t st = wst_a + uint32_t(c % NS) * L::kStage;
-      const int pc = lane % PPT;
-#pragma unroll
-      for (int k = 0; k < PPT; ++k) {
-        const int r = lane / PPT + (32 / PPT) * k;
-        const int64_t vec = vec_of(t0 + r);
-        if (r < nt && dbg_ok(vec < a.rows * a.heads, a.guard)) {
-          const uint32_t o = uint32_t(r * CB + ((pc ^ L::swz(r)) * 16));
-          cp_async<16>(st + L::KC + o, a.k_codes + vec * CB + pc * 16);
-          cp_async<16>(st + L::VC + o, a.v_codes + vec * CB + pc * 16);
-        }
-      }
-      const int64_t svec = vec_of(t0 + lane);
-      if (lane < nt && dbg_ok(svec < a.rows * a.heads, a.guard)) {
-        const int64_t vec = svec;
-        const uint32_t o = uint32_t(lane * SBS);
-        const uint16_t* ks = a.k_scales + vec * NG;
-        const uint16_t* vs = a.v_scales + vec * NG;
-        if constexpr (SB >= 16) {
-#pragma unroll
-          for (int q = 0; q < SB / 16; ++q) {
-            cp_async<16>(st + L::KS + o + 16 * q, ks + 8 * q);
-            cp_async<16>(st + L::VS + o + 16 * q, vs + 8 * q);
-          }
-        } else if constexpr (SB >= 4) {
-          cp_async<SB>(st + L::KS + o, ks);
-          cp_async<SB>(st + L::VS + o, vs);
-        } else {
-          // one scale per vector (2 bytes, below the smallest cp.async)
-          *reinterpret_cast<uint16_t*>(wst + (c % NS) * L::kStage + L::KS + o) = ks[0];
-          *reinterpret_cast<uint16_t*>(wst + (c % NS) * L::kStage + L::VS + o) = vs[0];
-        }
-      } else {
-        // past the end: value scale 0, so the stale codes there decode to 0
-        uint8_t* z = wst + (c % NS) * L::kStage + L::VS + lane * SBS;
-#pragma unroll
-        for (int q = 0; q < SBS / 4; ++q) reinterpret_cast<uint32_t*>(z)[q] = 0u;
-      }
-    }
-    cp_async_commit();
-  };
-
   float m[NQ], l[NQ];          // running max (warp-uniform) and this lane's sum
   float2 vacc[NQ][4 * VW];     // sum p sigma c, coordinates 8 VW vwi ..
 #pragma unroll
@@ -466,8 +478,6 @@ __global__ void __cluster_dims__(kAttnSplit, 1, 1)
   const int vwi = lane % LPT;  // value phase: words VW vwi .. of the row
   const int vt0 = lane / LPT;  // value phase: tokens vt0, vt0 + TPI, ... of the chunk
 
-#pragma unroll
-  for (int c = 0; c < NS - 1; ++c) issue(c);
   for (int64_t c = 0; c < n_chunks; ++c) {
     issue(c + NS - 1);
     cp_async_wait<NS - 1>();   // chunk c has landed (this lane's copies) ...
@@ -664,6 +674,8 @@ __global__ void __cluster_dims__(kAttnSplit, 1, 1)
   }
   cp_async_wait<0>();
   __syncwarp();
+  // the unrotation may be scheduled once every CTA is merging
+  asm volatile("griddepcontrol.launch_dependents;");
 
   // warp totals: the lanes' sums, and the lanes vwi, vwi + LPT, ... (same
   // coordinates), into the warp's first stage

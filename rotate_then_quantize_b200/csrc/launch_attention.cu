@@ -35,8 +35,32 @@ int launch_decode_attention_d128(const AttnCall& c) {
             rc = prepare_kernel<K>(smem, kAttnWarps * 32, &bps);
             if (rc != SRFTQ_OK) return;
             attn_query_kernel<ROT, NQ><<<g1, 128, 0, c.stream>>>(a);
-            K<<<int(blocks), kAttnWarps * 32, smem, c.stream>>>(a);
-            attn_unrotate_kernel<ROT, NQ><<<g1, 128, 0, c.stream>>>(a);
+            // the attention and unrotation grids are programmatic launches:
+            // each may start while the grid before it finishes and waits for
+            // its results with griddepcontrol.wait (attention.cuh)
+            cudaLaunchAttribute pdl[1];
+            pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+            pdl[0].val.programmaticStreamSerializationAllowed = SRFTQ_ATTN_PDL;
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3(unsigned(blocks));
+            cfg.blockDim = dim3(kAttnWarps * 32);
+            cfg.dynamicSmemBytes = size_t(smem);
+            cfg.stream = c.stream;
+            cfg.attrs = pdl;
+            cfg.numAttrs = 1;
+            if (cudaLaunchKernelEx(&cfg, K, a) != cudaSuccess) {
+              (void)cudaGetLastError();
+              rc = SRFTQ_ERR_CUDA;
+              return;
+            }
+            cfg.gridDim = dim3(unsigned(g1));
+            cfg.blockDim = dim3(128);
+            cfg.dynamicSmemBytes = 0;
+            if (cudaLaunchKernelEx(&cfg, attn_unrotate_kernel<ROT, NQ>, a) != cudaSuccess) {
+              (void)cudaGetLastError();
+              rc = SRFTQ_ERR_CUDA;
+              return;
+            }
             rc = finish_launch();
           }
         });
