@@ -19,6 +19,10 @@
 //                         (the rotated-domain output) back into `out`;
 //   attn_unrotate_kernel  one thread per output: s_V * R_V^T, in place.
 // The main kernel then carries no transform and stays small in registers.
+// The second and third are programmatic launches: each may start while the
+// grid before it finishes, and waits (griddepcontrol.wait) before it reads
+// that grid's results. The attention CTAs issue their first chunk's copies
+// before that wait, since those read only the caches.
 //
 // Main kernel: one cluster of kAttnSplit CTAs per (b, h); CTA r takes the
 // r-th slice of the tokens and each of its warps every kAttnWarps-th chunk
